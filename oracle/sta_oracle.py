@@ -1,0 +1,286 @@
+"""fp64 CPU oracle (test infrastructure only; see the package docstring).
+
+Readings taken where the pages leave a step open are stated beside each
+function. Arrays are numpy; floating-point work is float64 on values that
+are exactly the bf16 inputs.
+"""
+import math
+
+import numpy as np
+
+TILE = (1, 8, 8)  # tokens per tile along (t, y, x); 64 tokens
+TILE_TOKENS = 64
+MASS_ONE = 1 << 24  # fixed-point unit of the selection mass
+
+
+# --------------------------------------------------------------------------
+# Token layout (Compact Attention abstract: "tile-aligned mask family";
+# Table III "Cubic" component).
+# Reading: 1x8x8 tiles; tiles numbered in (t, tile-row, tile-column) raster
+# order; tokens inside a tile row-major in (y, x); heads moved to dim 1;
+# grids not divisible by 8 are padded with zero rows at the right / bottom.
+# --------------------------------------------------------------------------
+def tile_grid(T, H, W):
+    """(NH, NW, Nt, Lpad) for a T x H x W token grid."""
+    nh = (H + 7) // 8
+    nw = (W + 7) // 8
+    nt = T * nh * nw
+    return nh, nw, nt, TILE_TOKENS * nt
+
+
+def tiled_row_of_raster(T, H, W):
+    """For each raster token i = (t*H + y)*W + x, its row in the tiled layout."""
+    nh, nw, _, _ = tile_grid(T, H, W)
+    out = np.empty(T * H * W, dtype=np.int64)
+    i = 0
+    for t in range(T):
+        for y in range(H):
+            for x in range(W):
+                n = (t * nh + y // 8) * nw + x // 8
+                out[i] = TILE_TOKENS * n + (y % 8) * 8 + (x % 8)
+                i += 1
+    return out
+
+
+def valid_rows(T, H, W):
+    """Boolean [Lpad]: True where the tiled row holds a real token."""
+    _, _, _, lpad = tile_grid(T, H, W)
+    v = np.zeros(lpad, dtype=bool)
+    v[tiled_row_of_raster(T, H, W)] = True
+    return v
+
+
+def reorder_fwd(x, T, H, W):
+    """Raster [B, L, heads, d] -> tiled [B, heads, Lpad, d]; pad rows are 0."""
+    x = np.asarray(x)
+    B, L, Hh, d = x.shape
+    assert L == T * H * W
+    _, _, _, lpad = tile_grid(T, H, W)
+    out = np.zeros((B, Hh, lpad, d), dtype=x.dtype)
+    rows = tiled_row_of_raster(T, H, W)
+    out[:, :, rows, :] = np.transpose(x, (0, 2, 1, 3))
+    return out
+
+
+def reorder_inv(xt, T, H, W):
+    """Tiled [B, heads, Lpad, d] -> raster [B, L, heads, d]; pad rows dropped."""
+    xt = np.asarray(xt)
+    rows = tiled_row_of_raster(T, H, W)
+    return np.ascontiguousarray(np.transpose(xt[:, :, rows, :], (0, 2, 1, 3)))
+
+
+# --------------------------------------------------------------------------
+# Pooled block scores (Rectified SpaAttn abstract: weights recovered from the
+# pooled query-key).
+# Reading: the mean over the real tokens of each tile (pads excluded); score
+# scale 1/sqrt(d) unless given; softmax over all key tiles of the row.
+# --------------------------------------------------------------------------
+def pool(xt, T, H, W):
+    """Tiled [B, heads, Lpad, d] -> per-tile means [B, heads, Nt, d] (fp64)."""
+    xt = np.asarray(xt)
+    B, Hh, lpad, d = xt.shape
+    _, _, nt, lp = tile_grid(T, H, W)
+    assert lpad == lp
+    valid = valid_rows(T, H, W).reshape(nt, TILE_TOKENS)
+    cnt = valid.sum(axis=1).astype(np.float64)
+    out = np.empty((B, Hh, nt, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hh):
+            tiles = xt[b, h].astype(np.float64).reshape(nt, TILE_TOKENS, d)
+            s = np.einsum("nr,nrd->nd", valid.astype(np.float64), tiles)
+            out[b, h] = s / cnt[:, None]
+    return out
+
+
+def block_scores(qbar, kbar, scale):
+    """S = scale * qbar kbar^T and its row softmax P, both [B, heads, Nt, Nt]."""
+    qbar = np.asarray(qbar, dtype=np.float64)
+    kbar = np.asarray(kbar, dtype=np.float64)
+    s = np.einsum("bhqd,bhkd->bhqk", qbar, kbar) * float(scale)
+    m = s.max(axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    p = e / e.sum(axis=-1, keepdims=True)
+    return s, p
+
+
+# --------------------------------------------------------------------------
+# Hybrid top-p / fixed top-k selection (SCOPE review, Eqs. (7)-(8) as quoted:
+# keep the smallest set reaching mass rho, with a fixed floor of keys).
+# Reading, at tile granularity:
+#   order  : key tiles by P descending, ties to the lower key-tile index;
+#   mass   : w_j = floor(P_j * 2^24) (integers, exact in any summation order);
+#   thr    : ceil(double(top_p) * double(sum_j w_j)), top_p taken as float32;
+#   m_p    : smallest m whose first m tiles reach thr; Nt if top_p >= 1,
+#            0 if top_p <= 0;
+#   keep   : the first max(m_p, min(k_min, Nt)) tiles of the order.
+# --------------------------------------------------------------------------
+def select_row(p_row, top_p, k_min):
+    """Boolean [Nt] keep-set for one row of block probabilities."""
+    p = np.asarray(p_row, dtype=np.float64)
+    nt = p.shape[0]
+    order = sorted(range(nt), key=lambda j: (-p[j], j))
+    w = [int(math.floor(float(p[j]) * MASS_ONE)) for j in range(nt)]
+    total = sum(w)
+    tp = float(np.float32(top_p))
+    if tp >= 1.0:
+        m_p = nt
+    elif tp <= 0.0:
+        m_p = 0
+    else:
+        thr = math.ceil(tp * float(total))
+        acc = 0
+        m_p = nt
+        for m in range(nt + 1):
+            if acc >= thr:
+                m_p = m
+                break
+            if m < nt:
+                acc += w[order[m]]
+    m = max(m_p, min(int(k_min), nt))
+    keep = np.zeros(nt, dtype=bool)
+    keep[order[:m]] = True
+    return keep
+
+
+def select(P, top_p, k_min):
+    """Row-wise select() over the last axis of P."""
+    P = np.asarray(P)
+    flat = P.reshape(-1, P.shape[-1])
+    out = np.stack([select_row(r, top_p, k_min) for r in flat])
+    return out.reshape(P.shape)
+
+
+# --------------------------------------------------------------------------
+# Deformable dual window per temporal-distance group (Compact Attention
+# Fig. 1(3), Fig. 4; Table III "Frame-group" and "Dual Window").
+# Reading: in tile units, key tile kt is kept for query tile qt of head h iff
+# group g (the last g with group_lo[g] <= |dt|) exists and
+#   (|dy| <= ry1 and |dx| <= rx1) or (|dy| <= ry2 and |dx| <= rx2)
+# with (ry1, rx1, ry2, rx2) = windows[h, g]; -1 switches a window off;
+# rectangles are centred on the query tile and clipped at the grid edge.
+# --------------------------------------------------------------------------
+def window_mask(windows, group_lo, T, H, W):
+    """Boolean [heads, Nt, Nt] dual-window mask."""
+    windows = np.asarray(windows, dtype=np.int64)
+    Hh, G, four = windows.shape
+    assert four == 4 and len(group_lo) == G
+    nh, nw, nt, _ = tile_grid(T, H, W)
+    idx = np.arange(nt)
+    tt, ty, tx = idx // (nh * nw), (idx // nw) % nh, idx % nw
+    dt = np.abs(tt[:, None] - tt[None, :])
+    dy = np.abs(ty[:, None] - ty[None, :])
+    dx = np.abs(tx[:, None] - tx[None, :])
+    grp = np.full((nt, nt), -1, dtype=np.int64)
+    for g in range(G):
+        grp[dt >= int(group_lo[g])] = g
+    out = np.zeros((Hh, nt, nt), dtype=bool)
+    for h in range(Hh):
+        for g in range(G):
+            ry1, rx1, ry2, rx2 = windows[h, g]
+            in_g = grp == g
+            w1 = (dy <= ry1) & (dx <= rx1)
+            w2 = (dy <= ry2) & (dx <= rx2)
+            out[h] |= in_g & (w1 | w2)
+    return out
+
+
+def mask_to_csr(mask):
+    """Boolean [..., Nt, Nt] -> (row_ptr int32 [R+1], col_idx int32 [nnz]);
+    rows are the flattened leading axes, columns ascending."""
+    m = np.asarray(mask, dtype=bool)
+    nt = m.shape[-1]
+    flat = m.reshape(-1, nt)
+    counts = flat.sum(axis=1)
+    row_ptr = np.zeros(flat.shape[0] + 1, dtype=np.int64)
+    row_ptr[1:] = np.cumsum(counts)
+    cols = [np.nonzero(r)[0] for r in flat]
+    col_idx = np.concatenate(cols) if cols else np.zeros(0, dtype=np.int64)
+    return row_ptr.astype(np.int32), col_idx.astype(np.int32)
+
+
+def build_mask(q_tiled, k_tiled, T, H, W, use_scores, top_p, k_min,
+               windows=None, group_lo=None, sm_scale=0.0):
+    """Full mask construction: pool, score, select, OR windows, emit CSR.
+
+    Returns dict(mask [B,heads,Nt,Nt] bool, probs [B,heads,Nt,Nt] fp64 or
+    None, row_ptr, col_idx).
+    """
+    q_tiled = np.asarray(q_tiled)
+    B, Hh, _, d = q_tiled.shape
+    _, _, nt, _ = tile_grid(T, H, W)
+    scale = float(sm_scale) if sm_scale else 1.0 / math.sqrt(d)
+    mask = np.zeros((B, Hh, nt, nt), dtype=bool)
+    probs = None
+    if use_scores:
+        qbar = pool(q_tiled, T, H, W)
+        kbar = pool(k_tiled, T, H, W)
+        _, probs = block_scores(qbar, kbar, scale)
+        mask |= select(probs, top_p, k_min)
+    if windows is not None:
+        mask |= window_mask(windows, group_lo, T, H, W)[None]
+    row_ptr, col_idx = mask_to_csr(mask)
+    return dict(mask=mask, probs=probs, row_ptr=row_ptr, col_idx=col_idx)
+
+
+# --------------------------------------------------------------------------
+# Masked softmax attention over the listed key tiles (Compact Attention
+# Fig. 3: precomputed masks loaded into block-sparse attention kernels).
+# Definition: for each real query token of query tile qt,
+#   o = sum_j softmax_j(scale * q . k_j) v_j,  LSE = log sum_j exp(scale q.k_j)
+# over the real tokens j of the listed key tiles. An empty list gives o = 0
+# and LSE = -inf. Padded query rows are not defined and not returned.
+# --------------------------------------------------------------------------
+def attention_rows(q_tiled, k_tiled, v_tiled, row_ptr, col_idx, T, H, W,
+                   sm_scale, rows):
+    """Attention for the CSR rows listed in `rows` (flat (b*heads + h)*Nt + qt).
+
+    Returns a list of (row, token_rows, O [n_q, d] fp64, LSE [n_q] fp64),
+    token_rows being the tiled-layout rows of the real query tokens.
+    """
+    q_tiled = np.asarray(q_tiled)
+    B, Hh, lpad, d = q_tiled.shape
+    _, _, nt, _ = tile_grid(T, H, W)
+    valid = valid_rows(T, H, W)
+    scale = float(sm_scale) if sm_scale else 1.0 / math.sqrt(d)
+    out = []
+    for r in rows:
+        r = int(r)
+        bh, qt = divmod(r, nt)
+        b, h = divmod(bh, Hh)
+        qrows = np.arange(qt * 64, qt * 64 + 64)
+        qrows = qrows[valid[qrows]]
+        q = q_tiled[b, h, qrows].astype(np.float64)
+        tiles = np.asarray(col_idx[int(row_ptr[r]):int(row_ptr[r + 1])], dtype=np.int64)
+        if tiles.size == 0:
+            out.append((r, qrows, np.zeros((qrows.size, d)), np.full(qrows.size, -np.inf)))
+            continue
+        krows = (tiles[:, None] * 64 + np.arange(64)[None, :]).reshape(-1)
+        krows = krows[valid[krows]]
+        k = np.asarray(k_tiled)[b, h, krows].astype(np.float64)
+        v = np.asarray(v_tiled)[b, h, krows].astype(np.float64)
+        s = (q @ k.T) * scale
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        z = e.sum(axis=1, keepdims=True)
+        o = (e / z) @ v
+        lse = (m + np.log(z))[:, 0]
+        out.append((r, qrows, o, lse))
+    return out
+
+
+def attention_all(q_tiled, k_tiled, v_tiled, row_ptr, col_idx, T, H, W, sm_scale):
+    """Attention for every row; returns O [B, heads, Lpad, d] (pad rows NaN)
+    and LSE [B, heads, Lpad] (pad rows NaN)."""
+    q_tiled = np.asarray(q_tiled)
+    B, Hh, lpad, d = q_tiled.shape
+    _, _, nt, _ = tile_grid(T, H, W)
+    O = np.full((B, Hh, lpad, d), np.nan)
+    LSE = np.full((B, Hh, lpad), np.nan)
+    res = attention_rows(q_tiled, k_tiled, v_tiled, row_ptr, col_idx, T, H, W,
+                         sm_scale, range(B * Hh * nt))
+    for r, qrows, o, lse in res:
+        bh, _ = divmod(r, nt)
+        b, h = divmod(bh, Hh)
+        O[b, h, qrows] = o
+        LSE[b, h, qrows] = lse
+    return O, LSE

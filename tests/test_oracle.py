@@ -1,0 +1,387 @@
+"""Pins for the fp64 oracle: closed forms, textbook routines, brute force.
+
+None of these call the CUDA path. Each test is chosen so that a plausible
+slip in the oracle (a dropped pad exclusion, a wrong tile index, a flipped
+comparison, a transposed operand, an off-by-one in the threshold) fails it.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle as O
+
+RNG = np.random.default_rng(12345)
+
+
+def _bf16_exact(shape, rng, scale=1.0):
+    x = torch.from_numpy(rng.standard_normal(shape) * scale).to(torch.bfloat16)
+    return x.to(torch.float64).numpy()
+
+
+# ----------------------------------------------------------------- layout
+def test_tile_grid_matches_workload_table():
+    # Sizes of the five workloads (padded to whole 1x8x8 tiles).
+    assert O.tile_grid(4, 16, 16) == (2, 2, 16, 1024)
+    assert O.tile_grid(21, 30, 52) == (4, 7, 588, 37632)
+    assert O.tile_grid(21, 45, 80) == (6, 10, 1260, 80640)
+    assert O.tile_grid(33, 45, 80) == (6, 10, 1980, 126720)
+
+
+def test_reorder_golden(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "reorder_cases.json")))
+    T, H, W = g["grid"]["T"], g["grid"]["H"], g["grid"]["W"]
+    assert O.tile_grid(T, H, W) == (g["grid"]["NH"], g["grid"]["NW"], g["grid"]["Nt"], g["grid"]["Lpad"])
+    rows = O.tiled_row_of_raster(T, H, W)
+    for tok in g["tokens"]:
+        i = (tok["t"] * H + tok["y"]) * W + tok["x"]
+        assert rows[i] == tok["row"], tok
+    v = O.valid_rows(T, H, W).reshape(-1, 64).sum(axis=1)
+    assert v.tolist() == g["valid_rows_per_tile"]
+
+
+@pytest.mark.parametrize("T,H,W", [(2, 9, 10), (3, 13, 19), (1, 16, 8), (2, 1, 1)])
+def test_reorder_tiles_are_spatial_blocks(T, H, W):
+    """Every tile holds the tokens of one frame inside one 8x8 block, row-major;
+    pad rows are zero; the map is a bijection onto the real rows."""
+    nh, nw, nt, lpad = O.tile_grid(T, H, W)
+    L = T * H * W
+    t, y, x = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    # encode coordinates (+1 so that pads, which are 0, are distinguishable)
+    x_r = np.stack([t.ravel() + 1, y.ravel() + 1, x.ravel() + 1], axis=1).astype(np.float64)
+    x_r = x_r.reshape(1, L, 1, 3)
+    xt = O.reorder_fwd(x_r, T, H, W)[0, 0]  # [Lpad, 3]
+    assert xt.shape == (lpad, 3)
+    real = xt[:, 0] > 0
+    assert real.sum() == L
+    assert np.all(xt[~real] == 0)
+    tiles = xt.reshape(nt, 64, 3)
+    for n in range(nt):
+        tn, tyn, txn = n // (nh * nw), (n // nw) % nh, n % nw
+        for r in range(64):
+            if tiles[n, r, 0] == 0:
+                # a pad row must be outside the grid
+                yy, xx = 8 * tyn + r // 8, 8 * txn + r % 8
+                assert yy >= H or xx >= W
+                continue
+            tt, yy, xx = (tiles[n, r] - 1).astype(int)
+            assert tt == tn
+            assert yy == 8 * tyn + r // 8 and xx == 8 * txn + r % 8
+    back = O.reorder_inv(O.reorder_fwd(x_r, T, H, W), T, H, W)
+    assert np.array_equal(back, x_r)
+
+
+def test_reorder_roundtrip_multihead():
+    T, H, W = 3, 11, 17
+    x = _bf16_exact((2, T * H * W, 3, 8), RNG)
+    xt = O.reorder_fwd(x, T, H, W)
+    assert xt.shape == (2, 3, O.tile_grid(T, H, W)[3], 8)
+    assert np.array_equal(O.reorder_inv(xt, T, H, W), x)
+    # heads and batches do not mix: head h of the tiled tensor holds only head h
+    for b in range(2):
+        for h in range(3):
+            assert np.array_equal(O.reorder_inv(xt[b:b + 1, h:h + 1], T, H, W)[0, :, 0], x[b, :, h])
+
+
+# ---------------------------------------------------------------- pooling
+def test_pool_closed_form_linear_field():
+    """x(t, y, x) = a + b t + c y + e x: the mean over the real tokens of tile
+    (t, ty, tx) with vy x vx real tokens is a + b t + c (8 ty + (vy-1)/2)
+    + e (8 tx + (vx-1)/2) (arithmetic series)."""
+    T, H, W = 3, 13, 21
+    a, bb, c, e = 0.5, -1.25, 0.75, 2.0
+    t, y, x = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    f = (a + bb * t + c * y + e * x).ravel()
+    xr = f.reshape(1, -1, 1, 1)
+    p = O.pool(O.reorder_fwd(xr, T, H, W), T, H, W)[0, 0, :, 0]
+    nh, nw, nt, _ = O.tile_grid(T, H, W)
+    for n in range(nt):
+        tn, ty, tx = n // (nh * nw), (n // nw) % nh, n % nw
+        vy, vx = min(8, H - 8 * ty), min(8, W - 8 * tx)
+        want = a + bb * tn + c * (8 * ty + (vy - 1) / 2) + e * (8 * tx + (vx - 1) / 2)
+        assert abs(p[n] - want) < 1e-12
+
+
+def test_pool_excludes_pads():
+    T, H, W = 2, 9, 10
+    xr = np.ones((1, T * H * W, 2, 4))
+    p = O.pool(O.reorder_fwd(xr, T, H, W), T, H, W)
+    assert np.allclose(p, 1.0, atol=0, rtol=1e-15)
+
+
+def test_pooled_score_is_mean_of_token_pair_logits():
+    """scale * qbar . kbar equals the mean over all (query token, key token)
+    pairs of scale * q . k (bilinearity), computed here by brute force."""
+    T, H, W, d = 2, 9, 10, 6
+    q = _bf16_exact((1, T * H * W, 1, d), RNG)
+    k = _bf16_exact((1, T * H * W, 1, d), RNG)
+    qt, kt = O.reorder_fwd(q, T, H, W), O.reorder_fwd(k, T, H, W)
+    s, p = O.block_scores(O.pool(qt, T, H, W), O.pool(kt, T, H, W), 0.3)
+    valid = O.valid_rows(T, H, W)
+    nt = O.tile_grid(T, H, W)[2]
+    for a in range(nt):
+        for b in range(nt):
+            qa = [qt[0, 0, r] for r in range(64 * a, 64 * a + 64) if valid[r]]
+            kb = [kt[0, 0, r] for r in range(64 * b, 64 * b + 64) if valid[r]]
+            tot = 0.0
+            for u in qa:
+                for w in kb:
+                    tot += float(np.dot(u, w))
+            assert abs(s[0, 0, a, b] - 0.3 * tot / (len(qa) * len(kb))) < 1e-10
+    assert np.allclose(p[0, 0], scipy.special.softmax(s[0, 0], axis=-1), rtol=1e-13, atol=1e-15)
+    assert np.allclose(p.sum(-1), 1.0, atol=1e-13)
+
+
+# -------------------------------------------------------------- selection
+def test_select_golden(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "select_cases.json")))
+    for case in g["cases"]:
+        keep = O.select_row(np.array(case["p"]), case["top_p"], case["k_min"])
+        assert sorted(np.nonzero(keep)[0].tolist()) == case["keep"], case["name"]
+
+
+def test_select_top_p_one_keeps_all():
+    p = scipy.special.softmax(RNG.standard_normal((5, 37)) * 3, axis=-1)
+    for row in p:
+        assert O.select_row(row, 1.0, 0).all()
+        assert O.select_row(row, 1.5, 0).all()
+
+
+def test_select_top_p_zero_is_stable_topk():
+    p = scipy.special.softmax(RNG.standard_normal((6, 29)) * 2, axis=-1)
+    p[0, 3] = p[0, 7]  # a tie
+    for row in p:
+        for k in (0, 1, 5, 29, 40):
+            keep = O.select_row(row, 0.0, k)
+            want = np.argsort(-row, kind="stable")[: min(k, row.size)]
+            assert sorted(np.nonzero(keep)[0].tolist()) == sorted(want.tolist())
+
+
+def test_select_minimal_by_brute_force():
+    """On Nt = 12, the kept set (k_min = 0) is a smallest subset whose integer
+    mass reaches the threshold, and it is the prefix of the stated order."""
+    nt = 12
+    for trial in range(6):
+        row = scipy.special.softmax(RNG.standard_normal(nt) * (1 + trial), axis=-1)
+        for top_p in (0.3, 0.6, 0.9, 0.97):
+            keep = O.select_row(row, top_p, 0)
+            w = np.floor(row * 2 ** 24).astype(np.int64)
+            thr = math.ceil(float(np.float32(top_p)) * float(w.sum()))
+            best = None
+            for m in range(nt + 1):
+                if any(w[list(c)].sum() >= thr for c in itertools.combinations(range(nt), m)):
+                    best = m
+                    break
+            assert keep.sum() == best
+            assert w[keep].sum() >= thr
+            order = sorted(range(nt), key=lambda j: (-row[j], j))
+            assert set(np.nonzero(keep)[0]) == set(order[:best])
+
+
+def test_select_monotone_in_top_p_and_k_min():
+    row = scipy.special.softmax(RNG.standard_normal(50) * 2, axis=-1)
+    prev = np.zeros(50, dtype=bool)
+    for tp in np.linspace(0, 1, 21):
+        for km in (0, 3, 10):
+            keep = O.select_row(row, tp, km)
+            assert (O.select_row(row, tp, km + 1) >= keep).all()
+        keep0 = O.select_row(row, tp, 0)
+        assert (keep0 >= prev).all()
+        prev = keep0
+
+
+# ----------------------------------------------------------------- window
+def _window_count_closed_form(windows, group_lo, T, H, W, h, qt):
+    """Row count as a sum over frames of |R1 u R2| = |R1| + |R2| - |R1 n R2|
+    for two clipped rectangles centred on the query tile (inclusion-exclusion),
+    independent of the oracle's per-pair test."""
+    nh, nw, _, _ = O.tile_grid(T, H, W)
+    tq, yq, xq = qt // (nh * nw), (qt // nw) % nh, qt % nw
+
+    def span(c, r, n):
+        if r < 0:
+            return 0
+        return min(n - 1, c + r) - max(0, c - r) + 1
+
+    total = 0
+    for tk in range(T):
+        dt = abs(tq - tk)
+        gs = [g for g in range(len(group_lo)) if group_lo[g] <= dt]
+        if not gs:
+            continue
+        ry1, rx1, ry2, rx2 = windows[h, max(gs)]
+        a1 = span(yq, ry1, nh) * span(xq, rx1, nw)
+        a2 = span(yq, ry2, nh) * span(xq, rx2, nw)
+        ry3 = min(ry1, ry2) if min(ry1, rx1, ry2, rx2) >= 0 else -1
+        rx3 = min(rx1, rx2) if ry3 >= 0 else -1
+        a3 = span(yq, ry3, nh) * span(xq, rx3, nw)
+        total += a1 + a2 - a3
+    return total
+
+
+def test_window_counts_closed_form():
+    T, H, W = 5, 40, 56  # 5 x 5 x 7 tiles
+    windows = np.array([
+        [[1, 1, 0, 6], [0, 1, -1, -1], [-1, -1, -1, -1]],
+        [[2, 0, 0, 3], [1, 1, 4, 0], [0, 0, 0, 0]],
+        [[4, 6, -1, -1], [-1, -1, 2, 2], [1, 0, 0, 1]],
+    ], dtype=np.int32)
+    group_lo = [0, 1, 3]
+    m = O.window_mask(windows, group_lo, T, H, W)
+    nt = O.tile_grid(T, H, W)[2]
+    for h in range(3):
+        for qt in range(nt):
+            assert m[h, qt].sum() == _window_count_closed_form(windows, group_lo, T, H, W, h, qt)
+        assert np.array_equal(m[h], m[h].T)  # |dt|, |dy|, |dx| are symmetric
+
+
+def test_window_tiny_separates_local_and_axial():
+    """2 x 4 x 6 tile grid: local radius 1 plus full-row axial window for
+    |dt| = 0, nothing for |dt| >= 1: row count = 3x3-clipped block + rest of
+    the row, all in the query's own frame."""
+    T, H, W = 2, 32, 48
+    nh, nw, nt, _ = O.tile_grid(T, H, W)
+    windows = np.array([[[1, 1, 0, nw - 1], [-1, -1, -1, -1]]], dtype=np.int32)
+    m = O.window_mask(windows, [0, 1], T, H, W)[0]
+    # the last group is open-ended: one group [0] alone covers every frame
+    m_all = O.window_mask(windows[:, :1], [0], T, H, W)[0]
+    assert m_all.sum() == T * m.sum()
+    for qt in range(nt):
+        tq, yq, xq = qt // (nh * nw), (qt // nw) % nh, qt % nw
+        ny = min(nh - 1, yq + 1) - max(0, yq - 1) + 1
+        nx = min(nw - 1, xq + 1) - max(0, xq - 1) + 1
+        assert m[qt].sum() == ny * nx + (nw - nx)
+        # nothing in the other frame
+        other = [k for k in range(nt) if k // (nh * nw) != tq]
+        assert not m[qt, other].any()
+
+
+def test_window_monotone_in_extent():
+    T, H, W = 3, 24, 40
+    base = np.array([[[1, 1, 0, 2], [0, 0, -1, -1]]], dtype=np.int32)
+    m0 = O.window_mask(base, [0, 1], T, H, W)
+    for h_ in range(2):
+        for c in range(4):
+            wider = base.copy()
+            wider[0, h_, c] += 1
+            assert (O.window_mask(wider, [0, 1], T, H, W) >= m0).all()
+
+
+# -------------------------------------------------------------------- CSR
+def test_csr_invariants():
+    mask = RNG.random((2, 3, 9, 9)) < 0.3
+    mask[0, 1, 4] = False  # an empty row
+    rp, ci = O.mask_to_csr(mask)
+    assert rp[0] == 0 and rp[-1] == ci.size == mask.sum()
+    assert np.all(np.diff(rp) >= 0)
+    flat = mask.reshape(-1, 9)
+    for r in range(flat.shape[0]):
+        cols = ci[rp[r]:rp[r + 1]]
+        assert np.all(np.diff(cols) > 0)
+        assert set(cols.tolist()) == set(np.nonzero(flat[r])[0].tolist())
+
+
+def test_build_mask_union_of_parts():
+    T, H, W, d = 3, 16, 24, 8
+    q = _bf16_exact((1, T * H * W, 2, d), RNG, 2.0)
+    k = _bf16_exact((1, T * H * W, 2, d), RNG, 2.0)
+    qt, kt = O.reorder_fwd(q, T, H, W), O.reorder_fwd(k, T, H, W)
+    win = np.array([[[0, 0, -1, -1], [-1, -1, -1, -1]], [[1, 0, 0, 2], [0, 0, -1, -1]]], dtype=np.int32)
+    res = O.build_mask(qt, kt, T, H, W, True, 0.8, 2, win, [0, 1])
+    only_sel = O.build_mask(qt, kt, T, H, W, True, 0.8, 2, None, None)
+    only_win = O.build_mask(qt, kt, T, H, W, False, 0.0, 0, win, [0, 1])
+    assert np.array_equal(res["mask"], only_sel["mask"] | only_win["mask"])
+    assert np.array_equal(only_sel["mask"], O.select(res["probs"], 0.8, 2))
+    assert (only_sel["mask"].sum(-1) >= 2).all()
+
+
+# -------------------------------------------------------------- attention
+def _sdpa64(q, k, v, scale):
+    import torch.nn.functional as F
+    tq = torch.from_numpy(q)[None, None]
+    tk = torch.from_numpy(k)[None, None]
+    tv = torch.from_numpy(v)[None, None]
+    return F.scaled_dot_product_attention(tq, tk, tv, scale=scale)[0, 0].numpy()
+
+
+def test_dense_mask_equals_sdpa():
+    """A full mask reproduces dense softmax attention (torch SDPA, fp64)."""
+    T, H, W, d = 2, 16, 16, 16
+    q = _bf16_exact((1, T * H * W, 1, d), RNG)
+    k = _bf16_exact((1, T * H * W, 1, d), RNG)
+    v = _bf16_exact((1, T * H * W, 1, d), RNG)
+    qt, kt, vt = (O.reorder_fwd(a, T, H, W) for a in (q, k, v))
+    nt = O.tile_grid(T, H, W)[2]
+    rp, ci = O.mask_to_csr(np.ones((1, 1, nt, nt), dtype=bool))
+    Ot, lse = O.attention_all(qt, kt, vt, rp, ci, T, H, W, 0.0)
+    o_r = O.reorder_inv(Ot, T, H, W)[0, :, 0]
+    ref = _sdpa64(q[0, :, 0], k[0, :, 0], v[0, :, 0], 1 / math.sqrt(d))
+    assert np.allclose(o_r, ref, atol=1e-12, rtol=1e-12)
+    s = q[0, :, 0] @ k[0, :, 0].T / math.sqrt(d)
+    lse_ref = scipy.special.logsumexp(s, axis=1)
+    assert np.allclose(O.reorder_inv(lse[..., None], T, H, W)[0, :, 0, 0], lse_ref, atol=1e-12)
+
+
+def test_dense_mask_ragged_grid_equals_sdpa_over_real_tokens():
+    T, H, W, d = 2, 9, 13, 8
+    q = _bf16_exact((1, T * H * W, 1, d), RNG)
+    k = _bf16_exact((1, T * H * W, 1, d), RNG)
+    v = _bf16_exact((1, T * H * W, 1, d), RNG)
+    qt, kt, vt = (O.reorder_fwd(a, T, H, W) for a in (q, k, v))
+    nt = O.tile_grid(T, H, W)[2]
+    rp, ci = O.mask_to_csr(np.ones((1, 1, nt, nt), dtype=bool))
+    Ot, _ = O.attention_all(qt, kt, vt, rp, ci, T, H, W, 0.7)
+    ref = _sdpa64(q[0, :, 0], k[0, :, 0], v[0, :, 0], 0.7)
+    assert np.allclose(O.reorder_inv(Ot, T, H, W)[0, :, 0], ref, atol=1e-12)
+
+
+def test_attention_weights_convex():
+    """With V = 1 every output is exactly 1 (weights sum to one); outputs lie in
+    the per-coordinate range of the attended values."""
+    T, H, W, d = 2, 16, 24, 8
+    q = _bf16_exact((1, T * H * W, 2, d), RNG, 3.0)
+    k = _bf16_exact((1, T * H * W, 2, d), RNG, 3.0)
+    v = _bf16_exact((1, T * H * W, 2, d), RNG)
+    qt, kt, vt = (O.reorder_fwd(a, T, H, W) for a in (q, k, v))
+    nt = O.tile_grid(T, H, W)[2]
+    mask = RNG.random((1, 2, nt, nt)) < 0.4
+    mask[0, 0, 0] = False
+    rp, ci = O.mask_to_csr(mask)
+    ones = np.ones_like(vt)
+    res1 = O.attention_rows(qt, kt, ones, rp, ci, T, H, W, 0.0, range(2 * nt))
+    for r, qrows, o, lse in res1:
+        if rp[r + 1] > rp[r]:
+            assert np.allclose(o, 1.0, atol=1e-12)
+        else:
+            assert np.all(o == 0) and np.all(np.isneginf(lse))
+    res = O.attention_rows(qt, kt, vt, rp, ci, T, H, W, 0.0, range(2 * nt))
+    for r, qrows, o, lse in res:
+        tiles = ci[rp[r]:rp[r + 1]]
+        if tiles.size == 0:
+            continue
+        h = r // nt
+        rows = (tiles[:, None] * 64 + np.arange(64)).ravel()
+        vv = vt[0, h, rows]
+        assert np.all(o <= vv.max(axis=0) + 1e-12) and np.all(o >= vv.min(axis=0) - 1e-12)
+
+
+def test_single_tile_list_is_plain_softmax():
+    T, H, W, d = 1, 16, 16, 16
+    q = _bf16_exact((1, T * H * W, 1, d), RNG, 2.0)
+    k = _bf16_exact((1, T * H * W, 1, d), RNG, 2.0)
+    v = _bf16_exact((1, T * H * W, 1, d), RNG)
+    qt, kt, vt = (O.reorder_fwd(a, T, H, W) for a in (q, k, v))
+    rp = np.array([0, 1, 2, 3, 4], dtype=np.int32)
+    ci = np.array([3, 0, 2, 1], dtype=np.int32)
+    res = O.attention_rows(qt, kt, vt, rp, ci, T, H, W, 0.25, range(4))
+    for r, qrows, o, lse in res:
+        kk = kt[0, 0, 64 * ci[r]:64 * ci[r] + 64]
+        vv = vt[0, 0, 64 * ci[r]:64 * ci[r] + 64]
+        s = qt[0, 0, qrows] @ kk.T * 0.25
+        assert np.allclose(o, scipy.special.softmax(s, axis=1) @ vv, atol=1e-12)
+        assert np.allclose(lse, scipy.special.logsumexp(s, axis=1), atol=1e-12)
