@@ -1,0 +1,435 @@
+"""Benchmark of the block-sparse 3D-tile attention path on B200.
+
+One step = one pass of the whole hot path over one synthetic 720p video-DiT
+layer (75,600 tokens, 40 heads, d = 128, top-p 0.95 / k_min 8 OR dual
+windows, ~15% density): sta_reorder of Q, K, V -> sta_build_mask ->
+sta_attn_fwd -> sta_reorder of O back to raster order.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Rank 0 prints one JSON line. Under torchrun every rank runs its own layer
+(independent problems, no collective on the data path: weak scaling); the
+time is the max over ranks of the device-timed region.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import CONFIGS, make_qkv, window_params, window_scale  # noqa: E402
+
+METRIC = "kept-block attn TFLOP/s & % BF16 peak; ms/layer at 75,600 tokens, 15% density"
+UNIT = "TFLOP/s"
+CFG_INDEX = 2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def flops_per_pair(d):
+    return 4.0 * 64 * 64 * d
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attn_source_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "block_sparse_attention_28_b200", "csrc")
+    for name in ("sta_attn.cuh", "sta_tc.cuh", "sta_common.cuh"):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu
+    summary, or None when the summary is missing or the kernel changed."""
+    p = os.path.join(ROOT, "profiles", "attn_fwd_720p_traffic.md")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    for line in open(p):
+        if line.startswith("traffic_bytes_per_launch:"):
+            vals["t"] = float(line.split(":", 1)[1])
+        if line.startswith("kernel_source_hash:"):
+            vals["h"] = line.split(":", 1)[1].strip()
+    if vals.get("h") != attn_source_hash():
+        return None
+    return vals.get("t")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+class Layer:
+    """Device buffers and launches of one step of the path."""
+
+    def __init__(self, sta, cfg, dev, seed_offset=0):
+        from dataclasses import replace
+
+        self.sta = sta
+        self.cfg = replace(cfg, seed=cfg.seed + seed_offset)
+        c = self.cfg
+        self.B, self.Hh, self.d = c.B, c.heads, c.d
+        self.g = sta.grid(c.T, c.H, c.W)
+        self.nt = sta.sta_num_tiles(self.g)
+        self.lpad = sta.sta_tiled_len(self.g)
+        self.q, self.k, self.v = make_qkv(c, device=dev)
+        shape_t = (self.B, self.Hh, self.lpad, self.d)
+        self.qt, self.kt, self.vt, self.ot = (torch.empty(shape_t, dtype=torch.bfloat16, device=dev)
+                                              for _ in range(4))
+        self.o = torch.empty_like(self.q)
+        self.win = torch.from_numpy(window_params(cfg, window_scale(CFG_INDEX, 0))).to(dev)
+        self.params = sta.mask_params(c.top_p, c.k_min, c.use_scores, 0.0, c.group_lo, self.win)
+        self.bufs = sta.MaskBuffers(self.B, self.Hh, self.d, self.g, dev)
+        self.launches_per_step = 3 + 4 + 1 + 1  # reorder x3, pool/select/scan/fill, attn, inverse
+
+    def reorder_in(self):
+        s = self.sta
+        for src, dst in ((self.q, self.qt), (self.k, self.kt), (self.v, self.vt)):
+            s.sta_reorder(src, dst, self.B, self.Hh, self.d, self.g)
+
+    def build(self):
+        self.sta.build_mask(self.qt, self.kt, self.B, self.Hh, self.d, self.g, self.params, self.bufs)
+
+    def attn(self):
+        self.sta.sta_attn_fwd(self.qt, self.kt, self.vt, self.ot, None, self.bufs.row_ptr, self.bufs.col_idx,
+                              self.B, self.Hh, self.d, self.g)
+
+    def reorder_out(self):
+        self.sta.sta_reorder(self.ot, self.o, self.B, self.Hh, self.d, self.g, inverse=True)
+
+    def step(self, ev=None):
+        if ev is not None:
+            ev[0].record()
+        self.reorder_in()
+        if ev is not None:
+            ev[1].record()
+        self.build()
+        if ev is not None:
+            ev[2].record()
+        self.attn()
+        if ev is not None:
+            ev[3].record()
+        self.reorder_out()
+        if ev is not None:
+            ev[4].record()
+
+    def kept_pairs(self):
+        return int(self.bufs.nnz.item())
+
+    def pair_union_stats(self):
+        """Pairing efficiency (|A|+|B|) / (2 |A u B|) of the 128-row CTAs."""
+        rp = self.bufs.row_ptr.cpu().numpy()
+        ci = self.bufs.col_idx[: int(rp[-1])].cpu().numpy()
+        nt = self.nt
+        tot_ab, tot_u = 0, 0
+        for bh in range(self.B * self.Hh):
+            for p in range(0, nt, 2):
+                ra = bh * nt + p
+                a = ci[rp[ra]:rp[ra + 1]]
+                b = ci[rp[ra + 1]:rp[ra + 2]] if p + 1 < nt else np.zeros(0, np.int32)
+                tot_ab += a.size + b.size
+                tot_u += np.union1d(a, b).size
+        return tot_ab / (2.0 * tot_u) if tot_u else 1.0, tot_u
+
+
+def cpu_oracle_sample(cfg, layer, budget_s, rows_per_head=8, max_heads=None):
+    """Time the oracle (as it stands) on a bounded sample of the same layer:
+    for sampled heads, its reorder, pooling, scores, selection and windows
+    over the head, then masked attention for sampled query-tile rows.
+    Returns (kept-pair flops / s, description, seconds, threads)."""
+    import oracle as O
+
+    T, H, W, d = cfg.T, cfg.H, cfg.W, cfg.d
+    nt = layer.nt
+    win = window_params(cfg, window_scale(CFG_INDEX, 0))
+    rng = np.random.default_rng(123)
+    heads = rng.permutation(cfg.heads)
+    if max_heads:
+        heads = heads[:max_heads]
+    t0 = time.perf_counter()
+    pairs, nrows, nheads = 0, 0, 0
+    for h in heads:
+        q = layer.q[:, :, h:h + 1].float().cpu().numpy()
+        k = layer.k[:, :, h:h + 1].float().cpu().numpy()
+        v = layer.v[:, :, h:h + 1].float().cpu().numpy()
+        qt, kt, vt = (O.reorder_fwd(x.astype(np.float64), T, H, W) for x in (q, k, v))
+        _, p = O.block_scores(O.pool(qt, T, H, W), O.pool(kt, T, H, W), 1.0 / math.sqrt(d))
+        rows = rng.choice(nt, rows_per_head, replace=False)
+        wm = O.window_mask(win[h:h + 1], cfg.group_lo, T, H, W)[0]
+        mask = np.zeros((1, 1, nt, nt), dtype=bool)
+        for r in rows:
+            mask[0, 0, r] = O.select_row(p[0, 0, r], cfg.top_p, cfg.k_min) | wm[r]
+        rp, ci = O.mask_to_csr(mask)
+        O.attention_rows(qt, kt, vt, rp, ci, T, H, W, 1.0 / math.sqrt(d), rows)
+        pairs += int(mask.sum())
+        nrows += len(rows)
+        nheads += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    threads = len(os.sched_getaffinity(0))
+    desc = (f"{nheads} head(s) of the 75,600-token layer: full-head reorder, pooling, block scores and "
+            f"windows, then selection and masked attention for {nrows} query-tile rows "
+            f"({pairs} kept pairs)")
+    return pairs * flops_per_pair(d) / dt / 1e12, desc, dt, threads
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle timed as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    import block_sparse_attention_28_b200  # noqa: F401  (only to reuse tile counts)
+
+    cfg = CONFIGS[CFG_INDEX]
+
+    class _Stub:
+        pass
+
+    layer = _Stub()
+    layer.q, layer.k, layer.v = make_qkv(cfg, device="cpu")
+    from workloads import tile_counts
+
+    layer.nt = tile_counts(cfg.T, cfg.H, cfg.W)[2]
+    for _ in range(args.warmup):
+        cpu_oracle_sample(cfg, layer, 1.0, rows_per_head=2, max_heads=1)
+    vals, times = [], []
+    desc = ""
+    threads = 0
+    for _ in range(args.steps):
+        v, desc, dt, threads = cpu_oracle_sample(cfg, layer, 10.0, rows_per_head=4, max_heads=1)
+        vals.append(v)
+        times.append(dt)
+    value = float(statistics.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded random-Fourier-feature Q/K, Gaussian V)",
+        "config": {"workload": CONFIGS[CFG_INDEX].name, "tokens": cfg.L, "heads": cfg.heads, "d": cfg.d,
+                   "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import block_sparse_attention_28_b200 as sta
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    cfg = CONFIGS[CFG_INDEX]
+    layer = Layer(sta, cfg, dev, seed_offset=rank)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        layer.step()
+    barrier()
+    assert sta.sta_get_device_error() == sta.STA_OK
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(K):
+        layer.step(evs[i])
+    t_end.record()
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    assert sta.sta_get_device_error() == sta.STA_OK
+
+    reorder_ms = statistics.mean(e[0].elapsed_time(e[1]) + e[3].elapsed_time(e[4]) for e in evs)
+    build_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    t_max = torch.tensor([elapsed_ms], device=dev)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t_max.item())
+    pairs = layer.kept_pairs()
+    nt = layer.nt
+    density = pairs / (layer.B * layer.Hh * nt * nt)
+    flops = pairs * flops_per_pair(layer.d)
+    value = world * K * flops / (elapsed_ms * 1e-3) / 1e12
+    attn_tflops = flops / (attn_ms * 1e-3) / 1e12
+
+    # end to end through the C ABI from pinned host buffers (H2D in, D2H out)
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv = (x.cpu().pin_memory() for x in (layer.q, layer.k, layer.v))
+        ho = torch.empty(layer.o.shape, dtype=layer.o.dtype, pin_memory=True)
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv))
+        d2h = ho.numel() * ho.element_size()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.e2e_steps):
+            layer.q.copy_(hq, non_blocking=True)
+            layer.k.copy_(hk, non_blocking=True)
+            layer.v.copy_(hv, non_blocking=True)
+            layer.step()
+            ho.copy_(layer.o, non_blocking=True)
+        e1.record()
+        barrier()
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        t2 = torch.tensor([e2e_ms], device=dev)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * flops / (float(t2.item()) * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": float(t2.item())}
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    eff, union_tiles = layer.pair_union_stats() if rank == 0 else (None, None)
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            v_cpu, desc, dt, threads = cpu_oracle_sample(cfg, layer, args.cpu_budget)
+            cpu = {"value": v_cpu, "unit": UNIT, "cores": threads, "kind": "oracle",
+                   "sample": f"{desc}; {dt:.1f} s"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": max(3, args.warmup), "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded random-Fourier-feature Q/K, Gaussian V; no dataset)",
+            "config": {
+                "workload": cfg.name, "tokens": cfg.L, "padded_tokens": layer.lpad, "heads": cfg.heads,
+                "d": cfg.d, "grid": [cfg.T, cfg.H, cfg.W], "top_p": cfg.top_p, "k_min": cfg.k_min,
+                "density": density, "kept_pairs": pairs, "global_batch": world * cfg.B,
+                "parallelism": f"independent layer per GPU x{world}",
+                "l2": "inputs (Q,K,V 2.3 GB) larger than L2; no flush",
+                "step": "reorder Q,K,V + build_mask + attn_fwd + reorder O back",
+            },
+            "ms_per_layer": build_ms + attn_ms,
+            "ms_breakdown": {"reorder_in_out": reorder_ms, "build_mask": build_ms, "attn_fwd": attn_ms},
+            "attn_tflops": attn_tflops,
+            "attn_frac_of_peak": attn_tflops / peak,
+            "pairing_efficiency": eff,
+            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": attn_tflops / peak, "traffic": load_traffic(),
+                         "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                         "kernel": "attn_fwd_kernel<128>",
+                         "algorithmic": f"{pairs} kept pairs x 4*64*64*{cfg.d} flop"},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": K * layer.launches_per_step,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

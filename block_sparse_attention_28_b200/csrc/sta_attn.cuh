@@ -1,0 +1,389 @@
+// Block-sparse attention forward over listed key tiles (Compact Attention
+// Fig. 3: precomputed masks loaded into a block-sparse attention kernel).
+//
+// One CTA computes 128 query rows: the query tiles 2p and 2p+1 of one head
+// (a 128-row tcgen05 tile; a 64-token tile alone would leave half of the MMA
+// rows idle). The two CSR rows are merged into one ascending key-tile list
+// with a per-half membership flag; a half whose list lacks the key tile gets
+// P = 0 for that tile, so the work is |A u B| key tiles of 128 x 64.
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax + correction + epilogue; thread i owns query row i
+//              (TMEM lane i): S row -> online softmax (exp2, lazy rescale of
+//              O when the running max grows by more than 2^8) -> P (bf16) back
+//              into TMEM over S; at the end O / l -> bf16 -> global, and LSE.
+//   warp 4     TMA producer: Q once, then K_j and V_j per listed key tile
+//              into an NS-stage ring (128 B swizzle, no multicast).
+//   warp 5     MMA issuer (one thread): S_j = Q K_j^T (SS, M=128 N=64) into
+//              one of two TMEM S buffers, O += P_j V_j (A = P from TMEM,
+//              B = V MN-major from shared memory, M=128 N=d).
+// TMEM columns: S0 [0,64) S1 [64,128) O [128, 128+d).
+#pragma once
+#include "sta_common.cuh"
+#include "sta_tc.cuh"
+
+namespace sta {
+namespace attn {
+
+constexpr int NUM_THREADS = 192;
+constexpr int WARP_PRODUCER = 4;
+constexpr int WARP_MMA = 5;
+constexpr uint32_t FLAG_A = 1u << 30;
+constexpr uint32_t FLAG_B = 1u << 31;
+constexpr uint32_t KT_MASK = FLAG_A - 1u;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t O_COL = 128;
+constexpr long long WAIT_LIMIT = 2000000000LL;   // SM cycles (~1 s)
+constexpr long long DRAIN_LIMIT = 200000000LL;   // after an abort
+constexpr float RESCALE_LOG2 = 8.0f;             // lazy O rescale threshold
+
+template <int D>
+struct Cfg {
+  static constexpr int KB = D / 64;              // 128-byte swizzle atoms along d
+  static constexpr int NS = (D == 128) ? 4 : 6;  // K/V ring stages
+  static constexpr int TILE_BYTES = 64 * D * 2;  // one 64-token tile of Q, K or V
+  static constexpr int Q_REGION = 128 * 128;     // 128 rows x 128 B per d-atom
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + KB * Q_REGION;
+  static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NS * TILE_BYTES;
+  // q_full, k_full[NS], v_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done, mma_done
+  static constexpr int NUM_BARS = 1 + 3 * NS + 2 + 2 + 1 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_LIST = OFF_MISC + 64;
+  static constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 64, false);
+  static constexpr uint32_t IDESC_O = tc::idesc_bf16(128, D, true);
+};
+
+template <int D>
+inline size_t smem_bytes(int nt) {
+  const int wpr = (nt + 31) / 32;
+  return (size_t)Cfg<D>::OFF_LIST + (size_t)(2 * wpr + nt) * 4 + 1024;
+}
+
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16 *__restrict__ out,
+                float *__restrict__ lse, const int *__restrict__ row_ptr,
+                const int *__restrict__ col_idx, Geo g, float scale_log2) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = tc::smem_u32(smem);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nt = g.Nt;
+  const int bh = blockIdx.y;
+  const int qtA = 2 * blockIdx.x, qtB = qtA + 1;
+  const bool hasB = qtB < nt;
+  const int wpr = (nt + 31) / 32;
+
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+  uint64_t *q_full = bars;
+  uint64_t *k_full = bars + 1;
+  uint64_t *v_full = k_full + C::NS;
+  uint64_t *kv_empty = v_full + C::NS;
+  uint64_t *s_full = kv_empty + C::NS;
+  uint64_t *p_full = s_full + 2;
+  uint64_t *o_done = p_full + 2;
+  uint64_t *mma_done = o_done + 1;
+  uint32_t *misc = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);  // tmem, n, abort
+  volatile uint32_t *abort_flag = misc + 2;
+  uint32_t *bmA = reinterpret_cast<uint32_t *>(smem + C::OFF_LIST);
+  uint32_t *bmB = bmA + wpr;
+  uint32_t *U = bmB + wpr;
+
+  // ---- set-up: barriers, bitmaps, TMEM
+  if (tid == 0) {
+    tc::mbar_init(q_full, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      tc::mbar_init(k_full + s, 1);
+      tc::mbar_init(v_full + s, 1);
+      tc::mbar_init(kv_empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(s_full + b, 1);
+      tc::mbar_init(p_full + b, 4);
+    }
+    tc::mbar_init(o_done, 1);
+    tc::mbar_init(mma_done, 1);
+    misc[2] = 0u;
+    tc::fence_barrier_init();
+  }
+  for (int i = tid; i < 2 * wpr; i += NUM_THREADS) bmA[i] = 0u;
+  if (warp == WARP_MMA) {
+    tc::tmem_alloc(misc, TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  __syncthreads();
+
+  // ---- the two CSR rows as bitmaps, then their ascending union with flags
+  {
+    const long long rA = (long long)bh * nt + qtA;
+    const int a0 = row_ptr[rA], a1 = row_ptr[rA + 1];
+    for (int i = a0 + tid; i < a1; i += NUM_THREADS) {
+      const int c = col_idx[i];
+      if ((unsigned)c < (unsigned)nt)
+        atomicOr(bmA + (c >> 5), 1u << (c & 31));
+      else
+        record_error(DEV_ERR_BAD_MASK);
+    }
+    if (hasB) {
+      const int b0 = row_ptr[rA + 1], b1 = row_ptr[rA + 2];
+      for (int i = b0 + tid; i < b1; i += NUM_THREADS) {
+        const int c = col_idx[i];
+        if ((unsigned)c < (unsigned)nt)
+          atomicOr(bmB + (c >> 5), 1u << (c & 31));
+        else
+          record_error(DEV_ERR_BAD_MASK);
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int base = 0;
+    for (int w0 = 0; w0 < wpr; w0 += 32) {
+      const int w = w0 + lane;
+      const uint32_t a = (w < wpr) ? bmA[w] : 0u, b = (w < wpr) ? bmB[w] : 0u;
+      uint32_t u = a | b;
+      const int c = __popc(u);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int pos = base + incl - c;
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        const uint32_t m = 1u << bit;
+        U[pos++] = (uint32_t)(w * 32 + bit) | ((a & m) ? FLAG_A : 0u) | ((b & m) ? FLAG_B : 0u);
+        u &= u - 1u;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) misc[1] = (uint32_t)base;
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = misc[0];
+  const int n = (int)misc[1];
+
+  if (warp == WARP_PRODUCER) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0 && n > 0) {
+      const int rowA = (int)(((long long)bh * nt + qtA) * 64);
+      tc::mbar_expect_tx(q_full, (hasB ? 2 : 1) * C::TILE_BYTES);
+#pragma unroll
+      for (int kb = 0; kb < C::KB; ++kb) {
+        tc::tma_load_2d(sbase + C::OFF_Q + kb * C::Q_REGION, &tm_q, q_full, kb * 64, rowA);
+        if (hasB)
+          tc::tma_load_2d(sbase + C::OFF_Q + kb * C::Q_REGION + 8192, &tm_q, q_full, kb * 64,
+                          rowA + 64);
+      }
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int s = j % C::NS, u = j / C::NS;
+        if (u > 0 && !tc::mbar_wait(kv_empty + s, (u - 1) & 1, abort_flag, WAIT_LIMIT)) break;
+        const int kt = (int)(U[j] & KT_MASK);
+        const int row = (int)(((long long)bh * nt + kt) * 64);
+        tc::mbar_expect_tx(k_full + s, C::TILE_BYTES);
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb)
+          tc::tma_load_2d(sbase + C::OFF_K + s * C::TILE_BYTES + kb * 8192, &tm_k, k_full + s,
+                          kb * 64, row);
+        tc::mbar_expect_tx(v_full + s, C::TILE_BYTES);
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb)
+          tc::tma_load_2d(sbase + C::OFF_V + s * C::TILE_BYTES + kb * 8192, &tm_v, v_full + s,
+                          kb * 64, row);
+        issued = j + 1;
+      }
+      // Copies still in flight must land before the CTA can exit.
+      if (*abort_flag) {
+        tc::mbar_wait(q_full, 0, nullptr, DRAIN_LIMIT);
+        for (int j = (issued > C::NS ? issued - C::NS : 0); j < issued; ++j) {
+          tc::mbar_wait(k_full + j % C::NS, (j / C::NS) & 1, nullptr, DRAIN_LIMIT);
+          tc::mbar_wait(v_full + j % C::NS, (j / C::NS) & 1, nullptr, DRAIN_LIMIT);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == WARP_MMA) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0 && n > 0) {
+      bool ok = tc::mbar_wait(q_full, 0, abort_flag, WAIT_LIMIT);
+      tc::fence_after();
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % C::NS;
+        if (!tc::mbar_wait(k_full + s, (j / C::NS) & 1, abort_flag, WAIT_LIMIT)) return false;
+        tc::fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)((j & 1) * 64);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (uint32_t)((kk & 3) * 32);
+          const uint64_t a = tc::desc_k_sw128(sbase + C::OFF_Q + (kk >> 2) * C::Q_REGION + koff);
+          const uint64_t b =
+              tc::desc_k_sw128(sbase + C::OFF_K + s * C::TILE_BYTES + (kk >> 2) * 8192 + koff);
+          tc::mma_ss(d_tmem, a, b, C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(s_full + (j & 1));
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int s = j % C::NS;
+        if (!tc::mbar_wait(p_full + (j & 1), (j >> 1) & 1, abort_flag, WAIT_LIMIT)) return false;
+        if (!tc::mbar_wait(v_full + s, (j / C::NS) & 1, abort_flag, WAIT_LIMIT)) return false;
+        tc::fence_after();
+        const uint32_t p_tmem = tmem + (uint32_t)((j & 1) * 64);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t b =
+              tc::desc_mn_sw128(sbase + C::OFF_V + s * C::TILE_BYTES + kk * 2048, 8192u);
+          tc::mma_ts(tmem + O_COL, p_tmem + (uint32_t)(kk * 8), b, C::IDESC_O,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(kv_empty + s);
+        tc::mma_commit(o_done);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 1; ok && j < n; ++j) {
+        ok = issue_s(j);
+        if (ok) ok = issue_pv(j - 1);
+      }
+      if (ok) ok = issue_pv(n - 1);
+      // All issued MMAs must retire before TMEM is released.
+      tc::mma_commit(mma_done);
+      tc::mbar_wait(mma_done, 0, nullptr, ok ? WAIT_LIMIT : DRAIN_LIMIT);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------- softmax / correction / epilogue
+    const bool halfB = warp >= 2;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    float m = -INFINITY, l = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int buf = j & 1;
+      const bool got = tc::mbar_wait(s_full + buf, (j >> 1) & 1, abort_flag, WAIT_LIMIT);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc::fence_after();
+      const uint32_t e = U[j];
+      const bool mine = halfB ? (e & FLAG_B) != 0u : (e & FLAG_A) != 0u;
+      const uint32_t sS = tmem + lane_base + (uint32_t)(buf * 64);
+      uint32_t pk[32];
+      if (!mine) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+        tc::tmem_st32(sS, pk);
+      } else {
+        uint32_t r0[32], r1[32];
+        tc::tmem_ld32(sS, r0);
+        tc::tmem_ld32(sS + 32, r1);
+        float s[64];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          s[c] = __uint_as_float(r0[c]);
+          s[32 + c] = __uint_as_float(r1[c]);
+        }
+        // keys of partial tiles beyond the grid edge
+        const int kt = (int)(e & KT_MASK);
+        const int rem = kt % (g.NH * g.NW);
+        const int ty = rem / g.NW, tx = rem - ty * g.NW;
+        const int vy = valid_extent(g.H, ty), vx = valid_extent(g.W, tx);
+        if (vy < 8 || vx < 8) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if ((c >> 3) >= vy || (c & 7) >= vx) s[c] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < 64; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = fmaxf(m, mx * scale_log2);
+        const bool rescale = m_new > m + RESCALE_LOG2;
+        const float m_use = rescale ? m_new : m;
+        const float mref = (m_use == -INFINITY) ? 0.0f : m_use;
+        const float alpha = rescale ? tc::ex2(m - m_new) : 1.0f;
+        float sum = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float p0 = tc::ex2(fmaf(s[2 * c], scale_log2, -mref));
+          const float p1 = tc::ex2(fmaf(s[2 * c + 1], scale_log2, -mref));
+          sum += p0 + p1;
+          pk[c] = tc::pack_bf16(p0, p1);
+        }
+        tc::tmem_st32(sS, pk);
+        l = l * alpha + sum;
+        const bool need_o = rescale && (m != -INFINITY);
+        if (__any_sync(0xffffffffu, need_o)) {
+          // PV_{j-1} must have retired before O is scaled (j >= 1 here).
+          const bool got_o = tc::mbar_wait(o_done, (j - 1) & 1, abort_flag, WAIT_LIMIT);
+          if (!__all_sync(0xffffffffu, got_o)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after();
+          const float a = need_o ? alpha : 1.0f;
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tc::tmem_ld32(tmem + lane_base + O_COL + cc * 32, o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * a);
+            tc::tmem_st32(tmem + lane_base + O_COL + cc * 32, o);
+          }
+        }
+        m = m_use;
+      }
+      tc::tmem_wait_st();
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(p_full + buf);
+    }
+    // ---- epilogue
+    if (ok && n > 0) ok = tc::mbar_wait(o_done, (n - 1) & 1, abort_flag, WAIT_LIMIT);
+    ok = __all_sync(0xffffffffu, ok);
+    tc::fence_after();
+    const bool row_exists = !halfB || hasB;
+    if (ok && row_exists) {
+      const int qt = halfB ? qtB : qtA;
+      const long long orow = (long long)bh * g.Lpad + (long long)qt * 64 + (tid & 63);
+      const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+      uint4 *dst = reinterpret_cast<uint4 *>(out + orow * D);
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        if (n > 0) {
+          tc::tmem_ld32(tmem + lane_base + O_COL + cc * 32, o);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pk[c] = tc::pack_bf16(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          dst[cc * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+      }
+      if (lse != nullptr)
+        lse[orow] = (l > 0.0f) ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    }
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc::fence_after();
+    tc::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace attn
+}  // namespace sta

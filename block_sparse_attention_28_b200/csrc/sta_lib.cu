@@ -1,0 +1,268 @@
+// libsta: C ABI entry points (declared in include/sta.h).
+// Single translation unit: the kernels live in the included headers.
+#include <math.h>
+#include <string.h>
+
+#include "sta_attn.cuh"
+#include "sta_common.cuh"
+#include "sta_mask.cuh"
+#include "sta_reorder.cuh"
+
+using namespace sta;
+
+namespace {
+
+bool common_sizes_ok(int32_t B, int32_t heads, int32_t d, sta_grid g, Geo *geo, sta_status *st) {
+  if (B <= 0 || heads <= 0 || !make_geo(g, geo)) {
+    *st = STA_ERR_INVALID_ARG;
+    return false;
+  }
+  if (d != 64 && d != 128) {
+    *st = STA_ERR_UNSUPPORTED;
+    return false;
+  }
+  const long long bh = (long long)B * heads;
+  // 2D grids index (b*heads + h) in grid.y; TMA row coordinates and CSR
+  // offsets are 32-bit.
+  if (bh > 65535 || bh * geo->Lpad >= (1LL << 31) || bh * (long long)geo->Nt * geo->Nt >= (1LL << 31)) {
+    *st = STA_ERR_UNSUPPORTED;
+    return false;
+  }
+  return true;
+}
+
+struct MaskWs {
+  size_t qbar, kbar, bits, counts, total;
+};
+
+MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
+  const size_t R = (size_t)B * heads * g.Nt;
+  const size_t wpr = (size_t)(g.Nt + 31) / 32;
+  MaskWs w;
+  size_t off = 0;
+  w.qbar = off;
+  off = align_up(off + R * d * sizeof(float), 256);
+  w.kbar = off;
+  off = align_up(off + R * d * sizeof(float), 256);
+  w.bits = off;
+  off = align_up(off + R * wpr * sizeof(uint32_t), 256);
+  w.counts = off;
+  off = align_up(off + R * sizeof(int32_t), 256);
+  w.total = off;
+  return w;
+}
+
+size_t select_smem(int d, int nt, bool use_scores) {
+  return use_scores ? (size_t)(SEL_QB * d + SEL_QB * nt) * sizeof(float) : 0;
+}
+
+constexpr size_t MAX_DYN_SMEM = 227 * 1024;
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows, d] bf16 row-major; box = 64 rows x 64 elements (128 B), 128 B swizzle.
+bool make_tile_map(CUtensorMap *map, const void *base, unsigned long long rows, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool device_is_sm100() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return false;
+  return major == 10 && minor == 0;
+}
+
+template <int D>
+sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads,
+                        const Geo &g, const sta_mask_params *p, int32_t *row_ptr, int32_t *col_idx,
+                        int64_t *nnz_dev, uint8_t *block_mask, float *block_probs, uint8_t *ws,
+                        cudaStream_t s) {
+  const MaskWs L = mask_ws_layout(B, heads, D, g);
+  float *qbar = reinterpret_cast<float *>(ws + L.qbar);
+  float *kbar = reinterpret_cast<float *>(ws + L.kbar);
+  unsigned int *bits = reinterpret_cast<unsigned int *>(ws + L.bits);
+  int *counts = reinterpret_cast<int *>(ws + L.counts);
+  const long long R = (long long)B * heads * g.Nt;
+  const int wpr = (g.Nt + 31) / 32;
+  const bool use_scores = p->use_scores != 0;
+  const float scale = p->sm_scale != 0.0f ? p->sm_scale : 1.0f / sqrtf((float)D);
+
+  if (use_scores) {
+    const long long warps = 2 * R;
+    const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
+    pool_kernel<D><<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(q_tiled),
+                                           static_cast<const uint4 *>(k_tiled), qbar, kbar, R, g);
+    STA_CUDA_TRY(cudaGetLastError());
+  }
+  const size_t smem = select_smem(D, g.Nt, use_scores);
+  if (smem > 48 * 1024)
+    STA_CUDA_TRY(cudaFuncSetAttribute(score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem));
+  GroupLo glo;
+  for (int i = 0; i < STA_MAX_GROUPS; ++i) glo.v[i] = (i < p->num_groups) ? p->group_lo[i] : 0x7fffffff;
+  dim3 grid((unsigned)((g.Nt + SEL_QB - 1) / SEL_QB), (unsigned)(B * heads));
+  score_select_kernel<D><<<grid, SEL_THREADS, smem, s>>>(
+      qbar, kbar, heads, g, scale, p->top_p, p->k_min, use_scores ? 1 : 0, p->windows,
+      p->windows ? p->num_groups : 0, glo, bits, counts, block_probs, wpr);
+  STA_CUDA_TRY(cudaGetLastError());
+  scan_kernel<<<1, SCAN_THREADS, 0, s>>>(counts, row_ptr, reinterpret_cast<long long *>(nnz_dev), R);
+  STA_CUDA_TRY(cudaGetLastError());
+  const unsigned fblocks = (unsigned)((R * 32 + 255) / 256);
+  fill_kernel<<<fblocks, 256, 0, s>>>(bits, row_ptr, col_idx, block_mask, R, g.Nt, wpr);
+  STA_CUDA_TRY(cudaGetLastError());
+  if (block_probs != nullptr && !use_scores)
+    STA_CUDA_TRY(cudaMemsetAsync(block_probs, 0, (size_t)R * g.Nt * sizeof(float), s));
+  return STA_OK;
+}
+
+template <int D>
+sta_status launch_attn(const void *q, const void *k, const void *v, void *o, float *lse,
+                       const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
+                       const Geo &g, float sm_scale, cudaStream_t s) {
+  const unsigned long long rows = (unsigned long long)B * heads * g.Lpad;
+  CUtensorMap tq, tk, tv;
+  if (!make_tile_map(&tq, q, rows, D) || !make_tile_map(&tk, k, rows, D) || !make_tile_map(&tv, v, rows, D))
+    return STA_ERR_CUDA;
+  const size_t smem = attn::smem_bytes<D>(g.Nt);
+  if (smem > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
+  STA_CUDA_TRY(cudaFuncSetAttribute(attn::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem));
+  const float scale = sm_scale != 0.0f ? sm_scale : 1.0f / sqrtf((float)D);
+  const float scale_log2 = scale * 1.4426950408889634f;
+  dim3 grid((unsigned)((g.Nt + 1) / 2), (unsigned)(B * heads));
+  attn::attn_fwd_kernel<D><<<grid, attn::NUM_THREADS, smem, s>>>(
+      tq, tk, tv, static_cast<__nv_bfloat16 *>(o), lse, row_ptr, col_idx, g, scale_log2);
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t sta_num_tiles(sta_grid g) {
+  Geo geo;
+  return make_geo(g, &geo) ? (int64_t)geo.Nt : -1;
+}
+
+int64_t sta_tiled_len(sta_grid g) {
+  Geo geo;
+  return make_geo(g, &geo) ? (int64_t)geo.Lpad : -1;
+}
+
+sta_status sta_reorder(const void *src, void *dst, int32_t B, int32_t heads, int32_t d, sta_grid g,
+                       int32_t inverse, sta_stream_t stream) {
+  Geo geo;
+  sta_status st = STA_OK;
+  if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return st;
+  if (src == nullptr || dst == nullptr || !aligned16(src) || !aligned16(dst) || src == dst)
+    return STA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e = (d == 128) ? launch_reorder<128>(src, dst, B, heads, geo, inverse != 0, s)
+                                   : launch_reorder<64>(src, dst, B, heads, geo, inverse != 0, s);
+  return e == cudaSuccess ? STA_OK : STA_ERR_CUDA;
+}
+
+size_t sta_build_mask_workspace(int32_t B, int32_t heads, int32_t d, sta_grid g) {
+  Geo geo;
+  sta_status st;
+  if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return 0;
+  return mask_ws_layout(B, heads, d, geo).total;
+}
+
+sta_status sta_build_mask(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads, int32_t d,
+                          sta_grid g, const sta_mask_params *p, int32_t *row_ptr, int32_t *col_idx,
+                          int64_t *nnz_dev, uint8_t *block_mask, float *block_probs, void *workspace,
+                          size_t ws_bytes, sta_stream_t stream) {
+  Geo geo;
+  sta_status st = STA_OK;
+  if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return st;
+  if (p == nullptr || row_ptr == nullptr || col_idx == nullptr || nnz_dev == nullptr)
+    return STA_ERR_INVALID_ARG;
+  if (p->use_scores && (q_tiled == nullptr || k_tiled == nullptr || !aligned16(q_tiled) || !aligned16(k_tiled)))
+    return STA_ERR_INVALID_ARG;
+  if (p->windows != nullptr) {
+    if (p->num_groups < 1 || p->num_groups > STA_MAX_GROUPS || p->group_lo[0] != 0) return STA_ERR_INVALID_ARG;
+    for (int i = 1; i < p->num_groups; ++i)
+      if (p->group_lo[i] <= p->group_lo[i - 1]) return STA_ERR_INVALID_ARG;
+  }
+  if (p->k_min < 0 || !(p->top_p == p->top_p)) return STA_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      ws_bytes < mask_ws_layout(B, heads, d, geo).total)
+    return STA_ERR_WORKSPACE;
+  if (select_smem(d, geo.Nt, p->use_scores != 0) > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  return (d == 128) ? launch_build<128>(q_tiled, k_tiled, B, heads, geo, p, row_ptr, col_idx, nnz_dev,
+                                        block_mask, block_probs, ws, s)
+                    : launch_build<64>(q_tiled, k_tiled, B, heads, geo, p, row_ptr, col_idx, nnz_dev,
+                                       block_mask, block_probs, ws, s);
+}
+
+sta_status sta_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                        const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
+                        int32_t d, sta_grid g, float sm_scale, sta_stream_t stream) {
+  Geo geo;
+  sta_status st = STA_OK;
+  if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || row_ptr == nullptr || col_idx == nullptr)
+    return STA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return STA_ERR_INVALID_ARG;
+  if (!(sm_scale == sm_scale) || sm_scale < 0.0f) return STA_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return STA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return (d == 128) ? launch_attn<128>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s)
+                    : launch_attn<64>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s);
+}
+
+sta_status sta_get_device_error(sta_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  STA_CUDA_TRY(cudaStreamSynchronize(s));
+  unsigned int word = 0;
+  STA_CUDA_TRY(cudaMemcpyFromSymbol(&word, g_dev_error, sizeof(word)));
+  const unsigned int zero = 0;
+  STA_CUDA_TRY(cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(zero)));
+  if (word & DEV_ERR_TIMEOUT) return STA_ERR_TIMEOUT;
+  if (word & DEV_ERR_BAD_MASK) return STA_ERR_BAD_MASK;
+  return STA_OK;
+}
+
+const char *sta_status_string(sta_status s) {
+  switch (s) {
+    case STA_OK: return "ok";
+    case STA_ERR_INVALID_ARG: return "invalid argument";
+    case STA_ERR_UNSUPPORTED: return "unsupported size or device";
+    case STA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case STA_ERR_CUDA: return "CUDA call failed";
+    case STA_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case STA_ERR_BAD_MASK: return "CSR column index out of range";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,339 @@
+// Online mask construction: pooled block scores (Rectified SpaAttn), hybrid
+// top-p / k_min selection (SCOPE Eqs. (7)-(8) as quoted), OR'd with per-head
+// dual windows per temporal-distance group (Compact Attention Fig. 1(3),
+// Fig. 4), emitted as CSR lists (Compact Attention Fig. 3).
+//
+// Kernels, in launch order:
+//   pool_kernel          tile means of Q and K (HBM-bound, coalesced 16 B loads)
+//   score_select_kernel  16 query tiles x all key tiles per CTA: fp32 scores,
+//                        row softmax, selection, window test -> row bitsets
+//   scan_kernel          exclusive scan of the row counts -> row_ptr, nnz
+//   fill_kernel          bitsets -> ascending col_idx (+ optional byte mask)
+#pragma once
+#include "sta_common.cuh"
+
+namespace sta {
+
+constexpr float MASS_ONE_F = 16777216.0f;  // 2^24, fixed-point unit of the mass
+
+// ---------------------------------------------------------------- pooling
+// One warp per (b*heads + h, tile). Each lane owns one 16-byte chunk of a row
+// and walks the tile's real rows; the sum is exact in fp64 (64 bf16 values),
+// the mean is rounded once to fp32.
+template <int D>
+__global__ void __launch_bounds__(256)
+pool_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k, float *__restrict__ qbar,
+            float *__restrict__ kbar, long long n_tiles_total, Geo g) {
+  constexpr int CPR = D / 8;      // chunks per row
+  constexpr int RPI = 32 / CPR;   // rows per warp step
+  const long long warp_id = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const bool is_k = warp_id >= n_tiles_total;
+  const long long tile = is_k ? warp_id - n_tiles_total : warp_id;
+  if (tile >= n_tiles_total) return;
+  const uint4 *src = is_k ? k : q;
+  float *dst = is_k ? kbar : qbar;
+  const int n = (int)(tile % g.Nt);
+  const int tpf = g.NH * g.NW;
+  const int rem = n % tpf;
+  const int ty = rem / g.NW, tx = rem - ty * g.NW;
+  const int vy = valid_extent(g.H, ty), vx = valid_extent(g.W, tx);
+  const int sub = lane / CPR, c = lane - sub * CPR;
+  const uint4 *base = src + tile * 64 * CPR;
+  double acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+#pragma unroll 4
+  for (int i = 0; i < 64 / RPI; ++i) {
+    const int r = i * RPI + sub;
+    if ((r >> 3) < vy && (r & 7) < vx) {
+      const uint4 w = __ldcs(base + r * CPR + c);
+      const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&w);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(p[e]);
+        acc[2 * e] += (double)f.x;
+        acc[2 * e + 1] += (double)f.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int off = CPR; off < 32; off <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+  }
+  if (sub == 0) {
+    const double cnt = (double)(vy * vx);
+    float out[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = (float)(acc[e] / cnt);
+    float4 *o = reinterpret_cast<float4 *>(dst + tile * D + c * 8);
+    o[0] = make_float4(out[0], out[1], out[2], out[3]);
+    o[1] = make_float4(out[4], out[5], out[6], out[7]);
+  }
+}
+
+// ------------------------------------------------------ scores + selection
+constexpr int SEL_THREADS = 256;
+constexpr int SEL_QB = 16;  // query tiles per CTA
+
+struct GroupLo {
+  int v[STA_MAX_GROUPS];
+};
+
+__device__ __forceinline__ unsigned int warp_sum_u32(unsigned int x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ unsigned int mass_of(float p) {
+  return __float2uint_rd(p * MASS_ONE_F);  // exact: p in [0,1], scaling by 2^24
+}
+
+// Total mass (or count when `count_only`) of the row entries whose P bit
+// pattern is >= `key`. P >= 0, so float bits order like the values.
+__device__ __forceinline__ unsigned int mass_at_least(const float *row, int nt, unsigned int key,
+                                                      bool count_only, int lane) {
+  unsigned int s = 0;
+  for (int j = lane; j < nt; j += 32) {
+    const float p = row[j];
+    if (__float_as_uint(p) >= key) s += count_only ? 1u : mass_of(p);
+  }
+  return warp_sum_u32(s);
+}
+
+// Largest bit pattern v with f(v) >= target, f non-increasing (mass or count
+// of entries >= v). target must be >= 1 and f(0) >= target.
+__device__ unsigned int search_level(const float *row, int nt, unsigned int target, bool count_only,
+                                     int lane) {
+  unsigned int lo = 0u, hi = 0x3F800001u;  // f(lo) >= target > f(hi)
+  while (hi - lo > 1u) {
+    const unsigned int mid = lo + ((hi - lo) >> 1);
+    if (mass_at_least(row, nt, mid, count_only, lane) >= target)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  return lo;
+}
+
+// One CTA per (b*heads + h, block of SEL_QB query tiles).
+// Dynamic smem: qs [SEL_QB][D] fp32, then S [SEL_QB][Nt] fp32 (if use_scores).
+template <int D>
+__global__ void __launch_bounds__(SEL_THREADS)
+score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar, int heads, Geo g,
+                    float scale, float top_p, int k_min, int use_scores,
+                    const int *__restrict__ windows, int G, GroupLo glo,
+                    unsigned int *__restrict__ bits, int *__restrict__ counts,
+                    float *__restrict__ probs_out, int wpr) {
+  extern __shared__ __align__(16) float sm[];
+  const int nt = g.Nt;
+  const int bh = blockIdx.y;
+  const int h = bh % heads;
+  const int q0 = blockIdx.x * SEL_QB;
+  const int nq = min(SEL_QB, nt - q0);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float *qs = sm;
+  float *S = sm + SEL_QB * D;
+
+  if (use_scores) {
+    // Phase 1: S[i][kt] = scale * qbar[q0+i] . kbar[kt], sequential fp32 FMA over d.
+    for (int e = tid; e < SEL_QB * D; e += SEL_THREADS) {
+      const int i = e / D;
+      qs[e] = (i < nq) ? qbar[((long long)bh * nt + q0 + i) * D + (e - i * D)] : 0.0f;
+    }
+    __syncthreads();
+    for (int kt = tid; kt < nt; kt += SEL_THREADS) {
+      const float4 *kr = reinterpret_cast<const float4 *>(kbar + ((long long)bh * nt + kt) * D);
+      float acc[SEL_QB];
+#pragma unroll
+      for (int i = 0; i < SEL_QB; ++i) acc[i] = 0.0f;
+#pragma unroll 2
+      for (int d4 = 0; d4 < D / 4; ++d4) {
+        const float4 kv = __ldg(kr + d4);
+#pragma unroll
+        for (int i = 0; i < SEL_QB; ++i) {
+          const float4 qv = reinterpret_cast<const float4 *>(qs + i * D)[d4];
+          acc[i] = fmaf(qv.x, kv.x, acc[i]);
+          acc[i] = fmaf(qv.y, kv.y, acc[i]);
+          acc[i] = fmaf(qv.z, kv.z, acc[i]);
+          acc[i] = fmaf(qv.w, kv.w, acc[i]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < SEL_QB; ++i) S[i * nt + kt] = acc[i] * scale;
+    }
+    __syncthreads();
+  }
+
+  const int tpf = g.NH * g.NW;
+  for (int i = warp; i < nq; i += SEL_THREADS / 32) {
+    const int qt = q0 + i;
+    const long long row = (long long)bh * nt + qt;
+    float *Sr = S + i * nt;
+    unsigned int v_f = 0xFFFFFFFFu;  // keep P > v_f, plus c_f ties at v_f
+    unsigned int c_f = 0u;
+    if (use_scores) {
+      // Phase 2: row softmax in fp32 (max, expf, fixed-order sum, IEEE divide).
+      float mx = -INFINITY;
+      for (int j = lane; j < nt; j += 32) mx = fmaxf(mx, Sr[j]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float sum = 0.0f;
+      for (int j = lane; j < nt; j += 32) {
+        const float e = expf(Sr[j] - mx);
+        Sr[j] = e;
+        sum += e;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      for (int j = lane; j < nt; j += 32) {
+        const float p = Sr[j] / sum;
+        Sr[j] = p;
+        if (probs_out) probs_out[row * nt + j] = p;
+      }
+      __syncwarp();
+      // Phase 3: selection threshold as (level v_f, ties c_f).
+      const int kk = min(k_min, nt);
+      unsigned int m_p_level = 0xFFFFFFFFu, m_p_ties = 0u;
+      long long m_p = 0;
+      if (top_p >= 1.0f) {
+        m_p_level = 0u;  // every entry has P >= 0: keep all
+        m_p_ties = 0xFFFFFFFFu;
+        m_p = nt;
+      } else if (top_p > 0.0f) {
+        const unsigned int W = mass_at_least(Sr, nt, 0u, false, lane);
+        const double thr_d = ceil((double)top_p * (double)W);
+        const unsigned int thr = (unsigned int)thr_d;
+        if (thr > 0u) {
+          const unsigned int v = search_level(Sr, nt, thr, false, lane);
+          const unsigned int above = mass_at_least(Sr, nt, v + 1u, false, lane);
+          const unsigned int wv = mass_of(__uint_as_float(v));
+          const unsigned int need = (thr - above + wv - 1u) / wv;  // tied entries at level v
+          const unsigned int cnt_above = mass_at_least(Sr, nt, v + 1u, true, lane);
+          m_p_level = v;
+          m_p_ties = need;
+          m_p = (long long)cnt_above + need;
+        }
+      }
+      if ((long long)kk > m_p) {
+        const unsigned int u = search_level(Sr, nt, (unsigned int)kk, true, lane);
+        const unsigned int cnt_above = mass_at_least(Sr, nt, u + 1u, true, lane);
+        v_f = u;
+        c_f = (unsigned int)kk - cnt_above;
+      } else if (m_p > 0) {
+        v_f = m_p_level;
+        c_f = m_p_ties;
+      }
+    }
+    // Phase 4: membership bits = selected OR window, one 32-bit word per lane step.
+    const int tq = qt / tpf, remq = qt - tq * tpf;
+    const int yq = remq / g.NW, xq = remq - yq * g.NW;
+    const int *wh = windows ? windows + (long long)h * G * 4 : nullptr;
+    unsigned int ties_seen = 0u;
+    int total = 0;
+    unsigned int *brow = bits + row * wpr;
+    for (int w0 = 0; w0 < wpr; ++w0) {
+      const int kt = w0 * 32 + lane;
+      bool keep = false;
+      if (kt < nt) {
+        if (wh) {
+          const int tk = kt / tpf, remk = kt - tk * tpf;
+          const int yk = remk / g.NW, xk = remk - yk * g.NW;
+          const int dt = abs(tq - tk), dy = abs(yq - yk), dx = abs(xq - xk);
+          int grp = -1;
+          for (int gg = 0; gg < G; ++gg)
+            if (dt >= glo.v[gg]) grp = gg;
+          if (grp >= 0) {
+            const int *w4 = wh + grp * 4;
+            keep = (dy <= w4[0] && dx <= w4[1]) || (dy <= w4[2] && dx <= w4[3]);
+          }
+        }
+      }
+      // Selection membership needs the index-ordered rank among ties: warp-wide.
+      bool sel = false;
+      if (use_scores && v_f != 0xFFFFFFFFu) {
+        const unsigned int pb = (kt < nt) ? __float_as_uint(Sr[kt]) : 0u;
+        const bool tie = (kt < nt) && (pb == v_f);
+        const unsigned int tmask = __ballot_sync(0xffffffffu, tie);
+        const unsigned int before = __popc(tmask & ((1u << lane) - 1u));
+        sel = (kt < nt) && (pb > v_f || (tie && ties_seen + before < c_f));
+        ties_seen += __popc(tmask);
+      }
+      const unsigned int word = __ballot_sync(0xffffffffu, keep || sel);
+      if (lane == 0) brow[w0] = word;
+      total += __popc(word);
+    }
+    if (lane == 0) counts[row] = total;
+  }
+}
+
+// ---------------------------------------------------------------- scan
+// Single CTA: row_ptr[0] = 0, row_ptr[r+1] = sum of counts[0..r]; nnz = total.
+constexpr int SCAN_THREADS = 1024;
+
+__global__ void __launch_bounds__(SCAN_THREADS)
+scan_kernel(const int *__restrict__ counts, int *__restrict__ row_ptr, long long *__restrict__ nnz,
+            long long R) {
+  __shared__ long long part[SCAN_THREADS];
+  const int tid = threadIdx.x;
+  const long long per = (R + SCAN_THREADS - 1) / SCAN_THREADS;
+  const long long lo = min(R, tid * per), hi = min(R, lo + per);
+  long long s = 0;
+  for (long long r = lo; r < hi; ++r) s += counts[r];
+  part[tid] = s;
+  __syncthreads();
+  // Hillis-Steele inclusive scan over the per-thread sums.
+  for (int off = 1; off < SCAN_THREADS; off <<= 1) {
+    const long long add = (tid >= off) ? part[tid - off] : 0;
+    __syncthreads();
+    part[tid] += add;
+    __syncthreads();
+  }
+  long long run = part[tid] - s;  // exclusive prefix of this segment
+  if (tid == 0) row_ptr[0] = 0;
+  for (long long r = lo; r < hi; ++r) {
+    run += counts[r];
+    row_ptr[r + 1] = (int)run;
+  }
+  if (tid == SCAN_THREADS - 1) *nnz = part[tid];
+}
+
+// ---------------------------------------------------------------- fill
+// One warp per row: word prefix popcounts -> ascending column indices.
+__global__ void __launch_bounds__(256)
+fill_kernel(const unsigned int *__restrict__ bits, const int *__restrict__ row_ptr,
+            int *__restrict__ col_idx, unsigned char *__restrict__ block_mask, long long R, int nt,
+            int wpr) {
+  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= R) return;
+  const unsigned int *brow = bits + row * wpr;
+  int base = row_ptr[row];
+  for (int w0 = 0; w0 < wpr; w0 += 32) {
+    const int w = w0 + lane;
+    unsigned int word = (w < wpr) ? brow[w] : 0u;
+    const int c = __popc(word);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = base + incl - c;
+    if (block_mask && w < wpr) {
+      unsigned char *bm = block_mask + row * nt + (long long)w * 32;
+      const int lim = min(32, nt - w * 32);
+      for (int b = 0; b < lim; ++b) bm[b] = (unsigned char)((word >> b) & 1u);
+    }
+    while (word) {
+      const int b = __ffs(word) - 1;
+      col_idx[pos++] = w * 32 + b;
+      word &= word - 1u;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
+}  // namespace sta

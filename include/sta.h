@@ -1,0 +1,152 @@
+/*
+ * sta.h -- C ABI of libsta: block-sparse attention over a 3D video token grid
+ * with per-head tile masks, for NVIDIA B200 (sm_100a).
+ *
+ * The method (pages on training-free sparse attention for video diffusion
+ * transformers):
+ *   - Compact Attention (abstract; Fig. 1(3); Fig. 3; Fig. 4; Table III):
+ *     tile-aligned, head-specific masks made of two deformable windows with a
+ *     separate extent per temporal-distance group, computed once and loaded
+ *     into a block-sparse attention kernel that is reused across steps.
+ *   - Rectified SpaAttn (abstract): block importance from pooled query-key.
+ *   - SCOPE review (Eqs. (7)-(8) as quoted; abstract): hybrid top-p with a
+ *     fixed top-k floor.
+ *
+ * Conventions shared by every call
+ *   - Tiles are 1x8x8 tokens (64). For a T x H x W grid: NH = ceil(H/8),
+ *     NW = ceil(W/8), Nt = T*NH*NW tiles per head, Lpad = 64*Nt rows.
+ *     Tile n = (t*NH + y/8)*NW + x/8; token row inside the tile = (y%8)*8 + x%8.
+ *   - Raster tensors are [B, L, heads, d] bf16, L = T*H*W, token index
+ *     (t*H + y)*W + x. Tiled tensors are [B, heads, Lpad, d] bf16.
+ *   - Every pointer argument named as a tensor is DEVICE memory owned by the
+ *     caller; the library allocates nothing and keeps no pointer after return.
+ *   - All calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). Argument checks are synchronous and return a status
+ *     before anything is launched; a launch failure returns STA_ERR_CUDA.
+ *     Faults detected on the device (a bounded wait that ran out, an index out
+ *     of range) are recorded in a device error word read by
+ *     sta_get_device_error().
+ *   - d (head dim) must be 64 or 128. Device pointers must be 16-byte aligned.
+ */
+#ifndef STA_H
+#define STA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *sta_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+  STA_OK = 0,
+  STA_ERR_INVALID_ARG = 1, /* NULL pointer, bad size, misaligned pointer */
+  STA_ERR_UNSUPPORTED = 2, /* d not in {64,128}, grid too large, wrong GPU */
+  STA_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than required */
+  STA_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
+  STA_ERR_TIMEOUT = 5,     /* device: a bounded pipeline wait ran out */
+  STA_ERR_BAD_MASK = 6     /* device: a CSR column index out of range */
+} sta_status;
+
+typedef struct {
+  int32_t T, H, W; /* token grid; the tile is fixed at 1x8x8 */
+} sta_grid;
+
+#define STA_MAX_GROUPS 8
+
+/* Mask recipe of sta_build_mask.
+ * Selection (Rectified SpaAttn pooled scores; SCOPE hybrid top-p/top-k):
+ *   qbar, kbar = mean of Q, K over the real tokens of each tile;
+ *   P = softmax over key tiles of sm_scale * qbar . kbar (fp32);
+ *   order key tiles by P descending, ties to the lower index; with integer
+ *   mass w = floor(P * 2^24) and thr = ceil(double(top_p) * double(sum w)),
+ *   keep the shortest prefix reaching thr (all tiles if top_p >= 1, none if
+ *   top_p <= 0), extended to at least min(k_min, Nt) tiles.
+ * Windows (Compact Attention dual windows per temporal-distance group):
+ *   key tile kt is kept for query tile qt of head h iff the group
+ *   g = max{g : group_lo[g] <= |t_q - t_k|} exists and
+ *   (|dy| <= ry1 && |dx| <= rx1) || (|dy| <= ry2 && |dx| <= rx2)
+ *   with (ry1, rx1, ry2, rx2) = windows[(h*num_groups + g)*4 + 0..3], in
+ *   tile units; -1 switches a window off. The last group is open-ended.
+ * The mask is the union of the two parts. */
+typedef struct {
+  float top_p;            /* selection mass; >= 1 keeps all; ignored if !use_scores */
+  int32_t k_min;          /* floor on the selected count, clipped to Nt */
+  int32_t use_scores;     /* 0: window-only mask (no pooling / scoring) */
+  float sm_scale;         /* score scale; 0 means 1/sqrt(d) */
+  int32_t num_groups;     /* G in [1, STA_MAX_GROUPS] when windows != NULL */
+  int32_t group_lo[STA_MAX_GROUPS]; /* ascending, group_lo[0] == 0 */
+  const int32_t *windows; /* device int32 [heads][G][4]; NULL = no windows */
+} sta_mask_params;
+
+/* Number of tiles per head (Nt) and padded rows per head (Lpad) of a grid;
+ * -1 if the grid is invalid. */
+int64_t sta_num_tiles(sta_grid g);
+int64_t sta_tiled_len(sta_grid g);
+
+/* sta_reorder -- token layout change (Compact Attention: tile-aligned
+ * masks; Table III "Cubic" tiles).
+ *   inverse == 0: src raster [B, L, heads, d] -> dst tiled [B, heads, Lpad, d];
+ *                 rows of partial tiles beyond the grid are written as zero.
+ *   inverse != 0: src tiled -> dst raster; pad rows are dropped.
+ * bf16 elements are moved bit for bit. src and dst must not overlap. */
+sta_status sta_reorder(const void *src, void *dst, int32_t B, int32_t heads, int32_t d,
+                       sta_grid g, int32_t inverse, sta_stream_t stream);
+
+/* Bytes of device workspace sta_build_mask needs for these sizes. */
+size_t sta_build_mask_workspace(int32_t B, int32_t heads, int32_t d, sta_grid g);
+
+/* sta_build_mask -- per-head tile mask as CSR lists (Compact Attention Fig. 3:
+ * masks computed online are loaded into the block-sparse kernel; Fig. 4: the
+ * result is a binary mask over (query tile, key tile)).
+ *   q_tiled, k_tiled : [B, heads, Lpad, d] bf16 (read only if use_scores)
+ *   row_ptr          : int32 [B*heads*Nt + 1], written; row r = (b*heads+h)*Nt+qt
+ *   col_idx          : int32, capacity >= B*heads*Nt*Nt (worst case, so no
+ *                      host synchronisation is ever needed); each row's key
+ *                      tiles are written in ascending order
+ *   nnz_dev          : device int64 scalar, written with row_ptr[last]
+ *   block_mask       : optional uint8 [B, heads, Nt, Nt] (0/1); NULL to skip
+ *   block_probs      : optional fp32 [B, heads, Nt, Nt], the P the selection
+ *                      used (0 where !use_scores); NULL to skip
+ *   workspace        : device, >= sta_build_mask_workspace() bytes, 256-aligned
+ * The call is deterministic: the same inputs give bit-identical outputs. */
+sta_status sta_build_mask(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads,
+                          int32_t d, sta_grid g, const sta_mask_params *p, int32_t *row_ptr,
+                          int32_t *col_idx, int64_t *nnz_dev, uint8_t *block_mask,
+                          float *block_probs, void *workspace, size_t ws_bytes,
+                          sta_stream_t stream);
+
+/* sta_attn_fwd -- block-sparse attention forward over the listed key tiles
+ * (Compact Attention Fig. 3 "block-sparse attention kernels"; Fig. 5 "dense
+ * Compact kernel" is the same call with every tile listed).
+ * For every real query token of query tile qt in row r = (b*heads+h)*Nt+qt:
+ *   o   = sum_j softmax_j(sm_scale * q . k_j) v_j
+ *   lse = log(sum_j exp(sm_scale * q . k_j))           (natural log)
+ * over the real tokens j of tiles col_idx[row_ptr[r] .. row_ptr[r+1]).
+ *   q, k, v : tiled [B, heads, Lpad, d] bf16;  o : tiled [B, heads, Lpad, d] bf16
+ *   lse     : optional fp32 [B, heads, Lpad]; NULL to skip
+ *   row_ptr, col_idx : CSR as written by sta_build_mask (or the caller's own:
+ *             ascending, unique, in [0, Nt) per row; an index out of range is
+ *             reported as STA_ERR_BAD_MASK by sta_get_device_error and the
+ *             tile is skipped)
+ *   sm_scale: 0 means 1/sqrt(d)
+ * A row with an empty list gives o = 0 and lse = -inf. Output rows of pad
+ * tokens hold unspecified finite values. Accumulation is fp32; P is rounded
+ * to bf16 before the P.V product. */
+sta_status sta_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                        const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
+                        int32_t d, sta_grid g, float sm_scale, sta_stream_t stream);
+
+/* Reads and clears the device error word of the current device after
+ * synchronising `stream`. STA_OK if no device-side fault was recorded. */
+sta_status sta_get_device_error(sta_stream_t stream);
+
+/* Static description of a status code. */
+const char *sta_status_string(sta_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* STA_H */

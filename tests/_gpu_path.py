@@ -1,0 +1,66 @@
+"""Helpers for the GPU parity tests: run the CUDA path through the binding and
+bring results back as numpy. Imported only by tests marked gpu."""
+import math
+
+import numpy as np
+import torch
+
+import block_sparse_attention_28_b200 as sta
+
+DEV = "cuda"
+U32 = 2.0 ** -24
+
+
+def to_np64(x):
+    return x.float().cpu().numpy().astype(np.float64)
+
+
+def reorder(x, B, Hh, d, g):
+    lpad = sta.sta_tiled_len(g)
+    out = torch.full((B, Hh, lpad, d), float("nan"), dtype=torch.bfloat16, device=x.device)
+    sta.sta_reorder(x, out, B, Hh, d, g)
+    return out
+
+
+def build(qt, kt, B, Hh, d, g, params, with_mask=True, with_probs=True):
+    bufs = sta.MaskBuffers(B, Hh, d, g, qt.device if qt is not None else DEV, with_mask, with_probs)
+    sta.build_mask(qt, kt, B, Hh, d, g, params, bufs)
+    return bufs
+
+
+def csr_np(bufs):
+    nnz = int(bufs.nnz.item())
+    return bufs.row_ptr.cpu().numpy(), bufs.col_idx[:nnz].cpu().numpy(), nnz
+
+
+def attn(qt, kt, vt, row_ptr, col_idx, B, Hh, d, g, sm_scale=0.0):
+    o = torch.full_like(qt, float("nan"))
+    lse = torch.full(qt.shape[:3], float("nan"), dtype=torch.float32, device=qt.device)
+    sta.sta_attn_fwd(qt, kt, vt, o, lse, row_ptr, col_idx, B, Hh, d, g, sm_scale)
+    return o, lse
+
+
+def prob_bound(qbar, kbar, scale, p_ref):
+    """Per-element bound on |P_gpu - P_oracle| from the GPU arithmetic:
+    fp32 pooled means (one rounding each of an exact sum), a D-term fp32 FMA
+    chain for the score, fp32 exp / sum / divide. Returns an array like p_ref."""
+    d = qbar.shape[-1]
+    gam = d * U32 / (1 - d * U32)
+    cond = np.einsum("...qd,...kd->...qk", np.abs(qbar), np.abs(kbar)) * scale
+    ds = (gam + 2.0 * U32) * cond  # score error bound per element
+    E = ds.max(axis=-1, keepdims=True)
+    nt = p_ref.shape[-1]
+    rel = 2.2 * E + 4e-7 + 1.1 * nt * U32
+    return p_ref * rel + 1e-30
+
+
+def attn_errors(o_gpu_t, o_ref_t, valid_rows):
+    """max-abs and mean-abs error over real token rows (tiled layout)."""
+    a = to_np64(o_gpu_t)[:, :, valid_rows, :]
+    b = o_ref_t[:, :, valid_rows, :]
+    err = np.abs(a - b)
+    return float(err.max()), float(err.mean())
+
+
+def default_scale(d):
+    return 1.0 / math.sqrt(d)

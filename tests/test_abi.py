@@ -1,0 +1,83 @@
+"""The C-ABI library loads, exports every symbol the header declares, and its
+host-side logic (sizes, argument checks, status strings) behaves as stated.
+No compute call here needs a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sta.h")
+
+
+@pytest.fixture(scope="module")
+def sta():
+    from block_sparse_attention_28_b200 import build as b
+
+    b.build()
+    import block_sparse_attention_28_b200 as mod
+
+    return mod
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sta_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("sta_reorder", "sta_build_mask", "sta_build_mask_workspace", "sta_attn_fwd",
+                 "sta_get_device_error", "sta_status_string", "sta_num_tiles", "sta_tiled_len"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(sta):
+    lib = ctypes.CDLL(sta.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_tile_counts(sta):
+    assert sta.sta_num_tiles(sta.grid(21, 45, 80)) == 1260
+    assert sta.sta_tiled_len(sta.grid(21, 45, 80)) == 80640
+    assert sta.sta_num_tiles(sta.grid(33, 45, 80)) == 1980
+    assert sta.sta_num_tiles(sta.grid(21, 30, 52)) == 588
+    assert sta.sta_num_tiles(sta.grid(0, 4, 4)) == -1
+
+
+def test_workspace_size(sta):
+    g = sta.grid(21, 45, 80)
+    ws = sta.sta_build_mask_workspace(1, 40, 128, g)
+    R = 40 * 1260
+    assert ws >= 2 * R * 128 * 4 + R * 40 * 4 + R * 4
+    assert ws % 256 == 0
+    assert sta.sta_build_mask_workspace(1, 40, 96, g) == 0
+
+
+def test_argument_checks_return_before_any_launch(sta):
+    g = sta.grid(4, 16, 16)
+    lib = sta._lib
+    # unsupported head dim, bad batch, null pointers, misaligned pointers
+    assert lib.sta_reorder(16, 32, 1, 2, 96, g, 0, None) == sta.STA_ERR_UNSUPPORTED
+    assert lib.sta_reorder(16, 32, 0, 2, 64, g, 0, None) == sta.STA_ERR_INVALID_ARG
+    assert lib.sta_reorder(None, 32, 1, 2, 64, g, 0, None) == sta.STA_ERR_INVALID_ARG
+    assert lib.sta_reorder(17, 32, 1, 2, 64, g, 0, None) == sta.STA_ERR_INVALID_ARG
+    assert lib.sta_attn_fwd(None, 16, 16, 16, None, 16, 16, 1, 2, 64, g, 0.0, None) == sta.STA_ERR_INVALID_ARG
+    assert lib.sta_attn_fwd(16, 16, 16, 16, None, 16, 16, 1, 2, 64, g, -1.0, None) == sta.STA_ERR_INVALID_ARG
+    p = sta.mask_params(0.9, 2, True)
+    assert lib.sta_build_mask(16, 16, 1, 2, 64, g, ctypes.byref(p), 16, 16, 16, None, None, None, 0,
+                              None) == sta.STA_ERR_WORKSPACE
+    bad = sta.mask_params(0.9, 2, True, group_lo=(1, 2), windows=16)
+    assert lib.sta_build_mask(16, 16, 1, 2, 64, g, ctypes.byref(bad), 16, 16, 16, None, None, 256, 1 << 30,
+                              None) == sta.STA_ERR_INVALID_ARG
+    too_big = sta.grid(1 << 12, 1 << 10, 1 << 10)
+    assert lib.sta_reorder(16, 32, 1, 2, 64, too_big, 0, None) != sta.STA_OK
+
+
+def test_status_strings(sta):
+    for s in range(7):
+        assert sta.sta_status_string(s)
+    assert "out of range" in sta.sta_status_string(sta.STA_ERR_BAD_MASK)

@@ -1,0 +1,341 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Bars: reorder, CSR lists and byte masks bit-exact; block probabilities within
+a bound derived from the GPU's fp32 arithmetic; attention output within
+max-abs 2e-2 and mean-abs 2e-3 of the oracle, LSE within 1e-3, with masks
+built from identical block probabilities (the oracle's selection runs on the
+GPU's exported P).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from workloads import CONFIGS, fixed_windows_tiny, make_qkv, window_params, window_scale
+
+pytestmark = pytest.mark.gpu
+
+ATOL_MAX, ATOL_MEAN, LSE_TOL = 2e-2, 2e-3, 1e-3
+
+
+@pytest.fixture(scope="module")
+def sta():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    import block_sparse_attention_28_b200 as mod
+
+    return mod
+
+
+@pytest.fixture(scope="module")
+def gp(sta):
+    import _gpu_path
+
+    return _gpu_path
+
+
+def _rand_raster(B, L, Hh, d, seed, scale=1.0, device="cuda"):
+    g = torch.Generator(device=device).manual_seed(seed)
+    return (torch.randn(B, L, Hh, d, generator=g, device=device) * scale).to(torch.bfloat16)
+
+
+def _structured(T, H, W, Hh, d, seed, B=1):
+    """Small Q, K, V with the workload recipe (RFF positions + noise)."""
+    from workloads.configs import WorkloadConfig
+
+    cfg = WorkloadConfig(name="t", B=B, heads=Hh, d=d, T=T, H=H, W=W, seed=seed, use_scores=True)
+    return [x.cuda() for x in make_qkv(cfg, device="cpu")]
+
+
+# ------------------------------------------------------------------ reorder
+@pytest.mark.parametrize("T,H,W,d,B,Hh", [(4, 16, 16, 64, 1, 2), (3, 13, 19, 128, 2, 3),
+                                          (2, 9, 10, 64, 1, 1), (1, 8, 8, 128, 1, 5)])
+def test_reorder_bit_exact(sta, gp, T, H, W, d, B, Hh):
+    g = sta.grid(T, H, W)
+    x = _rand_raster(B, T * H * W, Hh, d, seed=T * 100 + H)
+    xt = gp.reorder(x, B, Hh, d, g)
+    want = O.reorder_fwd(gp.to_np64(x), T, H, W)
+    got = gp.to_np64(xt)
+    assert np.array_equal(got, want)  # also: pad rows are exactly zero
+    back = torch.full_like(x, float("nan"))
+    sta.sta_reorder(xt, back, B, Hh, d, g, inverse=True)
+    assert torch.equal(back.view(torch.int16), x.view(torch.int16))
+
+
+def test_reorder_full_size_720p(sta, gp):
+    cfg = CONFIGS[2]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    x = _rand_raster(B, cfg.L, Hh, d, seed=7)
+    xt = gp.reorder(x, B, Hh, d, g)
+    rows = O.tiled_row_of_raster(T, H, W)
+    rng = np.random.default_rng(0)
+    sample = rng.choice(cfg.L, 4096, replace=False)
+    got = xt[0][:, torch.from_numpy(rows[sample]).cuda(), :]
+    want = x[0][torch.from_numpy(sample).cuda()].transpose(0, 1)
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    valid = torch.from_numpy(O.valid_rows(T, H, W)).cuda()
+    assert int(valid.sum()) == cfg.L
+    assert torch.count_nonzero(xt[:, :, ~valid, :].float()) == 0
+    back = torch.empty_like(x)
+    sta.sta_reorder(xt, back, B, Hh, d, g, inverse=True)
+    assert torch.equal(back.view(torch.int16), x.view(torch.int16))
+
+
+# --------------------------------------------------------------- build_mask
+def _check_mask(sta, gp, qt, kt, B, Hh, d, T, H, W, top_p, k_min, use_scores, win, group_lo,
+                check_probs=True):
+    g = sta.grid(T, H, W)
+    win_d = torch.from_numpy(win).cuda() if win is not None else None
+    params = sta.mask_params(top_p, k_min, use_scores, 0.0, group_lo, win_d)
+    bufs = gp.build(qt, kt, B, Hh, d, g, params)
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    rp, ci, nnz = gp.csr_np(bufs)
+    nt = sta.sta_num_tiles(g)
+    mask = np.zeros((B, Hh, nt, nt), dtype=bool)
+    probs = bufs.block_probs.cpu().numpy()
+    if use_scores:
+        mask |= O.select(probs, top_p, k_min)
+        if check_probs:
+            scale = 1.0 / math.sqrt(d)
+            qb, kb = O.pool(gp.to_np64(qt), T, H, W), O.pool(gp.to_np64(kt), T, H, W)
+            _, p_ref = O.block_scores(qb, kb, scale)
+            bound = gp.prob_bound(qb, kb, scale, p_ref)
+            assert np.all(np.abs(probs - p_ref) <= bound)
+            # the oracle's own end-to-end mask differs only at near-ties
+            own = O.select(p_ref, top_p, k_min)
+            sel_gpu = O.select(probs, top_p, k_min)
+            assert (own != sel_gpu).mean() < 1e-3
+    else:
+        assert np.all(probs == 0)
+    if win is not None:
+        mask |= O.window_mask(win, group_lo, T, H, W)[None]
+    rp_o, ci_o = O.mask_to_csr(mask)
+    assert np.array_equal(rp, rp_o)
+    assert nnz == ci_o.size and np.array_equal(ci, ci_o)
+    assert np.array_equal(bufs.block_mask.cpu().numpy().astype(bool), mask)
+    return bufs, mask
+
+
+def test_build_mask_tiny_config(sta, gp):
+    cfg = CONFIGS[0]
+    q, k, _ = (x.cuda() for x in make_qkv(cfg, device="cpu"))
+    g = sta.grid(cfg.T, cfg.H, cfg.W)
+    qt, kt = gp.reorder(q, 1, cfg.heads, cfg.d, g), gp.reorder(k, 1, cfg.heads, cfg.d, g)
+    _check_mask(sta, gp, qt, kt, 1, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W, cfg.top_p, cfg.k_min, True,
+                fixed_windows_tiny(cfg), cfg.group_lo)
+
+
+@pytest.mark.parametrize("top_p,k_min,use_scores,with_win", [
+    (0.7, 3, True, True), (0.95, 8, True, False), (1.0, 0, True, False), (0.0, 0, True, False),
+    (0.0, 5, True, True), (0.5, 100, True, False), (0.0, 0, False, True), (0.3, 1, True, True)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_build_mask_ragged(sta, gp, top_p, k_min, use_scores, with_win, d):
+    T, H, W, Hh, B = 3, 19, 37, 3, 2  # 3 x 3 x 5 = 45 tiles, partial tiles on two edges
+    rng = np.random.default_rng(d + int(100 * top_p) + k_min)
+    q, k, _ = _structured(T, H, W, Hh, d, seed=11, B=B)
+    g = sta.grid(T, H, W)
+    qt, kt = gp.reorder(q, B, Hh, d, g), gp.reorder(k, B, Hh, d, g)
+    win = None
+    if with_win:
+        win = rng.integers(-1, 3, size=(Hh, 3, 4)).astype(np.int32)
+    _check_mask(sta, gp, qt, kt, B, Hh, d, T, H, W, top_p, k_min, use_scores, win, (0, 1, 3))
+
+
+def test_build_mask_window_only_full_480p(sta, gp):
+    cfg = CONFIGS[1]
+    g = sta.grid(cfg.T, cfg.H, cfg.W)
+    win = window_params(cfg, window_scale(1, 0))
+    win_d = torch.from_numpy(win).cuda()
+    params = sta.mask_params(0.0, 0, False, 0.0, cfg.group_lo, win_d)
+    bufs = gp.build(None, None, 1, cfg.heads, cfg.d, g, params, with_mask=False, with_probs=False)
+    rp, ci, nnz = gp.csr_np(bufs)
+    mask = O.window_mask(win, cfg.group_lo, cfg.T, cfg.H, cfg.W)[None]
+    rp_o, ci_o = O.mask_to_csr(mask)
+    assert np.array_equal(rp, rp_o) and np.array_equal(ci, ci_o)
+    assert abs(nnz / mask.size - 0.25) < 0.01
+
+
+def test_build_mask_full_720p_sampled_rows(sta, gp):
+    """The headline layer: full-size build; the oracle's selection on the GPU's
+    P for sampled rows, plus the windows, must give the same CSR rows."""
+    cfg = CONFIGS[2]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    q, k, _ = make_qkv(cfg, device="cuda")
+    qt, kt = gp.reorder(q, B, Hh, d, g), gp.reorder(k, B, Hh, d, g)
+    del q, k
+    win = window_params(cfg, window_scale(2, 0))
+    params = sta.mask_params(cfg.top_p, cfg.k_min, True, 0.0, cfg.group_lo, torch.from_numpy(win).cuda())
+    bufs = gp.build(qt, kt, B, Hh, d, g, params, with_mask=False, with_probs=True)
+    torch.cuda.synchronize()
+    rp, ci, nnz = gp.csr_np(bufs)
+    nt = sta.sta_num_tiles(g)
+    rng = np.random.default_rng(2)
+    heads = rng.choice(Hh, 3, replace=False)
+    wm = O.window_mask(win[heads], cfg.group_lo, T, H, W)
+    for hi, h in enumerate(heads):
+        rows = rng.choice(nt, 40, replace=False)
+        probs = bufs.block_probs[0, h, torch.from_numpy(rows).cuda()].cpu().numpy()
+        for ri, qtile in enumerate(rows):
+            keep = O.select_row(probs[ri], cfg.top_p, cfg.k_min) | wm[hi, qtile]
+            r = h * nt + qtile
+            assert np.array_equal(ci[rp[r]:rp[r + 1]], np.nonzero(keep)[0]), (h, qtile)
+    density = nnz / (B * Hh * nt * nt)
+    assert 0.10 < density < 0.20, density
+
+
+# ------------------------------------------------------------------ attention
+def _attn_check(sta, gp, qt, kt, vt, rp_t, ci_t, B, Hh, d, T, H, W, sm_scale=0.0, rows=None):
+    g = sta.grid(T, H, W)
+    o, lse = gp.attn(qt, kt, vt, rp_t, ci_t, B, Hh, d, g, sm_scale)
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    rp, ci = rp_t.cpu().numpy(), ci_t.cpu().numpy()
+    scale = sm_scale if sm_scale else 1.0 / math.sqrt(d)
+    nt = sta.sta_num_tiles(g)
+    if rows is None:
+        rows = range(B * Hh * nt)
+    q64, k64, v64 = gp.to_np64(qt), gp.to_np64(kt), gp.to_np64(vt)
+    res = O.attention_rows(q64, k64, v64, rp, ci, T, H, W, scale, rows)
+    o_np = o.float().cpu().numpy()
+    lse_np = lse.cpu().numpy()
+    errs = []
+    for r, qrows, o_ref, lse_ref in res:
+        bh, _ = divmod(r, nt)
+        b, h = divmod(bh, Hh)
+        got = o_np[b, h, qrows]
+        errs.append(np.abs(got - o_ref).ravel())
+        gl = lse_np[b, h, qrows]
+        fin = np.isfinite(lse_ref)
+        assert np.all(np.isneginf(gl[~fin]))
+        assert np.all(np.abs(gl[fin] - lse_ref[fin]) <= LSE_TOL * np.maximum(1.0, np.abs(lse_ref[fin])))
+    err = np.concatenate(errs)
+    assert np.isfinite(err).all()
+    assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (err.max(), err.mean())
+    return o, lse, err
+
+
+def test_attn_tiny_config(sta, gp):
+    cfg = CONFIGS[0]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    q, k, v = (x.cuda() for x in make_qkv(cfg, device="cpu"))
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    win = torch.from_numpy(fixed_windows_tiny(cfg)).cuda()
+    bufs = gp.build(qt, kt, B, Hh, d, g, sta.mask_params(cfg.top_p, cfg.k_min, True, 0.0, cfg.group_lo, win))
+    _attn_check(sta, gp, qt, kt, vt, bufs.row_ptr, bufs.col_idx, B, Hh, d, T, H, W)
+
+
+def _custom_csr(mask):
+    rp, ci = O.mask_to_csr(mask)
+    return torch.from_numpy(rp).cuda(), torch.from_numpy(np.ascontiguousarray(ci) if ci.size else
+                                                         np.zeros(1, np.int32)).cuda()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("kind", ["random", "dense", "empty_rows", "single_tile", "edge_tiles"])
+def test_attn_ragged_masks(sta, gp, d, kind):
+    T, H, W, Hh, B = 3, 19, 37, 2, 2  # 45 tiles: odd count, so the last CTA has one tile
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = _structured(T, H, W, Hh, d, seed=5, B=B)
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    rng = np.random.default_rng(len(kind) + d)
+    if kind == "random":
+        mask = rng.random((B, Hh, nt, nt)) < 0.3
+    elif kind == "dense":
+        mask = np.ones((B, Hh, nt, nt), dtype=bool)
+    elif kind == "empty_rows":
+        mask = rng.random((B, Hh, nt, nt)) < 0.2
+        mask[:, :, ::3] = False  # whole rows empty, including both halves of some CTAs
+        mask[0, 0, 0:2] = False
+    elif kind == "single_tile":
+        mask = np.zeros((B, Hh, nt, nt), dtype=bool)
+        for r in range(nt):
+            mask[:, :, r, (r * 7) % nt] = True
+    else:  # only the partial tiles at the right / bottom edges
+        nh, nw = (H + 7) // 8, (W + 7) // 8
+        edge = [t for t in range(nt) if (t % nw) == nw - 1 or ((t // nw) % nh) == nh - 1]
+        mask = np.zeros((B, Hh, nt, nt), dtype=bool)
+        mask[..., edge] = True
+    rp, ci = _custom_csr(mask)
+    _attn_check(sta, gp, qt, kt, vt, rp, ci, B, Hh, d, T, H, W, sm_scale=0.11 if d == 64 else 0.0)
+
+
+def test_attn_dense_large_logits(sta, gp):
+    """Dense mask on an unpadded grid with a large score scale, so that the
+    running max moves by more than the lazy-rescale threshold many times."""
+    T, H, W, Hh, B, d = 2, 32, 48, 2, 1, 128
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = _structured(T, H, W, Hh, d, seed=9)
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    rp, ci = _custom_csr(np.ones((B, Hh, nt, nt), dtype=bool))
+    _attn_check(sta, gp, qt, kt, vt, rp, ci, B, Hh, d, T, H, W, sm_scale=0.35)
+
+
+def test_attn_full_720p_sampled_rows(sta, gp):
+    """The headline layer end to end: full-size build and attention as timed by
+    the benchmark; the oracle recomputes sampled rows on the GPU's CSR."""
+    cfg = CONFIGS[2]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    q, k, v = make_qkv(cfg, device="cuda")
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    del q, k, v
+    win = torch.from_numpy(window_params(cfg, window_scale(2, 0))).cuda()
+    bufs = gp.build(qt, kt, B, Hh, d, g, sta.mask_params(cfg.top_p, cfg.k_min, True, 0.0, cfg.group_lo, win),
+                    with_mask=False, with_probs=False)
+    nt = sta.sta_num_tiles(g)
+    rng = np.random.default_rng(3)
+    rows = sorted(rng.choice(B * Hh * nt, 48, replace=False).tolist())
+    _attn_check(sta, gp, qt, kt, vt, bufs.row_ptr, bufs.col_idx, B, Hh, d, T, H, W, rows=rows)
+
+
+def test_attn_reuse_steps(sta, gp):
+    """Mask built once from step-0 inputs, reused after 10 perturbed steps."""
+    cfg = CONFIGS[4]
+    B, Hh, d, T, H, W = cfg.B, 8, cfg.d, cfg.T, cfg.H, cfg.W
+    from dataclasses import replace
+
+    c8 = replace(cfg, heads=Hh)
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = make_qkv(c8, device="cuda")
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    kmin = int(round(0.10 * nt))
+    bufs = gp.build(qt, kt, B, Hh, d, g, sta.mask_params(0.0, kmin, True), with_mask=False, with_probs=False)
+    rp, ci, nnz = gp.csr_np(bufs)
+    assert nnz == B * Hh * nt * kmin
+    gen = torch.Generator(device="cuda").manual_seed(44)
+    mq, mk = q.float(), k.float()
+    from workloads import perturb_step
+
+    for _ in range(cfg.reuse_steps):
+        mq, qb = perturb_step(mq, gen)
+        mk, kb = perturb_step(mk, gen)
+    qt10, kt10 = gp.reorder(qb, B, Hh, d, g), gp.reorder(kb, B, Hh, d, g)
+    rng = np.random.default_rng(4)
+    rows = sorted(rng.choice(B * Hh * nt, 24, replace=False).tolist())
+    _attn_check(sta, gp, qt, kt, vt, bufs.row_ptr, bufs.col_idx, B, Hh, d, T, H, W, rows=rows)
+    _attn_check(sta, gp, qt10, kt10, vt, bufs.row_ptr, bufs.col_idx, B, Hh, d, T, H, W, rows=rows)
+
+
+def test_attn_bad_column_index_is_reported(sta, gp):
+    T, H, W, Hh, B, d = 2, 16, 16, 1, 1, 64
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = _structured(T, H, W, Hh, d, seed=3)
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    mask = np.ones((B, Hh, nt, nt), dtype=bool)
+    rp, ci = _custom_csr(mask)
+    ci[3] = nt + 5  # out of range: skipped and reported, never read
+    sta.sta_get_device_error()
+    o, lse = gp.attn(qt, kt, vt, rp, ci, B, Hh, d, g)
+    assert sta.sta_get_device_error() == sta.STA_ERR_BAD_MASK
+    assert sta.sta_get_device_error() == sta.STA_OK  # the word was cleared
+    assert torch.isfinite(o.float()).all()
