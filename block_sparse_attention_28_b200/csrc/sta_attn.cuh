@@ -322,7 +322,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         l = l * alpha + sum;
         const bool need_o = rescale && (m != -INFINITY);
         if (__any_sync(0xffffffffu, need_o)) {
-          // PV_{j-1} must have retired before O is scaled (j >= 1 here).
+          // PV_{j-1} must have retired before O is scaled (j >= 1 here). S_j
+          // was issued after PV_{j-2}, so its completion proves PV_{j-2}
+          // retired: o_done has completed j-1 or j phases and the parity of
+          // phase j-1 is unambiguous.
           const bool got_o = tc::mbar_wait(o_done, (j - 1) & 1, abort_flag, WAIT_LIMIT);
           if (!__all_sync(0xffffffffu, got_o)) {
             ok = false;
@@ -347,7 +350,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (lane == 0) tc::mbar_arrive(p_full + buf);
     }
     // ---- epilogue
-    if (ok && n > 0) ok = tc::mbar_wait(o_done, (n - 1) & 1, abort_flag, WAIT_LIMIT);
+    // Wait on the single-use barrier committed after the last P.V: o_done's
+    // parity cannot tell PV_{n-1} from PV_{n-2} here, because the last S MMA
+    // was issued before PV_{n-2} and so proves only PV_{n-3} retired.
+    if (ok && n > 0) ok = tc::mbar_wait(mma_done, 0, abort_flag, WAIT_LIMIT);
     ok = __all_sync(0xffffffffu, ok);
     tc::fence_after();
     const bool row_exists = !halfB || hasB;
