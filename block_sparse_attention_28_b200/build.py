@@ -1,6 +1,9 @@
 """Build libsta.so in-tree with nvcc for sm_100a.
 
-    python -m block_sparse_attention_28_b200.build
+    python block_sparse_attention_28_b200/build.py [--force]
+
+Run it as a script (or load it by path): importing it through the package
+would first load the library it is meant to (re)build.
 """
 import os
 import shutil

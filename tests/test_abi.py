@@ -13,9 +13,9 @@ HEADER = os.path.join(ROOT, "include", "sta.h")
 
 @pytest.fixture(scope="module")
 def sta():
-    from block_sparse_attention_28_b200 import build as b
+    import runpy
 
-    b.build()
+    runpy.run_path(os.path.join(ROOT, "block_sparse_attention_28_b200", "build.py"), run_name="sta_build")["build"]()
     import block_sparse_attention_28_b200 as mod
 
     return mod
