@@ -49,7 +49,7 @@ class MaskParams(ctypes.Structure):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m block_sparse_attention_28_b200.build`")
+        f"{LIB_PATH} is missing: build it with `python block_sparse_attention_28_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 _vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -65,6 +65,9 @@ _lib.sta_build_mask_workspace.restype = _sz
 _lib.sta_build_mask.argtypes = [_vp, _vp, _i32, _i32, _i32, Grid, ctypes.POINTER(MaskParams), _vp, _vp,
                                 _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sta_build_mask.restype = ctypes.c_int
+_lib.sta_build_mask_noalloc.argtypes = [_vp, _vp, _i32, _i32, _i32, Grid, ctypes.POINTER(MaskParams), _vp,
+                                        _vp, _vp, _vp, _vp, _vp]
+_lib.sta_build_mask_noalloc.restype = ctypes.c_int
 _lib.sta_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, Grid, _f32, _vp]
 _lib.sta_attn_fwd.restype = ctypes.c_int
 _lib.sta_get_device_error.argtypes = [_vp]
@@ -139,6 +142,17 @@ def sta_build_mask(q_tiled, k_tiled, B, heads, d, g, params, row_ptr, col_idx, n
                                _ptr(row_ptr), _ptr(col_idx), _ptr(nnz_dev), _ptr(block_mask),
                                _ptr(block_probs), _ptr(workspace), int(ws_bytes), _stream(stream)),
            "sta_build_mask")
+
+
+def sta_build_mask_noalloc(q_tiled, k_tiled, B, heads, d, g, params, row_ptr, col_idx, nnz_dev,
+                           block_mask=None, block_probs=None, stream=None):
+    """sta_build_mask without a workspace argument, for callers that cannot
+    allocate device memory: the library's static 32 MiB device array serves as
+    the workspace (see include/sta.h for the size limit and sharing rules)."""
+    _check(_lib.sta_build_mask_noalloc(_ptr(q_tiled), _ptr(k_tiled), B, heads, d, g, ctypes.byref(params),
+                                       _ptr(row_ptr), _ptr(col_idx), _ptr(nnz_dev), _ptr(block_mask),
+                                       _ptr(block_probs), _stream(stream)),
+           "sta_build_mask_noalloc")
 
 
 def sta_attn_fwd(q, k, v, o, lse, row_ptr, col_idx, B, heads, d, g, sm_scale=0.0, stream=None):

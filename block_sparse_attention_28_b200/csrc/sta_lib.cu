@@ -3,6 +3,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "sta_attn.cuh"
 #include "sta_common.cuh"
 #include "sta_mask.cuh"
@@ -266,3 +268,48 @@ const char *sta_status_string(sta_status s) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free mask build: the workspace is this static device array.
+// Host code must not hand the array's name to a kernel (on the host it is only
+// a stand-in); its device address is looked up once per device with
+// cudaGetSymbolAddress and cached.
+namespace {
+
+constexpr int NOALLOC_MAX_DEVICES = 64;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[STA_NOALLOC_SCRATCH_BYTES];
+std::mutex g_noalloc_mutex;
+void *g_noalloc_addr[NOALLOC_MAX_DEVICES] = {};
+
+sta_status noalloc_scratch_address(void **out) {
+  int dev = -1;
+  STA_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return STA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void *addr = nullptr;
+    STA_CUDA_TRY(cudaGetSymbolAddress(&addr, g_noalloc_scratch));
+    if (addr == nullptr) return STA_ERR_CUDA;
+    g_noalloc_addr[dev] = addr;
+  }
+  *out = g_noalloc_addr[dev];
+  return STA_OK;
+}
+
+}  // namespace
+
+extern "C" sta_status sta_build_mask_noalloc(const void *q_tiled, const void *k_tiled, int32_t B,
+                                             int32_t heads, int32_t d, sta_grid g,
+                                             const sta_mask_params *p, int32_t *row_ptr,
+                                             int32_t *col_idx, int64_t *nnz_dev, uint8_t *block_mask,
+                                             float *block_probs, sta_stream_t stream) {
+  Geo geo;
+  sta_status st = STA_OK;
+  if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return st;
+  if (mask_ws_layout(B, heads, d, geo).total > (size_t)STA_NOALLOC_SCRATCH_BYTES) return STA_ERR_WORKSPACE;
+  void *scratch = nullptr;
+  st = noalloc_scratch_address(&scratch);
+  if (st != STA_OK) return st;
+  return sta_build_mask(q_tiled, k_tiled, B, heads, d, g, p, row_ptr, col_idx, nnz_dev, block_mask,
+                        block_probs, scratch, (size_t)STA_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -139,6 +139,35 @@ sta_status sta_attn_fwd(const void *q, const void *k, const void *v, void *o, fl
                         const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
                         int32_t d, sta_grid g, float sm_scale, sta_stream_t stream);
 
+/* Size in bytes of the static device scratch behind sta_build_mask_noalloc. */
+#define STA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* sta_build_mask_noalloc -- sta_build_mask for callers that cannot allocate.
+ * The pages have no counterpart to this call: it exists for callers whose
+ * device memory is laid out up front by a host framework or a fixed arena
+ * (embedded inference runtimes, plug-ins of engines that own every device
+ * allocation), so they can neither call cudaMalloc nor lend a workspace.
+ * Same arguments, results and determinism as sta_build_mask, minus the
+ * workspace: the workspace is a file-scope static device array of
+ * STA_NOALLOC_SCRATCH_BYTES (32 MiB), present on every GPU that loads the
+ * library until the process exits. The caller still passes inputs and outputs.
+ *   - Sizes whose workspace (sta_build_mask_workspace) exceeds the array are
+ *     rejected with STA_ERR_WORKSPACE before anything runs (e.g. 40 heads of a
+ *     21x30x52 grid fit; 40 heads of 21x45x80 do not).
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (the device must be current); make that first call
+ *     before any stream capture. Later calls reuse the cached address.
+ *   - No allocation of any kind (no cudaMalloc / cudaFree, no allocating
+ *     library routine). Nothing in the array has to start at zero: every
+ *     byte the kernels read is written earlier in the same call.
+ *   - All calls share the one array, which keeps the last call's contents:
+ *     calls that overlap on the GPU (different streams, or other host threads)
+ *     race on it and must be serialised by the caller. */
+sta_status sta_build_mask_noalloc(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads,
+                                  int32_t d, sta_grid g, const sta_mask_params *p, int32_t *row_ptr,
+                                  int32_t *col_idx, int64_t *nnz_dev, uint8_t *block_mask,
+                                  float *block_probs, sta_stream_t stream);
+
 /* Reads and clears the device error word of the current device after
  * synchronising `stream`. STA_OK if no device-side fault was recorded. */
 sta_status sta_get_device_error(sta_stream_t stream);
