@@ -133,7 +133,7 @@ class ClockSampler:
 class Layer:
     """Device buffers and launches of one step of the path."""
 
-    def __init__(self, sta, cfg, dev, seed_offset=0):
+    def __init__(self, sta, cfg, dev, seed_offset=0, cfg_index=CFG_INDEX, density_index=0):
         from dataclasses import replace
 
         self.sta = sta
@@ -148,7 +148,10 @@ class Layer:
         self.qt, self.kt, self.vt, self.ot = (torch.empty(shape_t, dtype=torch.bfloat16, device=dev)
                                               for _ in range(4))
         self.o = torch.empty_like(self.q)
-        self.win = torch.from_numpy(window_params(cfg, window_scale(CFG_INDEX, 0))).to(dev)
+        if c.window_density:
+            self.win = torch.from_numpy(window_params(cfg, window_scale(cfg_index, density_index))).to(dev)
+        else:
+            self.win = None
         self.params = sta.mask_params(c.top_p, c.k_min, c.use_scores, 0.0, c.group_lo, self.win)
         self.bufs = sta.MaskBuffers(self.B, self.Hh, self.d, self.g, dev)
         self.launches_per_step = 3 + 4 + 1 + 1  # reorder x3, pool/select/scan/fill, attn, inverse
@@ -293,6 +296,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config-index", type=int, default=CFG_INDEX,
+                    help="workload (profiling of smaller layers); the headline is the 720p layer")
+    ap.add_argument("--density-index", type=int, default=0)
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -310,8 +316,9 @@ def main():
         import torch.distributed as dist
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    cfg = CONFIGS[CFG_INDEX]
-    layer = Layer(sta, cfg, dev, seed_offset=rank)
+    cfg = CONFIGS[args.config_index]
+    layer = Layer(sta, cfg, dev, seed_offset=rank, cfg_index=args.config_index,
+                  density_index=args.density_index)
 
     def barrier():
         if world > 1:
@@ -391,7 +398,7 @@ def main():
     line = None
     if rank == 0:
         cpu = None
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.config_index == CFG_INDEX:
             v_cpu, desc, dt, threads = cpu_oracle_sample(cfg, layer, args.cpu_budget)
             cpu = {"value": v_cpu, "unit": UNIT, "cores": threads, "kind": "oracle",
                    "sample": f"{desc}; {dt:.1f} s"}

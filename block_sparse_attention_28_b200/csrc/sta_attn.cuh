@@ -36,11 +36,16 @@ constexpr uint32_t O_COL = 128;
 constexpr long long WAIT_LIMIT = 2000000000LL;   // SM cycles (~1 s)
 constexpr long long DRAIN_LIMIT = 200000000LL;   // after an abort
 constexpr float RESCALE_LOG2 = 8.0f;             // lazy O rescale threshold
+constexpr int MIN_BLOCKS_PER_SM = 2;             // two CTAs share an SM: one's softmax
+                                                 // overlaps the other's MMAs
+#ifndef STA_EXP2_POLY_EVERY
+#define STA_EXP2_POLY_EVERY 0                    // every k-th column pair uses ex2_poly
+#endif
 
 template <int D>
 struct Cfg {
   static constexpr int KB = D / 64;              // 128-byte swizzle atoms along d
-  static constexpr int NS = (D == 128) ? 4 : 6;  // K/V ring stages
+  static constexpr int NS = (D == 128) ? 2 : 4;  // K/V ring stages (2 CTAs per SM fit)
   static constexpr int TILE_BYTES = 64 * D * 2;  // one 64-token tile of Q, K or V
   static constexpr int Q_REGION = 128 * 128;     // 128 rows x 128 B per d-atom
   static constexpr int OFF_Q = 0;
@@ -62,7 +67,7 @@ inline size_t smem_bytes(int nt) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(NUM_THREADS, MIN_BLOCKS_PER_SM)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16 *__restrict__ out,
                 float *__restrict__ lse, const int *__restrict__ row_ptr,
@@ -302,22 +307,39 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int c = 0; c < 64; ++c)
             if ((c >> 3) >= vy || (c & 7) >= vx) s[c] = -INFINITY;
         }
-        float mx = s[0];
+        // tree reduction: max is exact in any order, and the tree is 6 deep
+        float t32[32];
 #pragma unroll
-        for (int c = 1; c < 64; ++c) mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < 32; ++c) t32[c] = fmaxf(s[c], s[c + 32]);
+#pragma unroll
+        for (int w = 16; w > 0; w >>= 1) {
+#pragma unroll
+          for (int c = 0; c < w; ++c) t32[c] = fmaxf(t32[c], t32[c + w]);
+        }
+        const float mx = t32[0];
         const float m_new = fmaxf(m, mx * scale_log2);
         const bool rescale = m_new > m + RESCALE_LOG2;
         const float m_use = rescale ? m_new : m;
         const float mref = (m_use == -INFINITY) ? 0.0f : m_use;
         const float alpha = rescale ? tc::ex2(m - m_new) : 1.0f;
-        float sum = 0.0f;
+        float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float p0 = tc::ex2(fmaf(s[2 * c], scale_log2, -mref));
-          const float p1 = tc::ex2(fmaf(s[2 * c + 1], scale_log2, -mref));
-          sum += p0 + p1;
+          const float x0 = fmaf(s[2 * c], scale_log2, -mref);
+          const float x1 = fmaf(s[2 * c + 1], scale_log2, -mref);
+          float p0, p1;
+          if (STA_EXP2_POLY_EVERY > 0 && (c % (STA_EXP2_POLY_EVERY > 0 ? STA_EXP2_POLY_EVERY : 1)) ==
+                                             STA_EXP2_POLY_EVERY - 1) {
+            p0 = tc::ex2_poly(x0);
+            p1 = tc::ex2_poly(x1);
+          } else {
+            p0 = tc::ex2(x0);
+            p1 = tc::ex2(x1);
+          }
+          part[c & 3] += p0 + p1;
           pk[c] = tc::pack_bf16(p0, p1);
         }
+        const float sum = (part[0] + part[1]) + (part[2] + part[3]);
         tc::tmem_st32(sS, pk);
         l = l * alpha + sum;
         const bool need_o = rescale && (m != -INFINITY);
