@@ -12,8 +12,10 @@
 //              (TMEM lane i): S row -> online softmax (exp2, lazy rescale of
 //              O when the running max grows by more than 2^8) -> P (bf16) back
 //              into TMEM over S; at the end O / l -> bf16 -> global, and LSE.
-//   warp 4     TMA producer: Q once, then K_j and V_j per listed key tile
-//              into an NS-stage ring (128 B swizzle, no multicast).
+//   warp 4     TMA producer: Q once, then K_{j+1} ahead of V_j per listed key
+//              tile, each into its own NS-stage ring (128 B swizzle, no
+//              multicast); a K slot is freed as soon as its S MMA retires, a V
+//              slot when its P.V MMA retires.
 //   warp 5     MMA issuer (one thread): S_j = Q K_j^T (SS, M=128 N=64) into
 //              one of two TMEM S buffers, O += P_j V_j (A = P from TMEM,
 //              B = V MN-major from shared memory, M=128 N=d).
@@ -52,8 +54,9 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + KB * Q_REGION;
   static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + NS * TILE_BYTES;
-  // q_full, k_full[NS], v_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done, mma_done
-  static constexpr int NUM_BARS = 1 + 3 * NS + 2 + 2 + 1 + 1;
+  // q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2],
+  // o_done, mma_done
+  static constexpr int NUM_BARS = 1 + 4 * NS + 2 + 2 + 1 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_LIST = OFF_MISC + 64;
   static constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 64, false);
@@ -87,9 +90,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
   uint64_t *q_full = bars;
   uint64_t *k_full = bars + 1;
-  uint64_t *v_full = k_full + C::NS;
-  uint64_t *kv_empty = v_full + C::NS;
-  uint64_t *s_full = kv_empty + C::NS;
+  uint64_t *k_empty = k_full + C::NS;
+  uint64_t *v_full = k_empty + C::NS;
+  uint64_t *v_empty = v_full + C::NS;
+  uint64_t *s_full = v_empty + C::NS;
   uint64_t *p_full = s_full + 2;
   uint64_t *o_done = p_full + 2;
   uint64_t *mma_done = o_done + 1;
@@ -104,8 +108,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc::mbar_init(q_full, 1);
     for (int s = 0; s < C::NS; ++s) {
       tc::mbar_init(k_full + s, 1);
+      tc::mbar_init(k_empty + s, 1);
       tc::mbar_init(v_full + s, 1);
-      tc::mbar_init(kv_empty + s, 1);
+      tc::mbar_init(v_empty + s, 1);
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(s_full + b, 1);
@@ -188,31 +193,39 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tc::tma_load_2d(sbase + C::OFF_Q + kb * C::Q_REGION + 8192, &tm_q, q_full, kb * 64,
                           rowA + 64);
       }
-      int issued = 0;
-      for (int j = 0; j < n; ++j) {
+      // K runs one tile ahead of V: K_{j+1} is needed by S_{j+1}, which the
+      // MMA warp issues before P.V_j.
+      auto load_tile = [&](const CUtensorMap *map, uint64_t *full, uint64_t *empty, int off,
+                           int j) -> bool {
         const int s = j % C::NS, u = j / C::NS;
-        if (u > 0 && !tc::mbar_wait(kv_empty + s, (u - 1) & 1, abort_flag, WAIT_LIMIT)) break;
+        if (u > 0 && !tc::mbar_wait(empty + s, (u - 1) & 1, abort_flag, WAIT_LIMIT)) return false;
         const int kt = (int)(U[j] & KT_MASK);
         const int row = (int)(((long long)bh * nt + kt) * 64);
-        tc::mbar_expect_tx(k_full + s, C::TILE_BYTES);
+        tc::mbar_expect_tx(full + s, C::TILE_BYTES);
 #pragma unroll
         for (int kb = 0; kb < C::KB; ++kb)
-          tc::tma_load_2d(sbase + C::OFF_K + s * C::TILE_BYTES + kb * 8192, &tm_k, k_full + s,
-                          kb * 64, row);
-        tc::mbar_expect_tx(v_full + s, C::TILE_BYTES);
-#pragma unroll
-        for (int kb = 0; kb < C::KB; ++kb)
-          tc::tma_load_2d(sbase + C::OFF_V + s * C::TILE_BYTES + kb * 8192, &tm_v, v_full + s,
-                          kb * 64, row);
-        issued = j + 1;
+          tc::tma_load_2d(sbase + off + s * C::TILE_BYTES + kb * 8192, map, full + s, kb * 64, row);
+        return true;
+      };
+      int issued_k = 0, issued_v = 0;
+      bool ok = load_tile(&tm_k, k_full, k_empty, C::OFF_K, 0);
+      if (ok) issued_k = 1;
+      for (int j = 0; ok && j < n; ++j) {
+        if (j + 1 < n) {
+          ok = load_tile(&tm_k, k_full, k_empty, C::OFF_K, j + 1);
+          if (!ok) break;
+          issued_k = j + 2;
+        }
+        ok = load_tile(&tm_v, v_full, v_empty, C::OFF_V, j);
+        if (ok) issued_v = j + 1;
       }
       // Copies still in flight must land before the CTA can exit.
       if (*abort_flag) {
         tc::mbar_wait(q_full, 0, nullptr, DRAIN_LIMIT);
-        for (int j = (issued > C::NS ? issued - C::NS : 0); j < issued; ++j) {
+        for (int j = (issued_k > C::NS ? issued_k - C::NS : 0); j < issued_k; ++j)
           tc::mbar_wait(k_full + j % C::NS, (j / C::NS) & 1, nullptr, DRAIN_LIMIT);
+        for (int j = (issued_v > C::NS ? issued_v - C::NS : 0); j < issued_v; ++j)
           tc::mbar_wait(v_full + j % C::NS, (j / C::NS) & 1, nullptr, DRAIN_LIMIT);
-        }
       }
     }
     __syncwarp();
@@ -235,6 +248,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tc::mma_ss(d_tmem, a, b, C::IDESC_S, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(s_full + (j & 1));
+        tc::mma_commit(k_empty + s);
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
@@ -250,7 +264,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tc::mma_ts(tmem + O_COL, p_tmem + (uint32_t)(kk * 8), b, C::IDESC_O,
                      (j > 0 || kk > 0) ? 1u : 0u);
         }
-        tc::mma_commit(kv_empty + s);
+        tc::mma_commit(v_empty + s);
         tc::mma_commit(o_done);
         return true;
       };
