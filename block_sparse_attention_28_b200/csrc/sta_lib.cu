@@ -54,8 +54,10 @@ MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
   return w;
 }
 
-size_t select_smem(int d, int nt, bool use_scores) {
-  return use_scores ? (size_t)(SEL_QB * d + SEL_QB * nt) * sizeof(float) : 0;
+size_t select_smem(int d, const Geo &g, bool use_scores) {
+  const size_t scores = use_scores ? (size_t)(SEL_QB * d + SEL_QB * g.Nt + (SEL_THREADS / 32) * 256) : 0;
+  const size_t tables = (size_t)((g.Nt + g.T + 3) & ~3) + 4 * STA_MAX_GROUPS;
+  return (scores + tables) * sizeof(float);
 }
 
 constexpr size_t MAX_DYN_SMEM = 227 * 1024;
@@ -121,7 +123,7 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
                                            static_cast<const uint4 *>(k_tiled), qbar, kbar, R, g);
     STA_CUDA_TRY(cudaGetLastError());
   }
-  const size_t smem = select_smem(D, g.Nt, use_scores);
+  const size_t smem = select_smem(D, g, use_scores);
   if (smem > 48 * 1024)
     STA_CUDA_TRY(cudaFuncSetAttribute(score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem));
@@ -217,7 +219,9 @@ sta_status sta_build_mask(const void *q_tiled, const void *k_tiled, int32_t B, i
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       ws_bytes < mask_ws_layout(B, heads, d, geo).total)
     return STA_ERR_WORKSPACE;
-  if (select_smem(d, geo.Nt, p->use_scores != 0) > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
+  if (select_smem(d, geo, p->use_scores != 0) > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
+  // window tables pack (t, tile row, tile column) into 12 + 10 + 10 bits
+  if (p->windows != nullptr && (geo.T >= 4096 || geo.NH >= 1024 || geo.NW >= 1024)) return STA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   return (d == 128) ? launch_build<128>(q_tiled, k_tiled, B, heads, geo, p, row_ptr, col_idx, nnz_dev,

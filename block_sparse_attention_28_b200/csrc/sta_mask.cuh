@@ -103,19 +103,63 @@ __device__ __forceinline__ unsigned int mass_at_least(const float *row, int nt, 
   return warp_sum_u32(s);
 }
 
-// Largest bit pattern v with f(v) >= target, f non-increasing (mass or count
-// of entries >= v). target must be >= 1 and f(0) >= target.
-__device__ unsigned int search_level(const float *row, int nt, unsigned int target, bool count_only,
-                                     int lane) {
-  unsigned int lo = 0u, hi = 0x3F800001u;  // f(lo) >= target > f(hi)
-  while (hi - lo > 1u) {
-    const unsigned int mid = lo + ((hi - lo) >> 1);
-    if (mass_at_least(row, nt, mid, count_only, lane) >= target)
-      lo = mid;
-    else
-      hi = mid;
+// Radix select over the P bit patterns (P >= 0, so the bits order like the
+// values). Finds the largest pattern v with f(v) >= target, where
+// f(v) = sum over entries with P >= v of (count_only ? 1 : mass), one digit at
+// a time from the most significant (bits 30-23, 22-15, 14-7, 6-0), with a
+// per-warp histogram of 256 bins in shared memory. Also returns f restricted
+// to entries strictly above v. target must be >= 1 and f(0) >= target.
+// All sums are integers, so the result does not depend on summation order.
+__device__ void radix_level(const float *row, int nt, unsigned int target, bool count_only, int lane,
+                            unsigned int *hist, unsigned int &v_out, unsigned int &above_out) {
+  unsigned int prefix = 0u, pmask = 0u, above = 0u;
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = pass == 0 ? 23 : (pass == 1 ? 15 : (pass == 2 ? 7 : 0));
+    const unsigned int dmask = pass == 3 ? 0x7Fu : 0xFFu;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hist[i * 32 + lane] = 0u;
+    __syncwarp();
+    for (int j = lane; j < nt; j += 32) {
+      const unsigned int b = __float_as_uint(row[j]);
+      if ((b & pmask) == prefix)
+        atomicAdd(hist + ((b >> shift) & dmask), count_only ? 1u : mass_of(__uint_as_float(b)));
+    }
+    __syncwarp();
+    // lane owns digits [8*lane, 8*lane + 8)
+    unsigned int hb[8], own = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      hb[k] = hist[8 * lane + k];
+      own += hb[k];
+    }
+    unsigned int suffix = own;  // digits owned by this lane and all higher lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned int y = __shfl_down_sync(0xffffffffu, suffix, o);
+      if (lane + o < 32) suffix += y;
+    }
+    unsigned int run = above + (suffix - own);
+    int found = -1;
+    unsigned int above_found = 0u;
+#pragma unroll
+    for (int k = 7; k >= 0; --k) {
+      if (found < 0 && run + hb[k] >= target) {
+        found = 8 * lane + k;
+        above_found = run;
+      }
+      run += hb[k];
+    }
+    const unsigned int hit = __ballot_sync(0xffffffffu, found >= 0);
+    const int src = 31 - __clz((int)hit);
+    const int digit = __shfl_sync(0xffffffffu, found, src);
+    above = __shfl_sync(0xffffffffu, above_found, src);
+    prefix |= (unsigned int)digit << shift;
+    pmask |= dmask << shift;
+    __syncwarp();
   }
-  return lo;
+  v_out = prefix;
+  above_out = above;
 }
 
 // One CTA per (b*heads + h, block of SEL_QB query tiles).
@@ -134,8 +178,33 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
   const int q0 = blockIdx.x * SEL_QB;
   const int nq = min(SEL_QB, nt - q0);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tpf = g.NH * g.NW;
+  // shared memory: [qs, S, histograms] if use_scores, then the window tables
   float *qs = sm;
-  float *S = sm + SEL_QB * D;
+  float *S = qs + (use_scores ? SEL_QB * D : 0);
+  unsigned int *hist = reinterpret_cast<unsigned int *>(S + (use_scores ? SEL_QB * nt : 0));
+  unsigned int *kcoord = hist + (use_scores ? (SEL_THREADS / 32) * 256 : 0);
+  int *gtab = reinterpret_cast<int *>(kcoord + nt);
+  int *wtab = gtab + ((nt + g.T + 3) & ~3) - nt;  // 16-byte aligned, 4 ints per group
+  unsigned int *whist = hist + warp * 256;
+
+  // Window tables, once per CTA: packed (t, tile row, tile column) of every
+  // key tile, the temporal group of every |dt|, and this head's extents.
+  if (windows != nullptr) {
+    for (int kt = tid; kt < nt; kt += SEL_THREADS) {
+      const int t = kt / tpf, rem = kt - t * tpf;
+      const int y = rem / g.NW, x = rem - y * g.NW;
+      kcoord[kt] = ((unsigned int)t << 20) | ((unsigned int)y << 10) | (unsigned int)x;
+    }
+    for (int dt = tid; dt < g.T; dt += SEL_THREADS) {
+      int grp = -1;
+      for (int gg = 0; gg < G; ++gg)
+        if (dt >= glo.v[gg]) grp = gg;
+      gtab[dt] = grp;
+    }
+    for (int i = tid; i < G * 4; i += SEL_THREADS) wtab[i] = windows[(long long)h * G * 4 + i];
+  }
+  if (!use_scores) __syncthreads();
 
   if (use_scores) {
     // Phase 1: S[i][kt] = scale * qbar[q0+i] . kbar[kt], sequential fp32 FMA over d.
@@ -167,7 +236,6 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
     __syncthreads();
   }
 
-  const int tpf = g.NH * g.NW;
   for (int i = warp; i < nq; i += SEL_THREADS / 32) {
     const int qt = q0 + i;
     const long long row = (long long)bh * nt + qt;
@@ -207,8 +275,8 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
         const double thr_d = ceil((double)top_p * (double)W);
         const unsigned int thr = (unsigned int)thr_d;
         if (thr > 0u) {
-          const unsigned int v = search_level(Sr, nt, thr, false, lane);
-          const unsigned int above = mass_at_least(Sr, nt, v + 1u, false, lane);
+          unsigned int v, above;
+          radix_level(Sr, nt, thr, false, lane, whist, v, above);
           const unsigned int wv = mass_of(__uint_as_float(v));
           const unsigned int need = (thr - above + wv - 1u) / wv;  // tied entries at level v
           const unsigned int cnt_above = mass_at_least(Sr, nt, v + 1u, true, lane);
@@ -218,8 +286,8 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
         }
       }
       if ((long long)kk > m_p) {
-        const unsigned int u = search_level(Sr, nt, (unsigned int)kk, true, lane);
-        const unsigned int cnt_above = mass_at_least(Sr, nt, u + 1u, true, lane);
+        unsigned int u, cnt_above;
+        radix_level(Sr, nt, (unsigned int)kk, true, lane, whist, u, cnt_above);
         v_f = u;
         c_f = (unsigned int)kk - cnt_above;
       } else if (m_p > 0) {
@@ -230,7 +298,6 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
     // Phase 4: membership bits = selected OR window, one 32-bit word per lane step.
     const int tq = qt / tpf, remq = qt - tq * tpf;
     const int yq = remq / g.NW, xq = remq - yq * g.NW;
-    const int *wh = windows ? windows + (long long)h * G * 4 : nullptr;
     unsigned int ties_seen = 0u;
     int total = 0;
     unsigned int *brow = bits + row * wpr;
@@ -238,16 +305,14 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
       const int kt = w0 * 32 + lane;
       bool keep = false;
       if (kt < nt) {
-        if (wh) {
-          const int tk = kt / tpf, remk = kt - tk * tpf;
-          const int yk = remk / g.NW, xk = remk - yk * g.NW;
-          const int dt = abs(tq - tk), dy = abs(yq - yk), dx = abs(xq - xk);
-          int grp = -1;
-          for (int gg = 0; gg < G; ++gg)
-            if (dt >= glo.v[gg]) grp = gg;
+        if (windows != nullptr) {
+          const unsigned int kc = kcoord[kt];
+          const int dt = abs(tq - (int)(kc >> 20));
+          const int dy = abs(yq - (int)((kc >> 10) & 1023u)), dx = abs(xq - (int)(kc & 1023u));
+          const int grp = gtab[dt];
           if (grp >= 0) {
-            const int *w4 = wh + grp * 4;
-            keep = (dy <= w4[0] && dx <= w4[1]) || (dy <= w4[2] && dx <= w4[3]);
+            const int4 w4 = reinterpret_cast<const int4 *>(wtab)[grp];
+            keep = (dy <= w4.x && dx <= w4.y) || (dy <= w4.z && dx <= w4.w);
           }
         }
       }
