@@ -187,6 +187,28 @@ class Layer:
         if ev is not None:
             ev[4].record()
 
+    def dense_run(self, reps=2):
+        """sta_attn_fwd on the same layer with every key tile listed (the dense
+        mask): CUDA-event time per launch and TFLOP/s over all Nt^2 pairs."""
+        R = self.B * self.Hh * self.nt
+        dev = self.qt.device
+        rp = (torch.arange(R + 1, device=dev, dtype=torch.int64) * self.nt).to(torch.int32)
+        ci = torch.arange(self.nt, device=dev, dtype=torch.int32).repeat(R)
+        self.sta.sta_attn_fwd(self.qt, self.kt, self.vt, self.ot, None, rp, ci, self.B, self.Hh, self.d, self.g)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            self.sta.sta_attn_fwd(self.qt, self.kt, self.vt, self.ot, None, rp, ci, self.B, self.Hh, self.d,
+                                  self.g)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        pairs = R * self.nt
+        del rp, ci
+        return {"ms": ms, "pairs": pairs, "tflops": pairs * flops_per_pair(self.d) / (ms * 1e-3) / 1e12,
+                "density": 1.0}
+
     def kept_pairs(self):
         return int(self.bufs.nnz.item())
 
@@ -296,6 +318,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense-mask run of the same kernel")
     ap.add_argument("--config-index", type=int, default=CFG_INDEX,
                     help="workload (profiling of smaller layers); the headline is the 720p layer")
     ap.add_argument("--density-index", type=int, default=0)
@@ -392,6 +415,11 @@ def main():
         e2e = {"value": world * flops / (float(t2.item()) * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": float(t2.item())}
 
+    # the same kernel with every key tile listed (dense-mask run), outside the timed region
+    dense = None
+    if rank == 0 and not args.no_dense:
+        dense = layer.dense_run(reps=2)
+
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     eff, union_tiles = layer.pair_union_stats() if rank == 0 else (None, None)
@@ -420,6 +448,7 @@ def main():
             "attn_tflops": attn_tflops,
             "attn_frac_of_peak": attn_tflops / peak,
             "pairing_efficiency": eff,
+            "dense_mask_run": dense,
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": attn_tflops / peak, "traffic": load_traffic(),
                          "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
