@@ -339,3 +339,88 @@ def test_attn_bad_column_index_is_reported(sta, gp):
     assert sta.sta_get_device_error() == sta.STA_ERR_BAD_MASK
     assert sta.sta_get_device_error() == sta.STA_OK  # the word was cleared
     assert torch.isfinite(o.float()).all()
+
+
+# ------------------------------------------------- full-size workload coverage
+@pytest.mark.parametrize("which", [0, 1, 2, 3])
+def test_build_mask_window_only_full_129_frames(sta, gp, which):
+    """129-frame layer (24 heads, 1,980 tiles per head), four temporal groups,
+    each density target: the whole CSR against the oracle's window mask."""
+    cfg = CONFIGS[3]
+    g = sta.grid(cfg.T, cfg.H, cfg.W)
+    win = window_params(cfg, window_scale(3, which))
+    params = sta.mask_params(0.0, 0, False, 0.0, cfg.group_lo, torch.from_numpy(win).cuda())
+    bufs = gp.build(None, None, 1, cfg.heads, cfg.d, g, params, with_mask=False, with_probs=False)
+    rp, ci, nnz = gp.csr_np(bufs)
+    mask = O.window_mask(win, cfg.group_lo, cfg.T, cfg.H, cfg.W)[None]
+    rp_o, ci_o = O.mask_to_csr(mask)
+    assert np.array_equal(rp, rp_o) and np.array_equal(ci, ci_o)
+    assert abs(nnz / mask.size - cfg.window_density[which]) < 0.01
+
+
+def test_attn_full_129_frames_sampled_rows(sta, gp):
+    cfg = CONFIGS[3]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    q, k, v = make_qkv(cfg, device="cuda")
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    del q, k, v
+    win = torch.from_numpy(window_params(cfg, window_scale(3, 2))).cuda()
+    bufs = gp.build(None, None, B, Hh, d, g, sta.mask_params(0.0, 0, False, 0.0, cfg.group_lo, win),
+                    with_mask=False, with_probs=False)
+    nt = sta.sta_num_tiles(g)
+    rng = np.random.default_rng(5)
+    rows = sorted(rng.choice(B * Hh * nt, 24, replace=False).tolist())
+    _attn_check(sta, gp, qt, kt, vt, bufs.row_ptr, bufs.col_idx, B, Hh, d, T, H, W, rows=rows)
+
+
+def test_attn_full_480p_sampled_rows(sta, gp):
+    cfg = CONFIGS[1]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    q, k, v = make_qkv(cfg, device="cuda")
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    del q, k, v
+    win = torch.from_numpy(window_params(cfg, window_scale(1, 0))).cuda()
+    bufs = gp.build(None, None, B, Hh, d, g, sta.mask_params(0.0, 0, False, 0.0, cfg.group_lo, win),
+                    with_mask=False, with_probs=False)
+    nt = sta.sta_num_tiles(g)
+    rng = np.random.default_rng(6)
+    rows = sorted(rng.choice(B * Hh * nt, 32, replace=False).tolist())
+    _attn_check(sta, gp, qt, kt, vt, bufs.row_ptr, bufs.col_idx, B, Hh, d, T, H, W, rows=rows)
+
+
+def test_attn_reuse_all_densities_full(sta, gp):
+    """Reuse layer, all 40 heads: masks of every density built once from step-0
+    inputs (fixed count per row, selection exact against the oracle on the
+    GPU's P for sampled rows), attention after 0 and 10 perturbed steps; the
+    100% run is the dense-mask reference of the same kernel."""
+    from workloads import perturb_step
+
+    cfg = CONFIGS[4]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = make_qkv(cfg, device="cuda")
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    gen = torch.Generator(device="cuda").manual_seed(404)
+    mq, mk = q.float(), k.float()
+    for _ in range(cfg.reuse_steps):
+        mq, qb = perturb_step(mq, gen)
+        mk, kb = perturb_step(mk, gen)
+    qt10, kt10 = gp.reorder(qb, B, Hh, d, g), gp.reorder(kb, B, Hh, d, g)
+    del q, k, mq, mk, qb, kb
+    rng = np.random.default_rng(7)
+    for rho in cfg.fixed_densities:
+        kmin = int(round(rho * nt))
+        bufs = gp.build(qt, kt, B, Hh, d, g, sta.mask_params(0.0, kmin, True), with_mask=False, with_probs=True)
+        rp, ci, nnz = gp.csr_np(bufs)
+        assert nnz == B * Hh * nt * kmin
+        rows = sorted(rng.choice(B * Hh * nt, 6, replace=False).tolist())
+        for r in rows:
+            bh, qtile = divmod(r, nt)
+            p_row = bufs.block_probs.view(-1, nt)[r].cpu().numpy()
+            assert np.array_equal(ci[rp[r]:rp[r + 1]], np.nonzero(O.select_row(p_row, 0.0, kmin))[0])
+        bufs.block_probs = None
+        _attn_check(sta, gp, qt, kt, vt, bufs.row_ptr, bufs.col_idx, B, Hh, d, T, H, W, rows=rows)
+        _attn_check(sta, gp, qt10, kt10, vt, bufs.row_ptr, bufs.col_idx, B, Hh, d, T, H, W, rows=rows)
