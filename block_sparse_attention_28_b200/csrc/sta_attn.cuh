@@ -302,14 +302,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
         tc::tmem_st32(sS, pk);
       } else {
-        uint32_t r0[32], r1[32];
-        tc::tmem_ld32(sS, r0);
-        tc::tmem_ld32(sS + 32, r1);
         float s[64];
+        {
+          uint32_t rr[64];
+          tc::tmem_ld64(sS, rr);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          s[c] = __uint_as_float(r0[c]);
-          s[32 + c] = __uint_as_float(r1[c]);
+          for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(rr[c]);
         }
         // keys of partial tiles beyond the grid edge
         const int kt = (int)(e & KT_MASK);
@@ -321,26 +319,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int c = 0; c < 64; ++c)
             if ((c >> 3) >= vy || (c & 7) >= vx) s[c] = -INFINITY;
         }
-        // tree reduction: max is exact in any order, and the tree is 6 deep
-        float t32[32];
+        // row max: a tree of three-input maxima (max is exact in any order)
+        float t22[22];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) t32[c] = fmaxf(s[c], s[c + 32]);
+        for (int c = 0; c < 21; ++c) t22[c] = tc::fmax3(s[3 * c], s[3 * c + 1], s[3 * c + 2]);
+        t22[21] = s[63];
+        float t8[8];
 #pragma unroll
-        for (int w = 16; w > 0; w >>= 1) {
-#pragma unroll
-          for (int c = 0; c < w; ++c) t32[c] = fmaxf(t32[c], t32[c + w]);
-        }
-        const float mx = t32[0];
+        for (int c = 0; c < 7; ++c) t8[c] = tc::fmax3(t22[3 * c], t22[3 * c + 1], t22[3 * c + 2]);
+        t8[7] = t22[21];
+        const float mx = tc::fmax3(tc::fmax3(t8[0], t8[1], t8[2]), tc::fmax3(t8[3], t8[4], t8[5]),
+                                   fmaxf(t8[6], t8[7]));
         const float m_new = fmaxf(m, mx * scale_log2);
         const bool rescale = m_new > m + RESCALE_LOG2;
         const float m_use = rescale ? m_new : m;
         const float mref = (m_use == -INFINITY) ? 0.0f : m_use;
         const float alpha = rescale ? tc::ex2(m - m_new) : 1.0f;
-        float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        // x = s * scale_log2 - mref two lanes at a time; p = 2^x; pairs summed
+        // in four packed accumulators
+        const uint64_t scale2 = tc::f2_pack(scale_log2, scale_log2);
+        const uint64_t negm2 = tc::f2_pack(-mref, -mref);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const float x0 = fmaf(s[2 * c], scale_log2, -mref);
-          const float x1 = fmaf(s[2 * c + 1], scale_log2, -mref);
+          float x0, x1;
+          tc::f2_unpack(tc::f2_fma(tc::f2_pack(s[2 * c], s[2 * c + 1]), scale2, negm2), x0, x1);
           float p0, p1;
           if (STA_EXP2_POLY_EVERY > 0 && (c % (STA_EXP2_POLY_EVERY > 0 ? STA_EXP2_POLY_EVERY : 1)) ==
                                              STA_EXP2_POLY_EVERY - 1) {
@@ -350,10 +353,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             p0 = tc::ex2(x0);
             p1 = tc::ex2(x1);
           }
-          part[c & 3] += p0 + p1;
+          acc[c & 3] = tc::f2_add(acc[c & 3], tc::f2_pack(p0, p1));
           pk[c] = tc::pack_bf16(p0, p1);
         }
-        const float sum = (part[0] + part[1]) + (part[2] + part[3]);
+        float sum;
+        {
+          float a0, a1;
+          tc::f2_unpack(tc::f2_add(tc::f2_add(acc[0], acc[1]), tc::f2_add(acc[2], acc[3])), a0, a1);
+          sum = a0 + a1;
+        }
         tc::tmem_st32(sS, pk);
         l = l * alpha + sum;
         const bool need_o = rescale && (m != -INFINITY);
