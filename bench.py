@@ -212,6 +212,19 @@ class Layer:
     def kept_pairs(self):
         return int(self.bufs.nnz.item())
 
+    def query_pairs(self):
+        """The two query tiles of each 128-row CTA, as the attention kernel pairs
+        them: the same spatial tile in frames 2u and 2u+1, and right-hand
+        neighbours within the last frame when the frame count is odd."""
+        c = self.cfg
+        nh, nw = -(-c.H // 8), -(-c.W // 8)
+        tpf = nh * nw
+        pairs = [(2 * u * tpf + r, (2 * u + 1) * tpf + r) for u in range(c.T // 2) for r in range(tpf)]
+        if c.T % 2:
+            base = (c.T - 1) * tpf
+            pairs += [(base + i, base + i + 1 if i + 1 < tpf else None) for i in range(0, tpf, 2)]
+        return pairs
+
     def pair_union_stats(self):
         """Pairing efficiency (|A|+|B|) / (2 |A u B|) of the 128-row CTAs."""
         rp = self.bufs.row_ptr.cpu().numpy()
@@ -219,10 +232,10 @@ class Layer:
         nt = self.nt
         tot_ab, tot_u = 0, 0
         for bh in range(self.B * self.Hh):
-            for p in range(0, nt, 2):
-                ra = bh * nt + p
+            for qa, qb in self.query_pairs():
+                ra = bh * nt + qa
                 a = ci[rp[ra]:rp[ra + 1]]
-                b = ci[rp[ra + 1]:rp[ra + 2]] if p + 1 < nt else np.zeros(0, np.int32)
+                b = ci[rp[bh * nt + qb]:rp[bh * nt + qb + 1]] if qb is not None else np.zeros(0, np.int32)
                 tot_ab += a.size + b.size
                 tot_u += np.union1d(a, b).size
         return tot_ab / (2.0 * tot_u) if tot_u else 1.0, tot_u

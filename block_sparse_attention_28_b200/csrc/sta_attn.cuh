@@ -1,9 +1,9 @@
 // Block-sparse attention forward over listed key tiles (Compact Attention
 // Fig. 3: precomputed masks loaded into a block-sparse attention kernel).
 //
-// One CTA computes 128 query rows: the query tiles 2p and 2p+1 of one head
-// (a 128-row tcgen05 tile; a 64-token tile alone would leave half of the MMA
-// rows idle). The two CSR rows are merged into one ascending key-tile list
+// One CTA computes 128 query rows: two query tiles of one head, the same
+// spatial tile in two consecutive frames (a 128-row tcgen05 tile; a 64-token
+// tile alone would leave half of the MMA rows idle). The two CSR rows are merged into one ascending key-tile list
 // with a per-half membership flag; a half whose list lacks the key tile gets
 // P = 0 for that tile, so the work is |A u B| key tiles of 128 x 64.
 //
@@ -44,19 +44,32 @@ constexpr int MIN_BLOCKS_PER_SM = 2;             // two CTAs share an SM: one's 
 #define STA_EXP2_POLY_EVERY 0                    // every k-th column pair uses ex2_poly
 #endif
 
+#ifndef STA_ATTN_NSK
+#define STA_ATTN_NSK 2                           // K ring stages at d = 128
+#endif
+#ifndef STA_ATTN_NSV
+#define STA_ATTN_NSV 2                           // V ring stages at d = 128
+#endif
+#ifndef STA_ATTN_KLEAD
+#define STA_ATTN_KLEAD 1                         // K tiles loaded ahead of the V tile
+#endif
+
 template <int D>
 struct Cfg {
   static constexpr int KB = D / 64;              // 128-byte swizzle atoms along d
-  static constexpr int NS = (D == 128) ? 2 : 4;  // K/V ring stages (2 CTAs per SM fit)
+  // ring stages: two CTAs per SM fit in shared memory
+  static constexpr int NSK = (D == 128) ? STA_ATTN_NSK : 4;
+  static constexpr int NSV = (D == 128) ? STA_ATTN_NSV : 4;
+  static constexpr int KLEAD = (D == 128) ? STA_ATTN_KLEAD : 1;
   static constexpr int TILE_BYTES = 64 * D * 2;  // one 64-token tile of Q, K or V
   static constexpr int Q_REGION = 128 * 128;     // 128 rows x 128 B per d-atom
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + KB * Q_REGION;
-  static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NS * TILE_BYTES;
-  // q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2],
+  static constexpr int OFF_V = OFF_K + NSK * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NSV * TILE_BYTES;
+  // q_full, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full[2], p_full[2],
   // o_done, mma_done
-  static constexpr int NUM_BARS = 1 + 4 * NS + 2 + 2 + 1 + 1;
+  static constexpr int NUM_BARS = 1 + 2 * NSK + 2 * NSV + 2 + 2 + 1 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_LIST = OFF_MISC + 64;
   static constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 64, false);
@@ -83,17 +96,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nt = g.Nt;
   const int bh = blockIdx.y;
-  const int qtA = 2 * blockIdx.x, qtB = qtA + 1;
+  // Query-tile pairing: the same spatial tile in frames 2u and 2u+1 (their
+  // lists overlap most: windows and pooled scores change little between
+  // neighbouring frames); with an odd frame count the last frame's tiles are
+  // paired with their right-hand neighbour.
+  const int tpf_q = g.NH * g.NW;
+  const int pairs_t = (g.T / 2) * tpf_q;
+  int qtA, qtB;
+  if ((int)blockIdx.x < pairs_t) {
+    const int u = (int)blockIdx.x / tpf_q, rem = (int)blockIdx.x - u * tpf_q;
+    qtA = 2 * u * tpf_q + rem;
+    qtB = qtA + tpf_q;
+  } else {
+    qtA = (g.T - 1) * tpf_q + 2 * ((int)blockIdx.x - pairs_t);
+    qtB = qtA + 1;
+  }
   const bool hasB = qtB < nt;
   const int wpr = (nt + 31) / 32;
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
   uint64_t *q_full = bars;
   uint64_t *k_full = bars + 1;
-  uint64_t *k_empty = k_full + C::NS;
-  uint64_t *v_full = k_empty + C::NS;
-  uint64_t *v_empty = v_full + C::NS;
-  uint64_t *s_full = v_empty + C::NS;
+  uint64_t *k_empty = k_full + C::NSK;
+  uint64_t *v_full = k_empty + C::NSK;
+  uint64_t *v_empty = v_full + C::NSV;
+  uint64_t *s_full = v_empty + C::NSV;
   uint64_t *p_full = s_full + 2;
   uint64_t *o_done = p_full + 2;
   uint64_t *mma_done = o_done + 1;
@@ -106,9 +133,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // ---- set-up: barriers, bitmaps, TMEM
   if (tid == 0) {
     tc::mbar_init(q_full, 1);
-    for (int s = 0; s < C::NS; ++s) {
+    for (int s = 0; s < C::NSK; ++s) {
       tc::mbar_init(k_full + s, 1);
       tc::mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < C::NSV; ++s) {
       tc::mbar_init(v_full + s, 1);
       tc::mbar_init(v_empty + s, 1);
     }
@@ -140,7 +169,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         record_error(DEV_ERR_BAD_MASK);
     }
     if (hasB) {
-      const int b0 = row_ptr[rA + 1], b1 = row_ptr[rA + 2];
+      const long long rB = (long long)bh * nt + qtB;
+      const int b0 = row_ptr[rB], b1 = row_ptr[rB + 1];
       for (int i = b0 + tid; i < b1; i += NUM_THREADS) {
         const int c = col_idx[i];
         if ((unsigned)c < (unsigned)nt)
@@ -185,19 +215,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ------------------------------------------------------ TMA producer
     if (lane == 0 && n > 0) {
       const int rowA = (int)(((long long)bh * nt + qtA) * 64);
+      const int rowB = (int)(((long long)bh * nt + qtB) * 64);
       tc::mbar_expect_tx(q_full, (hasB ? 2 : 1) * C::TILE_BYTES);
 #pragma unroll
       for (int kb = 0; kb < C::KB; ++kb) {
         tc::tma_load_2d(sbase + C::OFF_Q + kb * C::Q_REGION, &tm_q, q_full, kb * 64, rowA);
         if (hasB)
           tc::tma_load_2d(sbase + C::OFF_Q + kb * C::Q_REGION + 8192, &tm_q, q_full, kb * 64,
-                          rowA + 64);
+                          rowB);
       }
-      // K runs one tile ahead of V: K_{j+1} is needed by S_{j+1}, which the
+      // K runs KLEAD tiles ahead of V: K_{j+1} is needed by S_{j+1}, which the
       // MMA warp issues before P.V_j.
-      auto load_tile = [&](const CUtensorMap *map, uint64_t *full, uint64_t *empty, int off,
+      auto load_tile = [&](const CUtensorMap *map, uint64_t *full, uint64_t *empty, int off, int ns,
                            int j) -> bool {
-        const int s = j % C::NS, u = j / C::NS;
+        const int s = j % ns, u = j / ns;
         if (u > 0 && !tc::mbar_wait(empty + s, (u - 1) & 1, abort_flag, WAIT_LIMIT)) return false;
         const int kt = (int)(U[j] & KT_MASK);
         const int row = (int)(((long long)bh * nt + kt) * 64);
@@ -208,24 +239,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         return true;
       };
       int issued_k = 0, issued_v = 0;
-      bool ok = load_tile(&tm_k, k_full, k_empty, C::OFF_K, 0);
-      if (ok) issued_k = 1;
+      bool ok = true;
+      for (int j = 0; ok && j < C::KLEAD && j < n; ++j) {
+        ok = load_tile(&tm_k, k_full, k_empty, C::OFF_K, C::NSK, j);
+        if (ok) issued_k = j + 1;
+      }
       for (int j = 0; ok && j < n; ++j) {
-        if (j + 1 < n) {
-          ok = load_tile(&tm_k, k_full, k_empty, C::OFF_K, j + 1);
+        if (j + C::KLEAD < n) {
+          ok = load_tile(&tm_k, k_full, k_empty, C::OFF_K, C::NSK, j + C::KLEAD);
           if (!ok) break;
-          issued_k = j + 2;
+          issued_k = j + C::KLEAD + 1;
         }
-        ok = load_tile(&tm_v, v_full, v_empty, C::OFF_V, j);
+        ok = load_tile(&tm_v, v_full, v_empty, C::OFF_V, C::NSV, j);
         if (ok) issued_v = j + 1;
       }
       // Copies still in flight must land before the CTA can exit.
       if (*abort_flag) {
         tc::mbar_wait(q_full, 0, nullptr, DRAIN_LIMIT);
-        for (int j = (issued_k > C::NS ? issued_k - C::NS : 0); j < issued_k; ++j)
-          tc::mbar_wait(k_full + j % C::NS, (j / C::NS) & 1, nullptr, DRAIN_LIMIT);
-        for (int j = (issued_v > C::NS ? issued_v - C::NS : 0); j < issued_v; ++j)
-          tc::mbar_wait(v_full + j % C::NS, (j / C::NS) & 1, nullptr, DRAIN_LIMIT);
+        for (int j = (issued_k > C::NSK ? issued_k - C::NSK : 0); j < issued_k; ++j)
+          tc::mbar_wait(k_full + j % C::NSK, (j / C::NSK) & 1, nullptr, DRAIN_LIMIT);
+        for (int j = (issued_v > C::NSV ? issued_v - C::NSV : 0); j < issued_v; ++j)
+          tc::mbar_wait(v_full + j % C::NSV, (j / C::NSV) & 1, nullptr, DRAIN_LIMIT);
       }
     }
     __syncwarp();
@@ -235,8 +269,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       bool ok = tc::mbar_wait(q_full, 0, abort_flag, WAIT_LIMIT);
       tc::fence_after();
       auto issue_s = [&](int j) -> bool {
-        const int s = j % C::NS;
-        if (!tc::mbar_wait(k_full + s, (j / C::NS) & 1, abort_flag, WAIT_LIMIT)) return false;
+        const int s = j % C::NSK;
+        if (!tc::mbar_wait(k_full + s, (j / C::NSK) & 1, abort_flag, WAIT_LIMIT)) return false;
         tc::fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)((j & 1) * 64);
 #pragma unroll
@@ -252,9 +286,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
-        const int s = j % C::NS;
+        const int s = j % C::NSV;
         if (!tc::mbar_wait(p_full + (j & 1), (j >> 1) & 1, abort_flag, WAIT_LIMIT)) return false;
-        if (!tc::mbar_wait(v_full + s, (j / C::NS) & 1, abort_flag, WAIT_LIMIT)) return false;
+        if (!tc::mbar_wait(v_full + s, (j / C::NSV) & 1, abort_flag, WAIT_LIMIT)) return false;
         tc::fence_after();
         const uint32_t p_tmem = tmem + (uint32_t)((j & 1) * 64);
 #pragma unroll
