@@ -42,6 +42,30 @@ def flops_per_pair(d):
     return 4.0 * 64 * 64 * d
 
 
+def max_over_ranks(x, device, world):
+    """Largest value of x over all ranks (the job is as slow as its slowest rank)."""
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, device, world):
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def whole_job_tflops(total_flops_per_step, steps, elapsed_ms):
+    """Whole-job throughput: kept-pair flops of all ranks over the slowest rank's time."""
+    return steps * total_flops_per_step / (elapsed_ms * 1e-3) / 1e12
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -388,17 +412,13 @@ def main():
     reorder_ms = statistics.mean(e[0].elapsed_time(e[1]) + e[3].elapsed_time(e[4]) for e in evs)
     build_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    t_max = torch.tensor([elapsed_ms], device=dev)
-    if world > 1:
-        import torch.distributed as dist
-
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(t_max.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev, world)
     pairs = layer.kept_pairs()
     nt = layer.nt
     density = pairs / (layer.B * layer.Hh * nt * nt)
     flops = pairs * flops_per_pair(layer.d)
-    value = world * K * flops / (elapsed_ms * 1e-3) / 1e12
+    total_flops = sum_over_ranks(flops, dev, world)
+    value = whole_job_tflops(total_flops, K, elapsed_ms)
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
 
     # end to end through the C ABI from pinned host buffers (H2D in, D2H out)
@@ -419,14 +439,9 @@ def main():
             ho.copy_(layer.o, non_blocking=True)
         e1.record()
         barrier()
-        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        t2 = torch.tensor([e2e_ms], device=dev)
-        if world > 1:
-            import torch.distributed as dist
-
-            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * flops / (float(t2.item()) * 1e-3) / 1e12, "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": float(t2.item())}
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev, world)
+        e2e = {"value": whole_job_tflops(total_flops, 1, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     # the same kernel with every key tile listed (dense-mask run), outside the timed region
     dense = None
