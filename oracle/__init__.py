@@ -13,7 +13,7 @@ Sources (pages on block-sparse attention for video diffusion transformers):
     loaded into block-sparse attention kernels.
   * Rectified SpaAttn (abstract): pooled query-key block scores.
   * SCOPE review (Eqs. (7)-(8) as quoted; abstract): hybrid top-p / fixed
-    top-k selection.
+    top-k selection; Eqs. (9)-(10): the online per-head top-k floor.
 
 Parity pins: every function here is checked in tests/test_oracle_*.py
 against closed forms, textbook routines (torch SDPA in fp64, scipy
@@ -31,6 +31,9 @@ from .sta_oracle import (  # noqa: F401
     block_scores,
     select_row,
     select,
+    head_topk_floor,
+    select_with_head_floor,
+    tile_sizes,
     window_mask,
     build_mask,
     mask_to_csr,

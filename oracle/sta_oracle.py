@@ -151,6 +151,41 @@ def select(P, top_p, k_min):
 
 
 # --------------------------------------------------------------------------
+# Online per-head top-k floor (SCOPE review, Eqs. (9)-(10) as quoted: the
+# head's floor is the cluster-size-weighted mean of the base retained counts,
+# and clusters below it are extended to it).
+# Reading, at tile granularity: a cluster is a query tile, its size n_c the
+# number of real tokens in it, its base count b_c the size of the hybrid
+# top-p / k_min selection; k_head = ceil(sum n_c b_c / sum n_c) over the query
+# tiles of the head; a row keeps the first max(b_c, min(k_head, Nt)) tiles of
+# its order. The windows are OR'd in afterwards, as without the floor.
+# --------------------------------------------------------------------------
+def head_topk_floor(counts, sizes):
+    """k_head = ceil(sum(n_c * b_c) / sum(n_c)) in exact integer arithmetic."""
+    num = sum(int(n) * int(b) for n, b in zip(sizes, counts))
+    den = sum(int(n) for n in sizes)
+    return -(-num // den) if den else 0
+
+
+def select_with_head_floor(P_head, top_p, k_min, sizes):
+    """Selection of one head [Nt, Nt] with the per-head floor; returns
+    (keep [Nt, Nt] bool, k_head)."""
+    P_head = np.asarray(P_head)
+    base = np.stack([select_row(r, top_p, k_min) for r in P_head])
+    k_head = head_topk_floor(base.sum(axis=1), sizes)
+    out = base.copy()
+    for c in range(P_head.shape[0]):
+        if base[c].sum() < k_head:
+            out[c] = select_row(P_head[c], top_p, max(int(k_min), k_head))
+    return out, k_head
+
+
+def tile_sizes(T, H, W):
+    """Real tokens per tile, [Nt]."""
+    return valid_rows(T, H, W).reshape(-1, TILE_TOKENS).sum(axis=1)
+
+
+# --------------------------------------------------------------------------
 # Deformable dual window per temporal-distance group (Compact Attention
 # Fig. 1(3), Fig. 4; Table III "Frame-group" and "Dual Window").
 # Reading: in tile units, key tile kt is kept for query tile qt of head h iff
@@ -199,8 +234,9 @@ def mask_to_csr(mask):
 
 
 def build_mask(q_tiled, k_tiled, T, H, W, use_scores, top_p, k_min,
-               windows=None, group_lo=None, sm_scale=0.0):
-    """Full mask construction: pool, score, select, OR windows, emit CSR.
+               windows=None, group_lo=None, sm_scale=0.0, head_floor=False):
+    """Full mask construction: pool, score, select (with the per-head top-k
+    floor when head_floor), OR windows, emit CSR.
 
     Returns dict(mask [B,heads,Nt,Nt] bool, probs [B,heads,Nt,Nt] fp64 or
     None, row_ptr, col_idx).
@@ -215,7 +251,13 @@ def build_mask(q_tiled, k_tiled, T, H, W, use_scores, top_p, k_min,
         qbar = pool(q_tiled, T, H, W)
         kbar = pool(k_tiled, T, H, W)
         _, probs = block_scores(qbar, kbar, scale)
-        mask |= select(probs, top_p, k_min)
+        if head_floor:
+            sizes = tile_sizes(T, H, W)
+            for b in range(B):
+                for h in range(Hh):
+                    mask[b, h] |= select_with_head_floor(probs[b, h], top_p, k_min, sizes)[0]
+        else:
+            mask |= select(probs, top_p, k_min)
     if windows is not None:
         mask |= window_mask(windows, group_lo, T, H, W)[None]
     row_ptr, col_idx = mask_to_csr(mask)

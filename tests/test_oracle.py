@@ -385,3 +385,41 @@ def test_single_tile_list_is_plain_softmax():
         s = qt[0, 0, qrows] @ kk.T * 0.25
         assert np.allclose(o, scipy.special.softmax(s, axis=1) @ vv, atol=1e-12)
         assert np.allclose(lse, scipy.special.logsumexp(s, axis=1), atol=1e-12)
+
+
+# ------------------------------------------------- per-head top-k floor (f1)
+def test_head_floor_golden(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "head_floor_cases.json")))
+    for c in g["floor_cases"]:
+        assert O.head_topk_floor(c["counts"], c["sizes"]) == c["k_head"], c["why"]
+    sc = g["select_case"]
+    P = np.array(sc["p"])
+    base = np.stack([O.select_row(r, sc["top_p"], sc["k_min"]) for r in P])
+    assert [np.nonzero(r)[0].tolist() for r in base] == sc["base_keep"]
+    keep, k_head = O.select_with_head_floor(P, sc["top_p"], sc["k_min"], sc["sizes"])
+    assert k_head == sc["k_head"]
+    assert [np.nonzero(r)[0].tolist() for r in keep] == sc["keep"]
+
+
+def test_head_floor_properties():
+    """The floor never removes a tile, leaves rows at or above k_head alone,
+    brings every other row to exactly min(k_head, Nt), and with all base
+    counts equal changes nothing."""
+    rng = np.random.default_rng(8)
+    for trial in range(5):
+        P = scipy.special.softmax(rng.standard_normal((20, 31)) * (1 + trial), axis=-1)
+        sizes = rng.integers(1, 65, size=20)
+        base = np.stack([O.select_row(r, 0.8, 2) for r in P])
+        keep, k_head = O.select_with_head_floor(P, 0.8, 2, sizes)
+        assert (keep >= base).all()
+        bc = base.sum(1)
+        want = np.where(bc >= k_head, bc, min(k_head, 31))
+        assert np.array_equal(keep.sum(1), want)
+        assert k_head == -(-int((sizes * bc).sum()) // int(sizes.sum()))
+    P = np.full((4, 8), 1 / 8)
+    keep, k_head = O.select_with_head_floor(P, 0.5, 0, [64] * 4)
+    assert k_head == 4 and np.array_equal(keep, np.stack([O.select_row(r, 0.5, 0) for r in P]))
+
+
+def test_tile_sizes():
+    assert O.tile_sizes(2, 9, 10).tolist() == [64, 16, 8, 2] * 2
