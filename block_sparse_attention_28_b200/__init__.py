@@ -44,6 +44,7 @@ class MaskParams(ctypes.Structure):
         ("num_groups", ctypes.c_int32),
         ("group_lo", ctypes.c_int32 * MAX_GROUPS),
         ("windows", ctypes.c_void_p),
+        ("head_topk_floor", ctypes.c_int32),
     ]
 
 
@@ -122,9 +123,12 @@ def sta_build_mask_workspace(B, heads, d, g):
     return int(_lib.sta_build_mask_workspace(B, heads, d, g))
 
 
-def mask_params(top_p=0.0, k_min=0, use_scores=False, sm_scale=0.0, group_lo=(0,), windows=None):
-    """MaskParams; `windows` is a device int32 tensor [heads, G, 4] or None."""
+def mask_params(top_p=0.0, k_min=0, use_scores=False, sm_scale=0.0, group_lo=(0,), windows=None,
+                head_floor=False):
+    """MaskParams; `windows` is a device int32 tensor [heads, G, 4] or None;
+    `head_floor` turns on the per-head top-k floor of the selection."""
     p = MaskParams()
+    p.head_topk_floor = 1 if head_floor else 0
     p.top_p = float(top_p)
     p.k_min = int(k_min)
     p.use_scores = 1 if use_scores else 0

@@ -34,7 +34,7 @@ bool common_sizes_ok(int32_t B, int32_t heads, int32_t d, sta_grid g, Geo *geo, 
 }
 
 struct MaskWs {
-  size_t qbar, kbar, bits, counts, total;
+  size_t qbar, kbar, bits, counts, sel, kfloor, total;
 };
 
 MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
@@ -50,6 +50,10 @@ MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
   off = align_up(off + R * wpr * sizeof(uint32_t), 256);
   w.counts = off;
   off = align_up(off + R * sizeof(int32_t), 256);
+  w.sel = off;
+  off = align_up(off + R * sizeof(int32_t), 256);
+  w.kfloor = off;
+  off = align_up(off + (size_t)B * heads * sizeof(int32_t), 256);
   w.total = off;
   return w;
 }
@@ -130,9 +134,23 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
   GroupLo glo;
   for (int i = 0; i < STA_MAX_GROUPS; ++i) glo.v[i] = (i < p->num_groups) ? p->group_lo[i] : 0x7fffffff;
   dim3 grid((unsigned)((g.Nt + SEL_QB - 1) / SEL_QB), (unsigned)(B * heads));
+  const bool floor = use_scores && p->head_topk_floor != 0;
+  int *sel = reinterpret_cast<int *>(ws + L.sel);
+  int *kfloor = reinterpret_cast<int *>(ws + L.kfloor);
+  if (floor) {
+    // pass 1: base selection counts; per-head floor; pass 2 below re-selects
+    // with k_min raised to the floor
+    score_select_kernel<D><<<grid, SEL_THREADS, smem, s>>>(
+        qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, nullptr, 0, glo, bits, counts, nullptr,
+        wpr, nullptr, sel);
+    STA_CUDA_TRY(cudaGetLastError());
+    head_floor_kernel<<<(unsigned)(B * heads), FLOOR_THREADS, 0, s>>>(sel, kfloor, g);
+    STA_CUDA_TRY(cudaGetLastError());
+  }
   score_select_kernel<D><<<grid, SEL_THREADS, smem, s>>>(
       qbar, kbar, heads, g, scale, p->top_p, p->k_min, use_scores ? 1 : 0, p->windows,
-      p->windows ? p->num_groups : 0, glo, bits, counts, block_probs, wpr);
+      p->windows ? p->num_groups : 0, glo, bits, counts, block_probs, wpr, floor ? kfloor : nullptr,
+      nullptr);
   STA_CUDA_TRY(cudaGetLastError());
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(counts, row_ptr, reinterpret_cast<long long *>(nnz_dev), R);
   STA_CUDA_TRY(cudaGetLastError());

@@ -170,7 +170,8 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
                     float scale, float top_p, int k_min, int use_scores,
                     const int *__restrict__ windows, int G, GroupLo glo,
                     unsigned int *__restrict__ bits, int *__restrict__ counts,
-                    float *__restrict__ probs_out, int wpr) {
+                    float *__restrict__ probs_out, int wpr, const int *__restrict__ kmin_head,
+                    int *__restrict__ sel_count) {
   extern __shared__ __align__(16) float sm[];
   const int nt = g.Nt;
   const int bh = blockIdx.y;
@@ -263,7 +264,8 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
       }
       __syncwarp();
       // Phase 3: selection threshold as (level v_f, ties c_f).
-      const int kk = min(k_min, nt);
+      // per-head top-k floor (second pass): k_min raised to the head's floor
+      const int kk = min(kmin_head != nullptr ? max(k_min, kmin_head[bh]) : k_min, nt);
       unsigned int m_p_level = 0xFFFFFFFFu, m_p_ties = 0u;
       long long m_p = 0;
       if (top_p >= 1.0f) {
@@ -294,6 +296,7 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
         v_f = m_p_level;
         c_f = m_p_ties;
       }
+      if (sel_count != nullptr && lane == 0) sel_count[row] = (int)((long long)kk > m_p ? kk : m_p);
     }
     // Phase 4: membership bits = selected OR window, one 32-bit word per lane step.
     const int tq = qt / tpf, remq = qt - tq * tpf;
@@ -331,6 +334,45 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
       total += __popc(word);
     }
     if (lane == 0) counts[row] = total;
+  }
+}
+
+// ------------------------------------------------ per-head top-k floor
+// One CTA per (b*heads + h): k_head = ceil(sum_c n_c b_c / sum_c n_c), with
+// b_c the selected count of query tile c and n_c its number of real tokens
+// (SCOPE Eqs. (9)-(10) as quoted, query tiles as clusters). Integer sums.
+constexpr int FLOOR_THREADS = 256;
+
+__global__ void __launch_bounds__(FLOOR_THREADS)
+head_floor_kernel(const int *__restrict__ sel_count, int *__restrict__ kfloor, Geo g) {
+  __shared__ long long part[2][FLOOR_THREADS / 32];
+  const int bh = blockIdx.x, tid = threadIdx.x;
+  const int tpf = g.NH * g.NW;
+  long long num = 0, den = 0;
+  for (int qt = tid; qt < g.Nt; qt += FLOOR_THREADS) {
+    const int rem = qt % tpf;
+    const int ty = rem / g.NW, tx = rem - ty * g.NW;
+    const long long n = (long long)valid_extent(g.H, ty) * valid_extent(g.W, tx);
+    num += n * sel_count[(long long)bh * g.Nt + qt];
+    den += n;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    num += __shfl_xor_sync(0xffffffffu, num, o);
+    den += __shfl_xor_sync(0xffffffffu, den, o);
+  }
+  if ((tid & 31) == 0) {
+    part[0][tid >> 5] = num;
+    part[1][tid >> 5] = den;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    long long N = 0, Dn = 0;
+    for (int w = 0; w < FLOOR_THREADS / 32; ++w) {
+      N += part[0][w];
+      Dn += part[1][w];
+    }
+    kfloor[bh] = Dn > 0 ? (int)((N + Dn - 1) / Dn) : 0;
   }
 }
 

@@ -79,6 +79,12 @@ typedef struct {
   int32_t num_groups;     /* G in [1, STA_MAX_GROUPS] when windows != NULL */
   int32_t group_lo[STA_MAX_GROUPS]; /* ascending, group_lo[0] == 0 */
   const int32_t *windows; /* device int32 [heads][G][4]; NULL = no windows */
+  int32_t head_topk_floor; /* 1: raise each row's selection to its head's floor
+                              (SCOPE Eqs. (9)-(10) as quoted): with b_c the
+                              selected count of query tile c and n_c its real
+                              tokens, k_head = ceil(sum n_c b_c / sum n_c), and
+                              rows with b_c < k_head keep their first
+                              min(k_head, Nt) tiles; ignored if !use_scores */
 } sta_mask_params;
 
 /* Number of tiles per head (Nt) and padded rows per head (Lpad) of a grid;

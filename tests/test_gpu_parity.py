@@ -424,3 +424,60 @@ def test_attn_reuse_all_densities_full(sta, gp):
         bufs.block_probs = None
         _attn_check(sta, gp, qt, kt, vt, bufs.row_ptr, bufs.col_idx, B, Hh, d, T, H, W, rows=rows)
         _attn_check(sta, gp, qt10, kt10, vt, bufs.row_ptr, bufs.col_idx, B, Hh, d, T, H, W, rows=rows)
+
+
+# ---------------------------------------------- per-head top-k floor (SCOPE f1)
+def _floor_mask(probs, top_p, k_min, sizes):
+    B, Hh, nt, _ = probs.shape
+    out = np.zeros((B, Hh, nt, nt), dtype=bool)
+    for b in range(B):
+        for h in range(Hh):
+            out[b, h] = O.select_with_head_floor(probs[b, h], top_p, k_min, sizes)[0]
+    return out
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_build_mask_head_floor_ragged(sta, gp, d):
+    T, H, W, Hh, B = 3, 19, 37, 3, 2  # partial tiles: the cluster sizes n_c differ
+    q, k, _ = _structured(T, H, W, Hh, d, seed=21, B=B)
+    g = sta.grid(T, H, W)
+    qt, kt = gp.reorder(q, B, Hh, d, g), gp.reorder(k, B, Hh, d, g)
+    rng = np.random.default_rng(d)
+    win = rng.integers(-1, 2, size=(Hh, 3, 4)).astype(np.int32)
+    params = sta.mask_params(0.6, 1, True, 0.0, (0, 1, 3), torch.from_numpy(win).cuda(), head_floor=True)
+    bufs = gp.build(qt, kt, B, Hh, d, g, params)
+    torch.cuda.synchronize()
+    rp, ci, nnz = gp.csr_np(bufs)
+    probs = bufs.block_probs.cpu().numpy()
+    sizes = O.tile_sizes(T, H, W)
+    mask = _floor_mask(probs, 0.6, 1, sizes) | O.window_mask(win, (0, 1, 3), T, H, W)[None]
+    rp_o, ci_o = O.mask_to_csr(mask)
+    assert np.array_equal(rp, rp_o) and np.array_equal(ci, ci_o)
+    assert np.array_equal(bufs.block_mask.cpu().numpy().astype(bool), mask)
+    # the floor only adds tiles
+    base = O.select(probs, 0.6, 1)
+    assert (_floor_mask(probs, 0.6, 1, sizes) >= base).all()
+
+
+def test_build_mask_head_floor_720p_sampled_heads(sta, gp):
+    cfg = CONFIGS[2]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    q, k, _ = make_qkv(cfg, device="cuda")
+    qt, kt = gp.reorder(q, B, Hh, d, g), gp.reorder(k, B, Hh, d, g)
+    del q, k
+    win = window_params(cfg, window_scale(2, 0))
+    params = sta.mask_params(cfg.top_p, cfg.k_min, True, 0.0, cfg.group_lo, torch.from_numpy(win).cuda(),
+                             head_floor=True)
+    bufs = gp.build(qt, kt, B, Hh, d, g, params, with_mask=False, with_probs=True)
+    torch.cuda.synchronize()
+    rp, ci, nnz = gp.csr_np(bufs)
+    nt = sta.sta_num_tiles(g)
+    sizes = O.tile_sizes(T, H, W)
+    for h in (3, 29):
+        probs = bufs.block_probs[0, h].cpu().numpy()
+        keep, k_head = O.select_with_head_floor(probs, cfg.top_p, cfg.k_min, sizes)
+        keep |= O.window_mask(win[h:h + 1], cfg.group_lo, T, H, W)[0]
+        for qtile in range(0, nt, 7):
+            r = h * nt + qtile
+            assert np.array_equal(ci[rp[r]:rp[r + 1]], np.nonzero(keep[qtile])[0]), (h, qtile, k_head)
