@@ -14,6 +14,7 @@ Sources (pages on block-sparse attention for video diffusion transformers):
   * Rectified SpaAttn (abstract): pooled query-key block scores.
   * SCOPE review (Eqs. (7)-(8) as quoted; abstract): hybrid top-p / fixed
     top-k selection; Eqs. (9)-(10): the online per-head top-k floor.
+  * AdaSpa (abstract): exact block importance from a cached log-sum-exp.
 
 Parity pins: every function here is checked in tests/test_oracle_*.py
 against closed forms, textbook routines (torch SDPA in fp64, scipy
@@ -39,4 +40,5 @@ from .sta_oracle import (  # noqa: F401
     mask_to_csr,
     attention_rows,
     attention_all,
+    block_mass,
 )

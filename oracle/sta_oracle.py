@@ -326,3 +326,45 @@ def attention_all(q_tiled, k_tiled, v_tiled, row_ptr, col_idx, T, H, W, sm_scale
         O[b, h, qrows] = o
         LSE[b, h, qrows] = lse
     return O, LSE
+
+
+# --------------------------------------------------------------------------
+# LSE-cached exact block importance (AdaSpa abstract: exact block importance
+# computed during a full-attention step with a cached log-sum-exp, then
+# reused for the block-sparse steps that follow).
+# Reading: for query tile qt and listed key tile kt,
+#   mass(qt, kt) = (1 / n_q) * sum_i sum_j exp(scale * q_i . k_j - lse_i)
+# over the real query tokens i of qt (n_q of them) and the real key tokens j of
+# kt, with lse the cached per-token log-sum-exp (natural log); a token with
+# lse = -inf contributes nothing. With the exact LSE of the same inputs and
+# every tile listed, each row of masses sums to one.
+# --------------------------------------------------------------------------
+def block_mass(q_tiled, k_tiled, lse, row_ptr, col_idx, T, H, W, sm_scale, rows):
+    """Masses for the listed (row, key tile) pairs of the CSR rows in `rows`.
+
+    Returns {row: (tiles, masses)} with masses fp64 aligned to tiles."""
+    q_tiled = np.asarray(q_tiled)
+    B, Hh, lpad, d = q_tiled.shape
+    _, _, nt, _ = tile_grid(T, H, W)
+    valid = valid_rows(T, H, W)
+    scale = float(sm_scale) if sm_scale else 1.0 / math.sqrt(d)
+    out = {}
+    for r in rows:
+        r = int(r)
+        bh, qt = divmod(r, nt)
+        b, h = divmod(bh, Hh)
+        qrows = np.arange(qt * 64, qt * 64 + 64)
+        qrows = qrows[valid[qrows]]
+        q = q_tiled[b, h, qrows].astype(np.float64)
+        l = np.asarray(lse)[b, h, qrows].astype(np.float64)
+        live = np.isfinite(l)
+        tiles = np.asarray(col_idx[int(row_ptr[r]):int(row_ptr[r + 1])], dtype=np.int64)
+        masses = np.zeros(tiles.size)
+        for i, kt in enumerate(tiles):
+            krows = np.arange(kt * 64, kt * 64 + 64)
+            krows = krows[valid[krows]]
+            k = np.asarray(k_tiled)[b, h, krows].astype(np.float64)
+            s = (q[live] @ k.T) * scale - l[live][:, None]
+            masses[i] = np.exp(s).sum() / qrows.size
+        out[r] = (tiles, masses)
+    return out

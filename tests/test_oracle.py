@@ -423,3 +423,45 @@ def test_head_floor_properties():
 
 def test_tile_sizes():
     assert O.tile_sizes(2, 9, 10).tolist() == [64, 16, 8, 2] * 2
+
+
+# ------------------------------------------- LSE-cached block importance (f3)
+def test_block_mass_is_block_sum_of_dense_softmax():
+    """With the exact LSE and every tile listed, the block masses are the block
+    sums of the dense softmax matrix (scipy), averaged over the query tile's
+    real tokens; every row of masses sums to one."""
+    T, H, W, d = 2, 9, 13, 8  # ragged tiles
+    q = _bf16_exact((1, T * H * W, 1, d), RNG, 2.0)
+    k = _bf16_exact((1, T * H * W, 1, d), RNG, 2.0)
+    v = _bf16_exact((1, T * H * W, 1, d), RNG)
+    qt, kt, vt = (O.reorder_fwd(a, T, H, W) for a in (q, k, v))
+    nh, nw, nt, _ = O.tile_grid(T, H, W)
+    rp, ci = O.mask_to_csr(np.ones((1, 1, nt, nt), dtype=bool))
+    _, lse = O.attention_all(qt, kt, vt, rp, ci, T, H, W, 0.4)
+    res = O.block_mass(qt, kt, lse, rp, ci, T, H, W, 0.4, range(nt))
+    valid = O.valid_rows(T, H, W)
+    real = np.nonzero(valid)[0]
+    P = scipy.special.softmax(qt[0, 0, real] @ kt[0, 0, real].T * 0.4, axis=1)
+    tile_of = real // 64
+    for r in range(nt):
+        tiles, masses = res[r]
+        assert abs(masses.sum() - 1.0) < 1e-12
+        rows_r = tile_of == r
+        for kt_i, mval in zip(tiles, masses):
+            want = P[np.ix_(rows_r, tile_of == kt_i)].sum() / rows_r.sum()
+            assert abs(mval - want) < 1e-12
+
+
+def test_block_mass_with_stale_lse_scales_by_the_lse_gap():
+    """A cached LSE larger by delta scales every mass by exp(-delta)."""
+    T, H, W, d = 1, 16, 16, 8
+    q = _bf16_exact((1, T * H * W, 1, d), RNG)
+    k = _bf16_exact((1, T * H * W, 1, d), RNG)
+    qt, kt = O.reorder_fwd(q, T, H, W), O.reorder_fwd(k, T, H, W)
+    nt = O.tile_grid(T, H, W)[2]
+    rp, ci = O.mask_to_csr(np.ones((1, 1, nt, nt), dtype=bool))
+    lse = np.zeros((1, 1, 64 * nt))
+    a = O.block_mass(qt, kt, lse, rp, ci, T, H, W, 0.0, range(nt))
+    b = O.block_mass(qt, kt, lse + 0.5, rp, ci, T, H, W, 0.0, range(nt))
+    for r in range(nt):
+        assert np.allclose(b[r][1], a[r][1] * math.exp(-0.5), rtol=1e-13)
