@@ -45,6 +45,7 @@ class MaskParams(ctypes.Structure):
         ("group_lo", ctypes.c_int32 * MAX_GROUPS),
         ("windows", ctypes.c_void_p),
         ("head_topk_floor", ctypes.c_int32),
+        ("block_scores", ctypes.c_void_p),
     ]
 
 
@@ -71,6 +72,9 @@ _lib.sta_build_mask_noalloc.argtypes = [_vp, _vp, _i32, _i32, _i32, Grid, ctypes
 _lib.sta_build_mask_noalloc.restype = ctypes.c_int
 _lib.sta_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, Grid, _f32, _vp]
 _lib.sta_attn_fwd.restype = ctypes.c_int
+_lib.sta_attn_fwd_block_mass.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, Grid,
+                                         _f32, _vp]
+_lib.sta_attn_fwd_block_mass.restype = ctypes.c_int
 _lib.sta_get_device_error.argtypes = [_vp]
 _lib.sta_get_device_error.restype = ctypes.c_int
 _lib.sta_status_string.argtypes = [ctypes.c_int]
@@ -124,11 +128,13 @@ def sta_build_mask_workspace(B, heads, d, g):
 
 
 def mask_params(top_p=0.0, k_min=0, use_scores=False, sm_scale=0.0, group_lo=(0,), windows=None,
-                head_floor=False):
+                head_floor=False, block_scores=None):
     """MaskParams; `windows` is a device int32 tensor [heads, G, 4] or None;
-    `head_floor` turns on the per-head top-k floor of the selection."""
+    `head_floor` turns on the per-head top-k floor of the selection;
+    `block_scores` (device fp32 [B, heads, Nt, Nt]) replaces the pooled scores."""
     p = MaskParams()
     p.head_topk_floor = 1 if head_floor else 0
+    p.block_scores = _ptr(block_scores)
     p.top_p = float(top_p)
     p.k_min = int(k_min)
     p.use_scores = 1 if use_scores else 0
@@ -163,6 +169,14 @@ def sta_attn_fwd(q, k, v, o, lse, row_ptr, col_idx, B, heads, d, g, sm_scale=0.0
     _check(_lib.sta_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(row_ptr), _ptr(col_idx),
                              B, heads, d, g, float(sm_scale), _stream(stream)),
            "sta_attn_fwd")
+
+
+def sta_attn_fwd_block_mass(q, k, v, o, lse, row_ptr, col_idx, lse_cached, block_mass, B, heads, d, g,
+                            sm_scale=0.0, stream=None):
+    _check(_lib.sta_attn_fwd_block_mass(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(row_ptr),
+                                        _ptr(col_idx), _ptr(lse_cached), _ptr(block_mass), B, heads, d, g,
+                                        float(sm_scale), _stream(stream)),
+           "sta_attn_fwd_block_mass")
 
 
 def sta_get_device_error(stream=None):

@@ -82,12 +82,18 @@ inline size_t smem_bytes(int nt) {
   return (size_t)Cfg<D>::OFF_LIST + (size_t)(2 * wpr + nt) * 4 + 1024;
 }
 
-template <int D>
+// MASS: also accumulate the LSE-cached exact block importance (AdaSpa) of
+// every listed (query tile, key tile) pair into block_mass:
+//   mass = (1/n_q) sum_i sum_j 2^(s_ij * scale_log2 - lse_in_i * log2 e),
+// which is, per row and tile, the row's softmax sum (relative to its running
+// max m_i) times 2^(m_i - lse_in_i * log2 e): one extra exp2 per row and tile.
+template <int D, bool MASS>
 __global__ void __launch_bounds__(NUM_THREADS, MIN_BLOCKS_PER_SM)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16 *__restrict__ out,
                 float *__restrict__ lse, const int *__restrict__ row_ptr,
-                const int *__restrict__ col_idx, Geo g, float scale_log2) {
+                const int *__restrict__ col_idx, Geo g, float scale_log2,
+                const float *__restrict__ lse_in, float *__restrict__ block_mass) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -319,6 +325,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     float m = -INFINITY, l = 0.0f;
     bool ok = true;
+    // cached log-sum-exp of this thread's query token (MASS), in log2 units
+    float lin = -INFINITY, inv_nq = 0.0f;
+    const int qt_half = halfB ? qtB : qtA;
+    if (MASS && (!halfB || hasB)) {
+      const int rem = qt_half % (g.NH * g.NW);
+      const int ty = rem / g.NW, tx = rem - ty * g.NW;
+      const int vy = valid_extent(g.H, ty), vx = valid_extent(g.W, tx);
+      const int rr = tid & 63;
+      inv_nq = 1.0f / (float)(vy * vx);
+      if ((rr >> 3) < vy && (rr & 7) < vx)
+        lin = lse_in[(long long)bh * g.Lpad + (long long)qt_half * 64 + rr] * 1.4426950408889634f;
+    }
     for (int j = 0; j < n; ++j) {
       const int buf = j & 1;
       const bool got = tc::mbar_wait(s_full + buf, (j >> 1) & 1, abort_flag, WAIT_LIMIT);
@@ -398,6 +416,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         tc::tmem_st32(sS, pk);
         l = l * alpha + sum;
+        if (MASS) {
+          float c = (lin > -INFINITY) ? sum * tc::ex2(mref - lin) : 0.0f;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+          // two warps (32 rows each) per query tile: two adds onto zero, so the
+          // result does not depend on their order
+          if (lane == 0) atomicAdd(block_mass + ((long long)bh * nt + qt_half) * nt + kt, c * inv_nq);
+        }
         const bool need_o = rescale && (m != -INFINITY);
         if (__any_sync(0xffffffffu, need_o)) {
           // PV_{j-1} must have retired before O is scaled (j >= 1 here). S_j

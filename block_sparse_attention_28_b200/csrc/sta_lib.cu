@@ -120,7 +120,8 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
   const bool use_scores = p->use_scores != 0;
   const float scale = p->sm_scale != 0.0f ? p->sm_scale : 1.0f / sqrtf((float)D);
 
-  if (use_scores) {
+  const float *P_in = use_scores ? p->block_scores : nullptr;
+  if (use_scores && P_in == nullptr) {
     const long long warps = 2 * R;
     const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
     pool_kernel<D><<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(q_tiled),
@@ -142,7 +143,7 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
     // with k_min raised to the floor
     score_select_kernel<D><<<grid, SEL_THREADS, smem, s>>>(
         qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, nullptr, 0, glo, bits, counts, nullptr,
-        wpr, nullptr, sel);
+        wpr, nullptr, sel, P_in);
     STA_CUDA_TRY(cudaGetLastError());
     head_floor_kernel<<<(unsigned)(B * heads), FLOOR_THREADS, 0, s>>>(sel, kfloor, g);
     STA_CUDA_TRY(cudaGetLastError());
@@ -150,7 +151,7 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
   score_select_kernel<D><<<grid, SEL_THREADS, smem, s>>>(
       qbar, kbar, heads, g, scale, p->top_p, p->k_min, use_scores ? 1 : 0, p->windows,
       p->windows ? p->num_groups : 0, glo, bits, counts, block_probs, wpr, floor ? kfloor : nullptr,
-      nullptr);
+      nullptr, P_in);
   STA_CUDA_TRY(cudaGetLastError());
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(counts, row_ptr, reinterpret_cast<long long *>(nnz_dev), R);
   STA_CUDA_TRY(cudaGetLastError());
@@ -162,23 +163,27 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
   return STA_OK;
 }
 
-template <int D>
+template <int D, bool MASS>
 sta_status launch_attn(const void *q, const void *k, const void *v, void *o, float *lse,
                        const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
-                       const Geo &g, float sm_scale, cudaStream_t s) {
+                       const Geo &g, float sm_scale, cudaStream_t s, const float *lse_in = nullptr,
+                       float *block_mass = nullptr) {
   const unsigned long long rows = (unsigned long long)B * heads * g.Lpad;
   CUtensorMap tq, tk, tv;
   if (!make_tile_map(&tq, q, rows, D) || !make_tile_map(&tk, k, rows, D) || !make_tile_map(&tv, v, rows, D))
     return STA_ERR_CUDA;
   const size_t smem = attn::smem_bytes<D>(g.Nt);
   if (smem > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
-  STA_CUDA_TRY(cudaFuncSetAttribute(attn::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)smem));
+  STA_CUDA_TRY(cudaFuncSetAttribute(attn::attn_fwd_kernel<D, MASS>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (MASS)
+    STA_CUDA_TRY(cudaMemsetAsync(block_mass, 0, (size_t)B * heads * g.Nt * g.Nt * sizeof(float), s));
   const float scale = sm_scale != 0.0f ? sm_scale : 1.0f / sqrtf((float)D);
   const float scale_log2 = scale * 1.4426950408889634f;
   dim3 grid((unsigned)((g.Nt + 1) / 2), (unsigned)(B * heads));
-  attn::attn_fwd_kernel<D><<<grid, attn::NUM_THREADS, smem, s>>>(
-      tq, tk, tv, static_cast<__nv_bfloat16 *>(o), lse, row_ptr, col_idx, g, scale_log2);
+  attn::attn_fwd_kernel<D, MASS><<<grid, attn::NUM_THREADS, smem, s>>>(
+      tq, tk, tv, static_cast<__nv_bfloat16 *>(o), lse, row_ptr, col_idx, g, scale_log2, lse_in,
+      block_mass);
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }
@@ -226,7 +231,8 @@ sta_status sta_build_mask(const void *q_tiled, const void *k_tiled, int32_t B, i
   if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return st;
   if (p == nullptr || row_ptr == nullptr || col_idx == nullptr || nnz_dev == nullptr)
     return STA_ERR_INVALID_ARG;
-  if (p->use_scores && (q_tiled == nullptr || k_tiled == nullptr || !aligned16(q_tiled) || !aligned16(k_tiled)))
+  if (p->use_scores && p->block_scores == nullptr &&
+      (q_tiled == nullptr || k_tiled == nullptr || !aligned16(q_tiled) || !aligned16(k_tiled)))
     return STA_ERR_INVALID_ARG;
   if (p->windows != nullptr) {
     if (p->num_groups < 1 || p->num_groups > STA_MAX_GROUPS || p->group_lo[0] != 0) return STA_ERR_INVALID_ARG;
@@ -260,8 +266,29 @@ sta_status sta_attn_fwd(const void *q, const void *k, const void *v, void *o, fl
   if (!(sm_scale == sm_scale) || sm_scale < 0.0f) return STA_ERR_INVALID_ARG;
   if (!device_is_sm100()) return STA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return (d == 128) ? launch_attn<128>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s)
-                    : launch_attn<64>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s);
+  return (d == 128) ? launch_attn<128, false>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s)
+                    : launch_attn<64, false>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s);
+}
+
+sta_status sta_attn_fwd_block_mass(const void *q, const void *k, const void *v, void *o, float *lse,
+                                   const int32_t *row_ptr, const int32_t *col_idx,
+                                   const float *lse_cached, float *block_mass, int32_t B,
+                                   int32_t heads, int32_t d, sta_grid g, float sm_scale,
+                                   sta_stream_t stream) {
+  Geo geo;
+  sta_status st = STA_OK;
+  if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || row_ptr == nullptr ||
+      col_idx == nullptr || lse_cached == nullptr || block_mass == nullptr)
+    return STA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return STA_ERR_INVALID_ARG;
+  if (!(sm_scale == sm_scale) || sm_scale < 0.0f) return STA_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return STA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return (d == 128) ? launch_attn<128, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s,
+                                             lse_cached, block_mass)
+                    : launch_attn<64, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s,
+                                            lse_cached, block_mass);
 }
 
 sta_status sta_get_device_error(sta_stream_t stream) {

@@ -171,7 +171,7 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
                     const int *__restrict__ windows, int G, GroupLo glo,
                     unsigned int *__restrict__ bits, int *__restrict__ counts,
                     float *__restrict__ probs_out, int wpr, const int *__restrict__ kmin_head,
-                    int *__restrict__ sel_count) {
+                    int *__restrict__ sel_count, const float *__restrict__ P_in) {
   extern __shared__ __align__(16) float sm[];
   const int nt = g.Nt;
   const int bh = blockIdx.y;
@@ -207,7 +207,7 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
   }
   if (!use_scores) __syncthreads();
 
-  if (use_scores) {
+  if (use_scores && P_in == nullptr) {
     // Phase 1: S[i][kt] = scale * qbar[q0+i] . kbar[kt], sequential fp32 FMA over d.
     for (int e = tid; e < SEL_QB * D; e += SEL_THREADS) {
       const int i = e / D;
@@ -244,23 +244,32 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
     unsigned int v_f = 0xFFFFFFFFu;  // keep P > v_f, plus c_f ties at v_f
     unsigned int c_f = 0u;
     if (use_scores) {
-      // Phase 2: row softmax in fp32 (max, expf, fixed-order sum, IEEE divide).
-      float mx = -INFINITY;
-      for (int j = lane; j < nt; j += 32) mx = fmaxf(mx, Sr[j]);
+      if (P_in != nullptr) {
+        // caller-supplied block scores (e.g. exact block masses), clamped to [0, 1]
+        for (int j = lane; j < nt; j += 32) {
+          const float p = fminf(fmaxf(P_in[row * nt + j], 0.0f), 1.0f);
+          Sr[j] = p;
+          if (probs_out) probs_out[row * nt + j] = p;
+        }
+      } else {
+        // Phase 2: row softmax in fp32 (max, expf, fixed-order sum, IEEE divide).
+        float mx = -INFINITY;
+        for (int j = lane; j < nt; j += 32) mx = fmaxf(mx, Sr[j]);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      float sum = 0.0f;
-      for (int j = lane; j < nt; j += 32) {
-        const float e = expf(Sr[j] - mx);
-        Sr[j] = e;
-        sum += e;
-      }
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float sum = 0.0f;
+        for (int j = lane; j < nt; j += 32) {
+          const float e = expf(Sr[j] - mx);
+          Sr[j] = e;
+          sum += e;
+        }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      for (int j = lane; j < nt; j += 32) {
-        const float p = Sr[j] / sum;
-        Sr[j] = p;
-        if (probs_out) probs_out[row * nt + j] = p;
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        for (int j = lane; j < nt; j += 32) {
+          const float p = Sr[j] / sum;
+          Sr[j] = p;
+          if (probs_out) probs_out[row * nt + j] = p;
+        }
       }
       __syncwarp();
       // Phase 3: selection threshold as (level v_f, ties c_f).

@@ -85,6 +85,12 @@ typedef struct {
                               tokens, k_head = ceil(sum n_c b_c / sum n_c), and
                               rows with b_c < k_head keep their first
                               min(k_head, Nt) tiles; ignored if !use_scores */
+  const float *block_scores; /* device fp32 [B, heads, Nt, Nt] or NULL. When set
+                              (and use_scores), the selection runs on these
+                              rows instead of the pooled-score probabilities,
+                              e.g. the masses of sta_attn_fwd_block_mass;
+                              values are clamped to [0, 1] and q_tiled, k_tiled
+                              are not read */
 } sta_mask_params;
 
 /* Number of tiles per head (Nt) and padded rows per head (Lpad) of a grid;
@@ -173,6 +179,27 @@ sta_status sta_build_mask_noalloc(const void *q_tiled, const void *k_tiled, int3
                                   int32_t d, sta_grid g, const sta_mask_params *p, int32_t *row_ptr,
                                   int32_t *col_idx, int64_t *nnz_dev, uint8_t *block_mask,
                                   float *block_probs, sta_stream_t stream);
+
+/* sta_attn_fwd_block_mass -- sta_attn_fwd that also measures the exact block
+ * importance of every listed pair under a cached log-sum-exp (AdaSpa
+ * abstract: block importance computed during a full-attention step with the
+ * LSE cached from an earlier step, then reused by the sparse steps):
+ *   mass(qt, kt) = (1/n_q) sum_i sum_j exp(sm_scale * q_i . k_j - lse_cached_i)
+ * over the real query tokens i of qt (n_q of them) and the real key tokens j
+ * of kt; a token whose cached LSE is -inf contributes nothing. With the exact
+ * LSE of the same inputs and every tile listed, each row sums to one.
+ *   lse_cached : fp32 [B, heads, Lpad] (natural log), e.g. the lse output of
+ *                an earlier call on the same layer
+ *   block_mass : fp32 [B, heads, Nt, Nt], written: listed pairs get their
+ *                mass, every other entry 0
+ * All other arguments, outputs and errors are those of sta_attn_fwd. The
+ * masses are accumulated in fp32 (per-row sums relative to the running max,
+ * one exp2 per row and tile, two adds per pair onto zero: deterministic). */
+sta_status sta_attn_fwd_block_mass(const void *q, const void *k, const void *v, void *o, float *lse,
+                                   const int32_t *row_ptr, const int32_t *col_idx,
+                                   const float *lse_cached, float *block_mass, int32_t B,
+                                   int32_t heads, int32_t d, sta_grid g, float sm_scale,
+                                   sta_stream_t stream);
 
 /* Reads and clears the device error word of the current device after
  * synchronising `stream`. STA_OK if no device-side fault was recorded. */

@@ -481,3 +481,92 @@ def test_build_mask_head_floor_720p_sampled_heads(sta, gp):
         for qtile in range(0, nt, 7):
             r = h * nt + qtile
             assert np.array_equal(ci[rp[r]:rp[r + 1]], np.nonzero(keep[qtile])[0]), (h, qtile, k_head)
+
+
+# ---------------------------------------- LSE-cached block importance (AdaSpa f3)
+def _mass_check(sta, gp, qt, kt, vt, rp_t, ci_t, lse_cached, B, Hh, d, T, H, W, rows, sm_scale=0.0):
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    o_ref, lse_ref = gp.attn(qt, kt, vt, rp_t, ci_t, B, Hh, d, g, sm_scale)
+    o = torch.full_like(qt, float("nan"))
+    lse = torch.full(qt.shape[:3], float("nan"), dtype=torch.float32, device=qt.device)
+    mass = torch.full((B, Hh, nt, nt), float("nan"), dtype=torch.float32, device=qt.device)
+    sta.sta_attn_fwd_block_mass(qt, kt, vt, o, lse, rp_t, ci_t, lse_cached, mass, B, Hh, d, g, sm_scale)
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    # the attention outputs are those of sta_attn_fwd, bit for bit
+    assert torch.equal(o.view(torch.int16), o_ref.view(torch.int16))
+    assert torch.equal(lse, lse_ref)
+    rp, ci = rp_t.cpu().numpy(), ci_t.cpu().numpy()
+    res = O.block_mass(gp.to_np64(qt), gp.to_np64(kt), lse_cached.double().cpu().numpy(), rp, ci, T, H, W,
+                       sm_scale, rows)
+    m_np = mass.view(-1, nt).cpu().numpy()
+    listed = np.zeros_like(m_np, dtype=bool)
+    for r in range(m_np.shape[0]):
+        listed[r, ci[rp[r]:rp[r + 1]]] = True
+    assert np.all(m_np[~listed] == 0)
+    for r, (tiles, want) in res.items():
+        got = m_np[r, tiles]
+        assert np.allclose(got, want, rtol=2e-4, atol=1e-9), (r, np.abs(got - want).max())
+    return mass, lse
+
+
+def test_block_mass_tiny_dense_exact_lse(sta, gp):
+    """Dense list and the exact LSE of the same inputs: masses match the
+    oracle and every row sums to one."""
+    cfg = CONFIGS[0]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = (x.cuda() for x in make_qkv(cfg, device="cpu"))
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    rp, ci = _custom_csr(np.ones((B, Hh, nt, nt), dtype=bool))
+    _, lse_exact = gp.attn(qt, kt, vt, rp, ci, B, Hh, d, g)
+    mass, _ = _mass_check(sta, gp, qt, kt, vt, rp, ci, lse_exact, B, Hh, d, T, H, W, range(B * Hh * nt))
+    sums = mass.sum(-1).cpu().numpy()
+    assert np.allclose(sums, 1.0, atol=1e-4)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_block_mass_ragged_sparse_stale_lse(sta, gp, d):
+    """Ragged grid, random lists (odd tile count), a cached LSE from perturbed
+    inputs; then the selection on the masses is bit-exact."""
+    T, H, W, Hh, B = 3, 19, 37, 2, 2
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = _structured(T, H, W, Hh, d, seed=31, B=B)
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    rng = np.random.default_rng(d + 1)
+    mask = rng.random((B, Hh, nt, nt)) < 0.4
+    rp, ci = _custom_csr(mask)
+    q2 = (q.float() * 0.95 + 0.3 * torch.randn(q.shape, device="cuda")).to(torch.bfloat16)
+    _, lse_stale = gp.attn(gp.reorder(q2, B, Hh, d, g), kt, vt, rp, ci, B, Hh, d, g)
+    mass, _ = _mass_check(sta, gp, qt, kt, vt, rp, ci, lse_stale, B, Hh, d, T, H, W, range(B * Hh * nt))
+    # selection on the exact masses
+    params = sta.mask_params(0.8, 2, True, block_scores=mass)
+    bufs = gp.build(None, None, B, Hh, d, g, params)
+    rp_g, ci_g, nnz = gp.csr_np(bufs)
+    used = np.clip(mass.cpu().numpy(), 0.0, 1.0).astype(np.float32)
+    assert np.array_equal(bufs.block_probs.cpu().numpy(), used)
+    rp_o, ci_o = O.mask_to_csr(O.select(used.astype(np.float64), 0.8, 2))
+    assert np.array_equal(rp_g, rp_o) and np.array_equal(ci_g, ci_o)
+
+
+def test_block_mass_720p_dense_sampled_rows(sta, gp):
+    """The headline layer, dense list, exact LSE: sampled rows of masses."""
+    cfg = CONFIGS[2]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = make_qkv(cfg, device="cuda")
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    del q, k, v
+    R = B * Hh * nt
+    rp = (torch.arange(R + 1, device="cuda", dtype=torch.int64) * nt).to(torch.int32)
+    ci = torch.arange(nt, device="cuda", dtype=torch.int32).repeat(R)
+    _, lse_exact = gp.attn(qt, kt, vt, rp, ci, B, Hh, d, g)
+    rng = np.random.default_rng(9)
+    rows = sorted(rng.choice(R, 4, replace=False).tolist())
+    mass, _ = _mass_check(sta, gp, qt, kt, vt, rp, ci, lse_exact, B, Hh, d, T, H, W, rows)
+    sums = mass.view(-1, nt)[torch.tensor(rows, device="cuda")].sum(-1).cpu().numpy()
+    assert np.allclose(sums, 1.0, atol=1e-4)
