@@ -75,6 +75,8 @@ _lib.sta_attn_fwd.restype = ctypes.c_int
 _lib.sta_attn_fwd_block_mass.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, Grid,
                                          _f32, _vp]
 _lib.sta_attn_fwd_block_mass.restype = ctypes.c_int
+_lib.sta_selftest_wait_timeout.argtypes = [_i64, _vp]
+_lib.sta_selftest_wait_timeout.restype = ctypes.c_int
 _lib.sta_get_device_error.argtypes = [_vp]
 _lib.sta_get_device_error.restype = ctypes.c_int
 _lib.sta_status_string.argtypes = [ctypes.c_int]
@@ -177,6 +179,10 @@ def sta_attn_fwd_block_mass(q, k, v, o, lse, row_ptr, col_idx, lse_cached, block
                                         _ptr(col_idx), _ptr(lse_cached), _ptr(block_mass), B, heads, d, g,
                                         float(sm_scale), _stream(stream)),
            "sta_attn_fwd_block_mass")
+
+
+def sta_selftest_wait_timeout(limit_cycles=2000000, stream=None):
+    _check(_lib.sta_selftest_wait_timeout(int(limit_cycles), _stream(stream)), "sta_selftest_wait_timeout")
 
 
 def sta_get_device_error(stream=None):

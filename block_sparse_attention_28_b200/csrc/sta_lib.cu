@@ -105,6 +105,19 @@ bool device_is_sm100() {
   return major == 10 && minor == 0;
 }
 
+// One thread waits, with the pipeline's bounded wait, on a barrier that
+// expects one arrival that never comes.
+__global__ void selftest_wait_kernel(long long limit) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar, 1);
+    abort_flag = 0u;
+    tc::fence_barrier_init();
+    tc::mbar_wait(&bar, 0, &abort_flag, limit);
+  }
+}
+
 template <int D>
 sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads,
                         const Geo &g, const sta_mask_params *p, int32_t *row_ptr, int32_t *col_idx,
@@ -289,6 +302,14 @@ sta_status sta_attn_fwd_block_mass(const void *q, const void *k, const void *v, 
                                              lse_cached, block_mass)
                     : launch_attn<64, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s,
                                             lse_cached, block_mass);
+}
+
+sta_status sta_selftest_wait_timeout(int64_t limit_cycles, sta_stream_t stream) {
+  if (limit_cycles < 1000 || limit_cycles > 2000000000LL) return STA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  selftest_wait_kernel<<<1, 32, 0, s>>>((long long)limit_cycles);
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
 }
 
 sta_status sta_get_device_error(sta_stream_t stream) {

@@ -201,6 +201,15 @@ sta_status sta_attn_fwd_block_mass(const void *q, const void *k, const void *v, 
                                    int32_t heads, int32_t d, sta_grid g, float sm_scale,
                                    sta_stream_t stream);
 
+/* sta_selftest_wait_timeout -- exercises the bounded wait that every pipeline
+ * stage of sta_attn_fwd uses, without a fault: one thread initialises a
+ * shared-memory mbarrier that nothing will ever complete, waits on it for at
+ * most `limit_cycles` SM cycles (1e3 .. 2e9), records STA_ERR_TIMEOUT in the
+ * device error word and returns. The pages have no counterpart; it lets a
+ * caller check that a stalled pipeline is reported through
+ * sta_get_device_error() and leaves the context usable. */
+sta_status sta_selftest_wait_timeout(int64_t limit_cycles, sta_stream_t stream);
+
 /* Reads and clears the device error word of the current device after
  * synchronising `stream`. STA_OK if no device-side fault was recorded. */
 sta_status sta_get_device_error(sta_stream_t stream);

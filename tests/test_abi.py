@@ -81,3 +81,8 @@ def test_status_strings(sta):
     for s in range(7):
         assert sta.sta_status_string(s)
     assert "out of range" in sta.sta_status_string(sta.STA_ERR_BAD_MASK)
+
+
+def test_selftest_limit_is_checked_on_the_host(sta):
+    assert sta._lib.sta_selftest_wait_timeout(10, None) == sta.STA_ERR_INVALID_ARG
+    assert sta._lib.sta_selftest_wait_timeout(3_000_000_000, None) == sta.STA_ERR_INVALID_ARG

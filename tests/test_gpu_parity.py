@@ -570,3 +570,14 @@ def test_block_mass_720p_dense_sampled_rows(sta, gp):
     mass, _ = _mass_check(sta, gp, qt, kt, vt, rp, ci, lse_exact, B, Hh, d, T, H, W, rows)
     sums = mass.view(-1, nt)[torch.tensor(rows, device="cuda")].sum(-1).cpu().numpy()
     assert np.allclose(sums, 1.0, atol=1e-4)
+
+
+# ------------------------------------------------------- failure detection
+def test_bounded_wait_reports_timeout_and_context_survives(sta, gp):
+    """The pipeline's bounded wait, on a barrier nothing completes, gives up
+    after its limit and reports STA_ERR_TIMEOUT; the context keeps working."""
+    sta.sta_get_device_error()
+    sta.sta_selftest_wait_timeout(2_000_000)  # about a millisecond of SM cycles
+    assert sta.sta_get_device_error() == sta.STA_ERR_TIMEOUT
+    assert sta.sta_get_device_error() == sta.STA_OK
+    test_attn_tiny_config(sta, gp)  # a full attention call still runs and matches
