@@ -15,6 +15,7 @@ Sources (pages on block-sparse attention for video diffusion transformers):
   * SCOPE review (Eqs. (7)-(8) as quoted; abstract): hybrid top-p / fixed
     top-k selection; Eqs. (9)-(10): the online per-head top-k floor.
   * AdaSpa (abstract): exact block importance from a cached log-sum-exp.
+  * Compact Attention Figs. 3-5: recall-driven offline window search.
 
 Parity pins: every function here is checked in tests/test_oracle_*.py
 against closed forms, textbook routines (torch SDPA in fp64, scipy
@@ -41,4 +42,6 @@ from .sta_oracle import (  # noqa: F401
     attention_rows,
     attention_all,
     block_mass,
+    search_windows,
+    SEARCH_MOVES,
 )

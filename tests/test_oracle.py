@@ -465,3 +465,73 @@ def test_block_mass_with_stale_lse_scales_by_the_lse_gap():
     b = O.block_mass(qt, kt, lse + 0.5, rp, ci, T, H, W, 0.0, range(nt))
     for r in range(nt):
         assert np.allclose(b[r][1], a[r][1] * math.exp(-0.5), rtol=1e-13)
+
+
+# ------------------------------------------------ recall-driven window search (f2)
+def _coverage(win, group_lo, T, H, W, mass):
+    m = O.window_mask(np.asarray(win)[None], group_lo, T, H, W)[0]
+    w = np.floor(np.clip(mass, 0, 1) * 2 ** 24).astype(np.int64)
+    return m, int(w[m].sum()), int(w.sum())
+
+
+def test_window_search_keeps_everything_at_full_recall_with_dense_mass():
+    """tau = 1 and every pair carries mass: no pair can go, the windows stay full."""
+    rng = np.random.default_rng(1)
+    T, H, W = 3, 24, 32
+    nh, nw, nt, _ = O.tile_grid(T, H, W)
+    mass = rng.random((nt, nt)) + 0.1
+    mass /= mass.sum(1, keepdims=True)
+    win, st = O.search_windows(mass, T, H, W, (0, 1), 1.0, 1.0)
+    assert st["steps"] == 0 and st["recall"] == 1.0 and st["density"] == 1.0
+    assert (win == np.array([nh - 1, nw - 1, nh - 1, nw - 1])).all()
+
+
+def test_window_search_diagonal_mass_shrinks_to_the_own_tile():
+    """All mass on the query's own tile: at tau = 1 the search removes every
+    other pair (closed form: density 1/Nt, recall 1)."""
+    T, H, W = 3, 24, 32
+    nt = O.tile_grid(T, H, W)[2]
+    mass = np.eye(nt)
+    win, st = O.search_windows(mass, T, H, W, (0, 1), 1.0, 1.0)
+    m, cov, tot = _coverage(win, (0, 1), T, H, W, mass)
+    assert st["recall"] == 1.0 and cov == tot
+    assert m.sum() == nt and np.array_equal(m, np.eye(nt, dtype=bool))
+
+
+def test_window_search_zero_target_removes_everything():
+    rng = np.random.default_rng(2)
+    T, H, W = 2, 16, 24
+    nt = O.tile_grid(T, H, W)[2]
+    mass = rng.random((nt, nt))
+    win, st = O.search_windows(mass, T, H, W, (0, 1), 0.0, 0.0)
+    assert st["density"] == 0.0
+    assert (win == -1).any(axis=1).all() or (win[:, [0, 2]] == -1).all()
+
+
+def test_window_search_result_is_feasible_and_locally_final():
+    """On local-looking masses: the final recall (recomputed from the windows)
+    meets tau, and no single move of the move set uncovers a pair while still
+    meeting tau (checked by direct enumeration)."""
+    T, H, W = 4, 24, 40
+    nh, nw, nt, _ = O.tile_grid(T, H, W)
+    idx = np.arange(nt)
+    t, y, x = idx // (nh * nw), (idx // nw) % nh, idx % nw
+    d2 = (t[:, None] - t[None]) ** 2 * 2.0 + (y[:, None] - y[None]) ** 2 + 0.3 * (x[:, None] - x[None]) ** 2
+    mass = np.exp(-d2)
+    mass /= mass.sum(1, keepdims=True)
+    group_lo = (0, 1, 3)
+    for tau, lam in ((0.9, 1.0), (0.97, 0.5), (0.8, 2.0)):
+        win, st = O.search_windows(mass, T, H, W, group_lo, tau, lam)
+        m, cov, tot = _coverage(win, group_lo, T, H, W, mass)
+        thr = math.ceil(float(np.float32(tau)) * tot)
+        assert cov == st["covered"] and cov >= thr
+        assert st["density"] == m.mean() < 1.0
+        for g in range(len(group_lo)):
+            for ext in O.SEARCH_MOVES:
+                cand = win.astype(np.int64).copy()
+                if any(cand[g, e] <= -1 for e in ext):
+                    continue
+                for e in ext:
+                    cand[g, e] -= 1
+                m2, cov2, _ = _coverage(cand, group_lo, T, H, W, mass)
+                assert (m & ~m2).sum() == 0 or cov2 < thr
