@@ -75,6 +75,9 @@ _lib.sta_attn_fwd.restype = ctypes.c_int
 _lib.sta_attn_fwd_block_mass.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, Grid,
                                          _f32, _vp]
 _lib.sta_attn_fwd_block_mass.restype = ctypes.c_int
+_lib.sta_search_windows.argtypes = [_vp, _i32, _i32, Grid, _i32, ctypes.POINTER(ctypes.c_int32), _f32, _f32,
+                                    _vp, _vp, _vp]
+_lib.sta_search_windows.restype = ctypes.c_int
 _lib.sta_selftest_wait_timeout.argtypes = [_i64, _vp]
 _lib.sta_selftest_wait_timeout.restype = ctypes.c_int
 _lib.sta_get_device_error.argtypes = [_vp]
@@ -179,6 +182,13 @@ def sta_attn_fwd_block_mass(q, k, v, o, lse, row_ptr, col_idx, lse_cached, block
                                         _ptr(col_idx), _ptr(lse_cached), _ptr(block_mass), B, heads, d, g,
                                         float(sm_scale), _stream(stream)),
            "sta_attn_fwd_block_mass")
+
+
+def sta_search_windows(block_mass, B, heads, g, group_lo, tau, lam, windows, stats=None, stream=None):
+    lo = (ctypes.c_int32 * len(group_lo))(*[int(v) for v in group_lo])
+    _check(_lib.sta_search_windows(_ptr(block_mass), B, heads, g, len(group_lo), lo, float(tau), float(lam),
+                                   _ptr(windows), _ptr(stats), _stream(stream)),
+           "sta_search_windows")
 
 
 def sta_selftest_wait_timeout(limit_cycles=2000000, stream=None):

@@ -9,6 +9,7 @@
 #include "sta_common.cuh"
 #include "sta_mask.cuh"
 #include "sta_reorder.cuh"
+#include "sta_search.cuh"
 
 using namespace sta;
 
@@ -302,6 +303,32 @@ sta_status sta_attn_fwd_block_mass(const void *q, const void *k, const void *v, 
                                              lse_cached, block_mass)
                     : launch_attn<64, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s,
                                             lse_cached, block_mass);
+}
+
+sta_status sta_search_windows(const float *block_mass, int32_t B, int32_t heads, sta_grid g,
+                              int32_t num_groups, const int32_t *group_lo, float tau, float lambda,
+                              int32_t *windows, float *stats, sta_stream_t stream) {
+  Geo geo;
+  if (B <= 0 || heads <= 0 || !make_geo(g, &geo)) return STA_ERR_INVALID_ARG;
+  if (block_mass == nullptr || windows == nullptr || group_lo == nullptr) return STA_ERR_INVALID_ARG;
+  if (num_groups < 1 || num_groups > STA_MAX_GROUPS || group_lo[0] != 0) return STA_ERR_INVALID_ARG;
+  for (int i = 1; i < num_groups; ++i)
+    if (group_lo[i] <= group_lo[i - 1]) return STA_ERR_INVALID_ARG;
+  if (!(tau >= 0.0f && tau <= 1.0f) || !(lambda >= 0.0f)) return STA_ERR_INVALID_ARG;
+  if ((long long)B * heads > 65535 || geo.T >= 4096 || geo.NH >= 1024 || geo.NW >= 1024)
+    return STA_ERR_UNSUPPORTED;
+  const size_t smem = (size_t)(geo.Nt + geo.T) * sizeof(uint32_t);
+  if (smem > 200 * 1024) return STA_ERR_UNSUPPORTED;
+  if (smem > 48 * 1024)
+    STA_CUDA_TRY(cudaFuncSetAttribute(search_windows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem));
+  GroupLo glo;
+  for (int i = 0; i < STA_MAX_GROUPS; ++i) glo.v[i] = (i < num_groups) ? group_lo[i] : 0x7fffffff;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  search_windows_kernel<<<(unsigned)(B * heads), SEARCH_THREADS, smem, s>>>(block_mass, geo, num_groups, glo,
+                                                                           tau, lambda, windows, stats);
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
 }
 
 sta_status sta_selftest_wait_timeout(int64_t limit_cycles, sta_stream_t stream) {

@@ -201,6 +201,33 @@ sta_status sta_attn_fwd_block_mass(const void *q, const void *k, const void *v, 
                                    int32_t heads, int32_t d, sta_grid g, float sm_scale,
                                    sta_stream_t stream);
 
+/* sta_search_windows -- recall-driven offline search of the dual windows
+ * (Compact Attention Fig. 3: the windows are shrunk iteratively under a recall
+ * target tau and a cost weight lambda, and the configurations are stored for
+ * reuse; Fig. 4: the search starts from full coverage in every
+ * temporal-distance group; Fig. 5(c): recall target vs achieved sparsity).
+ * One search per (b, h) on its block importances, e.g. the masses of
+ * sta_attn_fwd_block_mass over a dense list with the exact LSE:
+ *   masses w = floor(min(max(m, 0), 1) * 2^24); W = sum of w; the recall of a
+ *   window set is the covered w over W;
+ *   start: (ry1, rx1, ry2, rx2) = (NH-1, NW-1, NH-1, NW-1) in every group;
+ *   moves, per group g in order: ry1-1, rx1-1, ry2-1, rx2-1, (ry1-1, ry2-1),
+ *   (rx1-1, rx2-1); an extent never goes below -1;
+ *   each step applies, among the moves that uncover at least one pair and
+ *   keep covered >= ceil(double(tau) * W), the one with the largest
+ *   J = removed / Nt^2 - lambda * lost / W (ties to the lowest g*6 + m), and
+ *   the search stops when no move is left.
+ *   block_mass : device fp32 [B, heads, Nt, Nt]
+ *   group_lo   : HOST int32 [num_groups], ascending, group_lo[0] == 0
+ *   tau in [0, 1]; lambda >= 0
+ *   windows    : device int32 [B*heads][num_groups][4], written (the layout of
+ *                sta_mask_params.windows for one batch entry)
+ *   stats      : optional device fp32 [B*heads][2] = (recall, density); NULL ok
+ * Deterministic: integer sums, one double comparison per move. */
+sta_status sta_search_windows(const float *block_mass, int32_t B, int32_t heads, sta_grid g,
+                              int32_t num_groups, const int32_t *group_lo, float tau, float lambda,
+                              int32_t *windows, float *stats, sta_stream_t stream);
+
 /* sta_selftest_wait_timeout -- exercises the bounded wait that every pipeline
  * stage of sta_attn_fwd uses, without a fault: one thread initialises a
  * shared-memory mbarrier that nothing will ever complete, waits on it for at

@@ -572,6 +572,100 @@ def test_block_mass_720p_dense_sampled_rows(sta, gp):
     assert np.allclose(sums, 1.0, atol=1e-4)
 
 
+# ------------------------------------------ recall-driven window search (f2)
+def _local_masses(T, H, W, shapes):
+    """One [Nt, Nt] row-normalised mass per (st, sy, sx) spread of a Gaussian
+    in tile distance (local-looking heads of different shape)."""
+    nh, nw, nt, _ = O.tile_grid(T, H, W)
+    idx = np.arange(nt)
+    t, y, x = idx // (nh * nw), (idx // nw) % nh, idx % nw
+    out = []
+    for st, sy, sx in shapes:
+        d2 = st * (t[:, None] - t[None]) ** 2 + sy * (y[:, None] - y[None]) ** 2 + sx * (x[:, None] - x[None]) ** 2
+        m = np.exp(-d2)
+        out.append(m / m.sum(1, keepdims=True))
+    return np.stack(out)
+
+
+def _search_check(sta, masses32, B, Hh, T, H, W, group_lo, tau, lam, heads=None):
+    """Run the GPU search on fp32 masses [B*Hh, Nt, Nt]; compare the windows
+    (exactly) and the stats with the oracle on the same fp32 values."""
+    g = sta.grid(T, H, W)
+    G = len(group_lo)
+    mass_t = torch.from_numpy(masses32).cuda()
+    win = torch.full((B * Hh, G, 4), 12345, dtype=torch.int32, device="cuda")
+    stats = torch.full((B * Hh, 2), float("nan"), dtype=torch.float32, device="cuda")
+    sta.sta_search_windows(mass_t, B, Hh, g, group_lo, tau, lam, win, stats)
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    win_np, st_np = win.cpu().numpy(), stats.cpu().numpy()
+    for bh in (range(B * Hh) if heads is None else heads):
+        want, st = O.search_windows(masses32[bh].astype(np.float64), T, H, W, group_lo, tau, lam)
+        assert np.array_equal(win_np[bh], want), (bh, win_np[bh].tolist(), want.tolist())
+        assert st_np[bh, 0] == np.float32(st["recall"]), (bh, st_np[bh, 0], st["recall"])
+        assert st_np[bh, 1] == np.float32(st["density"]), (bh, st_np[bh, 1], st["density"])
+    return win_np, st_np
+
+
+@pytest.mark.parametrize("tau,lam", [(0.9, 1.0), (0.97, 0.5), (0.8, 2.0), (1.0, 1.0), (0.0, 0.0)])
+def test_search_windows_synthetic_heads(sta, tau, lam):
+    """Ragged grid, three groups, local heads of several shapes plus the
+    degenerate ones (all mass on the own tile; no mass at all; uniform)."""
+    T, H, W = 4, 24, 40
+    nt = O.tile_grid(T, H, W)[2]
+    local = _local_masses(T, H, W, [(2.0, 1.0, 0.3), (0.2, 0.05, 2.0), (5.0, 3.0, 3.0), (0.05, 0.5, 0.01)])
+    extra = np.stack([np.eye(nt), np.zeros((nt, nt)), np.full((nt, nt), 1.0 / nt)])
+    masses = np.concatenate([local, extra]).astype(np.float32)  # B = 1, 7 heads
+    _search_check(sta, masses, 1, masses.shape[0], T, H, W, (0, 1, 3), tau, lam)
+
+
+def test_search_windows_batch_and_single_group(sta):
+    """B = 2 with one open-ended group on an odd tile grid."""
+    T, H, W = 3, 19, 37
+    masses = _local_masses(T, H, W, [(1.0, 0.5, 0.5), (0.1, 2.0, 0.1), (3.0, 0.02, 0.02), (0.5, 0.5, 0.05)])
+    _search_check(sta, masses.astype(np.float32), 2, 2, T, H, W, (0,), 0.9, 1.0)
+
+
+def test_search_windows_on_480p_block_masses(sta, gp):
+    """The 480p layer: exact block masses of the dense attention (fused LSE
+    path), then the search for every head; sampled heads match the oracle
+    window for window, and every head's windows meet the recall target."""
+    cfg = CONFIGS[1]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = make_qkv(cfg, device="cuda")
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    del q, k, v
+    R = B * Hh * nt
+    rp = (torch.arange(R + 1, device="cuda", dtype=torch.int64) * nt).to(torch.int32)
+    ci = torch.arange(nt, device="cuda", dtype=torch.int32).repeat(R)
+    _, lse_exact = gp.attn(qt, kt, vt, rp, ci, B, Hh, d, g)
+    o = torch.empty_like(qt)
+    lse = torch.empty_like(lse_exact)
+    mass = torch.empty((B, Hh, nt, nt), dtype=torch.float32, device="cuda")
+    sta.sta_attn_fwd_block_mass(qt, kt, vt, o, lse, rp, ci, lse_exact, mass, B, Hh, d, g)
+    torch.cuda.synchronize()
+    masses = mass.view(B * Hh, nt, nt).cpu().numpy()
+    tau, lam = 0.9, 1.0
+    win, st = _search_check(sta, masses, B, Hh, T, H, W, cfg.group_lo, tau, lam, heads=(0, 17, 39))
+    for bh in range(B * Hh):
+        keep = O.window_mask(win[bh][None], cfg.group_lo, T, H, W)[0]
+        w = np.floor(np.clip(masses[bh].astype(np.float64), 0, 1) * 2 ** 24)
+        assert w[keep].sum() >= math.ceil(float(np.float32(tau)) * w.sum())
+        assert st[bh, 1] == np.float32(keep.mean())
+
+
+def test_search_windows_rejects_bad_groups(sta):
+    g = sta.grid(4, 24, 40)
+    nt = O.tile_grid(4, 24, 40)[2]
+    m = torch.zeros((1, nt, nt), device="cuda")
+    out = torch.empty((1, 2, 4), dtype=torch.int32, device="cuda")
+    for lo, tau in (((1, 2), 0.9), ((0, 0), 0.9), ((0, 2), 1.5), ((0,) * 9, 0.9)):
+        with pytest.raises(sta.StaError):
+            sta.sta_search_windows(m, 1, 1, g, lo, tau, 1.0, out)
+
+
 # ------------------------------------------------------- failure detection
 def test_bounded_wait_reports_timeout_and_context_survives(sta, gp):
     """The pipeline's bounded wait, on a barrier nothing completes, gives up
