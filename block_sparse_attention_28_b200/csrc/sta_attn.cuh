@@ -30,9 +30,13 @@ namespace attn {
 constexpr int NUM_THREADS = 192;
 constexpr int WARP_PRODUCER = 4;
 constexpr int WARP_MMA = 5;
+// Union-list entry: key tile (bits 0-19; the host keeps Nt <= 2^20), the
+// valid extent of a partial key tile (rows - 1 in bits 20-22, columns - 1 in
+// bits 23-25, flag bit 26), and the two halves' membership flags.
+constexpr uint32_t KT_MASK = (1u << 20) - 1u;
+constexpr uint32_t EXT_PARTIAL = 1u << 26;
 constexpr uint32_t FLAG_A = 1u << 30;
 constexpr uint32_t FLAG_B = 1u << 31;
-constexpr uint32_t KT_MASK = FLAG_A - 1u;
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t O_COL = 128;
 constexpr long long WAIT_LIMIT = 2000000000LL;   // SM cycles (~1 s)
@@ -44,6 +48,9 @@ constexpr int MIN_BLOCKS_PER_SM = 2;             // two CTAs share an SM: one's 
 #define STA_EXP2_POLY_EVERY 0                    // every k-th column pair uses ex2_poly
 #endif
 
+#ifndef STA_ATTN_EXT_LIST
+#define STA_ATTN_EXT_LIST 1
+#endif
 #ifndef STA_ATTN_NSK
 #define STA_ATTN_NSK 2                           // K ring stages at d = 128
 #endif
@@ -216,6 +223,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   tc::fence_after();
   const uint32_t tmem = misc[0];
   const int n = (int)misc[1];
+#if STA_ATTN_EXT_LIST
+  // Mark key tiles cut by the grid edge once per entry, so that the softmax
+  // loop needs no division to find them.
+  for (int i = tid; i < n; i += NUM_THREADS) {
+    const uint32_t e = U[i];
+    const int kt = (int)(e & KT_MASK);
+    const int rem = kt % (g.NH * g.NW);
+    const int ty = rem / g.NW, tx = rem - ty * g.NW;
+    const int vy = valid_extent(g.H, ty), vx = valid_extent(g.W, tx);
+    if (vy < 8 || vx < 8) U[i] = e | EXT_PARTIAL | ((uint32_t)(vy - 1) << 20) | ((uint32_t)(vx - 1) << 23);
+  }
+  __syncthreads();
+#endif
 
   if (warp == WARP_PRODUCER) {
     // ------------------------------------------------------ TMA producer
@@ -363,10 +383,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         // keys of partial tiles beyond the grid edge
         const int kt = (int)(e & KT_MASK);
+#if STA_ATTN_EXT_LIST
+        if (e & EXT_PARTIAL) {
+          const int vy = (int)((e >> 20) & 7u) + 1, vx = (int)((e >> 23) & 7u) + 1;
+#else
         const int rem = kt % (g.NH * g.NW);
         const int ty = rem / g.NW, tx = rem - ty * g.NW;
         const int vy = valid_extent(g.H, ty), vx = valid_extent(g.W, tx);
         if (vy < 8 || vx < 8) {
+#endif
 #pragma unroll
           for (int c = 0; c < 64; ++c)
             if ((c >> 3) >= vy || (c & 7) >= vx) s[c] = -INFINITY;

@@ -38,6 +38,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0u;
 }
 
+#ifndef STA_WAIT_SLEEP_NS
+#define STA_WAIT_SLEEP_NS 1000000
+#endif
+// try_wait with a suspend-time hint: a waiting thread sleeps until the phase
+// completes (or the hint in ns runs out) instead of spinning, so waiting
+// warps take no issue slots from the softmax warps of their SM sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity) {
+#if STA_WAIT_SLEEP_NS > 0
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(STA_WAIT_SLEEP_NS)
+      : "memory");
+  return ok != 0u;
+#else
+  return mbar_try_wait(bar, parity);
+#endif
+}
+
 // Bounded wait: gives up after `limit` SM cycles (or when another role has
 // raised `abort`), records DEV_ERR_TIMEOUT and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile uint32_t *abort,
@@ -45,7 +67,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity)) return true;
     if (abort != nullptr && *abort) return false;
     if (clock64() - t0 > limit) {
       if (abort != nullptr) *abort = 1u;
