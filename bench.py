@@ -6,6 +6,7 @@ windows, ~15% density): sta_reorder of Q, K, V -> sta_build_mask ->
 sta_attn_fwd -> sta_reorder of O back to raster order.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  python bench.py --search-curve [--config-index I]   (window search, recall vs density)
 
 Rank 0 prints one JSON line. Under torchrun every rank runs its own layer
 (independent problems, no collective on the data path: weak scaling); the
@@ -313,6 +314,57 @@ class Layer:
         return tot_ab / (2.0 * tot_u) if tot_u else 1.0, tot_u
 
 
+def search_curve(sta, cfg_index, dev, taus=(0.8, 0.9, 0.95, 0.99), lam=1.0):
+    """Recall target against achieved density (Compact Attention Fig. 5(c)):
+    exact block masses of the dense layer (dense list, exact LSE), the window
+    search for every head at each target, then the window-only mask built from
+    the searched windows and the attention on it, compared with the dense
+    output (relative Frobenius error over the whole layer)."""
+    cfg = CONFIGS[cfg_index]
+    layer = Layer(sta, cfg, dev, cfg_index=cfg_index)
+    layer.reorder_in()
+    B, Hh, d, g, nt = layer.B, layer.Hh, layer.d, layer.g, layer.nt
+    R = B * Hh * nt
+    rp = (torch.arange(R + 1, device=dev, dtype=torch.int64) * nt).to(torch.int32)
+    ci = torch.arange(nt, device=dev, dtype=torch.int32).repeat(R)
+    lse = torch.empty((B, Hh, layer.lpad), dtype=torch.float32, device=dev)
+    sta.sta_attn_fwd(layer.qt, layer.kt, layer.vt, layer.ot, lse, rp, ci, B, Hh, d, g)
+    o_dense = layer.ot.float()
+    mass = torch.empty((B, Hh, nt, nt), dtype=torch.float32, device=dev)
+    lse2 = torch.empty_like(lse)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    sta.sta_attn_fwd_block_mass(layer.qt, layer.kt, layer.vt, layer.ot, lse2, rp, ci, lse, mass, B, Hh, d, g)
+    e1.record()
+    torch.cuda.synchronize()
+    mass_ms = e0.elapsed_time(e1)
+    del rp, ci
+    G = len(cfg.group_lo)
+    rows = []
+    for tau in taus:
+        win = torch.empty((B * Hh, G, 4), dtype=torch.int32, device=dev)
+        stats = torch.empty((B * Hh, 2), dtype=torch.float32, device=dev)
+        sta.sta_search_windows(mass, B, Hh, g, cfg.group_lo, tau, lam, win, stats)  # warm-up
+        e0.record()
+        sta.sta_search_windows(mass, B, Hh, g, cfg.group_lo, tau, lam, win, stats)
+        e1.record()
+        torch.cuda.synchronize()
+        search_ms = e0.elapsed_time(e1)
+        st = stats.cpu().numpy()
+        params = sta.mask_params(0.0, 0, False, 0.0, cfg.group_lo, win[:Hh])
+        sta.build_mask(layer.qt, layer.kt, B, Hh, d, g, params, layer.bufs)
+        sta.sta_attn_fwd(layer.qt, layer.kt, layer.vt, layer.ot, None, layer.bufs.row_ptr,
+                         layer.bufs.col_idx, B, Hh, d, g)
+        torch.cuda.synchronize()
+        rel = float(torch.linalg.vector_norm(layer.ot.float() - o_dense) / torch.linalg.vector_norm(o_dense))
+        rows.append({"tau": tau, "lambda": lam, "recall_mean": float(st[:, 0].mean()),
+                     "recall_min": float(st[:, 0].min()), "density": layer.kept_pairs() / (R * nt),
+                     "density_min_head": float(st[:, 1].min()), "density_max_head": float(st[:, 1].max()),
+                     "attn_rel_err_vs_dense": rel, "search_ms": search_ms})
+    assert sta.sta_get_device_error() == sta.STA_OK
+    return {"workload": cfg.name, "block_mass_ms": mass_ms, "curve": rows}
+
+
 def cpu_oracle_sample(cfg, layer, budget_s, rows_per_head=8, max_heads=None):
     """Time the oracle (as it stands) on a bounded sample of the same layer:
     for sampled heads, its reorder, pooling, scores, selection and windows
@@ -407,6 +459,8 @@ def main():
     ap.add_argument("--config-index", type=int, default=CFG_INDEX,
                     help="workload (profiling of smaller layers); the headline is the 720p layer")
     ap.add_argument("--density-index", type=int, default=0)
+    ap.add_argument("--search-curve", action="store_true",
+                    help="print the recall-target vs density curve of the window search and exit")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -420,6 +474,10 @@ def main():
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    if args.search_curve:
+        if rank == 0:
+            print(json.dumps(search_curve(sta, args.config_index, dev)), flush=True)
+        return
     if world > 1:
         import torch.distributed as dist
 
