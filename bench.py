@@ -7,6 +7,7 @@ sta_attn_fwd -> sta_reorder of O back to raster order.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
   python bench.py --search-curve [--config-index I]   (window search, recall vs density)
+  python bench.py --sweep                              (every layer of the workload table)
 
 Rank 0 prints one JSON line. Under torchrun every rank runs its own layer
 (independent problems, no collective on the data path: weak scaling); the
@@ -31,7 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from workloads import CONFIGS, make_qkv, window_params, window_scale  # noqa: E402
+from workloads import CONFIGS, make_qkv, perturb_step, window_params, window_scale  # noqa: E402
 
 METRIC = "kept-block attn TFLOP/s & % BF16 peak; ms/layer at 75,600 tokens, 15% density"
 UNIT = "TFLOP/s"
@@ -102,57 +103,100 @@ def load_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """SM clock, power and clock-event (throttle) reasons sampled every 10 ms
+    through NVML (the library nvidia-smi reads) on a host thread; `stop`
+    keeps the samples taken inside the timed region's host window. Falls back
+    to `nvidia-smi -lms 100` when the NVML binding is missing. Read-only."""
 
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake", 0x80))
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
-        self.index = index
+    def __init__(self, device):
+        self.device = device
+        self.samples = []  # (host time, sm MHz, max MHz, reason names, watts)
+        self.stop_flag = threading.Event()
         self.proc = None
-        self.lines = []
+        self.thread = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+        return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + uuid)
 
     def start(self):
         try:
+            nv, h = self._nvml_handle()
+            smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self.source = "nvml"
+
+            def run():
+                while not self.stop_flag.is_set():
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        watts = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                    except Exception:
+                        break
+                    names = [nm for nm, b in self.REASONS if bits & b]
+                    self.samples.append((time.monotonic(), float(sm), float(smax), names, watts))
+                    time.sleep(0.01)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                ["nvidia-smi", f"--id=GPU-{uuid}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi"
+
+            def read():
+                names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+                for ln in self.proc.stdout:
+                    parts = [x.strip() for x in ln.split(",")]
+                    try:
+                        sm, smax, watts = float(parts[0]), float(parts[1]), float(parts[2])
+                    except (ValueError, IndexError):
+                        continue
+                    act = [nm for nm, v in zip(names, parts[4:8]) if v.lower() == "active"]
+                    self.samples.append((time.monotonic(), sm, smax, act, watts))
+
+            self.thread = threading.Thread(target=read, daemon=True)
             self.thread.start()
         except (OSError, FileNotFoundError):
             self.proc = None
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 8:
-                continue
+    def stop(self, t0=None, t1=None):
+        self.stop_flag.set()
+        if self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for nm, val in zip(names, parts[4:8]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        if self.source is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        win = [x for x in self.samples if (t0 is None or x[0] >= t0) and (t1 is None or x[0] <= t1)]
+        if not win:
+            win = self.samples
+        reasons = sorted({nm for x in win for nm in x[3]})
+        return {"sm_mhz": statistics.median(x[1] for x in win) if win else None,
+                "sm_min_mhz": min(x[1] for x in win) if win else None,
+                "sm_max_mhz": max(x[2] for x in win) if win else None,
+                "power_w_median": statistics.median(x[4] for x in win) if win else None,
+                "reasons": reasons, "samples": len(win), "source": self.source}
 
 
 class Layer:
@@ -365,6 +409,92 @@ def search_curve(sta, cfg_index, dev, taus=(0.8, 0.9, 0.95, 0.99), lam=1.0):
     return {"workload": cfg.name, "block_mass_ms": mass_ms, "curve": rows}
 
 
+def _median_ms(fn, reps):
+    """Median CUDA-event time of `reps` launches of fn (each timed alone)."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in evs:
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in evs)
+
+
+def sweep(sta, dev, peak, reps=20):
+    """Every timed row of the workload table, one JSON line each: the 480p
+    window layer, the 720p layer, the 129-frame layer at four window
+    densities, and the reuse layer (mask built once from step-0 inputs at
+    fixed densities, attention timed on each of the perturbed steps).
+    Inputs (Q, K, V tiled, >= 385 MB each) are larger than L2."""
+    rows = []
+
+    def attn_line(cfg_name, layer, extra):
+        pairs = layer.kept_pairs()
+        nt = layer.nt
+        ms = _median_ms(layer.attn, reps)
+        tf = pairs * flops_per_pair(layer.d) / (ms * 1e-3) / 1e12
+        eff, _ = layer.pair_union_stats()
+        line = {"workload": cfg_name, "density": pairs / (layer.B * layer.Hh * nt * nt), "kept_pairs": pairs,
+                "attn_ms": ms, "attn_tflops": tf, "frac_of_sustained_peak": tf / peak,
+                "pairing_efficiency": eff}
+        line.update(extra)
+        rows.append(line)
+        print(json.dumps(line), flush=True)
+
+    def build_extra(layer):
+        build_ms = _median_ms(layer.build, reps)
+        reo_ms = _median_ms(layer.reorder_in, reps) / 3.0
+        c = layer.cfg
+        raster = c.B * c.L * c.heads * c.d * 2
+        tiled = c.B * c.heads * layer.lpad * c.d * 2
+        nnz = layer.kept_pairs()
+        build_bytes = (2 * tiled if c.use_scores else 0) + 4 * nnz + 4 * (layer.B * layer.Hh * layer.nt + 1)
+        return {"build_ms": build_ms, "build_gbs_algorithmic": build_bytes / (build_ms * 1e-3) / 1e9,
+                "reorder_ms_per_tensor": reo_ms,
+                "reorder_gbs": (raster + tiled) / (reo_ms * 1e-3) / 1e9}
+
+    for ci, dens in ((1, (0,)), (2, (0,)), (3, (0, 1, 2, 3))):
+        for di in dens:
+            layer = Layer(sta, CONFIGS[ci], dev, cfg_index=ci, density_index=di)
+            layer.reorder_in()
+            layer.build()
+            extra = build_extra(layer)
+            extra["density_target"] = CONFIGS[ci].window_density[di]
+            attn_line(CONFIGS[ci].name, layer, extra)
+            del layer
+            torch.cuda.empty_cache()
+
+    # reuse layer: top_p = 0, k_min = round(rho * Nt), no windows; mask from step 0
+    cfg = CONFIGS[4]
+    layer = Layer(sta, cfg, dev, cfg_index=4)
+    gen = torch.Generator(device=dev).manual_seed(1234)
+    masters = [layer.q.float(), layer.k.float()]
+    steps_inputs = []
+    for _ in range(cfg.reuse_steps):
+        qm, qb = perturb_step(masters[0], gen)
+        km, kb = perturb_step(masters[1], gen)
+        masters = [qm, km]
+        steps_inputs.append((qb, kb))
+    del masters
+    for rho in cfg.fixed_densities:
+        k_min = int(round(rho * layer.nt))
+        layer.params = sta.mask_params(0.0, k_min, True, 0.0, cfg.group_lo, None)
+        layer.reorder_in()
+        layer.build()
+        extra = build_extra(layer)
+        per_step = []
+        for qb, kb in steps_inputs:
+            layer.reorder_in(qb, kb, None)
+            per_step.append(_median_ms(layer.attn, max(3, reps // 4)))
+        extra.update({"density_target": rho, "k_min": k_min, "reuse_steps": len(per_step),
+                      "attn_ms_per_reuse_step": per_step})
+        attn_line(cfg.name, layer, extra)
+    del layer, steps_inputs
+    torch.cuda.empty_cache()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    return rows
+
+
 def cpu_oracle_sample(cfg, layer, budget_s, rows_per_head=8, max_heads=None):
     """Time the oracle (as it stands) on a bounded sample of the same layer:
     for sampled heads, its reorder, pooling, scores, selection and windows
@@ -459,6 +589,8 @@ def main():
     ap.add_argument("--config-index", type=int, default=CFG_INDEX,
                     help="workload (profiling of smaller layers); the headline is the 720p layer")
     ap.add_argument("--density-index", type=int, default=0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every layer of the workload table (one JSON line per row) and exit")
     ap.add_argument("--search-curve", action="store_true",
                     help="print the recall-target vs density curve of the window search and exit")
     args = ap.parse_args()
@@ -474,6 +606,11 @@ def main():
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    if args.sweep:
+        if rank == 0:
+            peaks, _ = load_peaks()
+            sweep(sta, dev, float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))))
+        return
     if args.search_curve:
         if rank == 0:
             print(json.dumps(search_curve(sta, args.config_index, dev)), flush=True)
@@ -500,18 +637,20 @@ def main():
 
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    clocks = ClockSampler(local_rank)
+    clocks = ClockSampler(dev)
     clocks.start()
-    time.sleep(0.3)
+    time.sleep(0.1)
     barrier()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    h0 = time.monotonic()
     t_start.record()
     for i in range(K):
         layer.step(evs[i])
     t_end.record()
     barrier()
-    clk = clocks.stop()
+    h1 = time.monotonic()
+    clk = clocks.stop(h0, h1)
     elapsed_ms = t_start.elapsed_time(t_end)
     assert sta.sta_get_device_error() == sta.STA_OK
 
