@@ -589,6 +589,8 @@ def main():
     ap.add_argument("--config-index", type=int, default=CFG_INDEX,
                     help="workload (profiling of smaller layers); the headline is the 720p layer")
     ap.add_argument("--density-index", type=int, default=0)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="use only this many heads of the workload (small cases for ncu captures)")
     ap.add_argument("--sweep", action="store_true",
                     help="time every layer of the workload table (one JSON line per row) and exit")
     ap.add_argument("--search-curve", action="store_true",
@@ -620,6 +622,10 @@ def main():
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     cfg = CONFIGS[args.config_index]
+    if args.heads > 0:
+        from dataclasses import replace
+
+        cfg = replace(cfg, heads=args.heads)
     layer = Layer(sta, cfg, dev, seed_offset=rank, cfg_index=args.config_index,
                   density_index=args.density_index)
 

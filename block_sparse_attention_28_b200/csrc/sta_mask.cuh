@@ -76,6 +76,7 @@ pool_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k, float *__r
 // ------------------------------------------------------ scores + selection
 constexpr int SEL_THREADS = 256;
 constexpr int SEL_QB = 16;  // query tiles per CTA
+constexpr int SEL_KPT = 3;  // key tiles per thread in the score pass
 
 struct GroupLo {
   int v[STA_MAX_GROUPS];
@@ -122,8 +123,9 @@ __device__ void radix_level(const float *row, int nt, unsigned int target, bool 
     __syncwarp();
     for (int j = lane; j < nt; j += 32) {
       const unsigned int b = __float_as_uint(row[j]);
-      if ((b & pmask) == prefix)
-        atomicAdd(hist + ((b >> shift) & dmask), count_only ? 1u : mass_of(__uint_as_float(b)));
+      // entries of zero mass add nothing to a mass histogram: no atomic
+      const unsigned int add = count_only ? 1u : mass_of(__uint_as_float(b));
+      if ((b & pmask) == prefix && add != 0u) atomicAdd(hist + ((b >> shift) & dmask), add);
     }
     __syncwarp();
     // lane owns digits [8*lane, 8*lane + 8)
@@ -214,25 +216,52 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
       qs[e] = (i < nq) ? qbar[((long long)bh * nt + q0 + i) * D + (e - i * D)] : 0.0f;
     }
     __syncthreads();
-    for (int kt = tid; kt < nt; kt += SEL_THREADS) {
-      const float4 *kr = reinterpret_cast<const float4 *>(kbar + ((long long)bh * nt + kt) * D);
-      float acc[SEL_QB];
+    // Each thread owns up to SEL_KPT key tiles (kt = base + tid + u * threads)
+    // of a chunk, so every query value read from shared memory feeds
+    // SEL_KPT FMAs; the passes split Nt into equal chunks. Every score is
+    // still one sequential fp32 FMA chain over d.
+    const int per_pass = SEL_THREADS * SEL_KPT;
+    const int passes = (nt + per_pass - 1) / per_pass;
+    const int chunk = (nt + passes - 1) / passes;
+    for (int pass = 0; pass < passes; ++pass) {
+      const int lo = pass * chunk, hi = min(nt, lo + chunk);
+      const float4 *kr[SEL_KPT];
+      bool on[SEL_KPT];
 #pragma unroll
-      for (int i = 0; i < SEL_QB; ++i) acc[i] = 0.0f;
-#pragma unroll 2
+      for (int u = 0; u < SEL_KPT; ++u) {
+        const int kt = lo + tid + u * SEL_THREADS;
+        on[u] = kt < hi;
+        kr[u] = reinterpret_cast<const float4 *>(kbar + ((long long)bh * nt + (on[u] ? kt : lo)) * D);
+      }
+      float acc[SEL_KPT][SEL_QB];
+#pragma unroll
+      for (int u = 0; u < SEL_KPT; ++u)
+#pragma unroll
+        for (int i = 0; i < SEL_QB; ++i) acc[u][i] = 0.0f;
       for (int d4 = 0; d4 < D / 4; ++d4) {
-        const float4 kv = __ldg(kr + d4);
+        float4 kv[SEL_KPT];
+#pragma unroll
+        for (int u = 0; u < SEL_KPT; ++u) kv[u] = __ldg(kr[u] + d4);
 #pragma unroll
         for (int i = 0; i < SEL_QB; ++i) {
           const float4 qv = reinterpret_cast<const float4 *>(qs + i * D)[d4];
-          acc[i] = fmaf(qv.x, kv.x, acc[i]);
-          acc[i] = fmaf(qv.y, kv.y, acc[i]);
-          acc[i] = fmaf(qv.z, kv.z, acc[i]);
-          acc[i] = fmaf(qv.w, kv.w, acc[i]);
+#pragma unroll
+          for (int u = 0; u < SEL_KPT; ++u) {
+            acc[u][i] = fmaf(qv.x, kv[u].x, acc[u][i]);
+            acc[u][i] = fmaf(qv.y, kv[u].y, acc[u][i]);
+            acc[u][i] = fmaf(qv.z, kv[u].z, acc[u][i]);
+            acc[u][i] = fmaf(qv.w, kv[u].w, acc[u][i]);
+          }
         }
       }
 #pragma unroll
-      for (int i = 0; i < SEL_QB; ++i) S[i * nt + kt] = acc[i] * scale;
+      for (int u = 0; u < SEL_KPT; ++u) {
+        const int kt = lo + tid + u * SEL_THREADS;
+        if (on[u]) {
+#pragma unroll
+          for (int i = 0; i < SEL_QB; ++i) S[i * nt + kt] = acc[u][i] * scale;
+        }
+      }
     }
     __syncthreads();
   }
