@@ -2,8 +2,9 @@
 
 One step = one pass of the whole hot path over one synthetic 720p video-DiT
 layer (75,600 tokens, 40 heads, d = 128, top-p 0.95 / k_min 8 OR dual
-windows, ~15% density): sta_reorder of Q, K, V -> sta_build_mask ->
-sta_attn_fwd -> sta_reorder of O back to raster order.
+windows, ~15% density), on raster Q, K, V: sta_build_mask_raster ->
+sta_attn_fwd_raster (the tile gather of Q, K, V and the scatter of O back to
+raster order happen inside the kernels' loads and stores).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
   python bench.py --search-curve [--config-index I]   (window search, recall vs density)
@@ -212,10 +213,9 @@ class Layer:
         self.g = sta.grid(c.T, c.H, c.W)
         self.nt = sta.sta_num_tiles(self.g)
         self.lpad = sta.sta_tiled_len(self.g)
+        self.dev = dev
         self.q, self.k, self.v = make_qkv(c, device=dev)
-        shape_t = (self.B, self.Hh, self.lpad, self.d)
-        self.qt, self.kt, self.vt, self.ot = (torch.empty(shape_t, dtype=torch.bfloat16, device=dev)
-                                              for _ in range(4))
+        self._tiled = None  # tiled copies, made only for the reorder / tiled-call measurements
         self.o = torch.empty_like(self.q)
         if c.window_density:
             self.win = torch.from_numpy(window_params(cfg, window_scale(cfg_index, density_index))).to(dev)
@@ -223,7 +223,29 @@ class Layer:
             self.win = None
         self.params = sta.mask_params(c.top_p, c.k_min, c.use_scores, 0.0, c.group_lo, self.win)
         self.bufs = sta.MaskBuffers(self.B, self.Hh, self.d, self.g, dev)
-        self.launches_per_step = 3 + 4 + 1 + 1  # reorder x3, pool/select/scan/fill, attn, inverse
+        self.launches_per_step = 4 + 1  # pool/select/scan/fill, attn (the tile gather is the TMA box)
+
+    @property
+    def qt(self):
+        return self._tiled_bufs()[0]
+
+    @property
+    def kt(self):
+        return self._tiled_bufs()[1]
+
+    @property
+    def vt(self):
+        return self._tiled_bufs()[2]
+
+    @property
+    def ot(self):
+        return self._tiled_bufs()[3]
+
+    def _tiled_bufs(self):
+        if self._tiled is None:
+            shape_t = (self.B, self.Hh, self.lpad, self.d)
+            self._tiled = tuple(torch.empty(shape_t, dtype=torch.bfloat16, device=self.dev) for _ in range(4))
+        return self._tiled
 
     def reorder_in(self, q=None, k=None, v=None):
         s = self.sta
@@ -231,10 +253,21 @@ class Layer:
         for src, dst in ((q, self.qt), (k, self.kt), (v, self.vt)):
             s.sta_reorder(src, dst, self.B, self.Hh, self.d, self.g)
 
-    def build(self):
+    def build(self, q=None, k=None):
+        """Mask from raster Q, K (sta_build_mask_raster)."""
+        self.sta.build_mask(self.q if q is None else q, self.k if k is None else k, self.B, self.Hh, self.d,
+                            self.g, self.params, self.bufs, raster=True)
+
+    def attn(self, q=None, k=None, v=None, o=None):
+        """Attention on raster Q, K, V into raster O (sta_attn_fwd_raster)."""
+        self.sta.sta_attn_fwd_raster(self.q if q is None else q, self.k if k is None else k,
+                                     self.v if v is None else v, self.o if o is None else o, None,
+                                     self.bufs.row_ptr, self.bufs.col_idx, self.B, self.Hh, self.d, self.g)
+
+    def build_tiled(self):
         self.sta.build_mask(self.qt, self.kt, self.B, self.Hh, self.d, self.g, self.params, self.bufs)
 
-    def attn(self):
+    def attn_tiled(self):
         self.sta.sta_attn_fwd(self.qt, self.kt, self.vt, self.ot, None, self.bufs.row_ptr, self.bufs.col_idx,
                               self.B, self.Hh, self.d, self.g)
 
@@ -268,14 +301,12 @@ class Layer:
                     dst.copy_(src, non_blocking=True)
                 in_ready[b].record(s_in)
             comp.wait_event(in_ready[b])
-            self.reorder_in(*ins[b])
-            in_free[b] = ev()
-            in_free[b].record(comp)
-            self.build()
-            self.attn()
+            self.build(ins[b][0], ins[b][1])
             if out_free[b] is not None:
                 comp.wait_event(out_free[b])
-            self.reorder_out(outs[b])
+            self.attn(*ins[b], outs[b])
+            in_free[b] = ev()
+            in_free[b].record(comp)
             out_ready[b].record(comp)
             s_out.wait_event(out_ready[b])
             with torch.cuda.stream(s_out):
@@ -289,10 +320,11 @@ class Layer:
         return t0.elapsed_time(t1) / steps
 
     def step(self, ev=None):
+        """One pass of the path on raster Q, K, V: mask, then attention into
+        raster O. The 1x8x8 tile gather and scatter happen in the TMA boxes and
+        the epilogue, so no reorder pass runs (events 0-1 bracket nothing)."""
         if ev is not None:
             ev[0].record()
-        self.reorder_in()
-        if ev is not None:
             ev[1].record()
         self.build()
         if ev is not None:
@@ -300,8 +332,6 @@ class Layer:
         self.attn()
         if ev is not None:
             ev[3].record()
-        self.reorder_out()
-        if ev is not None:
             ev[4].record()
 
     def dense_run(self, reps=2):
@@ -311,13 +341,14 @@ class Layer:
         dev = self.qt.device
         rp = (torch.arange(R + 1, device=dev, dtype=torch.int64) * self.nt).to(torch.int32)
         ci = torch.arange(self.nt, device=dev, dtype=torch.int32).repeat(R)
-        self.sta.sta_attn_fwd(self.qt, self.kt, self.vt, self.ot, None, rp, ci, self.B, self.Hh, self.d, self.g)
+        self.sta.sta_attn_fwd_raster(self.q, self.k, self.v, self.o, None, rp, ci, self.B, self.Hh, self.d,
+                                     self.g)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         e0.record()
         for _ in range(reps):
-            self.sta.sta_attn_fwd(self.qt, self.kt, self.vt, self.ot, None, rp, ci, self.B, self.Hh, self.d,
-                                  self.g)
+            self.sta.sta_attn_fwd_raster(self.q, self.k, self.v, self.o, None, rp, ci, self.B, self.Hh, self.d,
+                                         self.g)
         e1.record()
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1) / reps
@@ -448,7 +479,7 @@ def sweep(sta, dev, peak, reps=20):
         raster = c.B * c.L * c.heads * c.d * 2
         tiled = c.B * c.heads * layer.lpad * c.d * 2
         nnz = layer.kept_pairs()
-        build_bytes = (2 * tiled if c.use_scores else 0) + 4 * nnz + 4 * (layer.B * layer.Hh * layer.nt + 1)
+        build_bytes = (2 * raster if c.use_scores else 0) + 4 * nnz + 4 * (layer.B * layer.Hh * layer.nt + 1)
         return {"build_ms": build_ms, "build_gbs_algorithmic": build_bytes / (build_ms * 1e-3) / 1e9,
                 "reorder_ms_per_tensor": reo_ms,
                 "reorder_gbs": (raster + tiled) / (reo_ms * 1e-3) / 1e9}
@@ -456,7 +487,6 @@ def sweep(sta, dev, peak, reps=20):
     for ci, dens in ((1, (0,)), (2, (0,)), (3, (0, 1, 2, 3))):
         for di in dens:
             layer = Layer(sta, CONFIGS[ci], dev, cfg_index=ci, density_index=di)
-            layer.reorder_in()
             layer.build()
             extra = build_extra(layer)
             extra["density_target"] = CONFIGS[ci].window_density[di]
@@ -479,13 +509,11 @@ def sweep(sta, dev, peak, reps=20):
     for rho in cfg.fixed_densities:
         k_min = int(round(rho * layer.nt))
         layer.params = sta.mask_params(0.0, k_min, True, 0.0, cfg.group_lo, None)
-        layer.reorder_in()
         layer.build()
         extra = build_extra(layer)
         per_step = []
         for qb, kb in steps_inputs:
-            layer.reorder_in(qb, kb, None)
-            per_step.append(_median_ms(layer.attn, max(3, reps // 4)))
+            per_step.append(_median_ms(lambda: layer.attn(qb, kb), max(3, reps // 4)))
         extra.update({"density_target": rho, "k_min": k_min, "reuse_steps": len(per_step),
                       "attn_ms_per_reuse_step": per_step})
         attn_line(cfg.name, layer, extra)
@@ -660,7 +688,6 @@ def main():
     elapsed_ms = t_start.elapsed_time(t_end)
     assert sta.sta_get_device_error() == sta.STA_OK
 
-    reorder_ms = statistics.mean(e[0].elapsed_time(e[1]) + e[3].elapsed_time(e[4]) for e in evs)
     build_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     elapsed_ms = max_over_ranks(elapsed_ms, dev, world)
@@ -715,10 +742,12 @@ def main():
                 "density": density, "kept_pairs": pairs, "global_batch": world * cfg.B,
                 "parallelism": f"independent layer per GPU x{world}",
                 "l2": "inputs (Q,K,V 2.3 GB) larger than L2; no flush",
-                "step": "reorder Q,K,V + build_mask + attn_fwd + reorder O back",
+                "step": ("build_mask_raster (pool, scores, selection, windows, CSR) + attn_fwd_raster; "
+                         "the 1x8x8 tile gather of Q/K/V and scatter of O are the attention kernel's "
+                         "5D TMA boxes and epilogue stores, so no reorder pass runs"),
             },
             "ms_per_layer": build_ms + attn_ms,
-            "ms_breakdown": {"reorder_in_out": reorder_ms, "build_mask": build_ms, "attn_fwd": attn_ms},
+            "ms_breakdown": {"build_mask": build_ms, "attn_fwd": attn_ms},
             "attn_tflops": attn_tflops,
             "attn_frac_of_peak": attn_tflops / peak,
             "pairing_efficiency": eff,
@@ -726,7 +755,7 @@ def main():
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": attn_tflops / peak, "traffic": load_traffic(),
                          "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
-                         "kernel": "attn_fwd_kernel<128>",
+                         "kernel": "attn_fwd_kernel<128, MASS=false, RASTER=true>",
                          "algorithmic": f"{pairs} kept pairs x 4*64*64*{cfg.d} flop"},
             "cpu_baseline": cpu,
             "e2e": e2e,

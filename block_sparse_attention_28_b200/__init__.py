@@ -72,6 +72,10 @@ _lib.sta_build_mask_noalloc.argtypes = [_vp, _vp, _i32, _i32, _i32, Grid, ctypes
 _lib.sta_build_mask_noalloc.restype = ctypes.c_int
 _lib.sta_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, Grid, _f32, _vp]
 _lib.sta_attn_fwd.restype = ctypes.c_int
+_lib.sta_build_mask_raster.argtypes = _lib.sta_build_mask.argtypes
+_lib.sta_build_mask_raster.restype = ctypes.c_int
+_lib.sta_attn_fwd_raster.argtypes = _lib.sta_attn_fwd.argtypes
+_lib.sta_attn_fwd_raster.restype = ctypes.c_int
 _lib.sta_attn_fwd_block_mass.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, Grid,
                                          _f32, _vp]
 _lib.sta_attn_fwd_block_mass.restype = ctypes.c_int
@@ -148,6 +152,8 @@ def mask_params(top_p=0.0, k_min=0, use_scores=False, sm_scale=0.0, group_lo=(0,
     for i, v in enumerate(group_lo):
         p.group_lo[i] = int(v)
     p.windows = _ptr(windows)
+    # the struct holds raw device pointers: keep the tensors alive with it
+    p._keep = (windows, block_scores)
     return p
 
 
@@ -174,6 +180,22 @@ def sta_attn_fwd(q, k, v, o, lse, row_ptr, col_idx, B, heads, d, g, sm_scale=0.0
     _check(_lib.sta_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(row_ptr), _ptr(col_idx),
                              B, heads, d, g, float(sm_scale), _stream(stream)),
            "sta_attn_fwd")
+
+
+def sta_build_mask_raster(q, k, B, heads, d, g, params, row_ptr, col_idx, nnz_dev, block_mask=None,
+                          block_probs=None, workspace=None, ws_bytes=0, stream=None):
+    """sta_build_mask on raster [B, L, heads, d] Q and K."""
+    _check(_lib.sta_build_mask_raster(_ptr(q), _ptr(k), B, heads, d, g, ctypes.byref(params), _ptr(row_ptr),
+                                      _ptr(col_idx), _ptr(nnz_dev), _ptr(block_mask), _ptr(block_probs),
+                                      _ptr(workspace), int(ws_bytes), _stream(stream)),
+           "sta_build_mask_raster")
+
+
+def sta_attn_fwd_raster(q, k, v, o, lse, row_ptr, col_idx, B, heads, d, g, sm_scale=0.0, stream=None):
+    """sta_attn_fwd on raster [B, L, heads, d] Q, K, V and O (LSE tiled-indexed)."""
+    _check(_lib.sta_attn_fwd_raster(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(row_ptr),
+                                    _ptr(col_idx), B, heads, d, g, float(sm_scale), _stream(stream)),
+           "sta_attn_fwd_raster")
 
 
 def sta_attn_fwd_block_mass(q, k, v, o, lse, row_ptr, col_idx, lse_cached, block_mass, B, heads, d, g,
@@ -215,7 +237,8 @@ class MaskBuffers:
         self.workspace = torch.empty(max(1, self.ws_bytes), dtype=torch.uint8, device=device)
 
 
-def build_mask(q_tiled, k_tiled, B, heads, d, g, params, bufs, stream=None):
-    sta_build_mask(q_tiled, k_tiled, B, heads, d, g, params, bufs.row_ptr, bufs.col_idx, bufs.nnz,
-                   bufs.block_mask, bufs.block_probs, bufs.workspace, bufs.ws_bytes, stream)
+def build_mask(q_tiled, k_tiled, B, heads, d, g, params, bufs, stream=None, raster=False):
+    fn = sta_build_mask_raster if raster else sta_build_mask
+    fn(q_tiled, k_tiled, B, heads, d, g, params, bufs.row_ptr, bufs.col_idx, bufs.nnz,
+       bufs.block_mask, bufs.block_probs, bufs.workspace, bufs.ws_bytes, stream)
     return bufs

@@ -94,13 +94,19 @@ inline size_t smem_bytes(int nt) {
 //   mass = (1/n_q) sum_i sum_j 2^(s_ij * scale_log2 - lse_in_i * log2 e),
 // which is, per row and tile, the row's softmax sum (relative to its running
 // max m_i) times 2^(m_i - lse_in_i * log2 e): one extra exp2 per row and tile.
-template <int D, bool MASS>
+//
+// RASTER: Q, K, V and O stay in the raster layout [B, L, heads, d]. A tile is
+// then one box of a 5D tensor map (d, head, x, y, frame), 64 d-values x 1
+// head x 8 columns x 8 rows x 1 frame, which TMA writes to shared memory in
+// the tile's token order (zeros beyond the grid edge), so the permutation to
+// tiles costs no pass over memory; O rows go straight to their raster rows.
+template <int D, bool MASS, bool RASTER>
 __global__ void __launch_bounds__(NUM_THREADS, MIN_BLOCKS_PER_SM)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16 *__restrict__ out,
                 float *__restrict__ lse, const int *__restrict__ row_ptr,
                 const int *__restrict__ col_idx, Geo g, float scale_log2,
-                const float *__restrict__ lse_in, float *__restrict__ block_mass) {
+                const float *__restrict__ lse_in, float *__restrict__ block_mass, int heads) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -240,16 +246,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == WARP_PRODUCER) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0 && n > 0) {
-      const int rowA = (int)(((long long)bh * nt + qtA) * 64);
-      const int rowB = (int)(((long long)bh * nt + qtB) * 64);
-      tc::mbar_expect_tx(q_full, (hasB ? 2 : 1) * C::TILE_BYTES);
+      // all d-atoms of tile `tile` of this (b, h) into dst (+ 8192 per atom
+      // for K and V, + Q_REGION for Q)
+      auto load_tile_atoms = [&](const CUtensorMap *map, uint64_t *bar, uint32_t dst, uint32_t atom_step,
+                                 int tile) {
+        if (RASTER) {
+          const int tpf = g.NH * g.NW;
+          const int t = tile / tpf, rem = tile - t * tpf;
+          const int ty = rem / g.NW, tx = rem - ty * g.NW;
+          const int b = bh / heads, h = bh - b * heads;
 #pragma unroll
-      for (int kb = 0; kb < C::KB; ++kb) {
-        tc::tma_load_2d(sbase + C::OFF_Q + kb * C::Q_REGION, &tm_q, q_full, kb * 64, rowA);
-        if (hasB)
-          tc::tma_load_2d(sbase + C::OFF_Q + kb * C::Q_REGION + 8192, &tm_q, q_full, kb * 64,
-                          rowB);
-      }
+          for (int kb = 0; kb < C::KB; ++kb)
+            tc::tma_load_5d(dst + kb * atom_step, map, bar, kb * 64, h, tx * 8, ty * 8, b * g.T + t);
+        } else {
+          const int row = (int)(((long long)bh * nt + tile) * 64);
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb) tc::tma_load_2d(dst + kb * atom_step, map, bar, kb * 64, row);
+        }
+      };
+      tc::mbar_expect_tx(q_full, (hasB ? 2 : 1) * C::TILE_BYTES);
+      load_tile_atoms(&tm_q, q_full, sbase + C::OFF_Q, C::Q_REGION, qtA);
+      if (hasB) load_tile_atoms(&tm_q, q_full, sbase + C::OFF_Q + 8192, C::Q_REGION, qtB);
       // K runs KLEAD tiles ahead of V: K_{j+1} is needed by S_{j+1}, which the
       // MMA warp issues before P.V_j.
       auto load_tile = [&](const CUtensorMap *map, uint64_t *full, uint64_t *empty, int off, int ns,
@@ -257,11 +274,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int s = j % ns, u = j / ns;
         if (u > 0 && !tc::mbar_wait(empty + s, (u - 1) & 1, abort_flag, WAIT_LIMIT)) return false;
         const int kt = (int)(U[j] & KT_MASK);
-        const int row = (int)(((long long)bh * nt + kt) * 64);
         tc::mbar_expect_tx(full + s, C::TILE_BYTES);
-#pragma unroll
-        for (int kb = 0; kb < C::KB; ++kb)
-          tc::tma_load_2d(sbase + off + s * C::TILE_BYTES + kb * 8192, map, full + s, kb * 64, row);
+        load_tile_atoms(map, full + s, sbase + off + s * C::TILE_BYTES, 8192u, kt);
         return true;
       };
       int issued_k = 0, issued_v = 0;
@@ -490,7 +504,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int qt = halfB ? qtB : qtA;
       const long long orow = (long long)bh * g.Lpad + (long long)qt * 64 + (tid & 63);
       const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
-      uint4 *dst = reinterpret_cast<uint4 *>(out + orow * D);
+      // destination row: tiled row orow, or the token's raster row (none for
+      // the pad rows of a tile cut by the grid edge)
+      long long dst_row = orow;
+      bool store_row = true;
+      if (RASTER) {
+        const int tpf = g.NH * g.NW;
+        const int t = qt / tpf, rem = qt - t * tpf;
+        const int ty = rem / g.NW, tx = rem - ty * g.NW;
+        const int r = tid & 63;
+        const int y = ty * 8 + (r >> 3), x = tx * 8 + (r & 7);
+        const int b = bh / heads, h = bh - b * heads;
+        store_row = y < g.H && x < g.W;
+        dst_row = (((long long)(b * g.T + t) * g.H + y) * g.W + x) * heads + h;
+      }
+      uint4 *dst = reinterpret_cast<uint4 *>(out + dst_row * D);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -504,9 +532,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int c = 0; c < 16; ++c)
           pk[c] = tc::pack_bf16(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
+        if (store_row) {
 #pragma unroll
-        for (int v = 0; v < 4; ++v)
-          dst[cc * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int v = 0; v < 4; ++v)
+            dst[cc * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
       }
       if (lse != nullptr)
         lse[orow] = (l > 0.0f) ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;

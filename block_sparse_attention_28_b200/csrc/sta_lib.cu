@@ -98,6 +98,23 @@ bool make_tile_map(CUtensorMap *map, const void *base, unsigned long long rows, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Raster [B, L, heads, d] bf16 as the 5D tensor (d, heads, W, H, B*T): a box
+// of 64 d-values x 1 head x 8 columns x 8 rows x 1 frame is one token tile
+// (zero-filled beyond the grid edge), 128 B swizzle.
+bool make_raster_map(CUtensorMap *map, const void *base, const Geo &g, int B, int heads, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t row = (cuuint64_t)heads * d * 2;  // bytes per token
+  cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)g.W, (cuuint64_t)g.H,
+                        (cuuint64_t)B * g.T};
+  cuuint64_t strides[4] = {(cuuint64_t)d * 2, row, row * g.W, row * g.W * g.H};
+  cuuint32_t box[5] = {64, 1, 8, 8, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool device_is_sm100() {
   int dev = 0, major = 0, minor = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
@@ -123,7 +140,7 @@ template <int D>
 sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads,
                         const Geo &g, const sta_mask_params *p, int32_t *row_ptr, int32_t *col_idx,
                         int64_t *nnz_dev, uint8_t *block_mask, float *block_probs, uint8_t *ws,
-                        cudaStream_t s) {
+                        cudaStream_t s, bool raster = false) {
   const MaskWs L = mask_ws_layout(B, heads, D, g);
   float *qbar = reinterpret_cast<float *>(ws + L.qbar);
   float *kbar = reinterpret_cast<float *>(ws + L.kbar);
@@ -138,8 +155,12 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
   if (use_scores && P_in == nullptr) {
     const long long warps = 2 * R;
     const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
-    pool_kernel<D><<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(q_tiled),
-                                           static_cast<const uint4 *>(k_tiled), qbar, kbar, R, g);
+    if (raster)
+      pool_kernel<D, true><<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(q_tiled),
+                                                  static_cast<const uint4 *>(k_tiled), qbar, kbar, R, g, heads);
+    else
+      pool_kernel<D, false><<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(q_tiled),
+                                                   static_cast<const uint4 *>(k_tiled), qbar, kbar, R, g, heads);
     STA_CUDA_TRY(cudaGetLastError());
   }
   const size_t smem = select_smem(D, g, use_scores);
@@ -177,27 +198,33 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
   return STA_OK;
 }
 
-template <int D, bool MASS>
+template <int D, bool MASS, bool RASTER = false>
 sta_status launch_attn(const void *q, const void *k, const void *v, void *o, float *lse,
                        const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
                        const Geo &g, float sm_scale, cudaStream_t s, const float *lse_in = nullptr,
                        float *block_mass = nullptr) {
   const unsigned long long rows = (unsigned long long)B * heads * g.Lpad;
   CUtensorMap tq, tk, tv;
-  if (!make_tile_map(&tq, q, rows, D) || !make_tile_map(&tk, k, rows, D) || !make_tile_map(&tv, v, rows, D))
+  if (RASTER) {
+    if (!make_raster_map(&tq, q, g, B, heads, D) || !make_raster_map(&tk, k, g, B, heads, D) ||
+        !make_raster_map(&tv, v, g, B, heads, D))
+      return STA_ERR_CUDA;
+  } else if (!make_tile_map(&tq, q, rows, D) || !make_tile_map(&tk, k, rows, D) ||
+             !make_tile_map(&tv, v, rows, D)) {
     return STA_ERR_CUDA;
+  }
   const size_t smem = attn::smem_bytes<D>(g.Nt);
   if (smem > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
-  STA_CUDA_TRY(cudaFuncSetAttribute(attn::attn_fwd_kernel<D, MASS>,
+  STA_CUDA_TRY(cudaFuncSetAttribute(attn::attn_fwd_kernel<D, MASS, RASTER>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   if (MASS)
     STA_CUDA_TRY(cudaMemsetAsync(block_mass, 0, (size_t)B * heads * g.Nt * g.Nt * sizeof(float), s));
   const float scale = sm_scale != 0.0f ? sm_scale : 1.0f / sqrtf((float)D);
   const float scale_log2 = scale * 1.4426950408889634f;
   dim3 grid((unsigned)((g.Nt + 1) / 2), (unsigned)(B * heads));
-  attn::attn_fwd_kernel<D, MASS><<<grid, attn::NUM_THREADS, smem, s>>>(
+  attn::attn_fwd_kernel<D, MASS, RASTER><<<grid, attn::NUM_THREADS, smem, s>>>(
       tq, tk, tv, static_cast<__nv_bfloat16 *>(o), lse, row_ptr, col_idx, g, scale_log2, lse_in,
-      block_mass);
+      block_mass, heads);
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }
@@ -236,10 +263,11 @@ size_t sta_build_mask_workspace(int32_t B, int32_t heads, int32_t d, sta_grid g)
   return mask_ws_layout(B, heads, d, geo).total;
 }
 
-sta_status sta_build_mask(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads, int32_t d,
-                          sta_grid g, const sta_mask_params *p, int32_t *row_ptr, int32_t *col_idx,
-                          int64_t *nnz_dev, uint8_t *block_mask, float *block_probs, void *workspace,
-                          size_t ws_bytes, sta_stream_t stream) {
+static sta_status build_mask_any(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads,
+                                 int32_t d, sta_grid g, const sta_mask_params *p, int32_t *row_ptr,
+                                 int32_t *col_idx, int64_t *nnz_dev, uint8_t *block_mask,
+                                 float *block_probs, void *workspace, size_t ws_bytes,
+                                 sta_stream_t stream, bool raster) {
   Geo geo;
   sta_status st = STA_OK;
   if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return st;
@@ -263,14 +291,30 @@ sta_status sta_build_mask(const void *q_tiled, const void *k_tiled, int32_t B, i
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   return (d == 128) ? launch_build<128>(q_tiled, k_tiled, B, heads, geo, p, row_ptr, col_idx, nnz_dev,
-                                        block_mask, block_probs, ws, s)
+                                        block_mask, block_probs, ws, s, raster)
                     : launch_build<64>(q_tiled, k_tiled, B, heads, geo, p, row_ptr, col_idx, nnz_dev,
-                                       block_mask, block_probs, ws, s);
+                                       block_mask, block_probs, ws, s, raster);
 }
 
-sta_status sta_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
-                        const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
-                        int32_t d, sta_grid g, float sm_scale, sta_stream_t stream) {
+sta_status sta_build_mask(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads, int32_t d,
+                          sta_grid g, const sta_mask_params *p, int32_t *row_ptr, int32_t *col_idx,
+                          int64_t *nnz_dev, uint8_t *block_mask, float *block_probs, void *workspace,
+                          size_t ws_bytes, sta_stream_t stream) {
+  return build_mask_any(q_tiled, k_tiled, B, heads, d, g, p, row_ptr, col_idx, nnz_dev, block_mask,
+                        block_probs, workspace, ws_bytes, stream, false);
+}
+
+sta_status sta_build_mask_raster(const void *q, const void *k, int32_t B, int32_t heads, int32_t d,
+                                 sta_grid g, const sta_mask_params *p, int32_t *row_ptr, int32_t *col_idx,
+                                 int64_t *nnz_dev, uint8_t *block_mask, float *block_probs,
+                                 void *workspace, size_t ws_bytes, sta_stream_t stream) {
+  return build_mask_any(q, k, B, heads, d, g, p, row_ptr, col_idx, nnz_dev, block_mask, block_probs,
+                        workspace, ws_bytes, stream, true);
+}
+
+static sta_status attn_fwd_any(const void *q, const void *k, const void *v, void *o, float *lse,
+                               const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
+                               int32_t d, sta_grid g, float sm_scale, sta_stream_t stream, bool raster) {
   Geo geo;
   sta_status st = STA_OK;
   if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return st;
@@ -280,8 +324,26 @@ sta_status sta_attn_fwd(const void *q, const void *k, const void *v, void *o, fl
   if (!(sm_scale == sm_scale) || sm_scale < 0.0f) return STA_ERR_INVALID_ARG;
   if (!device_is_sm100()) return STA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (raster) {
+    // TMA coordinates of the 5D map are 32-bit: B*T frames, W columns, H rows
+    if ((long long)B * geo.T >= (1LL << 31)) return STA_ERR_UNSUPPORTED;
+    return (d == 128) ? launch_attn<128, false, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s)
+                      : launch_attn<64, false, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s);
+  }
   return (d == 128) ? launch_attn<128, false>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s)
                     : launch_attn<64, false>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s);
+}
+
+sta_status sta_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                        const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
+                        int32_t d, sta_grid g, float sm_scale, sta_stream_t stream) {
+  return attn_fwd_any(q, k, v, o, lse, row_ptr, col_idx, B, heads, d, g, sm_scale, stream, false);
+}
+
+sta_status sta_attn_fwd_raster(const void *q, const void *k, const void *v, void *o, float *lse,
+                               const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
+                               int32_t d, sta_grid g, float sm_scale, sta_stream_t stream) {
+  return attn_fwd_any(q, k, v, o, lse, row_ptr, col_idx, B, heads, d, g, sm_scale, stream, true);
 }
 
 sta_status sta_attn_fwd_block_mass(const void *q, const void *k, const void *v, void *o, float *lse,

@@ -20,26 +20,39 @@ constexpr float MASS_ONE_F = 16777216.0f;  // 2^24, fixed-point unit of the mass
 // One warp per (b*heads + h, tile). Each lane owns one 16-byte chunk of a row
 // and walks the tile's real rows; the sum is exact in fp64 (64 bf16 values),
 // the mean is rounded once to fp32.
-template <int D>
+// RASTER: Q and K in the raster layout [B, L, heads, d]; consecutive warps
+// take the same tile of consecutive heads, so together they read whole
+// token rows (all heads) at a time.
+template <int D, bool RASTER>
 __global__ void __launch_bounds__(256)
 pool_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k, float *__restrict__ qbar,
-            float *__restrict__ kbar, long long n_tiles_total, Geo g) {
+            float *__restrict__ kbar, long long n_tiles_total, Geo g, int heads) {
   constexpr int CPR = D / 8;      // chunks per row
   constexpr int RPI = 32 / CPR;   // rows per warp step
   const long long warp_id = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const bool is_k = warp_id >= n_tiles_total;
-  const long long tile = is_k ? warp_id - n_tiles_total : warp_id;
-  if (tile >= n_tiles_total) return;
+  const long long idx = is_k ? warp_id - n_tiles_total : warp_id;
+  if (idx >= n_tiles_total) return;
   const uint4 *src = is_k ? k : q;
   float *dst = is_k ? kbar : qbar;
-  const int n = (int)(tile % g.Nt);
+  const long long BH = n_tiles_total / g.Nt;
+  const long long bh = RASTER ? idx % BH : idx / g.Nt;
+  const int n = (int)(RASTER ? idx / BH : idx % g.Nt);
+  const long long tile = bh * g.Nt + n;  // output row of qbar / kbar
   const int tpf = g.NH * g.NW;
-  const int rem = n % tpf;
+  const int t = n / tpf, rem = n - t * tpf;
   const int ty = rem / g.NW, tx = rem - ty * g.NW;
   const int vy = valid_extent(g.H, ty), vx = valid_extent(g.W, tx);
   const int sub = lane / CPR, c = lane - sub * CPR;
-  const uint4 *base = src + tile * 64 * CPR;
+  // chunk of tile row r: tiled row tile*64 + r, or raster row of token
+  // (t, 8*ty + r/8, 8*tx + r%8) and head h
+  const long long b = bh / heads, h = bh - b * heads;
+  const long long frame_row0 = ((b * g.T + t) * g.H + 8LL * ty) * g.W + 8LL * tx;
+  auto row_chunk = [&](int r) -> const uint4 * {
+    if (RASTER) return src + ((frame_row0 + (long long)(r >> 3) * g.W + (r & 7)) * heads + h) * CPR;
+    return src + (tile * 64 + r) * CPR;
+  };
   double acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.0;
@@ -47,7 +60,7 @@ pool_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k, float *__r
   for (int i = 0; i < 64 / RPI; ++i) {
     const int r = i * RPI + sub;
     if ((r >> 3) < vy && (r & 7) < vx) {
-      const uint4 w = __ldcs(base + r * CPR + c);
+      const uint4 w = __ldcs(row_chunk(r) + c);
       const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&w);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {

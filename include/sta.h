@@ -151,6 +151,25 @@ sta_status sta_attn_fwd(const void *q, const void *k, const void *v, void *o, fl
                         const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
                         int32_t d, sta_grid g, float sm_scale, sta_stream_t stream);
 
+/* Raster-layout forms of sta_build_mask and sta_attn_fwd: the same results
+ * (bit for bit) without the layout change of sta_reorder. The token tiles
+ * (Compact Attention: tile-aligned masks over 1x8x8 cubes) are gathered by
+ * the kernels' loads instead of a separate pass over memory.
+ *   q, k, v : raster [B, L, heads, d] bf16
+ *   o       : raster [B, L, heads, d] bf16, every real token row written
+ *   lse     : optional fp32 [B, heads, Lpad], indexed like the tiled layout
+ *             (row 64*qt + (y%8)*8 + x%8 of the head); pad rows unspecified
+ * Every other argument, check and error is that of the tiled call. */
+sta_status sta_build_mask_raster(const void *q, const void *k, int32_t B, int32_t heads, int32_t d,
+                                 sta_grid g, const sta_mask_params *p, int32_t *row_ptr,
+                                 int32_t *col_idx, int64_t *nnz_dev, uint8_t *block_mask,
+                                 float *block_probs, void *workspace, size_t ws_bytes,
+                                 sta_stream_t stream);
+sta_status sta_attn_fwd_raster(const void *q, const void *k, const void *v, void *o, float *lse,
+                               const int32_t *row_ptr, const int32_t *col_idx, int32_t B,
+                               int32_t heads, int32_t d, sta_grid g, float sm_scale,
+                               sta_stream_t stream);
+
 /* Size in bytes of the static device scratch behind sta_build_mask_noalloc. */
 #define STA_NOALLOC_SCRATCH_BYTES (32u << 20)
 

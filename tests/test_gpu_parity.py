@@ -666,6 +666,67 @@ def test_search_windows_rejects_bad_groups(sta):
             sta.sta_search_windows(m, 1, 1, g, lo, tau, 1.0, out)
 
 
+# ------------------------------------------ raster-layout path (no reorder)
+def _raster_vs_tiled(sta, gp, q, k, v, B, Hh, d, T, H, W, params, rows_check=None):
+    """Mask and attention through the raster entry points equal, bit for bit,
+    the tiled path followed by the inverse reorder; returns the raster O."""
+    g = sta.grid(T, H, W)
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    bt = gp.build(qt, kt, B, Hh, d, g, params, with_mask=True, with_probs=True)
+    br = sta.MaskBuffers(B, Hh, d, g, "cuda", True, True)
+    sta.build_mask(q, k, B, Hh, d, g, params, br, raster=True)
+    torch.cuda.synchronize()
+    assert int(bt.nnz.item()) == int(br.nnz.item())
+    nnz = int(bt.nnz.item())
+    assert torch.equal(bt.row_ptr, br.row_ptr) and torch.equal(bt.col_idx[:nnz], br.col_idx[:nnz])
+    assert torch.equal(bt.block_mask, br.block_mask)
+    assert torch.equal(bt.block_probs, br.block_probs)
+    o_t, lse_t = gp.attn(qt, kt, vt, bt.row_ptr, bt.col_idx, B, Hh, d, g)
+    o_back = torch.full_like(q, float("nan"))
+    sta.sta_reorder(o_t, o_back, B, Hh, d, g, inverse=True)
+    o_r = torch.full_like(q, float("nan"))
+    lse_r = torch.full_like(lse_t, float("nan"))
+    sta.sta_attn_fwd_raster(q, k, v, o_r, lse_r, br.row_ptr, br.col_idx, B, Hh, d, g)
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    assert torch.equal(o_r.view(torch.int16), o_back.view(torch.int16))  # every raster row written
+    valid = torch.from_numpy(O.valid_rows(T, H, W)).cuda()
+    assert torch.equal(lse_r[:, :, valid], lse_t[:, :, valid])
+    return o_r
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T,H,W,Hh,B", [(3, 19, 37, 2, 2), (4, 16, 16, 3, 1), (2, 9, 10, 1, 1), (5, 24, 13, 2, 1)])
+def test_raster_path_equals_tiled(sta, gp, d, T, H, W, Hh, B):
+    q, k, v = _structured(T, H, W, Hh, d, seed=T * 7 + W, B=B)
+    nh, nw, _, _ = O.tile_grid(T, H, W)
+    win = np.zeros((Hh, 2, 4), dtype=np.int32)
+    win[:, 0] = (1, 1, 0, nw - 1)
+    win[:, 1] = (0, 0, -1, -1)
+    win_t = torch.from_numpy(win).cuda()  # params holds only its pointer: keep it alive
+    params = sta.mask_params(0.8, 2, True, 0.0, (0, 1), win_t)
+    o_r = _raster_vs_tiled(sta, gp, q, k, v, B, Hh, d, T, H, W, params)
+    # and against the oracle directly, on the raster output
+    g = sta.grid(T, H, W)
+    bt = gp.build(gp.reorder(q, B, Hh, d, g), gp.reorder(k, B, Hh, d, g), B, Hh, d, g, params)
+    rp, ci, _ = gp.csr_np(bt)
+    o_ref, _ = O.attention_all(*(O.reorder_fwd(gp.to_np64(x), T, H, W) for x in (q, k, v)), rp, ci, T, H, W,
+                               1.0 / math.sqrt(d))
+    want = O.reorder_inv(o_ref, T, H, W)
+    err = np.abs(gp.to_np64(o_r) - want)
+    assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN
+
+
+def test_raster_path_equals_tiled_720p(sta, gp):
+    """The headline layer: raster mask and attention equal the tiled path."""
+    cfg = CONFIGS[2]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    q, k, v = make_qkv(cfg, device="cuda")
+    win = torch.from_numpy(window_params(cfg, window_scale(2, 0))).cuda()
+    params = sta.mask_params(cfg.top_p, cfg.k_min, True, 0.0, cfg.group_lo, win)
+    _raster_vs_tiled(sta, gp, q, k, v, B, Hh, d, T, H, W, params)
+
+
 # ------------------------------------------------------- failure detection
 def test_bounded_wait_reports_timeout_and_context_survives(sta, gp):
     """The pipeline's bounded wait, on a barrier nothing completes, gives up
