@@ -122,6 +122,7 @@ class ClockSampler:
         self.proc = None
         self.thread = None
         self.source = None
+        self.limit_w = None
 
     def _nvml_handle(self):
         import pynvml
@@ -135,13 +136,28 @@ class ClockSampler:
             nv, h = self._nvml_handle()
             smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
             self.source = "nvml"
+            try:
+                self.limit_w = nv.nvmlDeviceGetPowerManagementLimit(h) / 1000.0
+            except Exception:
+                self.limit_w = None
+
+            def power_w():
+                # instantaneous board power where the driver reports it, else
+                # the (about 1 s) averaged figure
+                try:
+                    fv = nv.nvmlDeviceGetFieldValues(h, [nv.NVML_FI_DEV_POWER_INSTANT])[0]
+                    if fv.nvmlReturn == 0:
+                        return fv.value.uiVal / 1000.0
+                except Exception:
+                    pass
+                return nv.nvmlDeviceGetPowerUsage(h) / 1000.0
 
             def run():
                 while not self.stop_flag.is_set():
                     try:
                         sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
                         bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                        watts = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        watts = power_w()
                     except Exception:
                         break
                     names = [nm for nm, b in self.REASONS if bits & b]
@@ -197,6 +213,8 @@ class ClockSampler:
                 "sm_min_mhz": min(x[1] for x in win) if win else None,
                 "sm_max_mhz": max(x[2] for x in win) if win else None,
                 "power_w_median": statistics.median(x[4] for x in win) if win else None,
+                "power_w_max": max(x[4] for x in win) if win else None,
+                "power_limit_w": self.limit_w,
                 "reasons": reasons, "samples": len(win), "source": self.source}
 
 
