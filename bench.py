@@ -541,6 +541,17 @@ def sweep(sta, dev, peak, reps=20):
     return rows
 
 
+def blas_threads():
+    """Threads of the BLAS library numpy uses (the oracle's matmuls)."""
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max((x.get("num_threads", 0) for x in threadpool_info() if x.get("user_api") == "blas"),
+                   default=None)
+    except Exception:
+        return None
+
+
 def cpu_oracle_sample(cfg, layer, budget_s, rows_per_head=8, max_heads=None):
     """Time the oracle (as it stands) on a bounded sample of the same layer:
     for sampled heads, its reorder, pooling, scores, selection and windows
@@ -616,7 +627,8 @@ def run_reference(args, rank, world):
         "data": "synthetic (seeded random-Fourier-feature Q/K, Gaussian V)",
         "config": {"workload": CONFIGS[CFG_INDEX].name, "tokens": cfg.L, "heads": cfg.heads, "d": cfg.d,
                    "sample": desc},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "blas_threads": blas_threads(),
+                         "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -628,7 +640,8 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=6)
+    ap.add_argument("--e2e-steps", type=int, default=16,
+                    help="pipelined end-to-end steps (fill and drain are amortised over them)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-mask run of the same kernel")
@@ -747,8 +760,8 @@ def main():
         cpu = None
         if world == 1 and not args.no_cpu_baseline and args.config_index == CFG_INDEX:
             v_cpu, desc, dt, threads = cpu_oracle_sample(cfg, layer, args.cpu_budget)
-            cpu = {"value": v_cpu, "unit": UNIT, "cores": threads, "kind": "oracle",
-                   "sample": f"{desc}; {dt:.1f} s"}
+            cpu = {"value": v_cpu, "unit": UNIT, "cores": threads, "blas_threads": blas_threads(),
+                   "kind": "oracle", "sample": f"{desc}; {dt:.1f} s"}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": max(3, args.warmup), "ms_per_step": elapsed_ms / K, "higher_is_better": True,
