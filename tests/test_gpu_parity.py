@@ -717,6 +717,26 @@ def test_raster_path_equals_tiled(sta, gp, d, T, H, W, Hh, B):
     assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T,H,W", [(1, 5, 3), (1, 20, 30), (2, 3, 40), (3, 1, 1), (7, 8, 8)])
+def test_degenerate_grids(sta, gp, d, T, H, W):
+    """One tile, one frame, tiles one token high, one token per frame, whole
+    tiles only: raster and tiled calls agree bit for bit and match the oracle."""
+    Hh, B = 2, 1
+    q, k, v = _structured(T, H, W, Hh, d, seed=H * 31 + W, B=B)
+    nh, nw, nt, _ = O.tile_grid(T, H, W)
+    win_t = torch.from_numpy(np.tile(np.array([[1, 1, 0, nw - 1]], dtype=np.int32), (Hh, 1, 1))).cuda()
+    params = sta.mask_params(0.9, 1, True, 0.0, (0,), win_t)
+    o_r = _raster_vs_tiled(sta, gp, q, k, v, B, Hh, d, T, H, W, params)
+    g = sta.grid(T, H, W)
+    bt = gp.build(gp.reorder(q, B, Hh, d, g), gp.reorder(k, B, Hh, d, g), B, Hh, d, g, params)
+    rp, ci, _ = gp.csr_np(bt)
+    o_ref, _ = O.attention_all(*(O.reorder_fwd(gp.to_np64(x), T, H, W) for x in (q, k, v)), rp, ci, T, H, W,
+                               1.0 / math.sqrt(d))
+    err = np.abs(gp.to_np64(o_r) - O.reorder_inv(o_ref, T, H, W))
+    assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN
+
+
 def test_raster_path_equals_tiled_720p(sta, gp):
     """The headline layer: raster mask and attention equal the tiled path."""
     cfg = CONFIGS[2]
