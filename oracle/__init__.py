@@ -16,6 +16,8 @@ Sources (pages on block-sparse attention for video diffusion transformers):
     top-k selection; Eqs. (9)-(10): the online per-head top-k floor.
   * AdaSpa (abstract): exact block importance from a cached log-sum-exp.
   * Compact Attention Figs. 3-5: recall-driven offline window search.
+  * Rectified SpaAttn (abstract): rectified attention, skipped tiles
+    recovered from pooled keys and values (reading stated in the module).
 
 Parity pins: every function here is checked in tests/test_oracle_*.py
 against closed forms, textbook routines (torch SDPA in fp64, scipy
@@ -43,5 +45,7 @@ from .sta_oracle import (  # noqa: F401
     attention_all,
     block_mass,
     search_windows,
+    pooled_kv,
+    rectified_attention_rows,
     SEARCH_MOVES,
 )

@@ -329,6 +329,71 @@ def attention_all(q_tiled, k_tiled, v_tiled, row_ptr, col_idx, T, H, W, sm_scale
 
 
 # --------------------------------------------------------------------------
+# Rectified attention (Rectified SpaAttn abstract: sparse attention inflates
+# the weights of the kept (critical) tokens, by a factor set by the weight it
+# drops, and loses the dropped (non-critical) tokens entirely; the fix
+# reallocates the kept weights with pooled weights and recovers the dropped
+# ones from the pooled query-key).
+# Reading (the abstract gives no formula): every key tile the row does not
+# list enters the softmax as one pooled key k_bar (mean of its real keys)
+# with multiplicity n (its real token count) and value v_bar (mean of its
+# real values); listed tiles enter token by token:
+#   Z_keep = sum_{j in listed}   exp(scale * q.k_j)
+#   Z_skip = sum_{t not listed}  n_t * exp(scale * q.k_bar_t)
+#   o      = (sum_listed exp(scale q.k_j) v_j + sum_skip n_t exp(scale q.k_bar_t) v_bar_t)
+#            / (Z_keep + Z_skip)
+#   lse    = log(Z_keep + Z_skip)
+# so the kept part is scaled by Z_keep / (Z_keep + Z_skip) (the reallocation)
+# and the skipped tiles add their pooled estimate. No gate is applied (the
+# abstract's gain-versus-error condition has no stated form).
+# --------------------------------------------------------------------------
+def pooled_kv(k_tiled, v_tiled, T, H, W):
+    """Per-tile means of K and V over real tokens and the real-token counts:
+    (k_bar [B, heads, Nt, d], v_bar [B, heads, Nt, d], n [Nt])."""
+    kb = pool(k_tiled, T, H, W)
+    vb = pool(v_tiled, T, H, W)
+    return kb, vb, tile_sizes(T, H, W).astype(np.float64)
+
+
+def rectified_attention_rows(q_tiled, k_tiled, v_tiled, row_ptr, col_idx, T, H, W, sm_scale, rows):
+    """Rectified attention for the CSR rows in `rows`; same return format as
+    attention_rows (row, token_rows, O, LSE)."""
+    q_tiled = np.asarray(q_tiled)
+    B, Hh, lpad, d = q_tiled.shape
+    _, _, nt, _ = tile_grid(T, H, W)
+    valid = valid_rows(T, H, W)
+    scale = float(sm_scale) if sm_scale else 1.0 / math.sqrt(d)
+    kbar, vbar, n = pooled_kv(k_tiled, v_tiled, T, H, W)
+    out = []
+    for r in rows:
+        r = int(r)
+        bh, qt = divmod(r, nt)
+        b, h = divmod(bh, Hh)
+        qrows = np.arange(qt * 64, qt * 64 + 64)
+        qrows = qrows[valid[qrows]]
+        q = q_tiled[b, h, qrows].astype(np.float64)
+        tiles = np.asarray(col_idx[int(row_ptr[r]):int(row_ptr[r + 1])], dtype=np.int64)
+        skip = np.setdiff1d(np.arange(nt), tiles)
+        krows = (tiles[:, None] * 64 + np.arange(64)[None, :]).reshape(-1)
+        krows = krows[valid[krows]]
+        k = np.asarray(k_tiled)[b, h, krows].astype(np.float64)
+        v = np.asarray(v_tiled)[b, h, krows].astype(np.float64)
+        # logits of kept tokens, and of skipped tiles with log-multiplicity
+        s_keep = (q @ k.T) * scale
+        s_skip = (q @ kbar[b, h, skip].T) * scale + np.log(n[skip])[None, :]
+        s = np.concatenate([s_keep, s_skip], axis=1)
+        vals = np.concatenate([v, vbar[b, h, skip]], axis=0)
+        if s.shape[1] == 0:
+            out.append((r, qrows, np.zeros((qrows.size, d)), np.full(qrows.size, -np.inf)))
+            continue
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        z = e.sum(axis=1, keepdims=True)
+        out.append((r, qrows, (e / z) @ vals, (m + np.log(z))[:, 0]))
+    return out
+
+
+# --------------------------------------------------------------------------
 # LSE-cached exact block importance (AdaSpa abstract: exact block importance
 # computed during a full-attention step with a cached log-sum-exp, then
 # reused for the block-sparse steps that follow).

@@ -535,3 +535,81 @@ def test_window_search_result_is_feasible_and_locally_final():
                     cand[g, e] -= 1
                 m2, cov2, _ = _coverage(cand, group_lo, T, H, W, mass)
                 assert (m & ~m2).sum() == 0 or cov2 < thr
+
+
+# ------------------------------------------- rectified attention (f4 reading)
+def _tile_constant(T, H, W, Hh, d, rng, scale=1.0):
+    """Raster [1, L, Hh, d] whose real tokens of each 1x8x8 tile share one
+    bf16-exact vector (so a tile's mean equals each of its tokens)."""
+    nh, nw, nt, _ = O.tile_grid(T, H, W)
+    per_tile = torch.from_numpy(rng.standard_normal((nt, Hh, d)) * scale).to(torch.bfloat16).double().numpy()
+    t, y, x = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    tile = ((t * nh + y // 8) * nw + x // 8).reshape(-1)
+    return per_tile[tile][None]
+
+
+def test_rectified_with_every_tile_listed_is_plain_attention():
+    T, H, W, d = 2, 9, 13, 8
+    q = _bf16_exact((1, T * H * W, 1, d), RNG, 2.0)
+    k = _bf16_exact((1, T * H * W, 1, d), RNG, 2.0)
+    v = _bf16_exact((1, T * H * W, 1, d), RNG)
+    qt, kt, vt = (O.reorder_fwd(a, T, H, W) for a in (q, k, v))
+    nt = O.tile_grid(T, H, W)[2]
+    rp, ci = O.mask_to_csr(np.ones((1, 1, nt, nt), dtype=bool))
+    plain = O.attention_rows(qt, kt, vt, rp, ci, T, H, W, 0.0, range(nt))
+    rect = O.rectified_attention_rows(qt, kt, vt, rp, ci, T, H, W, 0.0, range(nt))
+    for (r1, q1, o1, l1), (r2, q2, o2, l2) in zip(plain, rect):
+        assert r1 == r2 and np.array_equal(q1, q2)
+        assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+@pytest.mark.parametrize("density", [0.0, 0.3, 0.7])
+def test_rectified_is_exact_when_tiles_are_constant(density):
+    """If every token of a tile carries the tile's key and value, a skipped
+    tile's pooled term (multiplicity x exp(q.k_bar), value v_bar) is exactly
+    its tokens' contribution: for any mask the rectified output and LSE equal
+    dense attention over all real tokens (torch SDPA in fp64, scipy logsumexp).
+    Ragged grid, so multiplicities differ between tiles."""
+    rng = np.random.default_rng(int(density * 10) + 3)
+    T, H, W, d, Hh = 3, 11, 19, 8, 2
+    q = _bf16_exact((1, T * H * W, Hh, d), rng, 1.5)
+    k = _tile_constant(T, H, W, Hh, d, rng, 1.5)
+    v = _tile_constant(T, H, W, Hh, d, rng)
+    qt, kt, vt = (O.reorder_fwd(a, T, H, W) for a in (q, k, v))
+    nt = O.tile_grid(T, H, W)[2]
+    mask = rng.random((1, Hh, nt, nt)) < density
+    rp, ci = O.mask_to_csr(mask)
+    res = O.rectified_attention_rows(qt, kt, vt, rp, ci, T, H, W, 0.0, range(Hh * nt))
+    Ot = np.full(qt.shape, np.nan)
+    Lt = np.full(qt.shape[:3], np.nan)
+    for r, qrows, o, lse in res:
+        h, _ = divmod(r, nt)
+        Ot[0, h, qrows] = o
+        Lt[0, h, qrows] = lse
+    o_r = O.reorder_inv(Ot, T, H, W)[0]
+    l_r = O.reorder_inv(Lt[..., None], T, H, W)[0, :, :, 0]
+    for h in range(Hh):
+        ref = _sdpa64(q[0, :, h], k[0, :, h], v[0, :, h], 1 / math.sqrt(d))
+        assert np.allclose(o_r[:, h], ref, atol=1e-10, rtol=1e-10)
+        lse_ref = scipy.special.logsumexp(q[0, :, h] @ k[0, :, h].T / math.sqrt(d), axis=1)
+        assert np.allclose(l_r[:, h], lse_ref, atol=1e-10)
+
+
+def test_rectified_weights_sum_to_one_and_pool_over_real_tokens():
+    """V = 1 gives exactly 1 (kept and pooled weights share one normaliser);
+    the pooled key and value of a partial tile average only its real tokens."""
+    T, H, W, d = 2, 10, 12, 8
+    q = _bf16_exact((1, T * H * W, 1, d), RNG, 2.0)
+    k = _bf16_exact((1, T * H * W, 1, d), RNG, 2.0)
+    qt, kt = (O.reorder_fwd(a, T, H, W) for a in (q, k))
+    vt = O.reorder_fwd(np.ones((1, T * H * W, 1, d)), T, H, W)
+    nt = O.tile_grid(T, H, W)[2]
+    mask = RNG.random((1, 1, nt, nt)) < 0.4
+    rp, ci = O.mask_to_csr(mask)
+    for _, _, o, _ in O.rectified_attention_rows(qt, kt, vt, rp, ci, T, H, W, 0.0, range(nt)):
+        assert np.allclose(o, 1.0, atol=1e-12)
+    kb, vb, n = O.pooled_kv(kt, vt, T, H, W)
+    assert n.sum() == T * H * W and np.allclose(vb, 1.0)
+    # tile 1 is cut by the right edge (W = 12): 8 x 4 real tokens
+    real = kt[0, 0, 64:128][O.valid_rows(T, H, W)[64:128]]
+    assert real.shape[0] == n[1] == 32 and np.allclose(kb[0, 0, 1], real.mean(0))
