@@ -76,6 +76,11 @@ _lib.sta_build_mask_raster.argtypes = _lib.sta_build_mask.argtypes
 _lib.sta_build_mask_raster.restype = ctypes.c_int
 _lib.sta_attn_fwd_raster.argtypes = _lib.sta_attn_fwd.argtypes
 _lib.sta_attn_fwd_raster.restype = ctypes.c_int
+_lib.sta_rectified_workspace.argtypes = [_i32, _i32, _i32, Grid]
+_lib.sta_rectified_workspace.restype = _sz
+_lib.sta_attn_fwd_rectified.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i32, _i32, _i32, Grid,
+                                        _f32, _vp]
+_lib.sta_attn_fwd_rectified.restype = ctypes.c_int
 _lib.sta_attn_fwd_block_mass.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, Grid,
                                          _f32, _vp]
 _lib.sta_attn_fwd_block_mass.restype = ctypes.c_int
@@ -196,6 +201,19 @@ def sta_attn_fwd_raster(q, k, v, o, lse, row_ptr, col_idx, B, heads, d, g, sm_sc
     _check(_lib.sta_attn_fwd_raster(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(row_ptr),
                                     _ptr(col_idx), B, heads, d, g, float(sm_scale), _stream(stream)),
            "sta_attn_fwd_raster")
+
+
+def sta_rectified_workspace(B, heads, d, g):
+    return int(_lib.sta_rectified_workspace(B, heads, d, g))
+
+
+def sta_attn_fwd_rectified(q, k, v, o, lse, row_ptr, col_idx, workspace, ws_bytes, B, heads, d, g,
+                           sm_scale=0.0, stream=None):
+    """Rectified attention: unlisted tiles enter as pooled keys / values."""
+    _check(_lib.sta_attn_fwd_rectified(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(row_ptr),
+                                       _ptr(col_idx), _ptr(workspace), int(ws_bytes), B, heads, d, g,
+                                       float(sm_scale), _stream(stream)),
+           "sta_attn_fwd_rectified")
 
 
 def sta_attn_fwd_block_mass(q, k, v, o, lse, row_ptr, col_idx, lse_cached, block_mass, B, heads, d, g,

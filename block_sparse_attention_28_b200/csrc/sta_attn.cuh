@@ -35,6 +35,7 @@ constexpr int WARP_MMA = 5;
 // bits 23-25, flag bit 26), and the two halves' membership flags.
 constexpr uint32_t KT_MASK = (1u << 20) - 1u;
 constexpr uint32_t EXT_PARTIAL = 1u << 26;
+constexpr uint32_t VIRT = 1u << 27;  // pooled key tile of the rectified form (index in bits 0-19)
 constexpr uint32_t FLAG_A = 1u << 30;
 constexpr uint32_t FLAG_B = 1u << 31;
 constexpr uint32_t TMEM_COLS = 256;
@@ -83,10 +84,11 @@ struct Cfg {
   static constexpr uint32_t IDESC_O = tc::idesc_bf16(128, D, true);
 };
 
+// ntp: pooled key rows of the rectified form (Nt rounded up to 64), 0 otherwise.
 template <int D>
-inline size_t smem_bytes(int nt) {
+inline size_t smem_bytes(int nt, int ntp = 0) {
   const int wpr = (nt + 31) / 32;
-  return (size_t)Cfg<D>::OFF_LIST + (size_t)(2 * wpr + nt) * 4 + 1024;
+  return (size_t)Cfg<D>::OFF_LIST + (size_t)(2 * wpr + nt + ntp / 64 + ntp) * 4 + 1024;
 }
 
 // MASS: also accumulate the LSE-cached exact block importance (AdaSpa) of
@@ -100,13 +102,24 @@ inline size_t smem_bytes(int nt) {
 // head x 8 columns x 8 rows x 1 frame, which TMA writes to shared memory in
 // the tile's token order (zeros beyond the grid edge), so the permutation to
 // tiles costs no pass over memory; O rows go straight to their raster rows.
-template <int D, bool MASS, bool RASTER>
+//
+// RECT (rectified form, Rectified SpaAttn abstract): after the listed tiles
+// the CTA walks ntp/64 pooled tiles whose 64 "keys" are the tile means
+// k_bar of key tiles 64u .. 64u+63 (and values v_bar), each key carrying its
+// tile's real-token count n as a multiplicity: the score of column kt is
+// scale * q.k_bar_kt + ln n_kt, and columns of tiles the row lists (or past
+// Nt) are masked. The online softmax then weighs listed tokens and pooled
+// tiles against one normaliser.
+template <int D, bool MASS, bool RASTER, bool RECT = false>
 __global__ void __launch_bounds__(NUM_THREADS, MIN_BLOCKS_PER_SM)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16 *__restrict__ out,
                 float *__restrict__ lse, const int *__restrict__ row_ptr,
                 const int *__restrict__ col_idx, Geo g, float scale_log2,
-                const float *__restrict__ lse_in, float *__restrict__ block_mass, int heads) {
+                const float *__restrict__ lse_in, float *__restrict__ block_mass, int heads,
+                const __grid_constant__ CUtensorMap tm_kbar, const __grid_constant__ CUtensorMap tm_vbar,
+                int ntp) {
+  static_assert(!(MASS && RECT) && !(RASTER && RECT), "the rectified form is tiled and mass-free");
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -228,11 +241,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   __syncthreads();
   tc::fence_after();
   const uint32_t tmem = misc[0];
-  const int n = (int)misc[1];
+  const int n_list = (int)misc[1];
+  const int nv = RECT ? ntp / 64 : 0;  // pooled tiles after the listed ones
+  const int n = n_list + nv;
+  float *bias = reinterpret_cast<float *>(U + nt + nv);  // ln n_kt / scale, per pooled key
+  if (RECT) {
+    for (int u = tid; u < nv; u += NUM_THREADS) U[n_list + u] = (uint32_t)u | VIRT | FLAG_A | FLAG_B;
+    const float ln2_over = 1.0f / scale_log2;  // log2(n) / scale_log2 = ln(n) / scale
+    for (int kt = tid; kt < ntp; kt += NUM_THREADS) {
+      float b = 0.0f;
+      if (kt < nt) {
+        const int rem = kt % (g.NH * g.NW);
+        const int ty = rem / g.NW, tx = rem - ty * g.NW;
+        b = log2f((float)(valid_extent(g.H, ty) * valid_extent(g.W, tx))) * ln2_over;
+      }
+      bias[kt] = b;
+    }
+  }
 #if STA_ATTN_EXT_LIST
   // Mark key tiles cut by the grid edge once per entry, so that the softmax
   // loop needs no division to find them.
-  for (int i = tid; i < n; i += NUM_THREADS) {
+  for (int i = tid; i < n_list; i += NUM_THREADS) {
     const uint32_t e = U[i];
     const int kt = (int)(e & KT_MASK);
     const int rem = kt % (g.NH * g.NW);
@@ -241,6 +270,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (vy < 8 || vx < 8) U[i] = e | EXT_PARTIAL | ((uint32_t)(vy - 1) << 20) | ((uint32_t)(vx - 1) << 23);
   }
   __syncthreads();
+#else
+  if (RECT) __syncthreads();
 #endif
 
   if (warp == WARP_PRODUCER) {
@@ -269,28 +300,37 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (hasB) load_tile_atoms(&tm_q, q_full, sbase + C::OFF_Q + 8192, C::Q_REGION, qtB);
       // K runs KLEAD tiles ahead of V: K_{j+1} is needed by S_{j+1}, which the
       // MMA warp issues before P.V_j.
-      auto load_tile = [&](const CUtensorMap *map, uint64_t *full, uint64_t *empty, int off, int ns,
-                           int j) -> bool {
+      auto load_tile = [&](const CUtensorMap *map, const CUtensorMap *pooled_map, uint64_t *full,
+                           uint64_t *empty, int off, int ns, int j) -> bool {
         const int s = j % ns, u = j / ns;
         if (u > 0 && !tc::mbar_wait(empty + s, (u - 1) & 1, abort_flag, WAIT_LIMIT)) return false;
-        const int kt = (int)(U[j] & KT_MASK);
+        const uint32_t e = U[j];
+        const int kt = (int)(e & KT_MASK);
         tc::mbar_expect_tx(full + s, C::TILE_BYTES);
-        load_tile_atoms(map, full + s, sbase + off + s * C::TILE_BYTES, 8192u, kt);
+        if (RECT && (e & VIRT) != 0u) {
+          // 64 pooled rows [64 kt, 64 kt + 64) of this head
+          const int row = (int)((long long)bh * ntp + 64LL * kt);
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb)
+            tc::tma_load_2d(sbase + off + s * C::TILE_BYTES + kb * 8192, pooled_map, full + s, kb * 64, row);
+        } else {
+          load_tile_atoms(map, full + s, sbase + off + s * C::TILE_BYTES, 8192u, kt);
+        }
         return true;
       };
       int issued_k = 0, issued_v = 0;
       bool ok = true;
       for (int j = 0; ok && j < C::KLEAD && j < n; ++j) {
-        ok = load_tile(&tm_k, k_full, k_empty, C::OFF_K, C::NSK, j);
+        ok = load_tile(&tm_k, &tm_kbar, k_full, k_empty, C::OFF_K, C::NSK, j);
         if (ok) issued_k = j + 1;
       }
       for (int j = 0; ok && j < n; ++j) {
         if (j + C::KLEAD < n) {
-          ok = load_tile(&tm_k, k_full, k_empty, C::OFF_K, C::NSK, j + C::KLEAD);
+          ok = load_tile(&tm_k, &tm_kbar, k_full, k_empty, C::OFF_K, C::NSK, j + C::KLEAD);
           if (!ok) break;
           issued_k = j + C::KLEAD + 1;
         }
-        ok = load_tile(&tm_v, v_full, v_empty, C::OFF_V, C::NSV, j);
+        ok = load_tile(&tm_v, &tm_vbar, v_full, v_empty, C::OFF_V, C::NSV, j);
         if (ok) issued_v = j + 1;
       }
       // Copies still in flight must land before the CTA can exit.
@@ -394,6 +434,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tc::tmem_ld64(sS, rr);
 #pragma unroll
           for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(rr[c]);
+        }
+        // pooled tiles (rectified form): columns of listed tiles and past Nt
+        // are masked; the others get their multiplicity bias ln n / scale
+        if (RECT && (e & VIRT) != 0u) {
+          const int u = (int)(e & KT_MASK);
+          const uint32_t *bm = halfB ? bmB : bmA;
+          const uint32_t w0 = (2 * u < wpr) ? bm[2 * u] : 0u;
+          const uint32_t w1 = (2 * u + 1 < wpr) ? bm[2 * u + 1] : 0u;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const int kp = 64 * u + c;
+            const bool listed = (((c < 32) ? (w0 >> c) : (w1 >> (c - 32))) & 1u) != 0u;
+            s[c] = (kp < nt && !listed) ? s[c] + bias[kp] : -INFINITY;
+          }
         }
         // keys of partial tiles beyond the grid edge
         const int kt = (int)(e & KT_MASK);

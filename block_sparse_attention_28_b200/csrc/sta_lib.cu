@@ -198,13 +198,17 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
   return STA_OK;
 }
 
-template <int D, bool MASS, bool RASTER = false>
+// Pooled key rows per head of the rectified form: Nt rounded up to 64.
+inline int pooled_rows(const Geo &g) { return (g.Nt + 63) / 64 * 64; }
+
+template <int D, bool MASS, bool RASTER = false, bool RECT = false>
 sta_status launch_attn(const void *q, const void *k, const void *v, void *o, float *lse,
                        const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
                        const Geo &g, float sm_scale, cudaStream_t s, const float *lse_in = nullptr,
-                       float *block_mass = nullptr) {
+                       float *block_mass = nullptr, const void *kbar = nullptr, const void *vbar = nullptr) {
   const unsigned long long rows = (unsigned long long)B * heads * g.Lpad;
-  CUtensorMap tq, tk, tv;
+  const int ntp = RECT ? pooled_rows(g) : 0;
+  CUtensorMap tq, tk, tv, tkb, tvb;
   if (RASTER) {
     if (!make_raster_map(&tq, q, g, B, heads, D) || !make_raster_map(&tk, k, g, B, heads, D) ||
         !make_raster_map(&tv, v, g, B, heads, D))
@@ -213,18 +217,25 @@ sta_status launch_attn(const void *q, const void *k, const void *v, void *o, flo
              !make_tile_map(&tv, v, rows, D)) {
     return STA_ERR_CUDA;
   }
-  const size_t smem = attn::smem_bytes<D>(g.Nt);
+  if (RECT) {
+    const unsigned long long prow = (unsigned long long)B * heads * ntp;
+    if (!make_tile_map(&tkb, kbar, prow, D) || !make_tile_map(&tvb, vbar, prow, D)) return STA_ERR_CUDA;
+  } else {
+    tkb = tk;  // unused
+    tvb = tv;
+  }
+  const size_t smem = attn::smem_bytes<D>(g.Nt, ntp);
   if (smem > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
-  STA_CUDA_TRY(cudaFuncSetAttribute(attn::attn_fwd_kernel<D, MASS, RASTER>,
+  STA_CUDA_TRY(cudaFuncSetAttribute(attn::attn_fwd_kernel<D, MASS, RASTER, RECT>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   if (MASS)
     STA_CUDA_TRY(cudaMemsetAsync(block_mass, 0, (size_t)B * heads * g.Nt * g.Nt * sizeof(float), s));
   const float scale = sm_scale != 0.0f ? sm_scale : 1.0f / sqrtf((float)D);
   const float scale_log2 = scale * 1.4426950408889634f;
   dim3 grid((unsigned)((g.Nt + 1) / 2), (unsigned)(B * heads));
-  attn::attn_fwd_kernel<D, MASS, RASTER><<<grid, attn::NUM_THREADS, smem, s>>>(
+  attn::attn_fwd_kernel<D, MASS, RASTER, RECT><<<grid, attn::NUM_THREADS, smem, s>>>(
       tq, tk, tv, static_cast<__nv_bfloat16 *>(o), lse, row_ptr, col_idx, g, scale_log2, lse_in,
-      block_mass, heads);
+      block_mass, heads, tkb, tvb, ntp);
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }
@@ -365,6 +376,51 @@ sta_status sta_attn_fwd_block_mass(const void *q, const void *k, const void *v, 
                                              lse_cached, block_mass)
                     : launch_attn<64, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s,
                                             lse_cached, block_mass);
+}
+
+size_t sta_rectified_workspace(int32_t B, int32_t heads, int32_t d, sta_grid g) {
+  Geo geo;
+  sta_status st = STA_OK;
+  if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return 0;
+  const size_t one = align_up((size_t)B * heads * pooled_rows(geo) * d * 2, 256);
+  return 2 * one;
+}
+
+sta_status sta_attn_fwd_rectified(const void *q, const void *k, const void *v, void *o, float *lse,
+                                  const int32_t *row_ptr, const int32_t *col_idx, void *workspace,
+                                  size_t ws_bytes, int32_t B, int32_t heads, int32_t d, sta_grid g,
+                                  float sm_scale, sta_stream_t stream) {
+  Geo geo;
+  sta_status st = STA_OK;
+  if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || row_ptr == nullptr || col_idx == nullptr)
+    return STA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return STA_ERR_INVALID_ARG;
+  if (!(sm_scale == sm_scale) || sm_scale < 0.0f) return STA_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      ws_bytes < sta_rectified_workspace(B, heads, d, g))
+    return STA_ERR_WORKSPACE;
+  if (!device_is_sm100()) return STA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int ntp = pooled_rows(geo);
+  const size_t one = align_up((size_t)B * heads * ntp * d * 2, 256);
+  uint8_t *kbar = static_cast<uint8_t *>(workspace);
+  uint8_t *vbar = kbar + one;
+  const long long bh = (long long)B * heads;
+  const unsigned blocks = (unsigned)((2 * bh * ntp * 32 + 255) / 256);
+  if (d == 128)
+    pool_kv_kernel<128><<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
+                                                reinterpret_cast<uint4 *>(kbar), reinterpret_cast<uint4 *>(vbar),
+                                                bh, ntp, geo);
+  else
+    pool_kv_kernel<64><<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
+                                               reinterpret_cast<uint4 *>(kbar), reinterpret_cast<uint4 *>(vbar),
+                                               bh, ntp, geo);
+  STA_CUDA_TRY(cudaGetLastError());
+  return (d == 128) ? launch_attn<128, false, false, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo,
+                                                           sm_scale, s, nullptr, nullptr, kbar, vbar)
+                    : launch_attn<64, false, false, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo,
+                                                          sm_scale, s, nullptr, nullptr, kbar, vbar);
 }
 
 sta_status sta_search_windows(const float *block_mass, int32_t B, int32_t heads, sta_grid g,

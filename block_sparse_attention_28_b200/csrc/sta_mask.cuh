@@ -86,6 +86,67 @@ pool_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k, float *__r
   }
 }
 
+// Pooled K and V of the rectified attention: row (bh, kt) of kbar / vbar is
+// the mean over the real tokens of tile kt (fp64 sum, rounded once to bf16),
+// for kt < Nt; rows Nt .. ntp-1 are zero. One warp per (tensor, bh, kt).
+template <int D>
+__global__ void __launch_bounds__(256)
+pool_kv_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v, uint4 *__restrict__ kbar,
+               uint4 *__restrict__ vbar, long long bh_total, int ntp, Geo g) {
+  constexpr int CPR = D / 8;
+  constexpr int RPI = 32 / CPR;
+  const long long warp_id = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long rows = bh_total * ntp;
+  const bool is_v = warp_id >= rows;
+  const long long idx = is_v ? warp_id - rows : warp_id;
+  if (idx >= rows) return;
+  const long long bh = idx / ntp;
+  const int kt = (int)(idx - bh * ntp);
+  const uint4 *src = is_v ? v : k;
+  uint4 *dst = (is_v ? vbar : kbar) + idx * CPR;
+  const int sub = lane / CPR, c = lane - sub * CPR;
+  if (kt >= g.Nt) {
+    if (sub == 0) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  const int rem = kt % (g.NH * g.NW);
+  const int ty = rem / g.NW, tx = rem - ty * g.NW;
+  const int vy = valid_extent(g.H, ty), vx = valid_extent(g.W, tx);
+  const uint4 *base = src + (bh * g.Nt + kt) * 64 * CPR;
+  double acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+  for (int i = 0; i < 64 / RPI; ++i) {
+    const int r = i * RPI + sub;
+    if ((r >> 3) < vy && (r & 7) < vx) {
+      const uint4 w = base[r * CPR + c];
+      const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&w);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(p[e]);
+        acc[2 * e] += (double)f.x;
+        acc[2 * e + 1] += (double)f.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int off = CPR; off < 32; off <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+  }
+  if (sub == 0) {
+    const double cnt = (double)(vy * vx);
+    uint32_t pk[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __nv_bfloat162 b2 = __floats2bfloat162_rn((float)(acc[2 * e] / cnt), (float)(acc[2 * e + 1] / cnt));
+      pk[e] = *reinterpret_cast<uint32_t *>(&b2);
+    }
+    dst[c] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
 // ------------------------------------------------------ scores + selection
 constexpr int SEL_THREADS = 256;
 constexpr int SEL_QB = 16;  // query tiles per CTA

@@ -220,6 +220,27 @@ sta_status sta_attn_fwd_block_mass(const void *q, const void *k, const void *v, 
                                    int32_t heads, int32_t d, sta_grid g, float sm_scale,
                                    sta_stream_t stream);
 
+/* sta_attn_fwd_rectified -- rectified block-sparse attention (Rectified
+ * SpaAttn abstract: dropping tiles inflates the kept weights and loses the
+ * dropped ones; the kept weights are reallocated with pooled weights and the
+ * dropped ones recovered from the pooled query-key). Reading (the abstract
+ * gives no formula): every key tile NOT listed for the row enters the softmax
+ * as one pooled key k_bar (mean of its real keys) with value v_bar (mean of
+ * its real values) and multiplicity n (its real token count):
+ *   o   = (sum_listed e^{s q.k_j} v_j + sum_unlisted n_t e^{s q.k_bar_t} v_bar_t)
+ *         / (sum_listed e^{s q.k_j} + sum_unlisted n_t e^{s q.k_bar_t})
+ *   lse = ln(denominator), s = sm_scale (0 -> 1/sqrt(d))
+ * With every tile listed this is sta_attn_fwd (bit for bit).
+ *   q, k, v, o, lse, row_ptr, col_idx : as sta_attn_fwd (tiled layout)
+ *   workspace : device, >= sta_rectified_workspace() bytes, 256-aligned;
+ *               receives the pooled K and V (bf16) of every head
+ * Errors as sta_attn_fwd, plus STA_ERR_WORKSPACE. */
+size_t sta_rectified_workspace(int32_t B, int32_t heads, int32_t d, sta_grid g);
+sta_status sta_attn_fwd_rectified(const void *q, const void *k, const void *v, void *o, float *lse,
+                                  const int32_t *row_ptr, const int32_t *col_idx, void *workspace,
+                                  size_t ws_bytes, int32_t B, int32_t heads, int32_t d, sta_grid g,
+                                  float sm_scale, sta_stream_t stream);
+
 /* sta_search_windows -- recall-driven offline search of the dual windows
  * (Compact Attention Fig. 3: the windows are shrunk iteratively under a recall
  * target tau and a cost weight lambda, and the configurations are stored for

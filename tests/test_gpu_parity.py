@@ -747,6 +747,97 @@ def test_raster_path_equals_tiled_720p(sta, gp):
     _raster_vs_tiled(sta, gp, q, k, v, B, Hh, d, T, H, W, params)
 
 
+# ---------------------------------------------- rectified attention (f4)
+def _rect(sta, qt, kt, vt, rp, ci, B, Hh, d, g, sm_scale=0.0):
+    ws_bytes = sta.sta_rectified_workspace(B, Hh, d, g)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    o = torch.full_like(qt, float("nan"))
+    lse = torch.full(qt.shape[:3], float("nan"), dtype=torch.float32, device="cuda")
+    sta.sta_attn_fwd_rectified(qt, kt, vt, o, lse, rp, ci, ws, ws_bytes, B, Hh, d, g, sm_scale)
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    return o, lse
+
+
+def _rect_check(sta, gp, qt, kt, vt, rp_t, ci_t, B, Hh, d, T, H, W, rows):
+    """Rows of the GPU's rectified attention against the oracle, one head at
+    a time (the oracle pools the whole head's K and V)."""
+    g = sta.grid(T, H, W)
+    o, lse = _rect(sta, qt, kt, vt, rp_t, ci_t, B, Hh, d, g)
+    nt = sta.sta_num_tiles(g)
+    rp, ci = rp_t.cpu().numpy(), ci_t.cpu().numpy()
+    by_head = {}
+    for r in rows:
+        by_head.setdefault(int(r) // nt, []).append(int(r) % nt)
+    errs = []
+    for bh, qts in sorted(by_head.items()):
+        b, h = divmod(bh, Hh)
+        one = [gp.to_np64(x[b:b + 1, h:h + 1]) for x in (qt, kt, vt)]
+        rp_h = rp[bh * nt:(bh + 1) * nt + 1] - rp[bh * nt]
+        ci_h = ci[rp[bh * nt]:rp[(bh + 1) * nt]]
+        o_np = gp.to_np64(o[b, h])
+        l_np = lse[b, h].double().cpu().numpy()
+        for _, qrows, o_ref, l_ref in O.rectified_attention_rows(*one, rp_h, ci_h, T, H, W, 0.0, qts):
+            errs.append(np.abs(o_np[qrows] - o_ref).ravel())
+            assert np.all(np.abs(l_np[qrows] - l_ref) <= LSE_TOL * np.maximum(1.0, np.abs(l_ref)))
+    err = np.concatenate(errs)
+    assert np.isfinite(err).all()
+    assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (err.max(), err.mean())
+    return o, lse
+
+
+def test_rectified_with_every_tile_listed_equals_plain(sta, gp):
+    """All tiles listed: every pooled column is masked and the output is that
+    of sta_attn_fwd, bit for bit."""
+    T, H, W, Hh, B, d = 3, 19, 37, 2, 2, 128
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = _structured(T, H, W, Hh, d, seed=5, B=B)
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    rp, ci = _custom_csr(np.ones((B, Hh, nt, nt), dtype=bool))
+    o_p, l_p = gp.attn(qt, kt, vt, rp, ci, B, Hh, d, g)
+    o_r, l_r = _rect(sta, qt, kt, vt, rp, ci, B, Hh, d, g)
+    valid = torch.from_numpy(O.valid_rows(T, H, W)).cuda()
+    assert torch.equal(o_r[:, :, valid].view(torch.int16), o_p[:, :, valid].view(torch.int16))
+    assert torch.equal(l_r[:, :, valid], l_p[:, :, valid])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("density", [0.0, 0.1, 0.5])
+def test_rectified_ragged_sparse(sta, gp, d, density):
+    """Ragged grid (odd tile count, partial tiles, Nt not a multiple of 64),
+    random lists incl. empty rows: every row against the oracle."""
+    T, H, W, Hh, B = 3, 19, 37, 2, 2
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = _structured(T, H, W, Hh, d, seed=11, B=B)
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    rng = np.random.default_rng(int(density * 100) + d)
+    mask = rng.random((B, Hh, nt, nt)) < density
+    mask[0, 0, 3] = False  # an empty row
+    rp, ci = _custom_csr(mask)
+    _rect_check(sta, gp, qt, kt, vt, rp, ci, B, Hh, d, T, H, W, range(B * Hh * nt))
+
+
+def test_rectified_720p_sampled_rows(sta, gp):
+    """The headline layer with its own mask: sampled rows against the oracle."""
+    cfg = CONFIGS[2]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = make_qkv(cfg, device="cuda")
+    qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
+    del q, k, v
+    win = torch.from_numpy(window_params(cfg, window_scale(2, 0))).cuda()
+    params = sta.mask_params(cfg.top_p, cfg.k_min, True, 0.0, cfg.group_lo, win)
+    bufs = gp.build(qt, kt, B, Hh, d, g, params, with_mask=False, with_probs=False)
+    rng = np.random.default_rng(17)
+    rows = sorted(rng.choice(B * Hh * nt, 6, replace=False).tolist())
+    nnz = int(bufs.nnz.item())
+    _rect_check(sta, gp, qt, kt, vt, bufs.row_ptr, bufs.col_idx[:max(nnz, 1)], B, Hh, d, T, H, W, rows)
+    del qt, kt, vt
+
+
 # ------------------------------------------------------- failure detection
 def test_bounded_wait_reports_timeout_and_context_survives(sta, gp):
     """The pipeline's bounded wait, on a barrier nothing completes, gives up
