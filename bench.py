@@ -458,6 +458,17 @@ def search_curve(sta, cfg_index, dev, taus=(0.8, 0.9, 0.95, 0.99), lam=1.0):
     return {"workload": cfg.name, "block_mass_ms": mass_ms, "curve": rows}
 
 
+def real_tiled_rows(cfg):
+    """Boolean [Lpad]: tiled rows that hold a real token (not grid padding)."""
+    nh, nw = -(-cfg.H // 8), -(-cfg.W // 8)
+    n = np.arange(cfg.T * nh * nw * 64)
+    tile, r = n // 64, n % 64
+    rem = tile % (nh * nw)
+    y = (rem // nw) * 8 + r // 8
+    x = (rem % nw) * 8 + r % 8
+    return (y < cfg.H) & (x < cfg.W)
+
+
 def _median_ms(fn, reps):
     """Median CUDA-event time of `reps` launches of fn (each timed alone)."""
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
@@ -511,6 +522,44 @@ def sweep(sta, dev, peak, reps=20):
             attn_line(CONFIGS[ci].name, layer, extra)
             del layer
             torch.cuda.empty_cache()
+
+    # rectified form on the 720p layer: time, and the error against dense
+    # attention of the plain and of the rectified output on the same mask
+    layer = Layer(sta, CONFIGS[2], dev, cfg_index=2)
+    layer.reorder_in()
+    layer.build_tiled()
+    B, Hh, d, g, nt = layer.B, layer.Hh, layer.d, layer.g, layer.nt
+    ws_bytes = sta.sta_rectified_workspace(B, Hh, d, g)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    o_rect = torch.empty_like(layer.qt)
+
+    def rect():
+        sta.sta_attn_fwd_rectified(layer.qt, layer.kt, layer.vt, o_rect, None, layer.bufs.row_ptr,
+                                   layer.bufs.col_idx, ws, ws_bytes, B, Hh, d, g)
+
+    rect_ms = _median_ms(rect, reps)
+    plain_ms = _median_ms(layer.attn_tiled, reps)
+    o_plain = layer.ot.float()
+    R = B * Hh * nt
+    rp = (torch.arange(R + 1, device=dev, dtype=torch.int64) * nt).to(torch.int32)
+    ci = torch.arange(nt, device=dev, dtype=torch.int32).repeat(R)
+    sta.sta_attn_fwd(layer.qt, layer.kt, layer.vt, layer.ot, None, rp, ci, B, Hh, d, g)
+    torch.cuda.synchronize()
+    o_dense = layer.ot.float()
+    real = torch.from_numpy(real_tiled_rows(layer.cfg)).to(dev)
+
+    def rel(a):
+        diff = (a - o_dense)[:, :, real]
+        return float(torch.linalg.vector_norm(diff) / torch.linalg.vector_norm(o_dense[:, :, real]))
+
+    line = {"workload": CONFIGS[2].name + " (rectified form)", "density": layer.kept_pairs() / (R * nt),
+            "kept_pairs": layer.kept_pairs(), "rectified_ms": rect_ms, "plain_ms_same_mask": plain_ms,
+            "pooled_steps_per_cta": (nt + 63) // 64,
+            "rel_err_vs_dense_plain": rel(o_plain), "rel_err_vs_dense_rectified": rel(o_rect.float())}
+    rows.append(line)
+    print(json.dumps(line), flush=True)
+    del layer, o_rect, o_plain, o_dense, ws, rp, ci
+    torch.cuda.empty_cache()
 
     # reuse layer: top_p = 0, k_min = round(rho * Nt), no windows; mask from step 0
     cfg = CONFIGS[4]
