@@ -45,13 +45,6 @@ constexpr long long DRAIN_LIMIT = 200000000LL;   // after an abort
 constexpr float RESCALE_LOG2 = 8.0f;             // lazy O rescale threshold
 constexpr int MIN_BLOCKS_PER_SM = 2;             // two CTAs share an SM: one's softmax
                                                  // overlaps the other's MMAs
-#ifndef STA_EXP2_POLY_EVERY
-#define STA_EXP2_POLY_EVERY 0                    // every k-th column pair uses ex2_poly
-#endif
-
-#ifndef STA_ATTN_EXT_LIST
-#define STA_ATTN_EXT_LIST 1
-#endif
 #ifndef STA_ATTN_NSK
 #define STA_ATTN_NSK 2                           // K ring stages at d = 128
 #endif
@@ -258,7 +251,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       bias[kt] = b;
     }
   }
-#if STA_ATTN_EXT_LIST
   // Mark key tiles cut by the grid edge once per entry, so that the softmax
   // loop needs no division to find them.
   for (int i = tid; i < n_list; i += NUM_THREADS) {
@@ -270,9 +262,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (vy < 8 || vx < 8) U[i] = e | EXT_PARTIAL | ((uint32_t)(vy - 1) << 20) | ((uint32_t)(vx - 1) << 23);
   }
   __syncthreads();
-#else
-  if (RECT) __syncthreads();
-#endif
 
   if (warp == WARP_PRODUCER) {
     // ------------------------------------------------------ TMA producer
@@ -451,15 +440,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         // keys of partial tiles beyond the grid edge
         const int kt = (int)(e & KT_MASK);
-#if STA_ATTN_EXT_LIST
         if (e & EXT_PARTIAL) {
           const int vy = (int)((e >> 20) & 7u) + 1, vx = (int)((e >> 23) & 7u) + 1;
-#else
-        const int rem = kt % (g.NH * g.NW);
-        const int ty = rem / g.NW, tx = rem - ty * g.NW;
-        const int vy = valid_extent(g.H, ty), vx = valid_extent(g.W, tx);
-        if (vy < 8 || vx < 8) {
-#endif
 #pragma unroll
           for (int c = 0; c < 64; ++c)
             if ((c >> 3) >= vy || (c & 7) >= vx) s[c] = -INFINITY;
@@ -489,15 +471,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int c = 0; c < 32; ++c) {
           float x0, x1;
           tc::f2_unpack(tc::f2_fma(tc::f2_pack(s[2 * c], s[2 * c + 1]), scale2, negm2), x0, x1);
-          float p0, p1;
-          if (STA_EXP2_POLY_EVERY > 0 && (c % (STA_EXP2_POLY_EVERY > 0 ? STA_EXP2_POLY_EVERY : 1)) ==
-                                             STA_EXP2_POLY_EVERY - 1) {
-            p0 = tc::ex2_poly(x0);
-            p1 = tc::ex2_poly(x1);
-          } else {
-            p0 = tc::ex2(x0);
-            p1 = tc::ex2(x1);
-          }
+          const float p0 = tc::ex2(x0), p1 = tc::ex2(x1);
           acc[c & 3] = tc::f2_add(acc[c & 3], tc::f2_pack(p0, p1));
           pk[c] = tc::pack_bf16(p0, p1);
         }

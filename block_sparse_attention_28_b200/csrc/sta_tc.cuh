@@ -209,27 +209,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA / integer pipes, to take part of the softmax exponentials off
-// the MUFU unit. Range reduction x = n + f with n = round(x) (the 1.5 * 2^23
-// shifter leaves n in the low mantissa bits), f in [-1/2, 1/2]; 2^f from a
-// degree-3 polynomial whose coefficients were fitted for this library by
-// weighted least squares on Chebyshev nodes with Lawson reweighting toward
-// the minimax relative error (7.5e-5 on [-1/2, 1/2], far below the 2^-9
-// relative rounding of the bf16 P it feeds); 2^n is added to the exponent
-// field. x < -125 returns 0, so masked keys (-inf) contribute nothing.
-__device__ __forceinline__ float ex2_poly(float x) {
-  const float shifter = 12582912.0f;  // 1.5 * 2^23
-  const float xc = fmaxf(x, -125.0f);
-  const float t = xc + shifter;
-  const float n = t - shifter;
-  const float f = xc - n;
-  float p = fmaf(0.055171623826026917f, f, 0.2426111251115799f);
-  p = fmaf(p, f, 0.6932609677314758f);
-  p = fmaf(p, f, 0.9999280571937561f);
-  const int bits = __float_as_int(p) + (__float_as_int(t) << 23);
-  return x < -125.0f ? 0.0f : __int_as_float(bits);
-}
-
 // Packed f32x2 arithmetic (two lanes of fp32 per instruction): half the issue
 // slots of scalar FFMA / FADD at the same per-element throughput.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
