@@ -7,7 +7,7 @@ sta_attn_fwd_raster (the tile gather of Q, K, V and the scatter of O back to
 raster order happen inside the kernels' loads and stores).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-  python bench.py --search-curve [--config-index I]   (window search, recall vs density)
+  python bench.py --search-curve [--workload NAME]   (window search, recall vs density)
   python bench.py --sweep                              (every layer of the workload table)
 
 Rank 0 prints one JSON line. Under torchrun every rank runs its own layer
@@ -37,7 +37,7 @@ from workloads import CONFIGS, make_qkv, perturb_step, window_params, window_sca
 
 METRIC = "kept-block attn TFLOP/s & % BF16 peak; ms/layer at 75,600 tokens, 15% density"
 UNIT = "TFLOP/s"
-CFG_INDEX = 2
+HEADLINE = "dit720p"  # the 75,600-token 720p layer
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -221,7 +221,7 @@ class ClockSampler:
 class Layer:
     """Device buffers and launches of one step of the path."""
 
-    def __init__(self, sta, cfg, dev, seed_offset=0, cfg_index=CFG_INDEX, density_index=0):
+    def __init__(self, sta, cfg, dev, seed_offset=0, workload=HEADLINE, density_index=0):
         from dataclasses import replace
 
         self.sta = sta
@@ -236,7 +236,7 @@ class Layer:
         self._tiled = None  # tiled copies, made only for the reorder / tiled-call measurements
         self.o = torch.empty_like(self.q)
         if c.window_density:
-            self.win = torch.from_numpy(window_params(cfg, window_scale(cfg_index, density_index))).to(dev)
+            self.win = torch.from_numpy(window_params(cfg, window_scale(workload, density_index))).to(dev)
         else:
             self.win = None
         self.params = sta.mask_params(c.top_p, c.k_min, c.use_scores, 0.0, c.group_lo, self.win)
@@ -407,14 +407,14 @@ class Layer:
         return tot_ab / (2.0 * tot_u) if tot_u else 1.0, tot_u
 
 
-def search_curve(sta, cfg_index, dev, taus=(0.8, 0.9, 0.95, 0.99), lam=1.0):
+def search_curve(sta, workload, dev, taus=(0.8, 0.9, 0.95, 0.99), lam=1.0):
     """Recall target against achieved density (Compact Attention Fig. 5(c)):
     exact block masses of the dense layer (dense list, exact LSE), the window
     search for every head at each target, then the window-only mask built from
     the searched windows and the attention on it, compared with the dense
     output (relative Frobenius error over the whole layer)."""
-    cfg = CONFIGS[cfg_index]
-    layer = Layer(sta, cfg, dev, cfg_index=cfg_index)
+    cfg = CONFIGS[workload]
+    layer = Layer(sta, cfg, dev, workload=workload)
     layer.reorder_in()
     B, Hh, d, g, nt = layer.B, layer.Hh, layer.d, layer.g, layer.nt
     R = B * Hh * nt
@@ -513,19 +513,19 @@ def sweep(sta, dev, peak, reps=20):
                 "reorder_ms_per_tensor": reo_ms,
                 "reorder_gbs": (raster + tiled) / (reo_ms * 1e-3) / 1e9}
 
-    for ci, dens in ((1, (0,)), (2, (0,)), (3, (0, 1, 2, 3))):
+    for wl, dens in (("dit480p", (0,)), (HEADLINE, (0,)), ("dit720p_129f", (0, 1, 2, 3))):
         for di in dens:
-            layer = Layer(sta, CONFIGS[ci], dev, cfg_index=ci, density_index=di)
+            layer = Layer(sta, CONFIGS[wl], dev, workload=wl, density_index=di)
             layer.build()
             extra = build_extra(layer)
-            extra["density_target"] = CONFIGS[ci].window_density[di]
-            attn_line(CONFIGS[ci].name, layer, extra)
+            extra["density_target"] = CONFIGS[wl].window_density[di]
+            attn_line(CONFIGS[wl].name, layer, extra)
             del layer
             torch.cuda.empty_cache()
 
     # rectified form on the 720p layer: time, and the error against dense
     # attention of the plain and of the rectified output on the same mask
-    layer = Layer(sta, CONFIGS[2], dev, cfg_index=2)
+    layer = Layer(sta, CONFIGS[HEADLINE], dev, workload=HEADLINE)
     layer.reorder_in()
     layer.build_tiled()
     B, Hh, d, g, nt = layer.B, layer.Hh, layer.d, layer.g, layer.nt
@@ -552,7 +552,7 @@ def sweep(sta, dev, peak, reps=20):
         diff = (a - o_dense)[:, :, real]
         return float(torch.linalg.vector_norm(diff) / torch.linalg.vector_norm(o_dense[:, :, real]))
 
-    line = {"workload": CONFIGS[2].name + " (rectified form)", "density": layer.kept_pairs() / (R * nt),
+    line = {"workload": CONFIGS[HEADLINE].name + " (rectified form)", "density": layer.kept_pairs() / (R * nt),
             "kept_pairs": layer.kept_pairs(), "rectified_ms": rect_ms, "plain_ms_same_mask": plain_ms,
             "pooled_steps_per_cta": (nt + 63) // 64,
             "rel_err_vs_dense_plain": rel(o_plain), "rel_err_vs_dense_rectified": rel(o_rect.float())}
@@ -562,8 +562,8 @@ def sweep(sta, dev, peak, reps=20):
     torch.cuda.empty_cache()
 
     # reuse layer: top_p = 0, k_min = round(rho * Nt), no windows; mask from step 0
-    cfg = CONFIGS[4]
-    layer = Layer(sta, cfg, dev, cfg_index=4)
+    cfg = CONFIGS["reuse480p"]
+    layer = Layer(sta, cfg, dev, workload="reuse480p")
     gen = torch.Generator(device=dev).manual_seed(1234)
     masters = [layer.q.float(), layer.k.float()]
     steps_inputs = []
@@ -610,7 +610,7 @@ def cpu_oracle_sample(cfg, layer, budget_s, rows_per_head=8, max_heads=None):
 
     T, H, W, d = cfg.T, cfg.H, cfg.W, cfg.d
     nt = layer.nt
-    win = window_params(cfg, window_scale(CFG_INDEX, 0))
+    win = window_params(cfg, window_scale(HEADLINE, 0))
     rng = np.random.default_rng(123)
     heads = rng.permutation(cfg.heads)
     if max_heads:
@@ -649,7 +649,7 @@ def run_reference(args, rank, world):
         return
     import block_sparse_attention_28_b200  # noqa: F401  (only to reuse tile counts)
 
-    cfg = CONFIGS[CFG_INDEX]
+    cfg = CONFIGS[HEADLINE]
 
     class _Stub:
         pass
@@ -674,7 +674,7 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded random-Fourier-feature Q/K, Gaussian V)",
-        "config": {"workload": CONFIGS[CFG_INDEX].name, "tokens": cfg.L, "heads": cfg.heads, "d": cfg.d,
+        "config": {"workload": CONFIGS[HEADLINE].name, "tokens": cfg.L, "heads": cfg.heads, "d": cfg.d,
                    "sample": desc},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "blas_threads": blas_threads(),
                          "kind": "oracle", "sample": desc},
@@ -694,7 +694,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-mask run of the same kernel")
-    ap.add_argument("--config-index", type=int, default=CFG_INDEX,
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(CONFIGS),
                     help="workload (profiling of smaller layers); the headline is the 720p layer")
     ap.add_argument("--density-index", type=int, default=0)
     ap.add_argument("--heads", type=int, default=0,
@@ -723,18 +723,18 @@ def main():
         return
     if args.search_curve:
         if rank == 0:
-            print(json.dumps(search_curve(sta, args.config_index, dev)), flush=True)
+            print(json.dumps(search_curve(sta, args.workload, dev)), flush=True)
         return
     if world > 1:
         import torch.distributed as dist
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    cfg = CONFIGS[args.config_index]
+    cfg = CONFIGS[args.workload]
     if args.heads > 0:
         from dataclasses import replace
 
         cfg = replace(cfg, heads=args.heads)
-    layer = Layer(sta, cfg, dev, seed_offset=rank, cfg_index=args.config_index,
+    layer = Layer(sta, cfg, dev, seed_offset=rank, workload=args.workload,
                   density_index=args.density_index)
 
     def barrier():
@@ -807,7 +807,7 @@ def main():
     line = None
     if rank == 0:
         cpu = None
-        if world == 1 and not args.no_cpu_baseline and args.config_index == CFG_INDEX:
+        if world == 1 and not args.no_cpu_baseline and args.workload == HEADLINE:
             v_cpu, desc, dt, threads = cpu_oracle_sample(cfg, layer, args.cpu_budget)
             cpu = {"value": v_cpu, "unit": UNIT, "cores": threads, "blas_threads": blas_threads(),
                    "kind": "oracle", "sample": f"{desc}; {dt:.1f} s"}

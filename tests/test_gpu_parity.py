@@ -65,7 +65,7 @@ def test_reorder_bit_exact(sta, gp, T, H, W, d, B, Hh):
 
 
 def test_reorder_full_size_720p(sta, gp):
-    cfg = CONFIGS[2]
+    cfg = CONFIGS["dit720p"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     g = sta.grid(T, H, W)
     x = _rand_raster(B, cfg.L, Hh, d, seed=7)
@@ -121,7 +121,7 @@ def _check_mask(sta, gp, qt, kt, B, Hh, d, T, H, W, top_p, k_min, use_scores, wi
 
 
 def test_build_mask_tiny_config(sta, gp):
-    cfg = CONFIGS[0]
+    cfg = CONFIGS["tiny"]
     q, k, _ = (x.cuda() for x in make_qkv(cfg, device="cpu"))
     g = sta.grid(cfg.T, cfg.H, cfg.W)
     qt, kt = gp.reorder(q, 1, cfg.heads, cfg.d, g), gp.reorder(k, 1, cfg.heads, cfg.d, g)
@@ -146,9 +146,9 @@ def test_build_mask_ragged(sta, gp, top_p, k_min, use_scores, with_win, d):
 
 
 def test_build_mask_window_only_full_480p(sta, gp):
-    cfg = CONFIGS[1]
+    cfg = CONFIGS["dit480p"]
     g = sta.grid(cfg.T, cfg.H, cfg.W)
-    win = window_params(cfg, window_scale(1, 0))
+    win = window_params(cfg, window_scale("dit480p", 0))
     win_d = torch.from_numpy(win).cuda()
     params = sta.mask_params(0.0, 0, False, 0.0, cfg.group_lo, win_d)
     bufs = gp.build(None, None, 1, cfg.heads, cfg.d, g, params, with_mask=False, with_probs=False)
@@ -162,13 +162,13 @@ def test_build_mask_window_only_full_480p(sta, gp):
 def test_build_mask_full_720p_sampled_rows(sta, gp):
     """The headline layer: full-size build; the oracle's selection on the GPU's
     P for sampled rows, plus the windows, must give the same CSR rows."""
-    cfg = CONFIGS[2]
+    cfg = CONFIGS["dit720p"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     g = sta.grid(T, H, W)
     q, k, _ = make_qkv(cfg, device="cuda")
     qt, kt = gp.reorder(q, B, Hh, d, g), gp.reorder(k, B, Hh, d, g)
     del q, k
-    win = window_params(cfg, window_scale(2, 0))
+    win = window_params(cfg, window_scale("dit720p", 0))
     params = sta.mask_params(cfg.top_p, cfg.k_min, True, 0.0, cfg.group_lo, torch.from_numpy(win).cuda())
     bufs = gp.build(qt, kt, B, Hh, d, g, params, with_mask=False, with_probs=True)
     torch.cuda.synchronize()
@@ -220,7 +220,7 @@ def _attn_check(sta, gp, qt, kt, vt, rp_t, ci_t, B, Hh, d, T, H, W, sm_scale=0.0
 
 
 def test_attn_tiny_config(sta, gp):
-    cfg = CONFIGS[0]
+    cfg = CONFIGS["tiny"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     g = sta.grid(T, H, W)
     q, k, v = (x.cuda() for x in make_qkv(cfg, device="cpu"))
@@ -281,13 +281,13 @@ def test_attn_dense_large_logits(sta, gp):
 def test_attn_full_720p_sampled_rows(sta, gp):
     """The headline layer end to end: full-size build and attention as timed by
     the benchmark; the oracle recomputes sampled rows on the GPU's CSR."""
-    cfg = CONFIGS[2]
+    cfg = CONFIGS["dit720p"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     g = sta.grid(T, H, W)
     q, k, v = make_qkv(cfg, device="cuda")
     qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
     del q, k, v
-    win = torch.from_numpy(window_params(cfg, window_scale(2, 0))).cuda()
+    win = torch.from_numpy(window_params(cfg, window_scale("dit720p", 0))).cuda()
     bufs = gp.build(qt, kt, B, Hh, d, g, sta.mask_params(cfg.top_p, cfg.k_min, True, 0.0, cfg.group_lo, win),
                     with_mask=False, with_probs=False)
     nt = sta.sta_num_tiles(g)
@@ -298,7 +298,7 @@ def test_attn_full_720p_sampled_rows(sta, gp):
 
 def test_attn_reuse_steps(sta, gp):
     """Mask built once from step-0 inputs, reused after 10 perturbed steps."""
-    cfg = CONFIGS[4]
+    cfg = CONFIGS["reuse480p"]
     B, Hh, d, T, H, W = cfg.B, 8, cfg.d, cfg.T, cfg.H, cfg.W
     from dataclasses import replace
 
@@ -346,9 +346,9 @@ def test_attn_bad_column_index_is_reported(sta, gp):
 def test_build_mask_window_only_full_129_frames(sta, gp, which):
     """129-frame layer (24 heads, 1,980 tiles per head), four temporal groups,
     each density target: the whole CSR against the oracle's window mask."""
-    cfg = CONFIGS[3]
+    cfg = CONFIGS["dit720p_129f"]
     g = sta.grid(cfg.T, cfg.H, cfg.W)
-    win = window_params(cfg, window_scale(3, which))
+    win = window_params(cfg, window_scale("dit720p_129f", which))
     params = sta.mask_params(0.0, 0, False, 0.0, cfg.group_lo, torch.from_numpy(win).cuda())
     bufs = gp.build(None, None, 1, cfg.heads, cfg.d, g, params, with_mask=False, with_probs=False)
     rp, ci, nnz = gp.csr_np(bufs)
@@ -359,13 +359,13 @@ def test_build_mask_window_only_full_129_frames(sta, gp, which):
 
 
 def test_attn_full_129_frames_sampled_rows(sta, gp):
-    cfg = CONFIGS[3]
+    cfg = CONFIGS["dit720p_129f"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     g = sta.grid(T, H, W)
     q, k, v = make_qkv(cfg, device="cuda")
     qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
     del q, k, v
-    win = torch.from_numpy(window_params(cfg, window_scale(3, 2))).cuda()
+    win = torch.from_numpy(window_params(cfg, window_scale("dit720p_129f", 2))).cuda()
     bufs = gp.build(None, None, B, Hh, d, g, sta.mask_params(0.0, 0, False, 0.0, cfg.group_lo, win),
                     with_mask=False, with_probs=False)
     nt = sta.sta_num_tiles(g)
@@ -375,13 +375,13 @@ def test_attn_full_129_frames_sampled_rows(sta, gp):
 
 
 def test_attn_full_480p_sampled_rows(sta, gp):
-    cfg = CONFIGS[1]
+    cfg = CONFIGS["dit480p"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     g = sta.grid(T, H, W)
     q, k, v = make_qkv(cfg, device="cuda")
     qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
     del q, k, v
-    win = torch.from_numpy(window_params(cfg, window_scale(1, 0))).cuda()
+    win = torch.from_numpy(window_params(cfg, window_scale("dit480p", 0))).cuda()
     bufs = gp.build(None, None, B, Hh, d, g, sta.mask_params(0.0, 0, False, 0.0, cfg.group_lo, win),
                     with_mask=False, with_probs=False)
     nt = sta.sta_num_tiles(g)
@@ -397,7 +397,7 @@ def test_attn_reuse_all_densities_full(sta, gp):
     100% run is the dense-mask reference of the same kernel."""
     from workloads import perturb_step
 
-    cfg = CONFIGS[4]
+    cfg = CONFIGS["reuse480p"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     g = sta.grid(T, H, W)
     nt = sta.sta_num_tiles(g)
@@ -460,13 +460,13 @@ def test_build_mask_head_floor_ragged(sta, gp, d):
 
 
 def test_build_mask_head_floor_720p_sampled_heads(sta, gp):
-    cfg = CONFIGS[2]
+    cfg = CONFIGS["dit720p"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     g = sta.grid(T, H, W)
     q, k, _ = make_qkv(cfg, device="cuda")
     qt, kt = gp.reorder(q, B, Hh, d, g), gp.reorder(k, B, Hh, d, g)
     del q, k
-    win = window_params(cfg, window_scale(2, 0))
+    win = window_params(cfg, window_scale("dit720p", 0))
     params = sta.mask_params(cfg.top_p, cfg.k_min, True, 0.0, cfg.group_lo, torch.from_numpy(win).cuda(),
                              head_floor=True)
     bufs = gp.build(qt, kt, B, Hh, d, g, params, with_mask=False, with_probs=True)
@@ -514,7 +514,7 @@ def _mass_check(sta, gp, qt, kt, vt, rp_t, ci_t, lse_cached, B, Hh, d, T, H, W, 
 def test_block_mass_tiny_dense_exact_lse(sta, gp):
     """Dense list and the exact LSE of the same inputs: masses match the
     oracle and every row sums to one."""
-    cfg = CONFIGS[0]
+    cfg = CONFIGS["tiny"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     g = sta.grid(T, H, W)
     nt = sta.sta_num_tiles(g)
@@ -554,7 +554,7 @@ def test_block_mass_ragged_sparse_stale_lse(sta, gp, d):
 
 def test_block_mass_720p_dense_sampled_rows(sta, gp):
     """The headline layer, dense list, exact LSE: sampled rows of masses."""
-    cfg = CONFIGS[2]
+    cfg = CONFIGS["dit720p"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     g = sta.grid(T, H, W)
     nt = sta.sta_num_tiles(g)
@@ -630,7 +630,7 @@ def test_search_windows_on_480p_block_masses(sta, gp):
     """The 480p layer: exact block masses of the dense attention (fused LSE
     path), then the search for every head; sampled heads match the oracle
     window for window, and every head's windows meet the recall target."""
-    cfg = CONFIGS[1]
+    cfg = CONFIGS["dit480p"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     g = sta.grid(T, H, W)
     nt = sta.sta_num_tiles(g)
@@ -739,10 +739,10 @@ def test_degenerate_grids(sta, gp, d, T, H, W):
 
 def test_raster_path_equals_tiled_720p(sta, gp):
     """The headline layer: raster mask and attention equal the tiled path."""
-    cfg = CONFIGS[2]
+    cfg = CONFIGS["dit720p"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     q, k, v = make_qkv(cfg, device="cuda")
-    win = torch.from_numpy(window_params(cfg, window_scale(2, 0))).cuda()
+    win = torch.from_numpy(window_params(cfg, window_scale("dit720p", 0))).cuda()
     params = sta.mask_params(cfg.top_p, cfg.k_min, True, 0.0, cfg.group_lo, win)
     _raster_vs_tiled(sta, gp, q, k, v, B, Hh, d, T, H, W, params)
 
@@ -821,14 +821,14 @@ def test_rectified_ragged_sparse(sta, gp, d, density):
 
 def test_rectified_720p_sampled_rows(sta, gp):
     """The headline layer with its own mask: sampled rows against the oracle."""
-    cfg = CONFIGS[2]
+    cfg = CONFIGS["dit720p"]
     B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
     g = sta.grid(T, H, W)
     nt = sta.sta_num_tiles(g)
     q, k, v = make_qkv(cfg, device="cuda")
     qt, kt, vt = (gp.reorder(x, B, Hh, d, g) for x in (q, k, v))
     del q, k, v
-    win = torch.from_numpy(window_params(cfg, window_scale(2, 0))).cuda()
+    win = torch.from_numpy(window_params(cfg, window_scale("dit720p", 0))).cuda()
     params = sta.mask_params(cfg.top_p, cfg.k_min, True, 0.0, cfg.group_lo, win)
     bufs = gp.build(qt, kt, B, Hh, d, g, params, with_mask=False, with_probs=False)
     rng = np.random.default_rng(17)

@@ -48,24 +48,24 @@ def tile_counts(T: int, H: int, W: int):
 
 
 CONFIGS = {
-    0: WorkloadConfig(
+    "tiny": WorkloadConfig(
         name="tiny_4x16x16_h2_d64", B=1, heads=2, d=64, T=4, H=16, W=16, seed=0,
         use_scores=True, top_p=0.9, k_min=2, group_lo=(0, 1),
         ell=(2.0, 6.0), ell_fixed=True,
         note="tiny reference case; fixed local 1x1 + full-row axial window"),
-    1: WorkloadConfig(
+    "dit480p": WorkloadConfig(
         name="dit480p_21x30x52_h40_d128_win25", B=1, heads=40, d=128, T=21, H=30, W=52, seed=1,
         use_scores=False, group_lo=(0, 1, 4), window_density=(0.25,),
         note="dual-window masks only, ~25% density"),
-    2: WorkloadConfig(
+    "dit720p": WorkloadConfig(
         name="dit720p_21x45x80_h40_d128_p95k8_d15", B=1, heads=40, d=128, T=21, H=45, W=80, seed=2,
         use_scores=True, top_p=0.95, k_min=8, group_lo=(0, 1, 4), window_density=(0.15,),
         note="online top-p 0.95 / k_min 8 OR dual windows, ~15% overall density"),
-    3: WorkloadConfig(
+    "dit720p_129f": WorkloadConfig(
         name="dit720p129f_33x45x80_h24_d128_win", B=1, heads=24, d=128, T=33, H=45, W=80, seed=3,
         use_scores=False, group_lo=(0, 1, 3, 7), window_density=(0.05, 0.10, 0.20, 0.30),
         note="dual-window masks, 4 temporal groups, density sweep"),
-    4: WorkloadConfig(
+    "reuse480p": WorkloadConfig(
         name="reuse_21x30x52_h40_d128", B=1, heads=40, d=128, T=21, H=30, W=52, seed=4,
         use_scores=True, top_p=0.0, group_lo=(0,),
         fixed_densities=(0.05, 0.10, 0.25, 0.50, 1.00), reuse_steps=10,

@@ -99,7 +99,7 @@ KINDS = ("local", "axial_x", "axial_y", "cross", "global")
 _SCALES = None
 
 
-def window_scale(cfg_index: int, which: int = 0) -> float:
+def window_scale(workload: str, which: int = 0) -> float:
     """Window scale meeting the workload's density target number `which`
     (stored by the calibration script beside the oracle)."""
     global _SCALES
@@ -108,7 +108,7 @@ def window_scale(cfg_index: int, which: int = 0) -> float:
         import os
         with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "window_scales.json")) as f:
             _SCALES = json.load(f)
-    return float(_SCALES[str(cfg_index)][which]["scale"])
+    return float(_SCALES[workload][which]["scale"])
 
 
 def window_params(cfg: WorkloadConfig, scale: float) -> np.ndarray:
