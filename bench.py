@@ -647,8 +647,6 @@ def run_reference(args, rank, world):
     """The CPU oracle timed as the reference arm (rank 0 only)."""
     if rank != 0:
         return
-    import block_sparse_attention_28_b200  # noqa: F401  (only to reuse tile counts)
-
     cfg = CONFIGS[HEADLINE]
 
     class _Stub:
