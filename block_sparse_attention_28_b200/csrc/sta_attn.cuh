@@ -263,6 +263,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   }
   __syncthreads();
 
+  // Every role walks the list from the first key tile at or after the CTA's
+  // own query tile and wraps around (any order gives the same softmax up to
+  // rounding): CTAs that run side by side then start on different key tiles
+  // instead of all asking L2 for the same low-numbered ones at once.
+  int rot = 0;
+  {
+    int lo = 0, hi = n_list;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if ((int)(U[mid] & KT_MASK) < qtA) lo = mid + 1; else hi = mid;
+    }
+    rot = (lo < n) ? lo : 0;
+  }
+  auto uidx = [&](int j) { const int t = j + rot; return t < n ? t : t - n; };
+
   if (warp == WARP_PRODUCER) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0 && n > 0) {
@@ -293,7 +308,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                            uint64_t *empty, int off, int ns, int j) -> bool {
         const int s = j % ns, u = j / ns;
         if (u > 0 && !tc::mbar_wait(empty + s, (u - 1) & 1, abort_flag, WAIT_LIMIT)) return false;
-        const uint32_t e = U[j];
+        const uint32_t e = U[uidx(j)];
         const int kt = (int)(e & KT_MASK);
         tc::mbar_expect_tx(full + s, C::TILE_BYTES);
         if (RECT && (e & VIRT) != 0u) {
@@ -408,7 +423,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         break;
       }
       tc::fence_after();
-      const uint32_t e = U[j];
+      const uint32_t e = U[uidx(j)];
       const bool mine = halfB ? (e & FLAG_B) != 0u : (e & FLAG_A) != 0u;
       const uint32_t sS = tmem + lane_base + (uint32_t)(buf * 64);
       uint32_t pk[32];
