@@ -81,7 +81,7 @@ struct Cfg {
 template <int D>
 inline size_t smem_bytes(int nt, int ntp = 0) {
   const int wpr = (nt + 31) / 32;
-  return (size_t)Cfg<D>::OFF_LIST + (size_t)(2 * wpr + nt + ntp / 64 + ntp) * 4 + 1024;
+  return (size_t)Cfg<D>::OFF_LIST + (size_t)(2 * wpr + nt + ntp / 64 + ntp) * 4 + 16 + 1024;
 }
 
 // MASS: also accumulate the LSE-cached exact block importance (AdaSpa) of
@@ -237,12 +237,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int n_list = (int)misc[1];
   const int nv = RECT ? ntp / 64 : 0;  // pooled tiles after the listed ones
   const int n = n_list + nv;
-  float *bias = reinterpret_cast<float *>(U + nt + nv);  // ln n_kt / scale, per pooled key
+  // ln n_kt / scale per pooled key (-inf past Nt), 16-byte aligned for float4 reads
+  float *bias = reinterpret_cast<float *>((reinterpret_cast<uintptr_t>(U + nt + nv) + 15u) & ~uintptr_t(15));
   if (RECT) {
     for (int u = tid; u < nv; u += NUM_THREADS) U[n_list + u] = (uint32_t)u | VIRT | FLAG_A | FLAG_B;
     const float ln2_over = 1.0f / scale_log2;  // log2(n) / scale_log2 = ln(n) / scale
     for (int kt = tid; kt < ntp; kt += NUM_THREADS) {
-      float b = 0.0f;
+      float b = -INFINITY;
       if (kt < nt) {
         const int rem = kt % (g.NH * g.NW);
         const int ty = rem / g.NW, tx = rem - ty * g.NW;
@@ -444,13 +445,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (RECT && (e & VIRT) != 0u) {
           const int u = (int)(e & KT_MASK);
           const uint32_t *bm = halfB ? bmB : bmA;
-          const uint32_t w0 = (2 * u < wpr) ? bm[2 * u] : 0u;
-          const uint32_t w1 = (2 * u + 1 < wpr) ? bm[2 * u + 1] : 0u;
+          // columns the row does not list; the bias is -inf past Nt
+          const uint32_t a0 = (2 * u < wpr) ? ~bm[2 * u] : ~0u;
+          const uint32_t a1 = (2 * u + 1 < wpr) ? ~bm[2 * u + 1] : ~0u;
+          const float4 *b4 = reinterpret_cast<const float4 *>(bias + 64 * u);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int kp = 64 * u + c;
-            const bool listed = (((c < 32) ? (w0 >> c) : (w1 >> (c - 32))) & 1u) != 0u;
-            s[c] = (kp < nt && !listed) ? s[c] + bias[kp] : -INFINITY;
+          for (int c4 = 0; c4 < 16; ++c4) {
+            const float4 b = b4[c4];
+            const float bb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int c = 4 * c4 + q;
+              const bool on = (((c < 32) ? (a0 >> c) : (a1 >> (c - 32))) & 1u) != 0u;
+              s[c] = on ? s[c] + bb[q] : -INFINITY;
+            }
           }
         }
         // keys of partial tiles beyond the grid edge
