@@ -64,6 +64,8 @@ _lib.sta_reorder.argtypes = [_vp, _vp, _i32, _i32, _i32, Grid, _i32, _vp]
 _lib.sta_reorder.restype = ctypes.c_int
 _lib.sta_build_mask_workspace.argtypes = [_i32, _i32, _i32, Grid]
 _lib.sta_build_mask_workspace.restype = _sz
+_lib.sta_build_mask_workspace_min.argtypes = [_i32, _i32, _i32, Grid]
+_lib.sta_build_mask_workspace_min.restype = _sz
 _lib.sta_build_mask.argtypes = [_vp, _vp, _i32, _i32, _i32, Grid, ctypes.POINTER(MaskParams), _vp, _vp,
                                 _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sta_build_mask.restype = ctypes.c_int
@@ -139,6 +141,10 @@ def sta_reorder(src, dst, B, heads, d, g, inverse=False, stream=None):
 
 def sta_build_mask_workspace(B, heads, d, g):
     return int(_lib.sta_build_mask_workspace(B, heads, d, g))
+
+
+def sta_build_mask_workspace_min(B, heads, d, g):
+    return int(_lib.sta_build_mask_workspace_min(B, heads, d, g))
 
 
 def mask_params(top_p=0.0, k_min=0, use_scores=False, sm_scale=0.0, group_lo=(0,), windows=None,

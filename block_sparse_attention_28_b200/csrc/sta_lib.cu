@@ -34,8 +34,11 @@ bool common_sizes_ok(int32_t B, int32_t heads, int32_t d, sta_grid g, Geo *geo, 
   return true;
 }
 
+// total_min: the fused score/select pass; total: plus a P row buffer
+// [B*heads*Nt, Nt] fp32 for the split passes (scores, then a select pass
+// with four CTAs per SM).
 struct MaskWs {
-  size_t qbar, kbar, bits, counts, sel, kfloor, total;
+  size_t qbar, kbar, bits, counts, sel, kfloor, total_min, prows, total;
 };
 
 MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
@@ -55,14 +58,19 @@ MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
   off = align_up(off + R * sizeof(int32_t), 256);
   w.kfloor = off;
   off = align_up(off + (size_t)B * heads * sizeof(int32_t), 256);
+  w.total_min = off;
+  w.prows = off;
+  off = align_up(off + R * g.Nt * sizeof(float), 256);
   w.total = off;
   return w;
 }
 
-size_t select_smem(int d, const Geo &g, bool use_scores) {
-  const size_t scores = use_scores ? (size_t)(SEL_QB * d + SEL_QB * g.Nt + (SEL_THREADS / 32) * 256) : 0;
-  const size_t tables = (size_t)((g.Nt + g.T + 3) & ~3) + 4 * STA_MAX_GROUPS;
-  return (scores + tables) * sizeof(float);
+// Dynamic shared memory of score_select_kernel<D, qb, mode>.
+size_t select_smem(int d, const Geo &g, bool use_scores, int qb = SEL_QB, int mode = SEL_FUSED) {
+  const size_t q = (mode != SEL_SELECT && use_scores) ? (size_t)qb * d : 0;
+  const size_t scores = use_scores ? (size_t)(qb * g.Nt + (SEL_THREADS / 32) * 256) : 0;
+  const size_t tables = (mode == SEL_SCORES) ? 0 : (size_t)((g.Nt + g.T + 3) & ~3) + 4 * STA_MAX_GROUPS;
+  return (q + scores + tables) * sizeof(float);
 }
 
 constexpr size_t MAX_DYN_SMEM = 227 * 1024;
@@ -136,11 +144,14 @@ __global__ void selftest_wait_kernel(long long limit) {
   }
 }
 
+// ws_bytes decides the selection layout: with room for the P row buffer (or
+// a caller's block_probs to hold the rows) the scores pass and a separate,
+// smaller select pass run; otherwise the fused pass. Both give the same bits.
 template <int D>
 sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads,
                         const Geo &g, const sta_mask_params *p, int32_t *row_ptr, int32_t *col_idx,
                         int64_t *nnz_dev, uint8_t *block_mask, float *block_probs, uint8_t *ws,
-                        cudaStream_t s, bool raster = false) {
+                        size_t ws_bytes, cudaStream_t s, bool raster = false) {
   const MaskWs L = mask_ws_layout(B, heads, D, g);
   float *qbar = reinterpret_cast<float *>(ws + L.qbar);
   float *kbar = reinterpret_cast<float *>(ws + L.kbar);
@@ -163,31 +174,71 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
                                                    static_cast<const uint4 *>(k_tiled), qbar, kbar, R, g, heads);
     STA_CUDA_TRY(cudaGetLastError());
   }
-  const size_t smem = select_smem(D, g, use_scores);
-  if (smem > 48 * 1024)
-    STA_CUDA_TRY(cudaFuncSetAttribute(score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)smem));
   GroupLo glo;
   for (int i = 0; i < STA_MAX_GROUPS; ++i) glo.v[i] = (i < p->num_groups) ? p->group_lo[i] : 0x7fffffff;
-  dim3 grid((unsigned)((g.Nt + SEL_QB - 1) / SEL_QB), (unsigned)(B * heads));
   const bool floor = use_scores && p->head_topk_floor != 0;
   int *sel = reinterpret_cast<int *>(ws + L.sel);
   int *kfloor = reinterpret_cast<int *>(ws + L.kfloor);
-  if (floor) {
-    // pass 1: base selection counts; per-head floor; pass 2 below re-selects
-    // with k_min raised to the floor
-    score_select_kernel<D><<<grid, SEL_THREADS, smem, s>>>(
-        qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, nullptr, 0, glo, bits, counts, nullptr,
-        wpr, nullptr, sel, P_in);
+  const int *windows = p->windows;
+  const int G = p->windows ? p->num_groups : 0;
+  // P rows: the caller's block_probs, else the workspace's row buffer
+  float *prows = block_probs != nullptr ? block_probs
+                                        : (ws_bytes >= L.total ? reinterpret_cast<float *>(ws + L.prows) : nullptr);
+  const bool split = (use_scores && P_in == nullptr && prows != nullptr) || (use_scores && P_in != nullptr) ||
+                     !use_scores;
+  if (!split) {
+    // fused: scores, softmax, selection and windows per 16-row CTA
+    const size_t smem = select_smem(D, g, use_scores, SEL_QB, SEL_FUSED);
+    auto kern = score_select_kernel<D, SEL_QB, SEL_FUSED>;
+    if (smem > 48 * 1024)
+      STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    dim3 grid((unsigned)((g.Nt + SEL_QB - 1) / SEL_QB), (unsigned)(B * heads));
+    if (floor) {
+      // pass 1: base selection counts; per-head floor; pass 2 re-selects with
+      // k_min raised to the floor
+      kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, nullptr, 0, glo,
+                                           bits, counts, nullptr, wpr, nullptr, sel, nullptr);
+      STA_CUDA_TRY(cudaGetLastError());
+      head_floor_kernel<<<(unsigned)(B * heads), FLOOR_THREADS, 0, s>>>(sel, kfloor, g);
+      STA_CUDA_TRY(cudaGetLastError());
+    }
+    kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, windows, G, glo,
+                                         bits, counts, block_probs, wpr, floor ? kfloor : nullptr, nullptr,
+                                         nullptr);
     STA_CUDA_TRY(cudaGetLastError());
-    head_floor_kernel<<<(unsigned)(B * heads), FLOOR_THREADS, 0, s>>>(sel, kfloor, g);
+  } else {
+    const float *P_sel = P_in;        // rows the select pass reads
+    float *probs_sel = block_probs;   // and copies out (clamped) when from the caller
+    if (use_scores && P_in == nullptr) {
+      // scores pass: P rows into prows (the caller's block_probs when given)
+      const size_t smem = select_smem(D, g, true, SEL_QB, SEL_SCORES);
+      auto kern = score_select_kernel<D, SEL_QB, SEL_SCORES>;
+      if (smem > 48 * 1024)
+        STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      dim3 grid((unsigned)((g.Nt + SEL_QB - 1) / SEL_QB), (unsigned)(B * heads));
+      kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, nullptr, 0, glo,
+                                           bits, counts, prows, wpr, nullptr, nullptr, nullptr);
+      STA_CUDA_TRY(cudaGetLastError());
+      P_sel = prows;
+      probs_sel = nullptr;  // already written
+    }
+    const size_t smem = select_smem(D, g, use_scores, SEL_QB_SELECT, SEL_SELECT);
+    auto kern = score_select_kernel<D, SEL_QB_SELECT, SEL_SELECT>;
+    if (smem > 48 * 1024)
+      STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    dim3 grid((unsigned)((g.Nt + SEL_QB_SELECT - 1) / SEL_QB_SELECT), (unsigned)(B * heads));
+    if (floor) {
+      kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, nullptr, 0, glo,
+                                           bits, counts, nullptr, wpr, nullptr, sel, P_sel);
+      STA_CUDA_TRY(cudaGetLastError());
+      head_floor_kernel<<<(unsigned)(B * heads), FLOOR_THREADS, 0, s>>>(sel, kfloor, g);
+      STA_CUDA_TRY(cudaGetLastError());
+    }
+    kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, use_scores ? 1 : 0,
+                                         windows, G, glo, bits, counts, probs_sel, wpr,
+                                         floor ? kfloor : nullptr, nullptr, P_sel);
     STA_CUDA_TRY(cudaGetLastError());
   }
-  score_select_kernel<D><<<grid, SEL_THREADS, smem, s>>>(
-      qbar, kbar, heads, g, scale, p->top_p, p->k_min, use_scores ? 1 : 0, p->windows,
-      p->windows ? p->num_groups : 0, glo, bits, counts, block_probs, wpr, floor ? kfloor : nullptr,
-      nullptr, P_in);
-  STA_CUDA_TRY(cudaGetLastError());
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(counts, row_ptr, reinterpret_cast<long long *>(nnz_dev), R);
   STA_CUDA_TRY(cudaGetLastError());
   const unsigned fblocks = (unsigned)((R * 32 + 255) / 256);
@@ -274,6 +325,13 @@ size_t sta_build_mask_workspace(int32_t B, int32_t heads, int32_t d, sta_grid g)
   return mask_ws_layout(B, heads, d, geo).total;
 }
 
+size_t sta_build_mask_workspace_min(int32_t B, int32_t heads, int32_t d, sta_grid g) {
+  Geo geo;
+  sta_status st = STA_OK;
+  if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return 0;
+  return mask_ws_layout(B, heads, d, geo).total_min;
+}
+
 static sta_status build_mask_any(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads,
                                  int32_t d, sta_grid g, const sta_mask_params *p, int32_t *row_ptr,
                                  int32_t *col_idx, int64_t *nnz_dev, uint8_t *block_mask,
@@ -294,7 +352,7 @@ static sta_status build_mask_any(const void *q_tiled, const void *k_tiled, int32
   }
   if (p->k_min < 0 || !(p->top_p == p->top_p)) return STA_ERR_INVALID_ARG;
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
-      ws_bytes < mask_ws_layout(B, heads, d, geo).total)
+      ws_bytes < mask_ws_layout(B, heads, d, geo).total_min)
     return STA_ERR_WORKSPACE;
   if (select_smem(d, geo, p->use_scores != 0) > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
   // window tables pack (t, tile row, tile column) into 12 + 10 + 10 bits
@@ -302,9 +360,9 @@ static sta_status build_mask_any(const void *q_tiled, const void *k_tiled, int32
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   return (d == 128) ? launch_build<128>(q_tiled, k_tiled, B, heads, geo, p, row_ptr, col_idx, nnz_dev,
-                                        block_mask, block_probs, ws, s, raster)
+                                        block_mask, block_probs, ws, ws_bytes, s, raster)
                     : launch_build<64>(q_tiled, k_tiled, B, heads, geo, p, row_ptr, col_idx, nnz_dev,
-                                       block_mask, block_probs, ws, s, raster);
+                                       block_mask, block_probs, ws, ws_bytes, s, raster);
 }
 
 sta_status sta_build_mask(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads, int32_t d,
@@ -521,7 +579,7 @@ extern "C" sta_status sta_build_mask_noalloc(const void *q_tiled, const void *k_
   Geo geo;
   sta_status st = STA_OK;
   if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return st;
-  if (mask_ws_layout(B, heads, d, geo).total > (size_t)STA_NOALLOC_SCRATCH_BYTES) return STA_ERR_WORKSPACE;
+  if (mask_ws_layout(B, heads, d, geo).total_min > (size_t)STA_NOALLOC_SCRATCH_BYTES) return STA_ERR_WORKSPACE;
   void *scratch = nullptr;
   st = noalloc_scratch_address(&scratch);
   if (st != STA_OK) return st;

@@ -149,7 +149,15 @@ pool_kv_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v, uint4 *
 
 // ------------------------------------------------------ scores + selection
 constexpr int SEL_THREADS = 256;
-constexpr int SEL_QB = 16;  // query tiles per CTA
+constexpr int SEL_QB = 16;  // query tiles per CTA of the score pass (fused or scores-only)
+constexpr int SEL_QB_SELECT = 8;  // rows per CTA of the select-only pass (one per warp)
+// Modes of score_select_kernel:
+//   SEL_FUSED   scores, softmax, selection and windows in one CTA (16 rows
+//               kept in shared memory; used when no row buffer is available)
+//   SEL_SCORES  scores and softmax only: P rows written to P_out
+//   SEL_SELECT  selection and windows only, on P rows read from P_in (no
+//               score code, so the CTA is small and four fit on an SM)
+constexpr int SEL_FUSED = 0, SEL_SCORES = 1, SEL_SELECT = 2;
 constexpr int SEL_KPT = 3;  // key tiles per thread in the score pass
 
 struct GroupLo {
@@ -238,9 +246,11 @@ __device__ void radix_level(const float *row, int nt, unsigned int target, bool 
   above_out = above;
 }
 
-// One CTA per (b*heads + h, block of SEL_QB query tiles).
-// Dynamic smem: qs [SEL_QB][D] fp32, then S [SEL_QB][Nt] fp32 (if use_scores).
-template <int D>
+// One CTA per (b*heads + h, block of QB query tiles).
+// Dynamic smem: qs [QB][D] fp32 (score modes), S [QB][Nt] fp32 and the
+// per-warp histograms (if use_scores), then the window tables (not in
+// SEL_SCORES). In SEL_SCORES, probs_out is the row buffer P_out.
+template <int D, int QB, int MODE>
 __global__ void __launch_bounds__(SEL_THREADS)
 score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar, int heads, Geo g,
                     float scale, float top_p, int k_min, int use_scores,
@@ -248,18 +258,19 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
                     unsigned int *__restrict__ bits, int *__restrict__ counts,
                     float *__restrict__ probs_out, int wpr, const int *__restrict__ kmin_head,
                     int *__restrict__ sel_count, const float *__restrict__ P_in) {
+  constexpr bool HAS_SCORES = MODE != SEL_SELECT;
   extern __shared__ __align__(16) float sm[];
   const int nt = g.Nt;
   const int bh = blockIdx.y;
   const int h = bh % heads;
-  const int q0 = blockIdx.x * SEL_QB;
-  const int nq = min(SEL_QB, nt - q0);
+  const int q0 = blockIdx.x * QB;
+  const int nq = min(QB, nt - q0);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tpf = g.NH * g.NW;
-  // shared memory: [qs, S, histograms] if use_scores, then the window tables
+  // shared memory: [qs], [S, histograms] if use_scores, then the window tables
   float *qs = sm;
-  float *S = qs + (use_scores ? SEL_QB * D : 0);
-  unsigned int *hist = reinterpret_cast<unsigned int *>(S + (use_scores ? SEL_QB * nt : 0));
+  float *S = qs + ((HAS_SCORES && use_scores) ? QB * D : 0);
+  unsigned int *hist = reinterpret_cast<unsigned int *>(S + (use_scores ? QB * nt : 0));
   unsigned int *kcoord = hist + (use_scores ? (SEL_THREADS / 32) * 256 : 0);
   int *gtab = reinterpret_cast<int *>(kcoord + nt);
   int *wtab = gtab + ((nt + g.T + 3) & ~3) - nt;  // 16-byte aligned, 4 ints per group
@@ -267,7 +278,7 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
 
   // Window tables, once per CTA: packed (t, tile row, tile column) of every
   // key tile, the temporal group of every |dt|, and this head's extents.
-  if (windows != nullptr) {
+  if (MODE != SEL_SCORES && windows != nullptr) {
     for (int kt = tid; kt < nt; kt += SEL_THREADS) {
       const int t = kt / tpf, rem = kt - t * tpf;
       const int y = rem / g.NW, x = rem - y * g.NW;
@@ -283,9 +294,9 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
   }
   if (!use_scores) __syncthreads();
 
-  if (use_scores && P_in == nullptr) {
+  if (HAS_SCORES && use_scores && P_in == nullptr) {
     // Phase 1: S[i][kt] = scale * qbar[q0+i] . kbar[kt], sequential fp32 FMA over d.
-    for (int e = tid; e < SEL_QB * D; e += SEL_THREADS) {
+    for (int e = tid; e < QB * D; e += SEL_THREADS) {
       const int i = e / D;
       qs[e] = (i < nq) ? qbar[((long long)bh * nt + q0 + i) * D + (e - i * D)] : 0.0f;
     }
@@ -307,17 +318,17 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
         on[u] = kt < hi;
         kr[u] = reinterpret_cast<const float4 *>(kbar + ((long long)bh * nt + (on[u] ? kt : lo)) * D);
       }
-      float acc[SEL_KPT][SEL_QB];
+      float acc[SEL_KPT][QB];
 #pragma unroll
       for (int u = 0; u < SEL_KPT; ++u)
 #pragma unroll
-        for (int i = 0; i < SEL_QB; ++i) acc[u][i] = 0.0f;
+        for (int i = 0; i < QB; ++i) acc[u][i] = 0.0f;
       for (int d4 = 0; d4 < D / 4; ++d4) {
         float4 kv[SEL_KPT];
 #pragma unroll
         for (int u = 0; u < SEL_KPT; ++u) kv[u] = __ldg(kr[u] + d4);
 #pragma unroll
-        for (int i = 0; i < SEL_QB; ++i) {
+        for (int i = 0; i < QB; ++i) {
           const float4 qv = reinterpret_cast<const float4 *>(qs + i * D)[d4];
 #pragma unroll
           for (int u = 0; u < SEL_KPT; ++u) {
@@ -333,7 +344,7 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
         const int kt = lo + tid + u * SEL_THREADS;
         if (on[u]) {
 #pragma unroll
-          for (int i = 0; i < SEL_QB; ++i) S[i * nt + kt] = acc[u][i] * scale;
+          for (int i = 0; i < QB; ++i) S[i * nt + kt] = acc[u][i] * scale;
         }
       }
     }
@@ -347,8 +358,9 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
     unsigned int v_f = 0xFFFFFFFFu;  // keep P > v_f, plus c_f ties at v_f
     unsigned int c_f = 0u;
     if (use_scores) {
-      if (P_in != nullptr) {
-        // caller-supplied block scores (e.g. exact block masses), clamped to [0, 1]
+      if (!HAS_SCORES || P_in != nullptr) {
+        // P rows of the score pass, or caller-supplied block scores (e.g.
+        // exact block masses), clamped to [0, 1] (a no-op on softmax rows)
         for (int j = lane; j < nt; j += 32) {
           const float p = fminf(fmaxf(P_in[row * nt + j], 0.0f), 1.0f);
           Sr[j] = p;
@@ -374,6 +386,7 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
           if (probs_out) probs_out[row * nt + j] = p;
         }
       }
+      if (MODE == SEL_SCORES) continue;  // the select pass takes it from here
       __syncwarp();
       // Phase 3: selection threshold as (level v_f, ties c_f).
       // per-head top-k floor (second pass): k_min raised to the head's floor

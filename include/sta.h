@@ -107,8 +107,14 @@ int64_t sta_tiled_len(sta_grid g);
 sta_status sta_reorder(const void *src, void *dst, int32_t B, int32_t heads, int32_t d,
                        sta_grid g, int32_t inverse, sta_stream_t stream);
 
-/* Bytes of device workspace sta_build_mask needs for these sizes. */
+/* Bytes of device workspace of sta_build_mask for these sizes: the full size
+ * holds a row buffer of the block probabilities [B*heads*Nt, Nt] fp32, so the
+ * scores and the selection run as two passes (the selection pass keeps four
+ * CTAs per SM); any workspace of at least the _min size is accepted and runs
+ * the fused pass instead (same results, bit for bit). When block_probs is
+ * given, the rows go there and the minimum is enough for the two passes. */
 size_t sta_build_mask_workspace(int32_t B, int32_t heads, int32_t d, sta_grid g);
+size_t sta_build_mask_workspace_min(int32_t B, int32_t heads, int32_t d, sta_grid g);
 
 /* sta_build_mask -- per-head tile mask as CSR lists (Compact Attention Fig. 3:
  * masks computed online are loaded into the block-sparse kernel; Fig. 4: the
@@ -122,7 +128,9 @@ size_t sta_build_mask_workspace(int32_t B, int32_t heads, int32_t d, sta_grid g)
  *   block_mask       : optional uint8 [B, heads, Nt, Nt] (0/1); NULL to skip
  *   block_probs      : optional fp32 [B, heads, Nt, Nt], the P the selection
  *                      used (0 where !use_scores); NULL to skip
- *   workspace        : device, >= sta_build_mask_workspace() bytes, 256-aligned
+ *   workspace        : device, >= sta_build_mask_workspace_min() bytes (the
+ *                      full sta_build_mask_workspace() for the fastest
+ *                      layout), 256-aligned
  * The call is deterministic: the same inputs give bit-identical outputs. */
 sta_status sta_build_mask(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads,
                           int32_t d, sta_grid g, const sta_mask_params *p, int32_t *row_ptr,
@@ -182,9 +190,9 @@ sta_status sta_attn_fwd_raster(const void *q, const void *k, const void *v, void
  * workspace: the workspace is a file-scope static device array of
  * STA_NOALLOC_SCRATCH_BYTES (32 MiB), present on every GPU that loads the
  * library until the process exits. The caller still passes inputs and outputs.
- *   - Sizes whose workspace (sta_build_mask_workspace) exceeds the array are
- *     rejected with STA_ERR_WORKSPACE before anything runs (e.g. 40 heads of a
- *     21x30x52 grid fit; 40 heads of 21x45x80 do not).
+ *   - Sizes whose minimum workspace (sta_build_mask_workspace_min) exceeds
+ *     the array are rejected with STA_ERR_WORKSPACE before anything runs
+ *     (e.g. 40 heads of a 21x30x52 grid fit; 40 heads of 21x45x80 do not).
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress (the device must be current); make that first call
  *     before any stream capture. Later calls reuse the cached address.

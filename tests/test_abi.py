@@ -52,8 +52,10 @@ def test_workspace_size(sta):
     g = sta.grid(21, 45, 80)
     ws = sta.sta_build_mask_workspace(1, 40, 128, g)
     R = 40 * 1260
-    assert ws >= 2 * R * 128 * 4 + R * 40 * 4 + R * 4
-    assert ws % 256 == 0
+    ws_min = sta.sta_build_mask_workspace_min(1, 40, 128, g)
+    assert ws_min >= 2 * R * 128 * 4 + R * 40 * 4 + R * 4
+    assert ws >= ws_min + R * 1260 * 4  # plus the P row buffer of the two-pass layout
+    assert ws % 256 == 0 and ws_min % 256 == 0
     assert sta.sta_build_mask_workspace(1, 40, 96, g) == 0
 
 

@@ -666,6 +666,37 @@ def test_search_windows_rejects_bad_groups(sta):
             sta.sta_search_windows(m, 1, 1, g, lo, tau, 1.0, out)
 
 
+@pytest.mark.parametrize("floor", [False, True])
+@pytest.mark.parametrize("probs", [False, True])
+def test_build_mask_fused_and_two_pass_layouts_agree(sta, gp, floor, probs):
+    """The minimum workspace runs the fused score/select pass, the full one
+    the scores pass plus a separate select pass (and block_probs, when given,
+    holds the rows): the CSR, the byte mask and P agree bit for bit."""
+    T, H, W, Hh, B, d = 5, 24, 37, 3, 2, 128
+    g = sta.grid(T, H, W)
+    q, k, _ = _structured(T, H, W, Hh, d, seed=23, B=B)
+    qt, kt = (gp.reorder(x, B, Hh, d, g) for x in (q, k))
+    nh, nw, nt, _ = O.tile_grid(T, H, W)
+    win_t = torch.from_numpy(np.tile(np.array([[[1, 1, 0, nw - 1], [0, 0, -1, -1]]], dtype=np.int32),
+                                     (Hh, 1, 1))).cuda()
+    params = sta.mask_params(0.8, 3, True, 0.0, (0, 2), win_t, head_floor=floor)
+    outs = []
+    for ws_bytes in (sta.sta_build_mask_workspace_min(B, Hh, d, g), sta.sta_build_mask_workspace(B, Hh, d, g)):
+        bufs = sta.MaskBuffers(B, Hh, d, g, "cuda", True, probs)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        sta.sta_build_mask(qt, kt, B, Hh, d, g, params, bufs.row_ptr, bufs.col_idx, bufs.nnz, bufs.block_mask,
+                           bufs.block_probs, ws, ws_bytes)
+        torch.cuda.synchronize()
+        outs.append(bufs)
+    a, b = outs
+    n = int(a.nnz.item())
+    assert n == int(b.nnz.item()) and n > 0
+    assert torch.equal(a.row_ptr, b.row_ptr) and torch.equal(a.col_idx[:n], b.col_idx[:n])
+    assert torch.equal(a.block_mask, b.block_mask)
+    if probs:
+        assert torch.equal(a.block_probs.view(torch.int32), b.block_probs.view(torch.int32))
+
+
 # ------------------------------------------ raster-layout path (no reorder)
 def _raster_vs_tiled(sta, gp, q, k, v, B, Hh, d, T, H, W, params, rows_check=None):
     """Mask and attention through the raster entry points equal, bit for bit,

@@ -87,10 +87,10 @@ def test_noalloc_rejects_sizes_beyond_the_array(sta):
     # 40 heads of the 21x45x80 layer need ~60 MB of workspace: refused up
     # front, before any launch (the pointers are never touched).
     g = sta.grid(21, 45, 80)
-    assert sta.sta_build_mask_workspace(1, 40, 128, g) > (32 << 20)
+    assert sta.sta_build_mask_workspace_min(1, 40, 128, g) > (32 << 20)
     params = sta.mask_params(0.95, 8, True)
     status = sta._lib.sta_build_mask_noalloc(256, 256, 1, 40, 128, g, sta.ctypes.byref(params), 256, 256,
                                              256, None, None, None)
     assert status == sta.STA_ERR_WORKSPACE
     # 40 heads of the 21x30x52 layer fit
-    assert sta.sta_build_mask_workspace(1, 40, 128, sta.grid(21, 30, 52)) <= (32 << 20)
+    assert sta.sta_build_mask_workspace_min(1, 40, 128, sta.grid(21, 30, 52)) <= (32 << 20)
