@@ -869,6 +869,40 @@ def test_rectified_720p_sampled_rows(sta, gp):
     del qt, kt, vt
 
 
+def test_step_replays_from_a_cuda_graph(sta, gp):
+    """The raster mask build and attention launch nothing that breaks stream
+    capture (no allocation, no host synchronisation): a captured step replays
+    with the same outputs as the eager calls."""
+    T, H, W, Hh, B, d = 4, 30, 44, 4, 1, 128
+    g = sta.grid(T, H, W)
+    q, k, v = _structured(T, H, W, Hh, d, seed=41, B=B)
+    nh, nw, nt, _ = O.tile_grid(T, H, W)
+    win_t = torch.from_numpy(np.tile(np.array([[[1, 2, 0, nw - 1], [0, 0, -1, -1]]], dtype=np.int32),
+                                     (Hh, 1, 1))).cuda()
+    params = sta.mask_params(0.9, 2, True, 0.0, (0, 1), win_t)
+    bufs = sta.MaskBuffers(B, Hh, d, g, "cuda")
+    o_eager = torch.empty_like(q)
+    sta.build_mask(q, k, B, Hh, d, g, params, bufs, raster=True)
+    sta.sta_attn_fwd_raster(q, k, v, o_eager, None, bufs.row_ptr, bufs.col_idx, B, Hh, d, g)
+    torch.cuda.synchronize()
+    rp_eager = bufs.row_ptr.clone()
+    o = torch.zeros_like(q)
+    bufs.row_ptr.zero_()
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        sta.build_mask(q, k, B, Hh, d, g, params, bufs, raster=True)
+        sta.sta_attn_fwd_raster(q, k, v, o, None, bufs.row_ptr, bufs.col_idx, B, Hh, d, g)
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    assert torch.equal(bufs.row_ptr, rp_eager)
+    assert torch.equal(o.view(torch.int16), o_eager.view(torch.int16))
+    del graph
+
+
 # ------------------------------------------------------- failure detection
 def test_bounded_wait_reports_timeout_and_context_survives(sta, gp):
     """The pipeline's bounded wait, on a barrier nothing completes, gives up
