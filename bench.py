@@ -9,6 +9,7 @@ raster order happen inside the kernels' loads and stores).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
   python bench.py --search-curve [--workload NAME]   (window search, recall vs density)
   python bench.py --sweep                              (every layer of the workload table)
+  python bench.py --l2-probe                           (the attention's tile-load stream alone)
 
 Rank 0 prints one JSON line. Under torchrun every rank runs its own layer
 (independent problems, no collective on the data path: weak scaling); the
@@ -601,6 +602,31 @@ def blas_threads():
         return None
 
 
+def l2_probe(sta, dev, iters=2000):
+    """Rate of the attention kernel's load stream on its own (16 KB key-tile
+    TMA loads at pseudo-random tiles), from an L2-resident 40 MB region and
+    from a 4 GB region, at 1 and 2 CTAs per SM and 2 to 6 loads in flight."""
+    props = torch.cuda.get_device_properties(dev)
+    rows = []
+    for label, nbytes in (("L2-resident 40 MB", 40 << 20), ("4 GB (DRAM)", 4 << 30)):
+        buf = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        for cps in (1, 2):
+            for slots in (2, 4, 6):
+                if slots * 16384 * cps > 200 * 1024:
+                    continue
+                sta.sta_selftest_tma_stream(buf, cps, slots, 50)
+                ms = _median_ms(lambda: sta.sta_selftest_tma_stream(buf, cps, slots, iters), 5)
+                moved = props.multi_processor_count * cps * iters * 16384
+                line = {"source": label, "ctas_per_sm": cps, "loads_in_flight_per_cta": slots, "ms": ms,
+                        "tb_per_s": moved / (ms * 1e-3) / 1e12}
+                rows.append(line)
+                print(json.dumps(line), flush=True)
+        del buf
+        torch.cuda.empty_cache()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    return rows
+
+
 def cpu_oracle_sample(cfg, layer, budget_s, rows_per_head=8, max_heads=None):
     """Time the oracle (as it stands) on a bounded sample of the same layer:
     for sampled heads, its reorder, pooling, scores, selection and windows
@@ -699,6 +725,8 @@ def main():
                     help="use only this many heads of the workload (small cases for ncu captures)")
     ap.add_argument("--sweep", action="store_true",
                     help="time every layer of the workload table (one JSON line per row) and exit")
+    ap.add_argument("--l2-probe", action="store_true",
+                    help="rate of the attention's 16 KB TMA tile loads on their own, then exit")
     ap.add_argument("--search-curve", action="store_true",
                     help="print the recall-target vs density curve of the window search and exit")
     args = ap.parse_args()
@@ -714,6 +742,10 @@ def main():
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    if args.l2_probe:
+        if rank == 0:
+            l2_probe(sta, dev)
+        return
     if args.sweep:
         if rank == 0:
             peaks, _ = load_peaks()

@@ -131,6 +131,45 @@ bool device_is_sm100() {
   return major == 10 && minor == 0;
 }
 
+// The attention kernel's load stream without its compute: one thread per CTA
+// keeps `slots` 16 KB key-tile loads (two 64x64 bf16 boxes, 128 B swizzle,
+// as the kernel issues them) in flight from `tiles` tiles of buf, at
+// pseudo-random tile indices, for `iters` loads. Timed by the caller; it
+// gives the L2-to-SM rate TMA reaches on this GPU at a given depth.
+constexpr int STREAM_MAX_SLOTS = 6;
+__global__ void __launch_bounds__(32) tma_stream_kernel(const __grid_constant__ CUtensorMap tm, int tiles,
+                                                        int slots, int iters) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + slots * 16384);
+  if (threadIdx.x != 0) return;
+  for (int sl = 0; sl < slots; ++sl) tc::mbar_init(bar + sl, 1);
+  tc::fence_barrier_init();
+  uint32_t seed = blockIdx.x * 2654435761u + 12345u;
+  auto issue = [&](int sl) {
+    seed = seed * 1664525u + 1013904223u;
+    const int tile = (int)(seed % (uint32_t)tiles);
+    tc::mbar_expect_tx(bar + sl, 16384);
+    tc::tma_load_2d(tc::smem_u32(smem + sl * 16384), &tm, bar + sl, 0, tile * 64);
+    tc::tma_load_2d(tc::smem_u32(smem + sl * 16384 + 8192), &tm, bar + sl, 64, tile * 64);
+  };
+  int issued = 0;
+  for (; issued < slots && issued < iters; ++issued) issue(issued);
+  for (int i = 0; i < iters; ++i) {
+    const int sl = i % slots;
+    // spin without a suspend hint, so that the wait adds no wake-up delay to
+    // the rate being measured; bounded, then recorded like the pipeline waits
+    bool ok = false;
+    for (long long spin = 0; spin < 100000000LL && !ok; ++spin) ok = tc::mbar_try_wait(bar + sl, (i / slots) & 1);
+    if (!ok) {
+      record_error(DEV_ERR_TIMEOUT);
+      for (int j = i + 1; j < issued; ++j) tc::mbar_wait(bar + j % slots, (j / slots) & 1, nullptr, 200000000LL);
+      return;
+    }
+    if (issued < iters) issue(issued++ % slots);
+  }
+}
+
 // One thread waits, with the pipeline's bounded wait, on a barrier that
 // expects one arrival that never comes.
 __global__ void selftest_wait_kernel(long long limit) {
@@ -503,6 +542,31 @@ sta_status sta_search_windows(const float *block_mass, int32_t B, int32_t heads,
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   search_windows_kernel<<<(unsigned)(B * heads), SEARCH_THREADS, smem, s>>>(block_mass, geo, num_groups, glo,
                                                                            tau, lambda, windows, stats);
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
+}
+
+sta_status sta_selftest_tma_stream(const void *buf, size_t bytes, int32_t ctas_per_sm, int32_t slots,
+                                   int32_t iters, sta_stream_t stream) {
+  if (buf == nullptr || (reinterpret_cast<uintptr_t>(buf) & 15u) != 0 || bytes < 16384) return STA_ERR_INVALID_ARG;
+  if (ctas_per_sm < 1 || ctas_per_sm > 8 || slots < 1 || slots > STREAM_MAX_SLOTS || iters < 1 ||
+      (long long)slots * 16384 * ctas_per_sm > 200 * 1024)
+    return STA_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return STA_ERR_UNSUPPORTED;
+  const long long tiles = (long long)(bytes / 16384);
+  if (tiles * 64 >= (1LL << 31)) return STA_ERR_UNSUPPORTED;
+  CUtensorMap tm;
+  if (!make_tile_map(&tm, buf, (unsigned long long)tiles * 64, 128)) return STA_ERR_CUDA;
+  int dev = 0, sms = 0;
+  STA_CUDA_TRY(cudaGetDevice(&dev));
+  STA_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const size_t smem = (size_t)slots * 16384 + 64 + 1024;
+  STA_CUDA_TRY(cudaFuncSetAttribute(tma_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)((size_t)STREAM_MAX_SLOTS * 16384 + 64 + 1024)));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // ctas_per_sm CTAs per SM through the grid size; they fit on an SM at once
+  // (checked above)
+  tma_stream_kernel<<<(unsigned)(sms * ctas_per_sm), 32, smem, s>>>(tm, (int)tiles, slots, iters);
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }

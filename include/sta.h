@@ -285,6 +285,17 @@ sta_status sta_search_windows(const float *block_mass, int32_t B, int32_t heads,
  * sta_get_device_error() and leaves the context usable. */
 sta_status sta_selftest_wait_timeout(int64_t limit_cycles, sta_stream_t stream);
 
+/* sta_selftest_tma_stream -- the attention kernel's load stream on its own:
+ * ctas_per_sm CTAs per SM, each keeping `slots` (1..6) 16 KB key-tile loads
+ * in flight (two 64x64 bf16 TMA boxes with 128 B swizzle, as the kernel
+ * loads K and V), from pseudo-random tiles of buf (device, bytes >= 16 KB,
+ * 16-byte aligned), `iters` loads per CTA; slots x 16 KB x ctas_per_sm must
+ * fit in 200 KB. The caller times it; bytes moved = SMs x ctas_per_sm x
+ * iters x 16384. It measures the L2-to-SM rate the hardware gives such loads
+ * when nothing else runs (a denominator for the attention's load stream). */
+sta_status sta_selftest_tma_stream(const void *buf, size_t bytes, int32_t ctas_per_sm, int32_t slots,
+                                   int32_t iters, sta_stream_t stream);
+
 /* Reads and clears the device error word of the current device after
  * synchronising `stream`. STA_OK if no device-side fault was recorded. */
 sta_status sta_get_device_error(sta_stream_t stream);

@@ -903,6 +903,24 @@ def test_step_replays_from_a_cuda_graph(sta, gp):
     del graph
 
 
+def test_tma_stream_selftest_runs_and_checks_arguments(sta):
+    buf = torch.zeros(8 << 20, dtype=torch.uint8, device="cuda")
+    sta.sta_selftest_tma_stream(buf, 2, 4, 20)  # first launch loads the module
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    sta.sta_selftest_tma_stream(buf, 2, 4, 200)
+    e1.record()
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    moved = torch.cuda.get_device_properties(0).multi_processor_count * 2 * 200 * 16384
+    assert moved / (e0.elapsed_time(e1) * 1e-3) > 1e12  # well above 1 TB/s from L2
+    with pytest.raises(sta.StaError):
+        sta.sta_selftest_tma_stream(buf, 2, 7, 10)  # more than 6 loads in flight
+    with pytest.raises(sta.StaError):
+        sta.sta_selftest_tma_stream(buf, 8, 6, 10)  # does not fit in shared memory
+
+
 # ------------------------------------------------------- failure detection
 def test_bounded_wait_reports_timeout_and_context_survives(sta, gp):
     """The pipeline's bounded wait, on a barrier nothing completes, gives up
