@@ -54,6 +54,7 @@ search_windows_kernel(const float *__restrict__ mass, Geo g, int G, GroupLo glo,
   __shared__ unsigned long long mv_lost[STA_MAX_GROUPS][SEARCH_MOVES];
   __shared__ unsigned int mv_removed[STA_MAX_GROUPS][SEARCH_MOVES];
   __shared__ int done;
+  __shared__ int dirty;  // group whose moves must be re-evaluated (-1: all)
   const int nt = g.Nt, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = SEARCH_THREADS / 32;
   const long long bh = blockIdx.x;
@@ -73,7 +74,10 @@ search_windows_kernel(const float *__restrict__ mass, Geo g, int G, GroupLo glo,
     gtab[dt] = grp;
   }
   if (tid < G * 4) win[tid / 4][tid % 4] = (tid % 2 == 0) ? g.NH - 1 : g.NW - 1;
-  if (tid == 0) done = 0;
+  if (tid == 0) {
+    done = 0;
+    dirty = -1;
+  }
   // total integer mass W (every pair is covered at the start)
   unsigned long long tot = 0;
   for (int q = warp; q < nt; q += nwarps)
@@ -91,7 +95,12 @@ search_windows_kernel(const float *__restrict__ mass, Geo g, int G, GroupLo glo,
   const int max_steps = G * (2 * g.NH + 2 * g.NW + 4);
 
   for (int step = 0; step < max_steps && !done; ++step) {
+    // A move of group g changes only pairs whose |dt| falls in g, so the other
+    // groups' move costs from earlier steps still hold: only the group the
+    // last step moved is scanned again (all groups on the first step).
+    const int only = dirty;
     for (int gi = 0; gi < G; ++gi) {
+      if (only >= 0 && gi != only) continue;
       const int ry1 = win[gi][0], rx1 = win[gi][1], ry2 = win[gi][2], rx2 = win[gi][3];
       int cand[SEARCH_MOVES][4];
 #pragma unroll
@@ -173,6 +182,7 @@ search_windows_kernel(const float *__restrict__ mass, Geo g, int G, GroupLo glo,
         for (int e = 0; e < 4; ++e) win[gi][e] = w4[e];
         covered -= mv_lost[gi][mi];
         covered_pairs -= mv_removed[gi][mi];
+        dirty = gi;
       }
     }
     __syncthreads();
