@@ -79,11 +79,18 @@ def load_peaks():
 
 
 def attn_source_hash():
+    """Hash of the attention kernel's code (comments and blank space left
+    out, so that editing a comment keeps a traffic capture valid)."""
+    import re
+
     h = hashlib.sha256()
     d = os.path.join(ROOT, "block_sparse_attention_28_b200", "csrc")
     for name in ("sta_attn.cuh", "sta_tc.cuh", "sta_common.cuh"):
-        with open(os.path.join(d, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(d, name)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -3,9 +3,12 @@
 //
 // One CTA computes 128 query rows: two query tiles of one head, the same
 // spatial tile in two consecutive frames (a 128-row tcgen05 tile; a 64-token
-// tile alone would leave half of the MMA rows idle). The two CSR rows are merged into one ascending key-tile list
-// with a per-half membership flag; a half whose list lacks the key tile gets
-// P = 0 for that tile, so the work is |A u B| key tiles of 128 x 64.
+// tile alone would leave half of the MMA rows idle). The two CSR rows are
+// merged into one ascending key-tile list with a per-half membership flag; a
+// half whose list lacks the key tile gets P = 0 for that tile, so the work is
+// |A u B| key tiles of 128 x 64. All roles walk the list from the first key
+// tile at or after the CTA's own query tile and wrap around, which spreads
+// the requests of neighbouring CTAs over L2.
 //
 // Warp roles (192 threads):
 //   warps 0-3  softmax + correction + epilogue; thread i owns query row i
@@ -19,7 +22,9 @@
 //   warp 5     MMA issuer (one thread): S_j = Q K_j^T (SS, M=128 N=64) into
 //              one of two TMEM S buffers, O += P_j V_j (A = P from TMEM,
 //              B = V MN-major from shared memory, M=128 N=d).
-// TMEM columns: S0 [0,64) S1 [64,128) O [128, 128+d).
+// TMEM columns: S0 [0,64) S1 [64,128) O [128, 128+d). Two CTAs share an SM
+// (TMEM 2 x 256 columns, shared memory 2 x 103 KB), so one CTA's softmax runs
+// while the other's MMAs do.
 #pragma once
 #include "sta_common.cuh"
 #include "sta_tc.cuh"
