@@ -226,6 +226,24 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(win), "source": self.source}
 
 
+def count_step_launches(layer):
+    """Kernels that one step launches, as CUPTI records them (torch.profiler)
+    on an untimed step: (count, short kernel names), or (None, None) when the
+    profiler cannot record kernels here."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CPU, ProfilerActivity.CUDA]) as prof:
+            layer.step()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    except Exception:  # no CUPTI: the caller falls back to the static count
+        return None, None
+    kernels = [n.split("(")[0].replace("void ", "") for n in names if "Memcpy" not in n and "Memset" not in n]
+    return (len(kernels), kernels) if kernels else (None, None)
+
+
 class Layer:
     """Device buffers and launches of one step of the path."""
 
@@ -249,7 +267,9 @@ class Layer:
             self.win = None
         self.params = sta.mask_params(c.top_p, c.k_min, c.use_scores, 0.0, c.group_lo, self.win)
         self.bufs = sta.MaskBuffers(self.B, self.Hh, self.d, self.g, dev)
-        self.launches_per_step = 4 + 1  # pool/select/scan/fill, attn (the tile gather is the TMA box)
+        # pool, tensor-core scores, select, scan, fill; attention (the tile
+        # gather is the TMA box, so no reorder launch)
+        self.launches_per_step = 5 + 1
 
     @property
     def qt(self):
@@ -719,6 +739,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--no-launch-count", action="store_true",
+                    help="skip the CUPTI count of one step's kernels (for runs under ncu); "
+                         "gpu_launches is then the static count")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=16,
                     help="pipelined end-to-end steps (fill and drain are amortised over them)")
@@ -785,6 +808,11 @@ def main():
         layer.step()
     barrier()
     assert sta.sta_get_device_error() == sta.STA_OK
+    n_launch, step_kernels = (None, None) if args.no_launch_count else count_step_launches(layer)
+    launch_src = "cupti, one untimed step"
+    if n_launch is None:
+        n_launch, launch_src = layer.launches_per_step, "static count"
+    barrier()
 
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
@@ -876,7 +904,9 @@ def main():
                          "algorithmic": f"{pairs} kept pairs x 4*64*64*{cfg.d} flop"},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": K * layer.launches_per_step,
+            "gpu_launches": K * n_launch,
+            "gpu_launches_source": launch_src,
+            "step_kernels": step_kernels,
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)

@@ -178,11 +178,17 @@ def sta_build_mask(q_tiled, k_tiled, B, heads, d, g, params, row_ptr, col_idx, n
            "sta_build_mask")
 
 
+# bytes of the static device array behind sta_build_mask_noalloc (the
+# header's STA_NOALLOC_SCRATCH_BYTES)
+STA_NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
 def sta_build_mask_noalloc(q_tiled, k_tiled, B, heads, d, g, params, row_ptr, col_idx, nnz_dev,
                            block_mask=None, block_probs=None, stream=None):
     """sta_build_mask without a workspace argument, for callers that cannot
     allocate device memory: the library's static 32 MiB device array serves as
-    the workspace (see include/sta.h for the size limit and sharing rules)."""
+    the workspace, so the results are those of sta_build_mask with a workspace
+    of that size (see include/sta.h for the size limit and sharing rules)."""
     _check(_lib.sta_build_mask_noalloc(_ptr(q_tiled), _ptr(k_tiled), B, heads, d, g, ctypes.byref(params),
                                        _ptr(row_ptr), _ptr(col_idx), _ptr(nnz_dev), _ptr(block_mask),
                                        _ptr(block_probs), _stream(stream)),

@@ -9,6 +9,7 @@
 #include "sta_common.cuh"
 #include "sta_mask.cuh"
 #include "sta_reorder.cuh"
+#include "sta_score.cuh"
 #include "sta_search.cuh"
 
 using namespace sta;
@@ -34,11 +35,12 @@ bool common_sizes_ok(int32_t B, int32_t heads, int32_t d, sta_grid g, Geo *geo, 
   return true;
 }
 
-// total_min: the fused score/select pass; total: plus a P row buffer
-// [B*heads*Nt, Nt] fp32 for the split passes (scores, then a select pass
-// with four CTAs per SM).
+// total_min: the fused score/select pass; total: plus the low tf32 parts of
+// the pooled Q and K (qlo, klo) and a row buffer [B*heads*Nt, Nt] fp32 for
+// the split passes (tensor-core scores, then a select pass with four CTAs
+// per SM).
 struct MaskWs {
-  size_t qbar, kbar, bits, counts, sel, kfloor, total_min, prows, total;
+  size_t qbar, kbar, bits, counts, sel, kfloor, total_min, qlo, klo, prows, total;
 };
 
 MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
@@ -59,6 +61,10 @@ MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
   w.kfloor = off;
   off = align_up(off + (size_t)B * heads * sizeof(int32_t), 256);
   w.total_min = off;
+  w.qlo = off;
+  off = align_up(off + R * d * sizeof(float), 256);
+  w.klo = off;
+  off = align_up(off + R * d * sizeof(float), 256);
   w.prows = off;
   off = align_up(off + R * g.Nt * sizeof(float), 256);
   w.total = off;
@@ -67,9 +73,9 @@ MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
 
 // Dynamic shared memory of score_select_kernel<D, qb, mode>.
 size_t select_smem(int d, const Geo &g, bool use_scores, int qb = SEL_QB, int mode = SEL_FUSED) {
-  const size_t q = (mode != SEL_SELECT && use_scores) ? (size_t)qb * d : 0;
+  const size_t q = (mode == SEL_FUSED && use_scores) ? (size_t)qb * d : 0;
   const size_t scores = use_scores ? (size_t)(qb * g.Nt + (SEL_THREADS / 32) * 256) : 0;
-  const size_t tables = (mode == SEL_SCORES) ? 0 : (size_t)((g.Nt + g.T + 3) & ~3) + 4 * STA_MAX_GROUPS;
+  const size_t tables = (size_t)((g.Nt + g.T + 3) & ~3) + 4 * STA_MAX_GROUPS;
   return (q + scores + tables) * sizeof(float);
 }
 
@@ -121,6 +127,46 @@ bool make_raster_map(CUtensorMap *map, const void *base, const Geo &g, int B, in
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Pooled rows [bh, Nt, d] fp32 as a 3D tensor (d, Nt, bh); a box is 32 d-values
+// (128 B) x `rows` tiles x 1 head, zero-filled past Nt, 128 B swizzle.
+bool make_pooled_map(CUtensorMap *map, const float *base, long long bh, int nt, int d, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)nt, (cuuint64_t)bh};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)nt * d * 4};
+  cuuint32_t box[3] = {32, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor-core scores S = scale * qbar kbar^T of every head into rows
+// [bh*Nt + qt][kt] of S, from the split pooled parts.
+template <int D>
+sta_status launch_scores_tc(const float *qhi, const float *qlo, const float *khi, const float *klo, float *S,
+                            long long bh, const Geo &g, float scale, cudaStream_t s) {
+  CUtensorMap m_qhi, m_qlo;
+  if (!make_pooled_map(&m_qhi, qhi, bh, g.Nt, D, score::N) || !make_pooled_map(&m_qlo, qlo, bh, g.Nt, D, score::N))
+    return STA_ERR_CUDA;
+  auto kern = score::score_tc_kernel<D>;
+  const int smem = score::Cfg<D>::SMEM;
+  STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  // key blocks x query ranges x heads, with at least two waves of CTAs
+  // where the query range can be split
+  const int kblocks = (g.Nt + score::M - 1) / score::M;
+  const int qblocks = (g.Nt + score::N - 1) / score::N;
+  const long long base = (long long)kblocks * bh;
+  int parts = (int)((2LL * 148 + base - 1) / base);
+  parts = parts < 1 ? 1 : (parts > qblocks ? qblocks : parts);
+  const int per_part = (qblocks + parts - 1) / parts;
+  parts = (qblocks + per_part - 1) / per_part;  // no empty range
+  dim3 grid((unsigned)kblocks, (unsigned)parts, (unsigned)bh);
+  kern<<<grid, score::NUM_THREADS, smem, s>>>(khi, klo, m_qhi, m_qlo, S, g.Nt, scale, per_part * score::N);
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
 }
 
 bool device_is_sm100() {
@@ -183,9 +229,12 @@ __global__ void selftest_wait_kernel(long long limit) {
   }
 }
 
-// ws_bytes decides the selection layout: with room for the P row buffer (or
-// a caller's block_probs to hold the rows) the scores pass and a separate,
-// smaller select pass run; otherwise the fused pass. Both give the same bits.
+// ws_bytes decides the layout. With the full workspace the scores run on
+// the tensor cores into a row buffer (the caller's block_probs when given)
+// and a separate, smaller select pass does the softmax and the selection;
+// with the minimum workspace one fused pass computes the scores with fp32
+// FMA chains. Each layout is deterministic; both are within their stated
+// error bounds of the exact scores.
 template <int D>
 sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads,
                         const Geo &g, const sta_mask_params *p, int32_t *row_ptr, int32_t *col_idx,
@@ -200,17 +249,23 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
   const int wpr = (g.Nt + 31) / 32;
   const bool use_scores = p->use_scores != 0;
   const float scale = p->sm_scale != 0.0f ? p->sm_scale : 1.0f / sqrtf((float)D);
+  const bool full_ws = ws_bytes >= L.total;
 
   const float *P_in = use_scores ? p->block_scores : nullptr;
+  const bool tc_scores = use_scores && P_in == nullptr && full_ws;
+  float *qlo = tc_scores ? reinterpret_cast<float *>(ws + L.qlo) : nullptr;
+  float *klo = tc_scores ? reinterpret_cast<float *>(ws + L.klo) : nullptr;
   if (use_scores && P_in == nullptr) {
     const long long warps = 2 * R;
     const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
     if (raster)
       pool_kernel<D, true><<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(q_tiled),
-                                                  static_cast<const uint4 *>(k_tiled), qbar, kbar, R, g, heads);
+                                                  static_cast<const uint4 *>(k_tiled), qbar, kbar, qlo, klo, R,
+                                                  g, heads);
     else
       pool_kernel<D, false><<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(q_tiled),
-                                                   static_cast<const uint4 *>(k_tiled), qbar, kbar, R, g, heads);
+                                                   static_cast<const uint4 *>(k_tiled), qbar, kbar, qlo, klo, R,
+                                                   g, heads);
     STA_CUDA_TRY(cudaGetLastError());
   }
   GroupLo glo;
@@ -220,11 +275,7 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
   int *kfloor = reinterpret_cast<int *>(ws + L.kfloor);
   const int *windows = p->windows;
   const int G = p->windows ? p->num_groups : 0;
-  // P rows: the caller's block_probs, else the workspace's row buffer
-  float *prows = block_probs != nullptr ? block_probs
-                                        : (ws_bytes >= L.total ? reinterpret_cast<float *>(ws + L.prows) : nullptr);
-  const bool split = (use_scores && P_in == nullptr && prows != nullptr) || (use_scores && P_in != nullptr) ||
-                     !use_scores;
+  const bool split = !use_scores || P_in != nullptr || full_ws;
   if (!split) {
     // fused: scores, softmax, selection and windows per 16-row CTA
     const size_t smem = select_smem(D, g, use_scores, SEL_QB, SEL_FUSED);
@@ -236,30 +287,26 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
       // pass 1: base selection counts; per-head floor; pass 2 re-selects with
       // k_min raised to the floor
       kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, nullptr, 0, glo,
-                                           bits, counts, nullptr, wpr, nullptr, sel, nullptr);
+                                           bits, counts, nullptr, wpr, nullptr, sel, nullptr, 0);
       STA_CUDA_TRY(cudaGetLastError());
       head_floor_kernel<<<(unsigned)(B * heads), FLOOR_THREADS, 0, s>>>(sel, kfloor, g);
       STA_CUDA_TRY(cudaGetLastError());
     }
     kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, windows, G, glo,
                                          bits, counts, block_probs, wpr, floor ? kfloor : nullptr, nullptr,
-                                         nullptr);
+                                         nullptr, 0);
     STA_CUDA_TRY(cudaGetLastError());
   } else {
-    const float *P_sel = P_in;        // rows the select pass reads
-    float *probs_sel = block_probs;   // and copies out (clamped) when from the caller
-    if (use_scores && P_in == nullptr) {
-      // scores pass: P rows into prows (the caller's block_probs when given)
-      const size_t smem = select_smem(D, g, true, SEL_QB, SEL_SCORES);
-      auto kern = score_select_kernel<D, SEL_QB, SEL_SCORES>;
-      if (smem > 48 * 1024)
-        STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-      dim3 grid((unsigned)((g.Nt + SEL_QB - 1) / SEL_QB), (unsigned)(B * heads));
-      kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, nullptr, 0, glo,
-                                           bits, counts, prows, wpr, nullptr, nullptr, nullptr);
-      STA_CUDA_TRY(cudaGetLastError());
-      P_sel = prows;
-      probs_sel = nullptr;  // already written
+    const float *P_sel = P_in;  // rows the select pass reads
+    int logits = 0;             // whether they are scores still to be softmaxed
+    if (tc_scores) {
+      // scores into the caller's block_probs when given (the select pass
+      // overwrites them with P), else into the workspace's row buffer
+      float *rows = block_probs != nullptr ? block_probs : reinterpret_cast<float *>(ws + L.prows);
+      const sta_status st = launch_scores_tc<D>(qbar, qlo, kbar, klo, rows, (long long)B * heads, g, scale, s);
+      if (st != STA_OK) return st;
+      P_sel = rows;
+      logits = 1;
     }
     const size_t smem = select_smem(D, g, use_scores, SEL_QB_SELECT, SEL_SELECT);
     auto kern = score_select_kernel<D, SEL_QB_SELECT, SEL_SELECT>;
@@ -268,14 +315,14 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
     dim3 grid((unsigned)((g.Nt + SEL_QB_SELECT - 1) / SEL_QB_SELECT), (unsigned)(B * heads));
     if (floor) {
       kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, nullptr, 0, glo,
-                                           bits, counts, nullptr, wpr, nullptr, sel, P_sel);
+                                           bits, counts, nullptr, wpr, nullptr, sel, P_sel, logits);
       STA_CUDA_TRY(cudaGetLastError());
       head_floor_kernel<<<(unsigned)(B * heads), FLOOR_THREADS, 0, s>>>(sel, kfloor, g);
       STA_CUDA_TRY(cudaGetLastError());
     }
     kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, use_scores ? 1 : 0,
-                                         windows, G, glo, bits, counts, probs_sel, wpr,
-                                         floor ? kfloor : nullptr, nullptr, P_sel);
+                                         windows, G, glo, bits, counts, block_probs, wpr,
+                                         floor ? kfloor : nullptr, nullptr, P_sel, logits);
     STA_CUDA_TRY(cudaGetLastError());
   }
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(counts, row_ptr, reinterpret_cast<long long *>(nnz_dev), R);

@@ -5,8 +5,11 @@
 //
 // Kernels, in launch order:
 //   pool_kernel          tile means of Q and K (HBM-bound, coalesced 16 B loads)
-//   score_select_kernel  16 query tiles x all key tiles per CTA: fp32 scores,
-//                        row softmax, selection, window test -> row bitsets
+//   score_tc_kernel      (sta_score.cuh, full workspace) the scores on the
+//                        tensor cores, rows of S written to a row buffer
+//   score_select_kernel  row softmax, selection, window test -> row bitsets;
+//                        with the minimum workspace it also computes the
+//                        scores (fp32 FMA chains, 16 query tiles per CTA)
 //   scan_kernel          exclusive scan of the row counts -> row_ptr, nnz
 //   fill_kernel          bitsets -> ascending col_idx (+ optional byte mask)
 #pragma once
@@ -16,17 +19,28 @@ namespace sta {
 
 constexpr float MASS_ONE_F = 16777216.0f;  // 2^24, fixed-point unit of the mass
 
+// fp32 rounded to the nearest tf32 (10 explicit mantissa bits, ties away
+// from zero); the low 13 bits of the result are zero.
+__device__ __forceinline__ float round_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
 // ---------------------------------------------------------------- pooling
 // One warp per (b*heads + h, tile). Each lane owns one 16-byte chunk of a row
 // and walks the tile's real rows; the sum is exact in fp64 (64 bf16 values),
-// the mean is rounded once to fp32.
+// the mean is rounded once to fp32. With qlo / klo given, the mean x is
+// stored split for the tensor-core scores: tf32(x) in qbar / kbar and
+// tf32(x - tf32(x)) in qlo / klo (round to nearest, ties away).
 // RASTER: Q and K in the raster layout [B, L, heads, d]; consecutive warps
 // take the same tile of consecutive heads, so together they read whole
 // token rows (all heads) at a time.
 template <int D, bool RASTER>
 __global__ void __launch_bounds__(256)
 pool_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k, float *__restrict__ qbar,
-            float *__restrict__ kbar, long long n_tiles_total, Geo g, int heads) {
+            float *__restrict__ kbar, float *__restrict__ qlo, float *__restrict__ klo,
+            long long n_tiles_total, Geo g, int heads) {
   constexpr int CPR = D / 8;      // chunks per row
   constexpr int RPI = 32 / CPR;   // rows per warp step
   const long long warp_id = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -36,6 +50,7 @@ pool_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k, float *__r
   if (idx >= n_tiles_total) return;
   const uint4 *src = is_k ? k : q;
   float *dst = is_k ? kbar : qbar;
+  float *dst_lo = is_k ? klo : qlo;
   const long long BH = n_tiles_total / g.Nt;
   const long long bh = RASTER ? idx % BH : idx / g.Nt;
   const int n = (int)(RASTER ? idx / BH : idx % g.Nt);
@@ -80,6 +95,18 @@ pool_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k, float *__r
     float out[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) out[e] = (float)(acc[e] / cnt);
+    if (dst_lo != nullptr) {
+      float lo[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float hi = round_tf32(out[e]);
+        lo[e] = round_tf32(out[e] - hi);  // x - hi is exact in fp32
+        out[e] = hi;
+      }
+      float4 *ol = reinterpret_cast<float4 *>(dst_lo + tile * D + c * 8);
+      ol[0] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+      ol[1] = make_float4(lo[4], lo[5], lo[6], lo[7]);
+    }
     float4 *o = reinterpret_cast<float4 *>(dst + tile * D + c * 8);
     o[0] = make_float4(out[0], out[1], out[2], out[3]);
     o[1] = make_float4(out[4], out[5], out[6], out[7]);
@@ -149,16 +176,17 @@ pool_kv_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v, uint4 *
 
 // ------------------------------------------------------ scores + selection
 constexpr int SEL_THREADS = 256;
-constexpr int SEL_QB = 16;  // query tiles per CTA of the score pass (fused or scores-only)
-constexpr int SEL_QB_SELECT = 8;  // rows per CTA of the select-only pass (one per warp)
+constexpr int SEL_QB = 16;        // query tiles per CTA of the fused pass
+constexpr int SEL_QB_SELECT = 8;  // rows per CTA of the select pass (one per warp)
 // Modes of score_select_kernel:
-//   SEL_FUSED   scores, softmax, selection and windows in one CTA (16 rows
-//               kept in shared memory; used when no row buffer is available)
-//   SEL_SCORES  scores and softmax only: P rows written to P_out
-//   SEL_SELECT  selection and windows only, on P rows read from P_in (no
-//               score code, so the CTA is small and four fit on an SM)
-constexpr int SEL_FUSED = 0, SEL_SCORES = 1, SEL_SELECT = 2;
-constexpr int SEL_KPT = 3;  // key tiles per thread in the score pass
+//   SEL_FUSED   scores (fp32 FMA chains), softmax, selection and windows in
+//               one CTA of 16 rows kept in shared memory (the minimum
+//               workspace: no row buffer)
+//   SEL_SELECT  softmax (when the rows hold scores), selection and windows
+//               on rows read from P_in; no score code, so the CTA is small
+//               and four fit on an SM
+constexpr int SEL_FUSED = 0, SEL_SELECT = 1;
+constexpr int SEL_KPT = 3;  // key tiles per thread in the fused score loop
 
 struct GroupLo {
   int v[STA_MAX_GROUPS];
@@ -168,6 +196,29 @@ __device__ __forceinline__ unsigned int warp_sum_u32(unsigned int x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
+}
+
+// Row softmax in fp32 over Sr[0, nt): maximum, expf, a fixed-order sum
+// (lane-strided partial sums, then a butterfly), IEEE divide. P replaces the
+// scores in Sr and is copied to out when given.
+__device__ __forceinline__ void row_softmax(float *Sr, int nt, int lane, float *out) {
+  float mx = -INFINITY;
+  for (int j = lane; j < nt; j += 32) mx = fmaxf(mx, Sr[j]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float sum = 0.0f;
+  for (int j = lane; j < nt; j += 32) {
+    const float e = expf(Sr[j] - mx);
+    Sr[j] = e;
+    sum += e;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  for (int j = lane; j < nt; j += 32) {
+    const float p = Sr[j] / sum;
+    Sr[j] = p;
+    if (out) out[j] = p;
+  }
 }
 
 __device__ __forceinline__ unsigned int mass_of(float p) {
@@ -247,9 +298,10 @@ __device__ void radix_level(const float *row, int nt, unsigned int target, bool 
 }
 
 // One CTA per (b*heads + h, block of QB query tiles).
-// Dynamic smem: qs [QB][D] fp32 (score modes), S [QB][Nt] fp32 and the
-// per-warp histograms (if use_scores), then the window tables (not in
-// SEL_SCORES). In SEL_SCORES, probs_out is the row buffer P_out.
+// Dynamic smem: qs [QB][D] fp32 (fused mode), S [QB][Nt] fp32 and the
+// per-warp histograms (if use_scores), then the window tables.
+// SEL_SELECT reads its rows from P_in: scores to be softmaxed when p_logits
+// (the tensor-core score pass), else block scores clamped to [0, 1].
 template <int D, int QB, int MODE>
 __global__ void __launch_bounds__(SEL_THREADS)
 score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar, int heads, Geo g,
@@ -257,8 +309,8 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
                     const int *__restrict__ windows, int G, GroupLo glo,
                     unsigned int *__restrict__ bits, int *__restrict__ counts,
                     float *__restrict__ probs_out, int wpr, const int *__restrict__ kmin_head,
-                    int *__restrict__ sel_count, const float *__restrict__ P_in) {
-  constexpr bool HAS_SCORES = MODE != SEL_SELECT;
+                    int *__restrict__ sel_count, const float *__restrict__ P_in, int p_logits) {
+  constexpr bool HAS_SCORES = MODE == SEL_FUSED;
   extern __shared__ __align__(16) float sm[];
   const int nt = g.Nt;
   const int bh = blockIdx.y;
@@ -278,7 +330,7 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
 
   // Window tables, once per CTA: packed (t, tile row, tile column) of every
   // key tile, the temporal group of every |dt|, and this head's extents.
-  if (MODE != SEL_SCORES && windows != nullptr) {
+  if (windows != nullptr) {
     for (int kt = tid; kt < nt; kt += SEL_THREADS) {
       const int t = kt / tpf, rem = kt - t * tpf;
       const int y = rem / g.NW, x = rem - y * g.NW;
@@ -358,35 +410,24 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
     unsigned int v_f = 0xFFFFFFFFu;  // keep P > v_f, plus c_f ties at v_f
     unsigned int c_f = 0u;
     if (use_scores) {
-      if (!HAS_SCORES || P_in != nullptr) {
-        // P rows of the score pass, or caller-supplied block scores (e.g.
-        // exact block masses), clamped to [0, 1] (a no-op on softmax rows)
+      float *pout = probs_out ? probs_out + row * nt : nullptr;
+      if (!HAS_SCORES && p_logits) {
+        // Phase 2: scores of the tensor-core pass, then the row softmax (the
+        // rows may be the caller's block_probs: each lane reads its entries
+        // before it overwrites them with P)
+        for (int j = lane; j < nt; j += 32) Sr[j] = P_in[row * nt + j];
+        row_softmax(Sr, nt, lane, pout);
+      } else if (!HAS_SCORES || P_in != nullptr) {
+        // caller-supplied block scores (e.g. exact block masses), clamped to [0, 1]
         for (int j = lane; j < nt; j += 32) {
           const float p = fminf(fmaxf(P_in[row * nt + j], 0.0f), 1.0f);
           Sr[j] = p;
-          if (probs_out) probs_out[row * nt + j] = p;
+          if (pout) pout[j] = p;
         }
       } else {
-        // Phase 2: row softmax in fp32 (max, expf, fixed-order sum, IEEE divide).
-        float mx = -INFINITY;
-        for (int j = lane; j < nt; j += 32) mx = fmaxf(mx, Sr[j]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        float sum = 0.0f;
-        for (int j = lane; j < nt; j += 32) {
-          const float e = expf(Sr[j] - mx);
-          Sr[j] = e;
-          sum += e;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        for (int j = lane; j < nt; j += 32) {
-          const float p = Sr[j] / sum;
-          Sr[j] = p;
-          if (probs_out) probs_out[row * nt + j] = p;
-        }
+        // Phase 2: row softmax of the fused pass's scores
+        row_softmax(Sr, nt, lane, pout);
       }
-      if (MODE == SEL_SCORES) continue;  // the select pass takes it from here
       __syncwarp();
       // Phase 3: selection threshold as (level v_f, ties c_f).
       // per-head top-k floor (second pass): k_min raised to the head's floor

@@ -1,0 +1,256 @@
+// Pooled block scores on the tensor cores (Rectified SpaAttn: block
+// importance from pooled queries and keys). Per head, the scores are one
+// dense fp32 contraction over d, S = scale * qbar kbar^T [Nt x Nt]; here it
+// runs as tcgen05 kind::tf32 MMAs on split operands. Each pooled value x
+// (an fp32 mean) is stored as two tf32 parts, hi = tf32(x) and
+// lo = tf32(x - hi), so x = hi + lo + r with |r| <= 2^-22 |x|, and each term
+// q.k is taken as lo_q hi_k + hi_q lo_k + hi_q hi_k (the dropped lo_q lo_k is
+// below 2^-22 |q k|). The small products go into the accumulator first.
+// pool_kernel writes the parts.
+//
+// One CTA per (128 key tiles, range of query tiles, b*heads + h); 192 threads:
+//   warps 0-3  load the CTA's key block (hi and lo parts, one key tile per
+//              thread) into TMEM, where it is the A operand of every MMA;
+//              then the epilogue: TMEM lane = key tile, column = query tile,
+//              so each column is one 128-byte coalesced store into a row of S
+//   warp 4     TMA producer: blocks of 64 query tiles (hi and lo) through a
+//              ring in shared memory (the B operand)
+//   warp 5     TMEM allocation and the MMA issue (one thread); accumulators
+//              double-buffered in TMEM so the epilogue of block j overlaps
+//              the MMAs of block j + 1
+// With the key block in TMEM an MMA reads only its 64 query rows from shared
+// memory, so it runs at the tensor-core rate instead of the shared-memory
+// rate. Query operands are K-major with the 128-byte swizzle: a chunk of 32
+// fp32 along d per 128-byte row, 8-row groups 1024 B apart. Every wait is
+// bounded; on a timeout the kernel records DEV_ERR_TIMEOUT, waits (bounded)
+// for its own copies in flight, releases TMEM and returns.
+#pragma once
+#include "sta_tc.cuh"
+
+namespace sta {
+namespace score {
+
+constexpr int M = 128;           // key tiles per CTA (TMEM lanes)
+constexpr int N = 64;            // query tiles per MMA block (TMEM columns)
+constexpr int NUM_THREADS = 192;
+constexpr int WARP_TMA = 4, WARP_MMA = 5;
+constexpr long long WAIT_LIMIT = 2000000000LL;  // SM cycles (~1 s)
+constexpr long long DRAIN_LIMIT = 200000000LL;  // after an abort
+
+template <int D>
+struct Cfg {
+  static constexpr int CH = D / 32;            // 128-byte chunks along d
+  static constexpr int B_CHUNK = N * 128;      // bytes of one chunk of a query block
+  static constexpr int B_PART = CH * B_CHUNK;  // one split part of a query block
+  static constexpr int STAGES = D == 128 ? 3 : 6;
+  static constexpr int STAGE_BYTES = 2 * B_PART;  // hi part, then lo part
+  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  // a_full, full[STAGES], empty[STAGES], t_full[2], t_empty[2], mma_done
+  static constexpr int NBAR = 1 + 2 * STAGES + 4 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem address, abort flag
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM = BYTES + 1024;    // slack for the 1024-byte alignment
+  // TMEM columns: two accumulators of N, then the key block's hi and lo
+  // parts (one fp32 / tf32 element per column, lane = key tile)
+  static constexpr uint32_t COL_HI = 2 * N, COL_LO = 2 * N + D;
+  static constexpr uint32_t TMEM_COLS = (2 * N + 2 * D) <= 256 ? 256 : 512;
+  static_assert(D % 32 == 0, "d must be a multiple of 32");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(2 * N + 2 * D <= 512, "tensor memory");
+};
+
+// instruction descriptor, kind::tf32: tf32 x tf32 -> fp32, B K-major
+// (D format bit 4, A / B format 2 = TF32 at bits 7-9 / 10-12, N >> 3 at
+// bit 17, M >> 4 at bit 24)
+constexpr uint32_t IDESC = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
+                           ((uint32_t)(M >> 4) << 24);
+
+// A from tensor memory (lane = row, one tf32 per column), B from shared memory.
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(IDESC), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint64_t *bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(tc::smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// khi / klo: the split parts of the pooled keys [b*heads][Nt][D] fp32, read
+// one row per thread; tm_qhi / tm_qlo: those of the pooled queries as 3D
+// tensors (d, Nt, b*heads), boxes of 32 x N x 1 (zero-filled past Nt).
+// S: [b*heads][Nt][Nt] fp32, row = query tile. The query tiles of this CTA
+// are [blockIdx.y * q_per_part, ... + q_per_part) clipped to Nt, q_per_part a
+// multiple of N.
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+score_tc_kernel(const float *__restrict__ khi, const float *__restrict__ klo,
+                const __grid_constant__ CUtensorMap tm_qhi, const __grid_constant__ CUtensorMap tm_qlo,
+                float *__restrict__ S, int nt, float scale, int q_per_part) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = tc::smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int k0 = blockIdx.x * M;
+  const int q_begin = blockIdx.y * q_per_part;
+  const int q_end = min(nt, q_begin + q_per_part);
+  const int bh = blockIdx.z;
+  const int nblk = q_end > q_begin ? (q_end - q_begin + N - 1) / N : 0;
+
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+  uint64_t *a_full = bars;
+  uint64_t *full = bars + 1;
+  uint64_t *empty = full + C::STAGES;
+  uint64_t *t_full = empty + C::STAGES;
+  uint64_t *t_empty = t_full + 2;
+  uint64_t *mma_done = t_empty + 2;
+  uint32_t *misc = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+  volatile uint32_t *abort_flag = misc + 1;
+
+  if (tid == 0) {
+    tc::mbar_init(a_full, 4);  // one arrival per loading warp
+    for (int s = 0; s < C::STAGES; ++s) {
+      tc::mbar_init(full + s, 1);
+      tc::mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(t_full + b, 1);
+      tc::mbar_init(t_empty + b, 4);  // one arrival per epilogue warp
+    }
+    tc::mbar_init(mma_done, 1);
+    misc[1] = 0u;
+    tc::fence_barrier_init();
+  }
+  if (warp == WARP_MMA) {
+    tc::tmem_alloc(misc, C::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == WARP_TMA) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0 && nblk > 0) {
+      int issued = 0;
+      for (int j = 0; j < nblk; ++j) {
+        const int s = j % C::STAGES, u = j / C::STAGES;
+        if (u > 0 && !tc::mbar_wait(empty + s, (u - 1) & 1, abort_flag, WAIT_LIMIT)) break;
+        const uint32_t dst = sbase + s * C::STAGE_BYTES;
+        const int q0 = q_begin + j * N;
+        tc::mbar_expect_tx(full + s, C::STAGE_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::CH; ++c) {
+          tma_load_3d(dst + c * C::B_CHUNK, &tm_qhi, full + s, 32 * c, q0, bh);
+          tma_load_3d(dst + C::B_PART + c * C::B_CHUNK, &tm_qlo, full + s, 32 * c, q0, bh);
+        }
+        issued = j + 1;
+      }
+      // copies still in flight must land before the CTA can exit
+      if (*abort_flag) {
+        for (int j = (issued > C::STAGES ? issued - C::STAGES : 0); j < issued; ++j)
+          tc::mbar_wait(full + j % C::STAGES, (j / C::STAGES) & 1, nullptr, DRAIN_LIMIT);
+      }
+    }
+    __syncwarp();
+  } else if (warp == WARP_MMA) {
+    // ---------------------------------------------------------- MMA issue
+    if (lane == 0 && nblk > 0) {
+      bool ok = tc::mbar_wait(a_full, 0, abort_flag, WAIT_LIMIT);
+      tc::fence_after();
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int s = j % C::STAGES, buf = j & 1;
+        if (!tc::mbar_wait(full + s, (j / C::STAGES) & 1, abort_flag, WAIT_LIMIT)) break;
+        if (j >= 2 && !tc::mbar_wait(t_empty + buf, ((j >> 1) - 1) & 1, abort_flag, WAIT_LIMIT)) break;
+        tc::fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(buf * N);
+        const uint32_t b_hi = sbase + s * C::STAGE_BYTES, b_lo = b_hi + C::B_PART;
+        // lo_k*hi_q and hi_k*lo_q first (small), then hi_k*hi_q; K = 8 tf32
+        // per MMA: 8 TMEM columns of A, 32 bytes of a swizzled B row
+#pragma unroll
+        for (int part = 0; part < 3; ++part) {
+          const uint32_t a = tmem + (part == 0 ? C::COL_LO : C::COL_HI);
+          const uint32_t b = part == 1 ? b_lo : b_hi;
+#pragma unroll
+          for (int kk = 0; kk < 4 * C::CH; ++kk) {
+            const uint32_t koff = (uint32_t)((kk & 3) * 32);
+            mma_tf32_ts(d_tmem, a + (uint32_t)(kk * 8), tc::desc_k_sw128(b + (kk >> 2) * C::B_CHUNK + koff),
+                        (part > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc::mma_commit(empty + s);
+        tc::mma_commit(t_full + buf);
+      }
+      // every issued MMA retires before TMEM is released
+      tc::mma_commit(mma_done);
+      tc::mbar_wait(mma_done, 0, nullptr, *abort_flag ? DRAIN_LIMIT : WAIT_LIMIT);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------- key block into TMEM, epilogue
+    const int k = k0 + tid;  // this thread's key tile (TMEM lane tid)
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    if (nblk > 0) {
+      const bool real = k < nt;
+      const long long roff = ((long long)bh * nt + (real ? k : 0)) * D;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const float4 *src = reinterpret_cast<const float4 *>((part == 0 ? khi : klo) + roff);
+#pragma unroll
+        for (int c = 0; c < C::CH; ++c) {
+          uint32_t r[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 v = real ? __ldg(src + c * 8 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            r[4 * i] = __float_as_uint(v.x);
+            r[4 * i + 1] = __float_as_uint(v.y);
+            r[4 * i + 2] = __float_as_uint(v.z);
+            r[4 * i + 3] = __float_as_uint(v.w);
+          }
+          tc::tmem_st32(tmem + lane_base + (part == 0 ? C::COL_HI : C::COL_LO) + (uint32_t)(32 * c), r);
+        }
+      }
+      tc::tmem_wait_st();
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(a_full);
+    }
+    float *col = S + (long long)bh * nt * nt + k;
+    for (int j = 0; j < nblk; ++j) {
+      const int buf = j & 1;
+      if (!tc::mbar_wait(t_full + buf, (j >> 1) & 1, abort_flag, WAIT_LIMIT)) break;
+      tc::fence_after();
+      uint32_t v[N];
+      tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * N), v);
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(t_empty + buf);
+      const int q0 = q_begin + j * N;
+      if (k < nt) {
+#pragma unroll
+        for (int c = 0; c < N; ++c) {
+          const int q = q0 + c;
+          if (q < q_end) col[(long long)q * nt] = __uint_as_float(v[c]) * scale;
+        }
+      }
+    }
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc::fence_after();
+    tc::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace score
+}  // namespace sta

@@ -107,12 +107,15 @@ int64_t sta_tiled_len(sta_grid g);
 sta_status sta_reorder(const void *src, void *dst, int32_t B, int32_t heads, int32_t d,
                        sta_grid g, int32_t inverse, sta_stream_t stream);
 
-/* Bytes of device workspace of sta_build_mask for these sizes: the full size
- * holds a row buffer of the block probabilities [B*heads*Nt, Nt] fp32, so the
- * scores and the selection run as two passes (the selection pass keeps four
- * CTAs per SM); any workspace of at least the _min size is accepted and runs
- * the fused pass instead (same results, bit for bit). When block_probs is
- * given, the rows go there and the minimum is enough for the two passes. */
+/* Bytes of device workspace of sta_build_mask for these sizes. The full size
+ * holds the pooled Q and K split into two tf32 parts each and a row buffer
+ * [B*heads*Nt, Nt] fp32: the pooled scores then run on the tensor cores
+ * (three tf32 products per term, within 2^-22 (3 d/8 + 3) of the sum of
+ * |q||k| per score) and a separate select pass does the softmax and the
+ * selection (four CTAs per SM). Any workspace of at least the _min size is
+ * accepted and runs one fused pass whose scores are fp32 FMA chains. The two
+ * layouts agree with the exact scores within their bounds, so a tile whose
+ * P sits at the selection threshold may be kept by one and not the other. */
 size_t sta_build_mask_workspace(int32_t B, int32_t heads, int32_t d, sta_grid g);
 size_t sta_build_mask_workspace_min(int32_t B, int32_t heads, int32_t d, sta_grid g);
 
@@ -131,7 +134,8 @@ size_t sta_build_mask_workspace_min(int32_t B, int32_t heads, int32_t d, sta_gri
  *   workspace        : device, >= sta_build_mask_workspace_min() bytes (the
  *                      full sta_build_mask_workspace() for the fastest
  *                      layout), 256-aligned
- * The call is deterministic: the same inputs give bit-identical outputs. */
+ * The call is deterministic: the same inputs and workspace size give
+ * bit-identical outputs. */
 sta_status sta_build_mask(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads,
                           int32_t d, sta_grid g, const sta_mask_params *p, int32_t *row_ptr,
                           int32_t *col_idx, int64_t *nnz_dev, uint8_t *block_mask,
@@ -186,8 +190,10 @@ sta_status sta_attn_fwd_raster(const void *q, const void *k, const void *v, void
  * device memory is laid out up front by a host framework or a fixed arena
  * (embedded inference runtimes, plug-ins of engines that own every device
  * allocation), so they can neither call cudaMalloc nor lend a workspace.
- * Same arguments, results and determinism as sta_build_mask, minus the
- * workspace: the workspace is a file-scope static device array of
+ * Same arguments as sta_build_mask minus the workspace, and the results of
+ * sta_build_mask with a workspace of STA_NOALLOC_SCRATCH_BYTES (the
+ * tensor-core layout when sta_build_mask_workspace() fits in it, else the
+ * fused one): the workspace is a file-scope static device array of
  * STA_NOALLOC_SCRATCH_BYTES (32 MiB), present on every GPU that loads the
  * library until the process exits. The caller still passes inputs and outputs.
  *   - Sizes whose minimum workspace (sta_build_mask_workspace_min) exceeds

@@ -40,12 +40,25 @@ def attn(qt, kt, vt, row_ptr, col_idx, B, Hh, d, g, sm_scale=0.0):
     return o, lse
 
 
-def prob_bound(qbar, kbar, scale, p_ref):
-    """Per-element bound on |P_gpu - P_oracle| from the GPU arithmetic:
-    fp32 pooled means (one rounding each of an exact sum), a D-term fp32 FMA
-    chain for the score, fp32 exp / sum / divide. Returns an array like p_ref."""
+def prob_bound(qbar, kbar, scale, p_ref, fused=False):
+    """Per-element bound on |P_gpu - P_oracle| from the GPU arithmetic.
+
+    Both layouts round the pooled means once to fp32 (an exact fp64 sum), and
+    run the softmax in fp32 (exp, fixed-order sum, divide). The score term
+    differs:
+    - fused (minimum workspace): a D-term sequential fp32 FMA chain,
+      error <= gamma_D |q||k|;
+    - tensor cores (full workspace): each mean x split as hi = tf32(x),
+      lo = tf32(x - hi), so |x - hi - lo| <= 2^-22 |x|; the products
+      lo*hi + hi*lo + hi*hi drop lo*lo, in all <= 3 * 2^-22 |q k|; the
+      fp32 accumulator passes through 3*D/8 MMAs (K = 8 each), each taken to
+      add at most 2 ulp (2^-22) of the sum of the magnitudes so far.
+    Returns an array like p_ref."""
     d = qbar.shape[-1]
-    gam = d * U32 / (1 - d * U32)
+    if fused:
+        gam = d * U32 / (1 - d * U32)
+    else:
+        gam = (3 * d / 8 + 3) * 2.0 ** -22
     cond = np.einsum("...qd,...kd->...qk", np.abs(qbar), np.abs(kbar)) * scale
     ds = (gam + 2.0 * U32) * cond  # score error bound per element
     E = ds.max(axis=-1, keepdims=True)

@@ -54,7 +54,9 @@ def test_workspace_size(sta):
     R = 40 * 1260
     ws_min = sta.sta_build_mask_workspace_min(1, 40, 128, g)
     assert ws_min >= 2 * R * 128 * 4 + R * 40 * 4 + R * 4
-    assert ws >= ws_min + R * 1260 * 4  # plus the P row buffer of the two-pass layout
+    # plus the low tf32 parts of the pooled Q and K and the row buffer of the
+    # tensor-core layout
+    assert ws >= ws_min + 2 * R * 128 * 4 + R * 1260 * 4
     assert ws % 256 == 0 and ws_min % 256 == 0
     assert sta.sta_build_mask_workspace(1, 40, 96, g) == 0
 
@@ -88,3 +90,9 @@ def test_status_strings(sta):
 def test_selftest_limit_is_checked_on_the_host(sta):
     assert sta._lib.sta_selftest_wait_timeout(10, None) == sta.STA_ERR_INVALID_ARG
     assert sta._lib.sta_selftest_wait_timeout(3_000_000_000, None) == sta.STA_ERR_INVALID_ARG
+
+
+def test_binding_mirrors_the_noalloc_array_size(sta):
+    m = re.search(r"#define\s+STA_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", open(HEADER).read())
+    assert m, "STA_NOALLOC_SCRATCH_BYTES not found in the header"
+    assert sta.STA_NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))

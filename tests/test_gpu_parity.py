@@ -692,34 +692,60 @@ def test_search_windows_rejects_bad_groups(sta):
 
 
 @pytest.mark.parametrize("floor", [False, True])
-@pytest.mark.parametrize("probs", [False, True])
-def test_build_mask_fused_and_two_pass_layouts_agree(sta, gp, floor, probs):
-    """The minimum workspace runs the fused score/select pass, the full one
-    the scores pass plus a separate select pass (and block_probs, when given,
-    holds the rows): the CSR, the byte mask and P agree bit for bit."""
-    T, H, W, Hh, B, d = 5, 24, 37, 3, 2, 128
+@pytest.mark.parametrize("d", [64, 128])
+def test_build_mask_fused_and_tensor_core_layouts(sta, gp, floor, d):
+    """The minimum workspace runs the fused pass (scores as fp32 FMA chains),
+    the full one the tensor-core scores and a separate select pass. For each
+    layout: P within that layout's own error bound of the oracle's P; the CSR
+    and the byte mask equal to the oracle's selection (with the per-head
+    floor when asked) on that layout's own P, OR the windows; without the
+    floor, the selection differs from the oracle's own only at near-threshold
+    tiles. The full layout without block_probs (rows in the workspace) gives
+    the same CSR as with them."""
+    T, H, W, Hh, B = 5, 24, 37, 3, 2
     g = sta.grid(T, H, W)
     q, k, _ = _structured(T, H, W, Hh, d, seed=23, B=B)
     qt, kt = (gp.reorder(x, B, Hh, d, g) for x in (q, k))
     nh, nw, nt, _ = O.tile_grid(T, H, W)
-    win_t = torch.from_numpy(np.tile(np.array([[[1, 1, 0, nw - 1], [0, 0, -1, -1]]], dtype=np.int32),
-                                     (Hh, 1, 1))).cuda()
-    params = sta.mask_params(0.8, 3, True, 0.0, (0, 2), win_t, head_floor=floor)
-    outs = []
-    for ws_bytes in (sta.sta_build_mask_workspace_min(B, Hh, d, g), sta.sta_build_mask_workspace(B, Hh, d, g)):
-        bufs = sta.MaskBuffers(B, Hh, d, g, "cuda", True, probs)
+    win = np.tile(np.array([[[1, 1, 0, nw - 1], [0, 0, -1, -1]]], dtype=np.int32), (Hh, 1, 1))
+    win_t = torch.from_numpy(win).cuda()
+    top_p, k_min, glo = 0.8, 3, (0, 2)
+    params = sta.mask_params(top_p, k_min, True, 0.0, glo, win_t, head_floor=floor)
+    scale = 1.0 / math.sqrt(d)
+    qb, kb = O.pool(gp.to_np64(qt), T, H, W), O.pool(gp.to_np64(kt), T, H, W)
+    _, p_ref = O.block_scores(qb, kb, scale)
+    wmask = O.window_mask(win, glo, T, H, W)[None]
+    sizes = O.tile_sizes(T, H, W)
+    own = O.select(p_ref, top_p, k_min)
+
+    def run(ws_bytes, with_probs):
+        bufs = sta.MaskBuffers(B, Hh, d, g, "cuda", True, with_probs)
         ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
         sta.sta_build_mask(qt, kt, B, Hh, d, g, params, bufs.row_ptr, bufs.col_idx, bufs.nnz, bufs.block_mask,
                            bufs.block_probs, ws, ws_bytes)
         torch.cuda.synchronize()
-        outs.append(bufs)
-    a, b = outs
-    n = int(a.nnz.item())
-    assert n == int(b.nnz.item()) and n > 0
-    assert torch.equal(a.row_ptr, b.row_ptr) and torch.equal(a.col_idx[:n], b.col_idx[:n])
-    assert torch.equal(a.block_mask, b.block_mask)
-    if probs:
-        assert torch.equal(a.block_probs.view(torch.int32), b.block_probs.view(torch.int32))
+        assert sta.sta_get_device_error() == sta.STA_OK
+        return bufs
+
+    for fused in (True, False):
+        ws_bytes = (sta.sta_build_mask_workspace_min if fused else sta.sta_build_mask_workspace)(B, Hh, d, g)
+        bufs = run(ws_bytes, True)
+        probs = bufs.block_probs.cpu().numpy()
+        bound = gp.prob_bound(qb, kb, scale, p_ref, fused=fused)
+        assert np.all(np.abs(probs.astype(np.float64) - p_ref) <= bound)
+        sel = _floor_mask(probs, top_p, k_min, sizes) if floor else O.select(probs, top_p, k_min)
+        mask = sel | wmask
+        assert np.array_equal(bufs.block_mask.cpu().numpy().astype(bool), mask)
+        rp, ci, nnz = gp.csr_np(bufs)
+        rp_o, ci_o = O.mask_to_csr(mask)
+        assert np.array_equal(rp, rp_o) and np.array_equal(ci, ci_o)
+        if not floor:
+            _assert_near_threshold(own, sel, p_ref, bound, top_p)
+        if not fused:
+            other = run(ws_bytes, False)
+            assert torch.equal(other.row_ptr, bufs.row_ptr)
+            assert torch.equal(other.col_idx[:nnz], bufs.col_idx[:nnz])
+            assert torch.equal(other.block_mask, bufs.block_mask)
 
 
 # ------------------------------------------ raster-layout path (no reorder)

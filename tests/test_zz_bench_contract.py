@@ -37,5 +37,11 @@ def test_bench_json_line():
     assert c["kind"] == "oracle" and c["value"] > 0 and c["cores"] >= 1
     e = d["e2e"]
     assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0
-    assert d["gpu_launches"] == 3 * 5
+    # pool, tensor-core scores, select, scan, fill, attention: six kernels of
+    # this library per step, as CUPTI recorded them
+    assert d["gpu_launches"] == 3 * 6
+    if d["gpu_launches_source"].startswith("cupti"):
+        ks = d["step_kernels"]
+        assert len(ks) == 6 and all(k.startswith("sta::") for k in ks), ks
+        assert sum("attn_fwd_kernel" in k for k in ks) == 1 and sum("score_tc_kernel" in k for k in ks) == 1
     assert d["clocks"]["sm_mhz"] is not None and isinstance(d["clocks"]["reasons"], list)
