@@ -148,8 +148,9 @@ bool make_pooled_map(CUtensorMap *map, const float *base, long long bh, int nt, 
 template <int D>
 sta_status launch_scores_tc(const float *qhi, const float *qlo, const float *khi, const float *klo, float *S,
                             long long bh, const Geo &g, float scale, cudaStream_t s) {
-  CUtensorMap m_qhi, m_qlo;
-  if (!make_pooled_map(&m_qhi, qhi, bh, g.Nt, D, score::N) || !make_pooled_map(&m_qlo, qlo, bh, g.Nt, D, score::N))
+  CUtensorMap m_khi, m_klo, m_qhi, m_qlo;
+  if (!make_pooled_map(&m_khi, khi, bh, g.Nt, D, score::M) || !make_pooled_map(&m_klo, klo, bh, g.Nt, D, score::M) ||
+      !make_pooled_map(&m_qhi, qhi, bh, g.Nt, D, score::N) || !make_pooled_map(&m_qlo, qlo, bh, g.Nt, D, score::N))
     return STA_ERR_CUDA;
   auto kern = score::score_tc_kernel<D>;
   const int smem = score::Cfg<D>::SMEM;
@@ -164,7 +165,7 @@ sta_status launch_scores_tc(const float *qhi, const float *qlo, const float *khi
   const int per_part = (qblocks + parts - 1) / parts;
   parts = (qblocks + per_part - 1) / per_part;  // no empty range
   dim3 grid((unsigned)kblocks, (unsigned)parts, (unsigned)bh);
-  kern<<<grid, score::NUM_THREADS, smem, s>>>(khi, klo, m_qhi, m_qlo, S, g.Nt, scale, per_part * score::N);
+  kern<<<grid, score::NUM_THREADS, smem, s>>>(m_khi, m_klo, m_qhi, m_qlo, S, g.Nt, scale, per_part * score::N);
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }

@@ -9,21 +9,23 @@
 // pool_kernel writes the parts.
 //
 // One CTA per (128 key tiles, range of query tiles, b*heads + h); 192 threads:
-//   warps 0-3  load the CTA's key block (hi and lo parts, one key tile per
-//              thread) into TMEM, where it is the A operand of every MMA;
-//              then the epilogue: TMEM lane = key tile, column = query tile,
-//              so each column is one 128-byte coalesced store into a row of S
-//   warp 4     TMA producer: blocks of 64 query tiles (hi and lo) through a
-//              ring in shared memory (the B operand)
+//   warp 4     TMA producer: first the CTA's key block (hi and lo parts) into
+//              the first ring stages, then, once it has moved to TMEM, blocks
+//              of 64 query tiles (hi and lo) through the ring (the B operand)
+//   warps 0-3  move the key block from shared memory to TMEM (one key tile
+//              per thread = TMEM lane), where it is the A operand of every
+//              MMA; then the epilogue of each block: TMEM -> registers ->
+//              a transposed tile in shared memory -> rows of S written as
+//              512-byte runs of 16-byte stores
 //   warp 5     TMEM allocation and the MMA issue (one thread); accumulators
 //              double-buffered in TMEM so the epilogue of block j overlaps
 //              the MMAs of block j + 1
 // With the key block in TMEM an MMA reads only its 64 query rows from shared
 // memory, so it runs at the tensor-core rate instead of the shared-memory
-// rate. Query operands are K-major with the 128-byte swizzle: a chunk of 32
-// fp32 along d per 128-byte row, 8-row groups 1024 B apart. Every wait is
-// bounded; on a timeout the kernel records DEV_ERR_TIMEOUT, waits (bounded)
-// for its own copies in flight, releases TMEM and returns.
+// rate. Operands in shared memory are K-major with the 128-byte swizzle: a
+// chunk of 32 fp32 along d per 128-byte row, 8-row groups 1024 B apart.
+// Every wait is bounded; on a timeout the kernel records DEV_ERR_TIMEOUT,
+// waits (bounded) for its own copies in flight, releases TMEM and returns.
 #pragma once
 #include "sta_tc.cuh"
 
@@ -40,13 +42,16 @@ constexpr long long DRAIN_LIMIT = 200000000LL;  // after an abort
 template <int D>
 struct Cfg {
   static constexpr int CH = D / 32;            // 128-byte chunks along d
+  static constexpr int A_CHUNK = M * 128;      // bytes of one chunk of the key block
+  static constexpr int A_PART = CH * A_CHUNK;  // one split part of the key block
   static constexpr int B_CHUNK = N * 128;      // bytes of one chunk of a query block
   static constexpr int B_PART = CH * B_CHUNK;  // one split part of a query block
   static constexpr int STAGES = D == 128 ? 3 : 6;
   static constexpr int STAGE_BYTES = 2 * B_PART;  // hi part, then lo part
-  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
-  // a_full, full[STAGES], empty[STAGES], t_full[2], t_empty[2], mma_done
-  static constexpr int NBAR = 1 + 2 * STAGES + 4 + 1;
+  static constexpr int OFF_T = STAGES * STAGE_BYTES;  // [N][M] fp32 epilogue tile
+  static constexpr int OFF_BAR = OFF_T + N * M * 4;
+  // a_tma, a_moved, a_full, full[STAGES], empty[STAGES], t_full[2], t_empty[2], mma_done
+  static constexpr int NBAR = 3 + 2 * STAGES + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem address, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM = BYTES + 1024;    // slack for the 1024-byte alignment
@@ -55,6 +60,7 @@ struct Cfg {
   static constexpr uint32_t COL_HI = 2 * N, COL_LO = 2 * N + D;
   static constexpr uint32_t TMEM_COLS = (2 * N + 2 * D) <= 256 ? 256 : 512;
   static_assert(D % 32 == 0, "d must be a multiple of 32");
+  static_assert(2 * A_PART <= STAGES * STAGE_BYTES, "key block staging");
   static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(2 * N + 2 * D <= 512, "tensor memory");
 };
@@ -74,6 +80,19 @@ __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// AND of `v` over the 128 threads of the epilogue warps (named barrier 1),
+// so that they all take the same branch around the barriers that follow.
+__device__ __forceinline__ bool all_epilogue(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0u;
+}
+
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint64_t *bar, int x, int y,
                                             int z) {
   asm volatile(
@@ -83,15 +102,15 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
-// khi / klo: the split parts of the pooled keys [b*heads][Nt][D] fp32, read
-// one row per thread; tm_qhi / tm_qlo: those of the pooled queries as 3D
-// tensors (d, Nt, b*heads), boxes of 32 x N x 1 (zero-filled past Nt).
-// S: [b*heads][Nt][Nt] fp32, row = query tile. The query tiles of this CTA
-// are [blockIdx.y * q_per_part, ... + q_per_part) clipped to Nt, q_per_part a
+// tm_khi / tm_klo / tm_qhi / tm_qlo: the split parts of the pooled keys and
+// queries as 3D tensors (d, Nt, b*heads) fp32, boxes of 32 x M x 1 (keys) and
+// 32 x N x 1 (queries), zero-filled past Nt. S: [b*heads][Nt][Nt] fp32,
+// row = query tile. The query tiles of this CTA are
+// [blockIdx.y * q_per_part, ... + q_per_part) clipped to Nt, q_per_part a
 // multiple of N.
 template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-score_tc_kernel(const float *__restrict__ khi, const float *__restrict__ klo,
+score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constant__ CUtensorMap tm_klo,
                 const __grid_constant__ CUtensorMap tm_qhi, const __grid_constant__ CUtensorMap tm_qlo,
                 float *__restrict__ S, int nt, float scale, int q_per_part) {
   using C = Cfg<D>;
@@ -106,8 +125,10 @@ score_tc_kernel(const float *__restrict__ khi, const float *__restrict__ klo,
   const int nblk = q_end > q_begin ? (q_end - q_begin + N - 1) / N : 0;
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-  uint64_t *a_full = bars;
-  uint64_t *full = bars + 1;
+  uint64_t *a_tma = bars;         // key block landed in shared memory
+  uint64_t *a_moved = bars + 1;   // key block read out of shared memory
+  uint64_t *a_full = bars + 2;    // key block in TMEM
+  uint64_t *full = bars + 3;
   uint64_t *empty = full + C::STAGES;
   uint64_t *t_full = empty + C::STAGES;
   uint64_t *t_empty = t_full + 2;
@@ -116,14 +137,16 @@ score_tc_kernel(const float *__restrict__ khi, const float *__restrict__ klo,
   volatile uint32_t *abort_flag = misc + 1;
 
   if (tid == 0) {
-    tc::mbar_init(a_full, 4);  // one arrival per loading warp
+    tc::mbar_init(a_tma, 1);
+    tc::mbar_init(a_moved, 4);  // one arrival per epilogue warp
+    tc::mbar_init(a_full, 4);
     for (int s = 0; s < C::STAGES; ++s) {
       tc::mbar_init(full + s, 1);
       tc::mbar_init(empty + s, 1);
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(t_full + b, 1);
-      tc::mbar_init(t_empty + b, 4);  // one arrival per epilogue warp
+      tc::mbar_init(t_empty + b, 4);
     }
     tc::mbar_init(mma_done, 1);
     misc[1] = 0u;
@@ -141,8 +164,16 @@ score_tc_kernel(const float *__restrict__ khi, const float *__restrict__ klo,
   if (warp == WARP_TMA) {
     // ---------------------------------------------------------- producer
     if (lane == 0 && nblk > 0) {
+      tc::mbar_expect_tx(a_tma, 2 * C::A_PART);
+#pragma unroll
+      for (int c = 0; c < C::CH; ++c) {
+        tma_load_3d(sbase + c * C::A_CHUNK, &tm_khi, a_tma, 32 * c, k0, bh);
+        tma_load_3d(sbase + C::A_PART + c * C::A_CHUNK, &tm_klo, a_tma, 32 * c, k0, bh);
+      }
       int issued = 0;
-      for (int j = 0; j < nblk; ++j) {
+      // the ring reuses the staging area once the key block is in TMEM
+      bool ok = tc::mbar_wait(a_moved, 0, abort_flag, WAIT_LIMIT);
+      for (int j = 0; ok && j < nblk; ++j) {
         const int s = j % C::STAGES, u = j / C::STAGES;
         if (u > 0 && !tc::mbar_wait(empty + s, (u - 1) & 1, abort_flag, WAIT_LIMIT)) break;
         const uint32_t dst = sbase + s * C::STAGE_BYTES;
@@ -157,6 +188,7 @@ score_tc_kernel(const float *__restrict__ khi, const float *__restrict__ klo,
       }
       // copies still in flight must land before the CTA can exit
       if (*abort_flag) {
+        tc::mbar_wait(a_tma, 0, nullptr, DRAIN_LIMIT);
         for (int j = (issued > C::STAGES ? issued - C::STAGES : 0); j < issued; ++j)
           tc::mbar_wait(full + j % C::STAGES, (j / C::STAGES) & 1, nullptr, DRAIN_LIMIT);
       }
@@ -197,51 +229,72 @@ score_tc_kernel(const float *__restrict__ khi, const float *__restrict__ klo,
     __syncwarp();
   } else {
     // ------------------------------------------- key block into TMEM, epilogue
-    const int k = k0 + tid;  // this thread's key tile (TMEM lane tid)
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    if (nblk > 0) {
-      const bool real = k < nt;
-      const long long roff = ((long long)bh * nt + (real ? k : 0)) * D;
+    bool ok = nblk > 0;
+    if (ok) {
+      // row tid of each swizzled chunk: 16-byte granule g sits at g ^ (tid % 8)
+      ok = tc::mbar_wait(a_tma, 0, abort_flag, WAIT_LIMIT);
+      if (ok) {
+#pragma unroll 1
+        for (int part = 0; part < 2; ++part) {
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const float4 *src = reinterpret_cast<const float4 *>((part == 0 ? khi : klo) + roff);
+          for (int c = 0; c < C::CH; ++c) {
+            const uint8_t *row = smem + part * C::A_PART + c * C::A_CHUNK + tid * 128;
+            uint32_t r[32];
 #pragma unroll
-        for (int c = 0; c < C::CH; ++c) {
-          uint32_t r[32];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 v = real ? __ldg(src + c * 8 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            r[4 * i] = __float_as_uint(v.x);
-            r[4 * i + 1] = __float_as_uint(v.y);
-            r[4 * i + 2] = __float_as_uint(v.z);
-            r[4 * i + 3] = __float_as_uint(v.w);
+            for (int g = 0; g < 8; ++g) {
+              const uint4 v = *reinterpret_cast<const uint4 *>(row + ((g ^ (tid & 7)) << 4));
+              r[4 * g] = v.x;
+              r[4 * g + 1] = v.y;
+              r[4 * g + 2] = v.z;
+              r[4 * g + 3] = v.w;
+            }
+            tc::tmem_st32(tmem + lane_base + (part == 0 ? C::COL_HI : C::COL_LO) + (uint32_t)(32 * c), r);
           }
-          tc::tmem_st32(tmem + lane_base + (part == 0 ? C::COL_HI : C::COL_LO) + (uint32_t)(32 * c), r);
         }
+        tc::tmem_wait_st();
       }
-      tc::tmem_wait_st();
       tc::fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(a_full);
+      if (lane == 0) {
+        tc::mbar_arrive(a_moved);
+        tc::mbar_arrive(a_full);
+      }
     }
-    float *col = S + (long long)bh * nt * nt + k;
-    for (int j = 0; j < nblk; ++j) {
+    float *T = reinterpret_cast<float *>(smem + C::OFF_T);
+    const bool vec = (nt & 3) == 0;  // every row segment of S is 16-byte aligned
+    // the four warps leave the loop together (they share barrier 1)
+    ok = all_epilogue(ok);
+    for (int j = 0; ok && j < nblk; ++j) {
       const int buf = j & 1;
-      if (!tc::mbar_wait(t_full + buf, (j >> 1) & 1, abort_flag, WAIT_LIMIT)) break;
+      if (!all_epilogue(tc::mbar_wait(t_full + buf, (j >> 1) & 1, abort_flag, WAIT_LIMIT))) break;
       tc::fence_after();
       uint32_t v[N];
       tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * N), v);
       tc::fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(t_empty + buf);
-      const int q0 = q_begin + j * N;
-      if (k < nt) {
+      // transposed tile T[query][key] (consecutive threads, consecutive keys)
 #pragma unroll
-        for (int c = 0; c < N; ++c) {
-          const int q = q0 + c;
-          if (q < q_end) col[(long long)q * nt] = __uint_as_float(v[c]) * scale;
+      for (int c = 0; c < N; ++c) T[c * M + tid] = __uint_as_float(v[c]) * scale;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // each warp writes query rows warp, warp + 4, ...: 128 keys per row,
+      // four per lane
+      const int q0 = q_begin + j * N;
+      const int kk = k0 + 4 * lane;
+      for (int c = warp; c < N && q0 + c < q_end; c += 4) {
+        const float4 val = reinterpret_cast<const float4 *>(T + c * M)[lane];
+        float *dst = S + ((long long)bh * nt + q0 + c) * nt + kk;
+        if (vec && kk + 3 < nt) {
+          *reinterpret_cast<float4 *>(dst) = val;
+        } else {
+          if (kk < nt) dst[0] = val.x;
+          if (kk + 1 < nt) dst[1] = val.y;
+          if (kk + 2 < nt) dst[2] = val.z;
+          if (kk + 3 < nt) dst[3] = val.w;
         }
       }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
     }
   }
   tc::fence_before();
