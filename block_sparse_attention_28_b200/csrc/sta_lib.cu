@@ -8,6 +8,7 @@
 #include "sta_attn.cuh"
 #include "sta_common.cuh"
 #include "sta_mask.cuh"
+#include "sta_pool.cuh"
 #include "sta_reorder.cuh"
 #include "sta_score.cuh"
 #include "sta_search.cuh"
@@ -127,6 +128,30 @@ bool make_raster_map(CUtensorMap *map, const void *base, const Geo &g, int B, in
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Raster [B, L, heads, d] bf16 as the 5D tensor (d, heads, W, H, B*T) with a
+// box of a whole token tile for `hb` heads: d x hb x 8 x 8 x 1 (zero-filled
+// beyond the grid edge and the last head), no swizzle.
+bool make_raster_pool_map(CUtensorMap *map, const void *base, const Geo &g, int B, int heads, int d, int hb) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t row = (cuuint64_t)heads * d * 2;  // bytes per token
+  cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)g.W, (cuuint64_t)g.H,
+                        (cuuint64_t)B * g.T};
+  cuuint64_t strides[4] = {(cuuint64_t)d * 2, row, row * g.W, row * g.W * g.H};
+  cuuint32_t box[5] = {(cuuint32_t)d, (cuuint32_t)hb, 8, 8, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 148;
+  return n > 0 ? n : 148;
 }
 
 // Pooled rows [bh, Nt, d] fp32 as a 3D tensor (d, Nt, bh); a box is 32 d-values
@@ -257,16 +282,24 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
   float *qlo = tc_scores ? reinterpret_cast<float *>(ws + L.qlo) : nullptr;
   float *klo = tc_scores ? reinterpret_cast<float *>(ws + L.klo) : nullptr;
   if (use_scores && P_in == nullptr) {
-    const long long warps = 2 * R;
-    const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
-    if (raster)
-      pool_kernel<D, true><<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(q_tiled),
-                                                  static_cast<const uint4 *>(k_tiled), qbar, kbar, qlo, klo, R,
-                                                  g, heads);
-    else
-      pool_kernel<D, false><<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(q_tiled),
-                                                   static_cast<const uint4 *>(k_tiled), qbar, kbar, qlo, klo, R,
-                                                   g, heads);
+    if (raster) {
+      // persistent TMA pooling: one CTA per SM over (tile, tensor, head group) boxes
+      using PC = pool::Cfg<D>;
+      CUtensorMap m_q, m_k;
+      if (!make_raster_pool_map(&m_q, q_tiled, g, B, heads, D, PC::HB) ||
+          !make_raster_pool_map(&m_k, k_tiled, g, B, heads, D, PC::HB))
+        return STA_ERR_CUDA;
+      auto kern = pool::pool_tma_kernel<D>;
+      STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PC::SMEM));
+      const long long units = 2LL * B * g.T * g.NH * g.NW * ((heads + PC::HB - 1) / PC::HB);
+      const long long ctas = units < sm_count() ? units : sm_count();
+      kern<<<(unsigned)ctas, pool::NUM_THREADS, PC::SMEM, s>>>(m_q, m_k, qbar, kbar, qlo, klo, g, heads, units);
+    } else {
+      const long long warps = 2 * R;
+      const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
+      pool_kernel<D><<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(q_tiled), static_cast<const uint4 *>(k_tiled),
+                                            qbar, kbar, qlo, klo, R, g);
+    }
     STA_CUDA_TRY(cudaGetLastError());
   }
   GroupLo glo;

@@ -4,7 +4,9 @@
 // Fig. 4), emitted as CSR lists (Compact Attention Fig. 3).
 //
 // Kernels, in launch order:
-//   pool_kernel          tile means of Q and K (HBM-bound, coalesced 16 B loads)
+//   pool_kernel          tile means of tiled Q and K (HBM-bound, coalesced 16 B
+//                        loads); the raster form pools with pool_tma_kernel
+//                        (sta_pool.cuh)
 //   score_tc_kernel      (sta_score.cuh, full workspace) the scores on the
 //                        tensor cores, rows of S written to a row buffer
 //   score_select_kernel  row softmax, selection, window test -> row bitsets;
@@ -28,19 +30,17 @@ __device__ __forceinline__ float round_tf32(float x) {
 }
 
 // ---------------------------------------------------------------- pooling
-// One warp per (b*heads + h, tile). Each lane owns one 16-byte chunk of a row
-// and walks the tile's real rows; the sum is exact in fp64 (64 bf16 values),
-// the mean is rounded once to fp32. With qlo / klo given, the mean x is
+// One warp per (b*heads + h, tile) of the tiled layout. Each lane owns one
+// 16-byte chunk of a row and walks the tile's real rows; the sum is exact in
+// fp64 (64 bf16 values whose magnitudes span less than 2^39), the mean is
+// rounded once to fp32. With qlo / klo given, the mean x is
 // stored split for the tensor-core scores: tf32(x) in qbar / kbar and
 // tf32(x - tf32(x)) in qlo / klo (round to nearest, ties away).
-// RASTER: Q and K in the raster layout [B, L, heads, d]; consecutive warps
-// take the same tile of consecutive heads, so together they read whole
-// token rows (all heads) at a time.
-template <int D, bool RASTER>
+template <int D>
 __global__ void __launch_bounds__(256)
 pool_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k, float *__restrict__ qbar,
             float *__restrict__ kbar, float *__restrict__ qlo, float *__restrict__ klo,
-            long long n_tiles_total, Geo g, int heads) {
+            long long n_tiles_total, Geo g) {
   constexpr int CPR = D / 8;      // chunks per row
   constexpr int RPI = 32 / CPR;   // rows per warp step
   const long long warp_id = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -51,23 +51,15 @@ pool_kernel(const uint4 *__restrict__ q, const uint4 *__restrict__ k, float *__r
   const uint4 *src = is_k ? k : q;
   float *dst = is_k ? kbar : qbar;
   float *dst_lo = is_k ? klo : qlo;
-  const long long BH = n_tiles_total / g.Nt;
-  const long long bh = RASTER ? idx % BH : idx / g.Nt;
-  const int n = (int)(RASTER ? idx / BH : idx % g.Nt);
+  const long long bh = idx / g.Nt;
+  const int n = (int)(idx % g.Nt);
   const long long tile = bh * g.Nt + n;  // output row of qbar / kbar
   const int tpf = g.NH * g.NW;
   const int t = n / tpf, rem = n - t * tpf;
   const int ty = rem / g.NW, tx = rem - ty * g.NW;
   const int vy = valid_extent(g.H, ty), vx = valid_extent(g.W, tx);
   const int sub = lane / CPR, c = lane - sub * CPR;
-  // chunk of tile row r: tiled row tile*64 + r, or raster row of token
-  // (t, 8*ty + r/8, 8*tx + r%8) and head h
-  const long long b = bh / heads, h = bh - b * heads;
-  const long long frame_row0 = ((b * g.T + t) * g.H + 8LL * ty) * g.W + 8LL * tx;
-  auto row_chunk = [&](int r) -> const uint4 * {
-    if (RASTER) return src + ((frame_row0 + (long long)(r >> 3) * g.W + (r & 7)) * heads + h) * CPR;
-    return src + (tile * 64 + r) * CPR;
-  };
+  auto row_chunk = [&](int r) -> const uint4 * { return src + (tile * 64 + r) * CPR; };
   double acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.0;

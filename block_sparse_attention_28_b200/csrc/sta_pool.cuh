@@ -1,0 +1,148 @@
+// Tile means of Q and K read straight from the raster layout through TMA:
+// the pooling of the mask build's raster form (Rectified SpaAttn abstract,
+// pooled queries and keys; tiles of 1 x 8 x 8 tokens).
+//
+// Persistent CTAs, one per SM, each walking the units u = blockIdx.x +
+// i * gridDim.x. A unit is one token tile of one tensor (Q or K) for HB
+// consecutive heads: a 5D TMA box (d, head, x, y, frame) of D x HB x 8 x 8 x 1
+// bf16 = 64 KB, zero-filled past the grid edge and past the last head.
+//   warp 8     TMA producer: boxes into a ring of STAGES buffers
+//   warps 0-7  each thread sums two adjacent (head, d) columns of the box over
+//              the 64 token rows in fp64 (exact for bf16 inputs whose
+//              magnitudes in a tile span less than 2^39), divides by the
+//              number of real tokens and rounds once to fp32; with qlo / klo
+//              given the mean x is stored split for the tensor-core scores,
+//              tf32(x) in qbar / kbar and tf32(x - tf32(x)) in qlo / klo
+// The ring keeps up to 192 KB of loads in flight per SM, which is what a
+// stream from HBM needs, without a thread per outstanding load.
+// Every wait is bounded; on a timeout the kernel records DEV_ERR_TIMEOUT,
+// waits (bounded) for its own copies in flight and returns.
+#pragma once
+#include "sta_mask.cuh"
+#include "sta_tc.cuh"
+
+namespace sta {
+namespace pool {
+
+constexpr int CONSUMERS = 256;                 // 8 warps, two columns per thread
+constexpr int NUM_THREADS = CONSUMERS + 32;    // + the producer warp
+constexpr int WARP_TMA = CONSUMERS / 32;
+constexpr int STAGES = 3;
+constexpr long long WAIT_LIMIT = 2000000000LL;  // SM cycles (~1 s)
+constexpr long long DRAIN_LIMIT = 200000000LL;  // after an abort
+
+template <int D>
+struct Cfg {
+  static constexpr int HB = 512 / D;                // heads per box: HB * D = 2 * CONSUMERS columns
+  static constexpr int COLS = HB * D;
+  static constexpr int BOX_BYTES = 64 * COLS * 2;   // 8 x 8 tokens x HB heads x D bf16
+  static constexpr int OFF_BAR = STAGES * BOX_BYTES;
+  static constexpr int SMEM = OFF_BAR + 16 * STAGES + 16 + 1024;  // + alignment slack
+  static_assert(COLS == 2 * CONSUMERS, "two columns per consumer thread");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+// Unit u = ((((b*T + t) * NH + ty) * NW + tx) * 2 + tensor) * G + group,
+// G = ceil(heads / HB); consecutive units are neighbouring boxes of memory.
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+pool_tma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                float *__restrict__ qbar, float *__restrict__ kbar, float *__restrict__ qlo,
+                float *__restrict__ klo, Geo g, int heads, long long units) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = tc::smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+  uint64_t *empty = full + STAGES;
+  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(empty + STAGES);
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(full + s, 1);
+      tc::mbar_init(empty + s, CONSUMERS / 32);  // one arrival per consumer warp
+    }
+    *abort_flag = 0u;
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  const int G = (heads + C::HB - 1) / C::HB;
+
+  if (warp == WARP_TMA) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      long long issued = 0, i = 0;
+      for (long long u = blockIdx.x; u < units; u += gridDim.x, ++i) {
+        const int s = (int)(i % STAGES);
+        const long long r = i / STAGES;
+        if (r > 0 && !tc::mbar_wait(empty + s, (uint32_t)((r - 1) & 1), abort_flag, WAIT_LIMIT)) break;
+        long long v = u;
+        const int grp = (int)(v % G);
+        v /= G;
+        const int tensor = (int)(v & 1);
+        v >>= 1;
+        const int tx = (int)(v % g.NW);
+        v /= g.NW;
+        const int ty = (int)(v % g.NH);
+        const int bt = (int)(v / g.NH);
+        tc::mbar_expect_tx(full + s, C::BOX_BYTES);
+        tc::tma_load_5d(sbase + s * C::BOX_BYTES, tensor ? &tm_k : &tm_q, full + s, 0, grp * C::HB, tx * 8,
+                        ty * 8, bt);
+        issued = i + 1;
+      }
+      // copies still in flight must land before the CTA can exit
+      if (*abort_flag) {
+        for (long long j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+          tc::mbar_wait(full + j % STAGES, (uint32_t)((j / STAGES) & 1), nullptr, DRAIN_LIMIT);
+      }
+    }
+    __syncwarp();
+    return;
+  }
+  // ------------------------------------------------------------ consumers
+  const int col = 2 * tid;  // columns col, col + 1 of the box: head col / D, dims col % D
+  const int h_in = col / D, dd = col - h_in * D;
+  long long i = 0;
+  for (long long u = blockIdx.x; u < units; u += gridDim.x, ++i) {
+    const int s = (int)(i % STAGES);
+    if (!tc::mbar_wait(full + s, (uint32_t)((i / STAGES) & 1), abort_flag, WAIT_LIMIT)) break;
+    // box row r = 8 y + x (token of the tile), columns [head][d]
+    const __nv_bfloat162 *box = reinterpret_cast<const __nv_bfloat162 *>(smem + s * C::BOX_BYTES) + tid;
+    double a0 = 0.0, a1 = 0.0;
+#pragma unroll 16
+    for (int r = 0; r < 64; ++r) {
+      const float2 f = __bfloat1622float2(box[r * (C::COLS / 2)]);
+      a0 += (double)f.x;
+      a1 += (double)f.y;
+    }
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(empty + s);
+    long long v = u;
+    const int grp = (int)(v % G);
+    v /= G;
+    const int tensor = (int)(v & 1);
+    v >>= 1;
+    const int tx = (int)(v % g.NW);
+    v /= g.NW;
+    const int ty = (int)(v % g.NH);
+    const int bt = (int)(v / g.NH);
+    const int h = grp * C::HB + h_in;
+    if (h < heads) {
+      const int b = bt / g.T, t = bt - b * g.T;
+      const double cnt = (double)(valid_extent(g.H, ty) * valid_extent(g.W, tx));
+      const long long row = ((long long)b * heads + h) * g.Nt + ((long long)t * g.NH + ty) * g.NW + tx;
+      float m0 = (float)(a0 / cnt), m1 = (float)(a1 / cnt);
+      float *lo = tensor ? klo : qlo;
+      if (lo != nullptr) {
+        const float h0 = round_tf32(m0), h1 = round_tf32(m1);
+        *reinterpret_cast<float2 *>(lo + row * D + dd) = make_float2(round_tf32(m0 - h0), round_tf32(m1 - h1));
+        m0 = h0;
+        m1 = h1;
+      }
+      *reinterpret_cast<float2 *>((tensor ? kbar : qbar) + row * D + dd) = make_float2(m0, m1);
+    }
+  }
+}
+
+}  // namespace pool
+}  // namespace sta
