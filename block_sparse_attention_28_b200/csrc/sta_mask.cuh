@@ -537,32 +537,60 @@ head_floor_kernel(const int *__restrict__ sel_count, int *__restrict__ kfloor, G
 // ---------------------------------------------------------------- scan
 // Single CTA: row_ptr[0] = 0, row_ptr[r+1] = sum of counts[0..r]; nnz = total.
 constexpr int SCAN_THREADS = 1024;
+constexpr int SCAN_BATCH = 4;  // chunks of 4 * SCAN_THREADS counts whose loads are issued together
 
+__device__ __forceinline__ int warp_incl_scan(int x, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  return x;
+}
+
+// Single-CTA exclusive scan of the row counts into row_ptr (row_ptr[0] = 0,
+// row_ptr[r + 1] = sum of counts[0..r]) and nnz = the total. The counts are
+// read in chunks of 4 per thread (4096 per chunk, coalesced), scanned with
+// warp shuffles plus one pass over the 32 warp totals, and chained by a
+// running carry. Integer sums: the result does not depend on the order.
 __global__ void __launch_bounds__(SCAN_THREADS)
 scan_kernel(const int *__restrict__ counts, int *__restrict__ row_ptr, long long *__restrict__ nnz,
             long long R) {
-  __shared__ long long part[SCAN_THREADS];
-  const int tid = threadIdx.x;
-  const long long per = (R + SCAN_THREADS - 1) / SCAN_THREADS;
-  const long long lo = min(R, tid * per), hi = min(R, lo + per);
-  long long s = 0;
-  for (long long r = lo; r < hi; ++r) s += counts[r];
-  part[tid] = s;
-  __syncthreads();
-  // Hillis-Steele inclusive scan over the per-thread sums.
-  for (int off = 1; off < SCAN_THREADS; off <<= 1) {
-    const long long add = (tid >= off) ? part[tid - off] : 0;
-    __syncthreads();
-    part[tid] += add;
-    __syncthreads();
-  }
-  long long run = part[tid] - s;  // exclusive prefix of this segment
+  __shared__ int wsum[SCAN_THREADS / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr long long CH = 4LL * SCAN_THREADS;
+  long long carry = 0;
   if (tid == 0) row_ptr[0] = 0;
-  for (long long r = lo; r < hi; ++r) {
-    run += counts[r];
-    row_ptr[r + 1] = (int)run;
+  for (long long base = 0; base < R; base += CH * SCAN_BATCH) {
+    int v[SCAN_BATCH][4];
+#pragma unroll
+    for (int bch = 0; bch < SCAN_BATCH; ++bch) {
+      const long long i0 = base + bch * CH + 4LL * tid;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[bch][e] = (i0 + e < R) ? counts[i0 + e] : 0;
+    }
+#pragma unroll
+    for (int bch = 0; bch < SCAN_BATCH; ++bch) {
+      if (base + bch * CH >= R) break;  // uniform over the CTA
+      int x[4];
+      x[0] = v[bch][0];
+#pragma unroll
+      for (int e = 1; e < 4; ++e) x[e] = x[e - 1] + v[bch][e];
+      const int incl = warp_incl_scan(x[3], lane);
+      if (lane == 31) wsum[warp] = incl;
+      __syncthreads();
+      if (warp == 0) wsum[lane] = warp_incl_scan(wsum[lane], lane);
+      __syncthreads();
+      const long long pre = carry + (warp > 0 ? wsum[warp - 1] : 0) + (incl - x[3]);
+      const long long i0 = base + bch * CH + 4LL * tid;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (i0 + e < R) row_ptr[i0 + e + 1] = (int)(pre + x[e]);
+      carry += wsum[SCAN_THREADS / 32 - 1];
+      __syncthreads();  // wsum is rewritten by the next chunk
+    }
   }
-  if (tid == SCAN_THREADS - 1) *nnz = part[tid];
+  if (tid == 0) *nnz = carry;
 }
 
 // ---------------------------------------------------------------- fill
