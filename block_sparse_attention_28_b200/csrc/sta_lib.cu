@@ -76,7 +76,9 @@ MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
 size_t select_smem(int d, const Geo &g, bool use_scores, int qb = SEL_QB, int mode = SEL_FUSED) {
   const size_t q = (mode == SEL_FUSED && use_scores) ? (size_t)qb * d : 0;
   const size_t scores = use_scores ? (size_t)(qb * g.Nt + (SEL_THREADS / 32) * 256) : 0;
-  const size_t tables = (size_t)((g.Nt + g.T + 3) & ~3) + 4 * STA_MAX_GROUPS;
+  // window tables (group of each |dt|, the head's extents) and one row of
+  // window bits per warp
+  const size_t tables = (size_t)((g.T + 3) & ~3) + 4 * STA_MAX_GROUPS + (SEL_THREADS / 32) * ((g.Nt + 31) / 32);
   return (q + scores + tables) * sizeof(float);
 }
 

@@ -311,23 +311,20 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
   const int nq = min(QB, nt - q0);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tpf = g.NH * g.NW;
-  // shared memory: [qs], [S, histograms] if use_scores, then the window tables
+  // shared memory: [qs], [S, histograms] if use_scores, then the window
+  // tables and one row of window bits per warp (all 16-byte aligned: QB * nt
+  // is a multiple of 8)
   float *qs = sm;
   float *S = qs + ((HAS_SCORES && use_scores) ? QB * D : 0);
   unsigned int *hist = reinterpret_cast<unsigned int *>(S + (use_scores ? QB * nt : 0));
-  unsigned int *kcoord = hist + (use_scores ? (SEL_THREADS / 32) * 256 : 0);
-  int *gtab = reinterpret_cast<int *>(kcoord + nt);
-  int *wtab = gtab + ((nt + g.T + 3) & ~3) - nt;  // 16-byte aligned, 4 ints per group
+  int *gtab = reinterpret_cast<int *>(hist + (use_scores ? (SEL_THREADS / 32) * 256 : 0));
+  int *wtab = gtab + ((g.T + 3) & ~3);  // 4 ints per group
+  unsigned int *wwin = reinterpret_cast<unsigned int *>(wtab + 4 * STA_MAX_GROUPS) + warp * wpr;
   unsigned int *whist = hist + warp * 256;
 
-  // Window tables, once per CTA: packed (t, tile row, tile column) of every
-  // key tile, the temporal group of every |dt|, and this head's extents.
+  // Window tables, once per CTA: the temporal group of every |dt| and this
+  // head's extents.
   if (windows != nullptr) {
-    for (int kt = tid; kt < nt; kt += SEL_THREADS) {
-      const int t = kt / tpf, rem = kt - t * tpf;
-      const int y = rem / g.NW, x = rem - y * g.NW;
-      kcoord[kt] = ((unsigned int)t << 20) | ((unsigned int)y << 10) | (unsigned int)x;
-    }
     for (int dt = tid; dt < g.T; dt += SEL_THREADS) {
       int grp = -1;
       for (int gg = 0; gg < G; ++gg)
@@ -336,7 +333,7 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
     }
     for (int i = tid; i < G * 4; i += SEL_THREADS) wtab[i] = windows[(long long)h * G * 4 + i];
   }
-  if (!use_scores) __syncthreads();
+  __syncthreads();  // every warp reads the tables
 
   if (HAS_SCORES && use_scores && P_in == nullptr) {
     // Phase 1: S[i][kt] = scale * qbar[q0+i] . kbar[kt], sequential fp32 FMA over d.
@@ -459,24 +456,35 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
     // Phase 4: membership bits = selected OR window, one 32-bit word per lane step.
     const int tq = qt / tpf, remq = qt - tq * tpf;
     const int yq = remq / g.NW, xq = remq - yq * g.NW;
+    if (windows != nullptr) {
+      // The row's window tiles, written as runs of bits: for each key frame,
+      // each of the two rectangles and each tile row it covers, the tile
+      // columns within the extent (clipped to the grid) are consecutive
+      // key tiles.
+      for (int w = lane; w < wpr; w += 32) wwin[w] = 0u;
+      __syncwarp();
+      const int items = g.T * 2 * g.NH;
+      for (int it = lane; it < items; it += 32) {
+        const int y = it % g.NH, rect = (it / g.NH) & 1, tk = it / (2 * g.NH);
+        const int grp = gtab[abs(tq - tk)];
+        if (grp < 0) continue;
+        const int4 w4 = reinterpret_cast<const int4 *>(wtab)[grp];
+        const int ry = rect ? w4.z : w4.x, rx = rect ? w4.w : w4.y;
+        if (ry < 0 || rx < 0 || abs(y - yq) > ry) continue;
+        const int base = (tk * g.NH + y) * g.NW;
+        const int k0 = base + max(0, xq - rx), k1 = base + min(g.NW - 1, xq + rx);
+        for (int w = k0 >> 5; w <= (k1 >> 5); ++w) {
+          const int lo = max(k0 - 32 * w, 0), hi = min(k1 - 32 * w, 31);
+          atomicOr(wwin + w, (0xFFFFFFFFu >> (31 - hi + lo)) << lo);  // bits lo..hi
+        }
+      }
+      __syncwarp();
+    }
     unsigned int ties_seen = 0u;
     int total = 0;
     unsigned int *brow = bits + row * wpr;
     for (int w0 = 0; w0 < wpr; ++w0) {
       const int kt = w0 * 32 + lane;
-      bool keep = false;
-      if (kt < nt) {
-        if (windows != nullptr) {
-          const unsigned int kc = kcoord[kt];
-          const int dt = abs(tq - (int)(kc >> 20));
-          const int dy = abs(yq - (int)((kc >> 10) & 1023u)), dx = abs(xq - (int)(kc & 1023u));
-          const int grp = gtab[dt];
-          if (grp >= 0) {
-            const int4 w4 = reinterpret_cast<const int4 *>(wtab)[grp];
-            keep = (dy <= w4.x && dx <= w4.y) || (dy <= w4.z && dx <= w4.w);
-          }
-        }
-      }
       // Selection membership needs the index-ordered rank among ties: warp-wide.
       bool sel = false;
       if (use_scores && v_f != 0xFFFFFFFFu) {
@@ -487,7 +495,7 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
         sel = (kt < nt) && (pb > v_f || (tie && ties_seen + before < c_f));
         ties_seen += __popc(tmask);
       }
-      const unsigned int word = __ballot_sync(0xffffffffu, keep || sel);
+      const unsigned int word = __ballot_sync(0xffffffffu, sel) | (windows != nullptr ? wwin[w0] : 0u);
       if (lane == 0) brow[w0] = word;
       total += __popc(word);
     }
