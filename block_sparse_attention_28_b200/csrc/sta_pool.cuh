@@ -6,13 +6,15 @@
 // i * gridDim.x. A unit is one token tile of one tensor (Q or K) for HB
 // consecutive heads: a 5D TMA box (d, head, x, y, frame) of D x HB x 8 x 8 x 1
 // bf16 = 64 KB, zero-filled past the grid edge and past the last head.
-//   warp 8     TMA producer: boxes into a ring of STAGES buffers
-//   warps 0-7  each thread sums two adjacent (head, d) columns of the box over
-//              the 64 token rows in fp64 (exact for bf16 inputs whose
-//              magnitudes in a tile span less than 2^39), divides by the
-//              number of real tokens and rounds once to fp32; with qlo / klo
-//              given the mean x is stored split for the tensor-core scores,
-//              tf32(x) in qbar / kbar and tf32(x - tf32(x)) in qlo / klo
+//   warp 16     TMA producer: boxes into a ring of STAGES buffers
+//   warps 0-15  each thread sums two adjacent (head, d) columns of the box
+//               over half of the 64 token rows in fp64; the two halves meet
+//               in shared memory (exact for bf16 inputs whose magnitudes in a
+//               tile span less than 2^39, so the split does not change the
+//               result); the sum is divided by the number of real tokens and
+//               rounded once to fp32; with qlo / klo given the mean x is stored
+//               split for the tensor-core scores, tf32(x) in qbar / kbar and
+//               tf32(x - tf32(x)) in qlo / klo
 // The ring keeps up to 192 KB of loads in flight per SM, which is what a
 // stream from HBM needs, without a thread per outstanding load.
 // Every wait is bounded; on a timeout the kernel records DEV_ERR_TIMEOUT,
@@ -24,7 +26,7 @@
 namespace sta {
 namespace pool {
 
-constexpr int CONSUMERS = 256;                 // 8 warps, two columns per thread
+constexpr int CONSUMERS = 512;                 // 16 warps: two columns x half the rows per thread
 constexpr int NUM_THREADS = CONSUMERS + 32;    // + the producer warp
 constexpr int WARP_TMA = CONSUMERS / 32;
 constexpr int STAGES = 3;
@@ -36,9 +38,10 @@ struct Cfg {
   static constexpr int HB = 512 / D;                // heads per box: HB * D = 2 * CONSUMERS columns
   static constexpr int COLS = HB * D;
   static constexpr int BOX_BYTES = 64 * COLS * 2;   // 8 x 8 tokens x HB heads x D bf16
-  static constexpr int OFF_BAR = STAGES * BOX_BYTES;
+  static constexpr int OFF_PART = STAGES * BOX_BYTES;  // [2][COLS] fp64 partial sums of the upper half
+  static constexpr int OFF_BAR = OFF_PART + 2 * COLS * 8;
   static constexpr int SMEM = OFF_BAR + 16 * STAGES + 16 + 1024;  // + alignment slack
-  static_assert(COLS == 2 * CONSUMERS, "two columns per consumer thread");
+  static_assert(COLS == CONSUMERS, "two columns per thread pair");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -100,23 +103,42 @@ pool_tma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     return;
   }
   // ------------------------------------------------------------ consumers
-  const int col = 2 * tid;  // columns col, col + 1 of the box: head col / D, dims col % D
+  const int pair = tid % (CONSUMERS / 2), half = tid / (CONSUMERS / 2);
+  const int col = 2 * pair;  // columns col, col + 1 of the box: head col / D, dims col % D
   const int h_in = col / D, dd = col - h_in * D;
+  double *part = reinterpret_cast<double *>(smem + C::OFF_PART);
   long long i = 0;
   for (long long u = blockIdx.x; u < units; u += gridDim.x, ++i) {
     const int s = (int)(i % STAGES);
-    if (!tc::mbar_wait(full + s, (uint32_t)((i / STAGES) & 1), abort_flag, WAIT_LIMIT)) break;
-    // box row r = 8 y + x (token of the tile), columns [head][d]
-    const __nv_bfloat162 *box = reinterpret_cast<const __nv_bfloat162 *>(smem + s * C::BOX_BYTES) + tid;
+    const bool got = tc::mbar_wait(full + s, (uint32_t)((i / STAGES) & 1), abort_flag, WAIT_LIMIT);
     double a0 = 0.0, a1 = 0.0;
+    if (got) {
+      // box row r = 8 y + x (token of the tile), columns [head][d]; this
+      // thread sums rows [32 half, 32 half + 32)
+      const __nv_bfloat162 *box = reinterpret_cast<const __nv_bfloat162 *>(smem + s * C::BOX_BYTES) + pair;
 #pragma unroll 16
-    for (int r = 0; r < 64; ++r) {
-      const float2 f = __bfloat1622float2(box[r * (C::COLS / 2)]);
-      a0 += (double)f.x;
-      a1 += (double)f.y;
+      for (int r = 32 * half; r < 32 * half + 32; ++r) {
+        const float2 f = __bfloat1622float2(box[r * (C::COLS / 2)]);
+        a0 += (double)f.x;
+        a1 += (double)f.y;
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(empty + s);
+      if (half == 1) {
+        part[(i & 1) * C::COLS + col] = a0;
+        part[(i & 1) * C::COLS + col + 1] = a1;
+      }
     }
-    __syncwarp();
-    if (lane == 0) tc::mbar_arrive(empty + s);
+    // the consumers leave the loop together (they share barrier 1), and the
+    // barrier also publishes the upper halves' partial sums
+    uint32_t all;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, %2, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}\n"
+                 : "=r"(all) : "r"((uint32_t)got), "n"(CONSUMERS) : "memory");
+    if (!all) break;
+    if (half == 1) continue;
+    a0 += part[(i & 1) * C::COLS + col];
+    a1 += part[(i & 1) * C::COLS + col + 1];
     long long v = u;
     const int grp = (int)(v % G);
     v /= G;
