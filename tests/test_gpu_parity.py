@@ -170,6 +170,21 @@ def test_build_mask_ragged(sta, gp, top_p, k_min, use_scores, with_win, d):
     _check_mask(sta, gp, qt, kt, B, Hh, d, T, H, W, top_p, k_min, use_scores, win, (0, 1, 3))
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_build_mask_several_key_blocks(sta, gp, d):
+    """Nt = 175 tiles: two 128-tile key blocks of the tensor-core scores, the
+    query range split over several CTAs, and rows of S whose length is not a
+    multiple of four (scalar stores)."""
+    T, H, W, Hh, B = 5, 40, 50, 2, 1  # 5 x 5 x 7 tiles
+    q, k, _ = _structured(T, H, W, Hh, d, seed=41, B=B)
+    g = sta.grid(T, H, W)
+    assert sta.sta_num_tiles(g) == 175
+    qt, kt = gp.reorder(q, B, Hh, d, g), gp.reorder(k, B, Hh, d, g)
+    rng = np.random.default_rng(d)
+    win = rng.integers(-1, 3, size=(Hh, 3, 4)).astype(np.int32)
+    _check_mask(sta, gp, qt, kt, B, Hh, d, T, H, W, 0.9, 4, True, win, (0, 1, 3))
+
+
 def test_build_mask_window_only_full_480p(sta, gp):
     cfg = CONFIGS["dit480p"]
     g = sta.grid(cfg.T, cfg.H, cfg.W)
@@ -778,8 +793,12 @@ def _raster_vs_tiled(sta, gp, q, k, v, B, Hh, d, T, H, W, params, rows_check=Non
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("T,H,W,Hh,B", [(3, 19, 37, 2, 2), (4, 16, 16, 3, 1), (2, 9, 10, 1, 1), (5, 24, 13, 2, 1)])
+@pytest.mark.parametrize("T,H,W,Hh,B", [(3, 19, 37, 2, 2), (4, 16, 16, 3, 1), (2, 9, 10, 1, 1), (5, 24, 13, 2, 1),
+                                        (3, 11, 20, 6, 1), (2, 8, 24, 10, 2)])
 def test_raster_path_equals_tiled(sta, gp, d, T, H, W, Hh, B):
+    """Raster and tiled calls agree bit for bit, and the raster output matches
+    the oracle. Head counts below, at and above one pooling box (4 heads at
+    d = 128, 8 at d = 64), with a partial last box."""
     q, k, v = _structured(T, H, W, Hh, d, seed=T * 7 + W, B=B)
     nh, nw, _, _ = O.tile_grid(T, H, W)
     win = np.zeros((Hh, 2, 4), dtype=np.int32)
