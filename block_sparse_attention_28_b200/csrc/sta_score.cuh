@@ -10,22 +10,24 @@
 //
 // One CTA per (128 key tiles, range of query tiles, b*heads + h); 192 threads:
 //   warp 4     TMA producer: first the CTA's key block (hi and lo parts) into
-//              the first ring stages, then, once it has moved to TMEM, blocks
-//              of 64 query tiles (hi and lo) through the ring (the B operand)
+//              the ring's buffers, then, once it has moved to TMEM, blocks of
+//              128 query tiles (the B operand), one 32-wide chunk of d (hi and
+//              lo, 32 KB) per ring stage
 //   warps 0-3  move the key block from shared memory to TMEM (one key tile
 //              per thread = TMEM lane), where it is the A operand of every
-//              MMA; then the epilogue of each block: TMEM -> registers ->
-//              a transposed tile in shared memory -> rows of S written as
-//              512-byte runs of 16-byte stores
+//              MMA; then the epilogue of each block, in two halves of 64
+//              query tiles: TMEM -> registers -> a transposed tile in shared
+//              memory -> rows of S written as 512-byte runs of 16-byte stores
 //   warp 5     TMEM allocation and the MMA issue (one thread); accumulators
 //              double-buffered in TMEM so the epilogue of block j overlaps
 //              the MMAs of block j + 1
-// With the key block in TMEM an MMA reads only its 64 query rows from shared
-// memory, so it runs at the tensor-core rate instead of the shared-memory
-// rate. Operands in shared memory are K-major with the 128-byte swizzle: a
-// chunk of 32 fp32 along d per 128-byte row, 8-row groups 1024 B apart.
-// Every wait is bounded; on a timeout the kernel records DEV_ERR_TIMEOUT,
-// waits (bounded) for its own copies in flight, releases TMEM and returns.
+// With the key block in TMEM an MMA reads only its query rows from shared
+// memory, and with N = 128 it runs at the full tensor-core rate (an N = 64
+// MMA takes ~46 cycles for the work of 32). Operands in shared memory are
+// K-major with the 128-byte swizzle: a chunk of 32 fp32 along d per 128-byte
+// row, 8-row groups 1024 B apart. Every wait is bounded; on a timeout the
+// kernel records DEV_ERR_TIMEOUT, waits (bounded) for its own copies in
+// flight, releases TMEM and returns.
 #pragma once
 #include "sta_tc.cuh"
 
@@ -33,7 +35,8 @@ namespace sta {
 namespace score {
 
 constexpr int M = 128;           // key tiles per CTA (TMEM lanes)
-constexpr int N = 64;            // query tiles per MMA block (TMEM columns)
+constexpr int N = 128;           // query tiles per MMA block (TMEM columns)
+constexpr int NH = 64;           // query tiles per epilogue half
 constexpr int NUM_THREADS = 192;
 constexpr int WARP_TMA = 4, WARP_MMA = 5;
 constexpr long long WAIT_LIMIT = 2000000000LL;  // SM cycles (~1 s)
@@ -45,11 +48,10 @@ struct Cfg {
   static constexpr int A_CHUNK = M * 128;      // bytes of one chunk of the key block
   static constexpr int A_PART = CH * A_CHUNK;  // one split part of the key block
   static constexpr int B_CHUNK = N * 128;      // bytes of one chunk of a query block
-  static constexpr int B_PART = CH * B_CHUNK;  // one split part of a query block
-  static constexpr int STAGES = D == 128 ? 3 : 6;
-  static constexpr int STAGE_BYTES = 2 * B_PART;  // hi part, then lo part
-  static constexpr int OFF_T = STAGES * STAGE_BYTES;  // [N][M] fp32 epilogue tile
-  static constexpr int OFF_BAR = OFF_T + N * M * 4;
+  static constexpr int STAGES = 5;             // ring stages of one chunk (hi part, then lo part)
+  static constexpr int STAGE_BYTES = 2 * B_CHUNK;
+  static constexpr int OFF_T = STAGES * STAGE_BYTES;  // [NH][M] fp32 epilogue tile
+  static constexpr int OFF_BAR = OFF_T + NH * M * 4;
   // a_tma, a_moved, a_full, full[STAGES], empty[STAGES], t_full[2], t_empty[2], mma_done
   static constexpr int NBAR = 3 + 2 * STAGES + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;  // tmem address, abort flag
@@ -58,7 +60,7 @@ struct Cfg {
   // TMEM columns: two accumulators of N, then the key block's hi and lo
   // parts (one fp32 / tf32 element per column, lane = key tile)
   static constexpr uint32_t COL_HI = 2 * N, COL_LO = 2 * N + D;
-  static constexpr uint32_t TMEM_COLS = (2 * N + 2 * D) <= 256 ? 256 : 512;
+  static constexpr uint32_t TMEM_COLS = 512;
   static_assert(D % 32 == 0, "d must be a multiple of 32");
   static_assert(2 * A_PART <= STAGES * STAGE_BYTES, "key block staging");
   static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -103,11 +105,10 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
 }
 
 // tm_khi / tm_klo / tm_qhi / tm_qlo: the split parts of the pooled keys and
-// queries as 3D tensors (d, Nt, b*heads) fp32, boxes of 32 x M x 1 (keys) and
-// 32 x N x 1 (queries), zero-filled past Nt. S: [b*heads][Nt][Nt] fp32,
-// row = query tile. The query tiles of this CTA are
-// [blockIdx.y * q_per_part, ... + q_per_part) clipped to Nt, q_per_part a
-// multiple of N.
+// queries as 3D tensors (d, Nt, b*heads) fp32, boxes of 32 x 128 x 1,
+// zero-filled past Nt. S: [b*heads][Nt][Nt] fp32, row = query tile. The query
+// tiles of this CTA are [blockIdx.y * q_per_part, ... + q_per_part) clipped to
+// Nt, q_per_part a multiple of N.
 template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constant__ CUtensorMap tm_klo,
@@ -160,6 +161,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
   __syncthreads();
   tc::fence_after();
   const uint32_t tmem = misc[0];
+  const int nchunks = nblk * C::CH;  // ring items: (block j, d-chunk c) = item j * CH + c
 
   if (warp == WARP_TMA) {
     // ---------------------------------------------------------- producer
@@ -173,24 +175,22 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
       int issued = 0;
       // the ring reuses the staging area once the key block is in TMEM
       bool ok = tc::mbar_wait(a_moved, 0, abort_flag, WAIT_LIMIT);
-      for (int j = 0; ok && j < nblk; ++j) {
-        const int s = j % C::STAGES, u = j / C::STAGES;
+      for (int it = 0; ok && it < nchunks; ++it) {
+        const int s = it % C::STAGES, u = it / C::STAGES;
         if (u > 0 && !tc::mbar_wait(empty + s, (u - 1) & 1, abort_flag, WAIT_LIMIT)) break;
+        const int j = it / C::CH, c = it - j * C::CH;
         const uint32_t dst = sbase + s * C::STAGE_BYTES;
         const int q0 = q_begin + j * N;
         tc::mbar_expect_tx(full + s, C::STAGE_BYTES);
-#pragma unroll
-        for (int c = 0; c < C::CH; ++c) {
-          tma_load_3d(dst + c * C::B_CHUNK, &tm_qhi, full + s, 32 * c, q0, bh);
-          tma_load_3d(dst + C::B_PART + c * C::B_CHUNK, &tm_qlo, full + s, 32 * c, q0, bh);
-        }
-        issued = j + 1;
+        tma_load_3d(dst, &tm_qhi, full + s, 32 * c, q0, bh);
+        tma_load_3d(dst + C::B_CHUNK, &tm_qlo, full + s, 32 * c, q0, bh);
+        issued = it + 1;
       }
       // copies still in flight must land before the CTA can exit
       if (*abort_flag) {
         tc::mbar_wait(a_tma, 0, nullptr, DRAIN_LIMIT);
-        for (int j = (issued > C::STAGES ? issued - C::STAGES : 0); j < issued; ++j)
-          tc::mbar_wait(full + j % C::STAGES, (j / C::STAGES) & 1, nullptr, DRAIN_LIMIT);
+        for (int it = (issued > C::STAGES ? issued - C::STAGES : 0); it < issued; ++it)
+          tc::mbar_wait(full + it % C::STAGES, (it / C::STAGES) & 1, nullptr, DRAIN_LIMIT);
       }
     }
     __syncwarp();
@@ -200,26 +200,31 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
       bool ok = tc::mbar_wait(a_full, 0, abort_flag, WAIT_LIMIT);
       tc::fence_after();
       for (int j = 0; ok && j < nblk; ++j) {
-        const int s = j % C::STAGES, buf = j & 1;
-        if (!tc::mbar_wait(full + s, (j / C::STAGES) & 1, abort_flag, WAIT_LIMIT)) break;
+        const int buf = j & 1;
         if (j >= 2 && !tc::mbar_wait(t_empty + buf, ((j >> 1) - 1) & 1, abort_flag, WAIT_LIMIT)) break;
-        tc::fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(buf * N);
-        const uint32_t b_hi = sbase + s * C::STAGE_BYTES, b_lo = b_hi + C::B_PART;
-        // lo_k*hi_q and hi_k*lo_q first (small), then hi_k*hi_q; K = 8 tf32
-        // per MMA: 8 TMEM columns of A, 32 bytes of a swizzled B row
-#pragma unroll
-        for (int part = 0; part < 3; ++part) {
-          const uint32_t a = tmem + (part == 0 ? C::COL_LO : C::COL_HI);
-          const uint32_t b = part == 1 ? b_lo : b_hi;
-#pragma unroll
-          for (int kk = 0; kk < 4 * C::CH; ++kk) {
-            const uint32_t koff = (uint32_t)((kk & 3) * 32);
-            mma_tf32_ts(d_tmem, a + (uint32_t)(kk * 8), tc::desc_k_sw128(b + (kk >> 2) * C::B_CHUNK + koff),
-                        (part > 0 || kk > 0) ? 1u : 0u);
+        for (int c = 0; ok && c < C::CH; ++c) {
+          const int it = j * C::CH + c, s = it % C::STAGES;
+          if (!tc::mbar_wait(full + s, (it / C::STAGES) & 1, abort_flag, WAIT_LIMIT)) {
+            ok = false;
+            break;
           }
+          tc::fence_after();
+          const uint32_t b_hi = sbase + s * C::STAGE_BYTES, b_lo = b_hi + C::B_CHUNK;
+          // lo_k*hi_q, hi_k*lo_q, then hi_k*hi_q over this chunk's four
+          // K = 8 steps: 8 TMEM columns of A, 32 bytes of a swizzled B row
+#pragma unroll
+          for (int part = 0; part < 3; ++part) {
+            const uint32_t a = tmem + (part == 0 ? C::COL_LO : C::COL_HI) + (uint32_t)(32 * c);
+            const uint32_t b = part == 1 ? b_lo : b_hi;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_tf32_ts(d_tmem, a + (uint32_t)(kk * 8), tc::desc_k_sw128(b + (uint32_t)(kk * 32)),
+                          (c > 0 || part > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc::mma_commit(empty + s);
         }
-        tc::mma_commit(empty + s);
+        if (!ok) break;
         tc::mma_commit(t_full + buf);
       }
       // every issued MMA retires before TMEM is released
@@ -263,38 +268,43 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
     }
     float *T = reinterpret_cast<float *>(smem + C::OFF_T);
     const bool vec = (nt & 3) == 0;  // every row segment of S is 16-byte aligned
+    const int kk = k0 + 4 * lane;
     // the four warps leave the loop together (they share barrier 1)
     ok = all_epilogue(ok);
     for (int j = 0; ok && j < nblk; ++j) {
       const int buf = j & 1;
       if (!all_epilogue(tc::mbar_wait(t_full + buf, (j >> 1) & 1, abort_flag, WAIT_LIMIT))) break;
       tc::fence_after();
-      uint32_t v[N];
-      tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * N), v);
-      tc::fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(t_empty + buf);
-      // transposed tile T[query][key] (consecutive threads, consecutive keys)
-#pragma unroll
-      for (int c = 0; c < N; ++c) T[c * M + tid] = __uint_as_float(v[c]) * scale;
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      // each warp writes query rows warp, warp + 4, ...: 128 keys per row,
-      // four per lane
-      const int q0 = q_begin + j * N;
-      const int kk = k0 + 4 * lane;
-      for (int c = warp; c < N && q0 + c < q_end; c += 4) {
-        const float4 val = reinterpret_cast<const float4 *>(T + c * M)[lane];
-        float *dst = S + ((long long)bh * nt + q0 + c) * nt + kk;
-        if (vec && kk + 3 < nt) {
-          *reinterpret_cast<float4 *>(dst) = val;
-        } else {
-          if (kk < nt) dst[0] = val.x;
-          if (kk + 1 < nt) dst[1] = val.y;
-          if (kk + 2 < nt) dst[2] = val.z;
-          if (kk + 3 < nt) dst[3] = val.w;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        uint32_t v[NH];
+        tc::tmem_ld64(tmem + lane_base + (uint32_t)(buf * N + half * NH), v);
+        if (half == 1) {
+          tc::fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(t_empty + buf);
         }
+        // transposed tile T[query][key] (consecutive threads, consecutive keys)
+#pragma unroll
+        for (int c = 0; c < NH; ++c) T[c * M + tid] = __uint_as_float(v[c]) * scale;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        // each warp writes query rows warp, warp + 4, ...: 128 keys per row,
+        // four per lane
+        const int q0 = q_begin + j * N + half * NH;
+        for (int c = warp; c < NH && q0 + c < q_end; c += 4) {
+          const float4 val = reinterpret_cast<const float4 *>(T + c * M)[lane];
+          float *dst = S + ((long long)bh * nt + q0 + c) * nt + kk;
+          if (vec && kk + 3 < nt) {
+            *reinterpret_cast<float4 *>(dst) = val;
+          } else {
+            if (kk < nt) dst[0] = val.x;
+            if (kk + 1 < nt) dst[1] = val.y;
+            if (kk + 2 < nt) dst[2] = val.z;
+            if (kk + 3 < nt) dst[3] = val.w;
+          }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
     }
   }
   tc::fence_before();
