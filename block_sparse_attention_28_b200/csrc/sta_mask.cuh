@@ -294,8 +294,10 @@ __device__ void radix_level(const float *row, int nt, unsigned int target, bool 
 // per-warp histograms (if use_scores), then the window tables.
 // SEL_SELECT reads its rows from P_in: scores to be softmaxed when p_logits
 // (the tensor-core score pass), else block scores clamped to [0, 1].
+// SEL_SELECT CTAs are capped at four per SM by shared memory; saying so lets
+// the compiler use the registers that occupancy leaves (56 instead of 40).
 template <int D, int QB, int MODE>
-__global__ void __launch_bounds__(SEL_THREADS)
+__global__ void __launch_bounds__(SEL_THREADS, MODE == SEL_SELECT ? 4 : 1)
 score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar, int heads, Geo g,
                     float scale, float top_p, int k_min, int use_scores,
                     const int *__restrict__ windows, int G, GroupLo glo,
