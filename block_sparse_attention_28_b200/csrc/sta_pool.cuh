@@ -15,8 +15,8 @@
 //               rounded once to fp32; with qlo / klo given the mean x is stored
 //               split for the tensor-core scores, tf32(x) in qbar / kbar and
 //               tf32(x - tf32(x)) in qlo / klo
-// The ring keeps up to 192 KB of loads in flight per SM, which is what a
-// stream from HBM needs, without a thread per outstanding load.
+// The ring keeps up to 192 KB of loads in flight per SM without a thread per
+// outstanding load.
 // Every wait is bounded; on a timeout the kernel records DEV_ERR_TIMEOUT,
 // waits (bounded) for its own copies in flight and returns.
 #pragma once

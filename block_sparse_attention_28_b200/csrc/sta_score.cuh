@@ -5,8 +5,9 @@
 // (an fp32 mean) is stored as two tf32 parts, hi = tf32(x) and
 // lo = tf32(x - hi), so x = hi + lo + r with |r| <= 2^-22 |x|, and each term
 // q.k is taken as lo_q hi_k + hi_q lo_k + hi_q hi_k (the dropped lo_q lo_k is
-// below 2^-22 |q k|). The small products go into the accumulator first.
-// pool_kernel writes the parts.
+// below 2^-22 |q k|). Within each 32-wide chunk of d the two small
+// products go into the accumulator before hi_q hi_k. The pooling kernels
+// write the parts.
 //
 // One CTA per (128 key tiles, range of query tiles, b*heads + h); 192 threads:
 //   warp 4     TMA producer: first the CTA's key block (hi and lo parts) into
