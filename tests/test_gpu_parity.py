@@ -108,10 +108,10 @@ def _assert_near_threshold(own, gpu, p_ref, bound, top_p):
 
 
 def _check_mask(sta, gp, qt, kt, B, Hh, d, T, H, W, top_p, k_min, use_scores, win, group_lo,
-                check_probs=True):
+                check_probs=True, sm_scale=0.0):
     g = sta.grid(T, H, W)
     win_d = torch.from_numpy(win).cuda() if win is not None else None
-    params = sta.mask_params(top_p, k_min, use_scores, 0.0, group_lo, win_d)
+    params = sta.mask_params(top_p, k_min, use_scores, sm_scale, group_lo, win_d)
     bufs = gp.build(qt, kt, B, Hh, d, g, params)
     torch.cuda.synchronize()
     assert sta.sta_get_device_error() == sta.STA_OK
@@ -122,7 +122,7 @@ def _check_mask(sta, gp, qt, kt, B, Hh, d, T, H, W, top_p, k_min, use_scores, wi
     if use_scores:
         mask |= O.select(probs, top_p, k_min)
         if check_probs:
-            scale = 1.0 / math.sqrt(d)
+            scale = sm_scale if sm_scale != 0.0 else 1.0 / math.sqrt(d)
             qb, kb = O.pool(gp.to_np64(qt), T, H, W), O.pool(gp.to_np64(kt), T, H, W)
             _, p_ref = O.block_scores(qb, kb, scale)
             bound = gp.prob_bound(qb, kb, scale, p_ref)
@@ -183,6 +183,18 @@ def test_build_mask_several_key_blocks(sta, gp, d):
     rng = np.random.default_rng(d)
     win = rng.integers(-1, 3, size=(Hh, 3, 4)).astype(np.int32)
     _check_mask(sta, gp, qt, kt, B, Hh, d, T, H, W, 0.9, 4, True, win, (0, 1, 3))
+
+
+@pytest.mark.parametrize("sm_scale", [0.05, 0.5])
+def test_build_mask_custom_scale(sta, gp, sm_scale):
+    """A caller-given score scale reaches the pooled scores (tensor-core
+    layout): P within its bound of the oracle's at that scale, CSR equal to
+    the oracle's selection on the GPU's P."""
+    T, H, W, Hh, B, d = 3, 19, 37, 3, 2, 128
+    q, k, _ = _structured(T, H, W, Hh, d, seed=17, B=B)
+    g = sta.grid(T, H, W)
+    qt, kt = gp.reorder(q, B, Hh, d, g), gp.reorder(k, B, Hh, d, g)
+    _check_mask(sta, gp, qt, kt, B, Hh, d, T, H, W, 0.8, 2, True, None, (0,), sm_scale=sm_scale)
 
 
 def test_build_mask_window_only_full_480p(sta, gp):
