@@ -10,6 +10,7 @@ raster order happen inside the kernels' loads and stores).
   python bench.py --search-curve [--workload NAME]   (window search, recall vs density)
   python bench.py --sweep                              (every layer of the workload table)
   python bench.py --l2-probe                           (the attention's tile-load stream alone)
+  python bench.py --mma-probe                          (cycles per tensor-core MMA by width)
 
 Rank 0 prints one JSON line. Under torchrun every rank runs its own layer
 (independent problems, no collective on the data path: weak scaling); the
@@ -654,6 +655,25 @@ def l2_probe(sta, dev, iters=2000):
     return rows
 
 
+def mma_probe(sta, iters=4096):
+    """Cost of one tcgen05.mma (bf16, M = 128, K = 16) of width N = 64, 128,
+    256, with A from shared memory or from tensor memory: SM cycles per MMA
+    (mean over the SMs, one CTA each) and multiply-adds per clock against the
+    SM's dense peak of 4096."""
+    rows = []
+    for a_tmem in (False, True):
+        for n in (64, 128, 256):
+            sta.sta_selftest_mma_rate(n, a_tmem, 64)  # warm-up
+            cyc = sta.sta_selftest_mma_rate(n, a_tmem, iters).double()
+            per = float(cyc.mean()) / iters
+            line = {"n": n, "a_operand": "tmem" if a_tmem else "smem", "cycles_per_mma": per,
+                    "mac_per_clock": 128 * n * 16 / per, "of_peak": 128 * n * 16 / per / 4096}
+            rows.append(line)
+            print(json.dumps(line), flush=True)
+    assert sta.sta_get_device_error() == sta.STA_OK
+    return rows
+
+
 def cpu_oracle_sample(cfg, layer, budget_s, rows_per_head=8, max_heads=None):
     """Time the oracle (as it stands) on a bounded sample of the same layer:
     for sampled heads, its reorder, pooling, scores, selection and windows
@@ -757,6 +777,8 @@ def main():
                     help="time every layer of the workload table (one JSON line per row) and exit")
     ap.add_argument("--l2-probe", action="store_true",
                     help="rate of the attention's 16 KB TMA tile loads on their own, then exit")
+    ap.add_argument("--mma-probe", action="store_true",
+                    help="cycles per tensor-core MMA (bf16, M=128, K=16) for N = 64 / 128 / 256")
     ap.add_argument("--search-curve", action="store_true",
                     help="print the recall-target vs density curve of the window search and exit")
     args = ap.parse_args()
@@ -775,6 +797,10 @@ def main():
     if args.l2_probe:
         if rank == 0:
             l2_probe(sta, dev)
+        return
+    if args.mma_probe:
+        if rank == 0:
+            mma_probe(sta)
         return
     if args.sweep:
         if rank == 0:

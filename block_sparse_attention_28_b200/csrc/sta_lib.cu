@@ -244,6 +244,67 @@ __global__ void __launch_bounds__(32) tma_stream_kernel(const __grid_constant__ 
   }
 }
 
+// Back-to-back tcgen05.mma (kind::f16, bf16 x bf16 -> fp32, M = 128, K = 16)
+// of one N, A from shared memory (A_TMEM = false) or from TMEM, B from shared
+// memory, all into one accumulator; the operands are zeros (their values do
+// not change the rate). One thread issues `iters` MMAs and waits for them;
+// cycles[blockIdx.x] gets the SM cycles from the first issue to completion.
+// One CTA per SM: the dynamic shared memory asked for keeps two off one SM.
+constexpr int MMA_RATE_SMEM = 120 * 1024;
+template <int N, bool A_TMEM>
+__global__ void __launch_bounds__(128, 1) mma_rate_kernel(long long *cycles, int iters) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+  __shared__ uint64_t bar;
+  __shared__ uint32_t taddr;
+  const int tid = threadIdx.x;
+  // A: 128 rows x 128 B; B: N rows x 128 B (K-major, 128-byte swizzle)
+  for (int i = tid; i < (16384 + N * 128) / 16; i += 128) reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0, 0, 0, 0);
+  if (tid == 0) {
+    tc::mbar_init(&bar, 1);
+    tc::fence_barrier_init();
+  }
+  if (tid < 32) {
+    tc::tmem_alloc(&taddr, 512);
+    tc::tmem_relinquish();
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // zeros visible to the tensor core
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tm = taddr;
+  if (tid == 0) {
+    const uint32_t sa = tc::smem_u32(smem), sb = sa + 16384;
+    constexpr uint32_t idesc = tc::idesc_bf16(128, N, false);
+    const long long t0 = clock64();
+    for (int i = 0; i < iters; ++i) {
+      const uint32_t koff = (uint32_t)((i & 3) * 32);  // the four K = 16 steps of a 128-byte row
+      if (A_TMEM)
+        tc::mma_ts(tm, tm + 256u + (uint32_t)((i & 3) * 8), tc::desc_k_sw128(sb + koff), idesc, i > 0 ? 1u : 0u);
+      else
+        tc::mma_ss(tm, tc::desc_k_sw128(sa + koff), tc::desc_k_sw128(sb + koff), idesc, i > 0 ? 1u : 0u);
+    }
+    tc::mma_commit(&bar);
+    const bool ok = tc::mbar_wait(&bar, 0, nullptr, 2000000000LL);
+    cycles[blockIdx.x] = ok ? clock64() - t0 : -1;
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (tid < 32) {
+    tc::fence_after();
+    tc::tmem_dealloc(tm, 512);
+  }
+}
+
+template <int N, bool A_TMEM>
+sta_status launch_mma_rate(long long *cycles, int iters, int sms, cudaStream_t s) {
+  auto kern = mma_rate_kernel<N, A_TMEM>;
+  STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MMA_RATE_SMEM));
+  kern<<<(unsigned)sms, 128, MMA_RATE_SMEM, s>>>(cycles, iters);
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
+}
+
 // One thread waits, with the pipeline's bounded wait, on a barrier that
 // expects one arrival that never comes.
 __global__ void selftest_wait_kernel(long long limit) {
@@ -652,6 +713,24 @@ sta_status sta_selftest_tma_stream(const void *buf, size_t bytes, int32_t ctas_p
   tma_stream_kernel<<<(unsigned)(sms * ctas_per_sm), 32, smem, s>>>(tm, (int)tiles, slots, iters);
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
+}
+
+sta_status sta_selftest_mma_rate(int32_t n, int32_t a_in_tmem, int32_t iters, int64_t *cycles,
+                                 sta_stream_t stream) {
+  if ((n != 64 && n != 128 && n != 256) || iters < 1 || iters > (1 << 20) || cycles == nullptr)
+    return STA_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return STA_ERR_UNSUPPORTED;
+  const int sms = sm_count();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  long long *out = reinterpret_cast<long long *>(cycles);
+  if (a_in_tmem) {
+    if (n == 64) return launch_mma_rate<64, true>(out, iters, sms, s);
+    if (n == 128) return launch_mma_rate<128, true>(out, iters, sms, s);
+    return launch_mma_rate<256, true>(out, iters, sms, s);
+  }
+  if (n == 64) return launch_mma_rate<64, false>(out, iters, sms, s);
+  if (n == 128) return launch_mma_rate<128, false>(out, iters, sms, s);
+  return launch_mma_rate<256, false>(out, iters, sms, s);
 }
 
 sta_status sta_selftest_wait_timeout(int64_t limit_cycles, sta_stream_t stream) {

@@ -302,6 +302,20 @@ sta_status sta_selftest_wait_timeout(int64_t limit_cycles, sta_stream_t stream);
 sta_status sta_selftest_tma_stream(const void *buf, size_t bytes, int32_t ctas_per_sm, int32_t slots,
                                    int32_t iters, sta_stream_t stream);
 
+/* sta_selftest_mma_rate -- the tensor-core rate of one MMA shape on its own:
+ * one CTA per SM of the current device issues `iters` (1..2^20) back-to-back
+ * tcgen05.mma of kind::f16 (bf16 x bf16 -> fp32) with M = 128, K = 16 and
+ * N = n (64, 128 or 256), A from shared memory (a_in_tmem = 0) or from
+ * tensor memory (a_in_tmem != 0), B from shared memory, into one
+ * accumulator. cycles: device int64 array with one entry per SM of the
+ * current device, written with each CTA's SM cycles from the first issue to
+ * completion (-1 if its bounded wait gave up, also recorded as
+ * STA_ERR_TIMEOUT). cycles / iters is the cost of one MMA; 128 * n * 16 /
+ * that is the multiply-adds per clock (4096 is the dense bf16 peak of an SM).
+ * Arguments out of range give STA_ERR_INVALID_ARG before anything runs. */
+sta_status sta_selftest_mma_rate(int32_t n, int32_t a_in_tmem, int32_t iters, int64_t *cycles,
+                                 sta_stream_t stream);
+
 /* Reads and clears the device error word of the current device after
  * synchronising `stream`. STA_OK if no device-side fault was recorded. */
 sta_status sta_get_device_error(sta_stream_t stream);

@@ -92,6 +92,13 @@ def test_selftest_limit_is_checked_on_the_host(sta):
     assert sta._lib.sta_selftest_wait_timeout(3_000_000_000, None) == sta.STA_ERR_INVALID_ARG
 
 
+def test_mma_rate_arguments_are_checked_on_the_host(sta):
+    buf = ctypes.c_int64(0)
+    for n, iters in ((96, 10), (64, 0), (128, (1 << 20) + 1)):
+        assert sta._lib.sta_selftest_mma_rate(n, 0, iters, ctypes.byref(buf), None) == sta.STA_ERR_INVALID_ARG
+    assert sta._lib.sta_selftest_mma_rate(64, 0, 10, None, None) == sta.STA_ERR_INVALID_ARG
+
+
 def test_binding_mirrors_the_noalloc_array_size(sta):
     m = re.search(r"#define\s+STA_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", open(HEADER).read())
     assert m, "STA_NOALLOC_SCRATCH_BYTES not found in the header"

@@ -1012,3 +1012,21 @@ def test_bounded_wait_reports_timeout_and_context_survives(sta, gp):
     assert sta.sta_get_device_error() == sta.STA_ERR_TIMEOUT
     assert sta.sta_get_device_error() == sta.STA_OK
     test_attn_tiny_config(sta, gp)  # a full attention call still runs and matches
+
+
+@pytest.mark.parametrize("a_tmem", [False, True])
+def test_mma_rate_selftest(sta, a_tmem):
+    """The MMA-rate self-test runs on every SM and reports a cost per MMA that
+    respects the tensor core's dense peak (4096 bf16 multiply-adds per SM per
+    clock): no width is measured faster than that bound."""
+    iters = 1024
+    for n in (64, 128, 256):
+        cyc = sta.sta_selftest_mma_rate(n, a_tmem, iters)
+        torch.cuda.synchronize()
+        assert sta.sta_get_device_error() == sta.STA_OK
+        assert cyc.numel() == torch.cuda.get_device_properties(0).multi_processor_count
+        assert bool((cyc > 0).all())
+        per = cyc.double() / iters
+        floor = 128 * n * 16 / 4096  # cycles of the multiply-adds alone at the peak
+        assert float(per.min()) >= 0.98 * floor
+        assert float(per.max()) < 20 * floor
