@@ -655,6 +655,21 @@ def l2_probe(sta, dev, iters=2000):
     return rows
 
 
+def build_roofline(layer, build_ms, peaks):
+    """The mask build against HBM: algorithmic bytes = the real rows of Q and
+    K read (when scores are on) + the CSR written (col_idx and row_ptr), over
+    the build's CUDA-event time, as a fraction of the measured copy
+    bandwidth. The select pass is instruction-bound, so the fraction is low
+    by design of the work, not by wasted traffic."""
+    c = layer.cfg
+    raster = c.B * c.L * c.heads * c.d * 2
+    nbytes = (2 * raster if c.use_scores else 0) + 4 * layer.kept_pairs() + 4 * (layer.B * layer.Hh * layer.nt + 1)
+    achieved = nbytes / (build_ms * 1e-3) / 1e9
+    peak = float(peaks.get("hbm_gbs", 6650.0))
+    return {"bound": "hbm", "algorithmic_bytes": nbytes, "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "kernels": "pool_tma, score_tc, score_select, scan, fill"}
+
+
 def mma_probe(sta, iters=4096):
     """Cost of one tcgen05.mma (bf16, M = 128, K = 16) of width N = 64, 128,
     256, with A from shared memory or from tensor memory: SM cycles per MMA
@@ -919,6 +934,7 @@ def main():
             },
             "ms_per_layer": build_ms + attn_ms,
             "ms_breakdown": {"build_mask": build_ms, "attn_fwd": attn_ms},
+            "build_roofline": build_roofline(layer, build_ms, peaks),
             "attn_tflops": attn_tflops,
             "attn_frac_of_peak": attn_tflops / peak,
             "pairing_efficiency": eff,

@@ -45,3 +45,6 @@ def test_bench_json_line():
         assert len(ks) == 6 and all(k.startswith("sta::") for k in ks), ks
         assert sum("attn_fwd_kernel" in k for k in ks) == 1 and sum("score_tc_kernel" in k for k in ks) == 1
     assert d["clocks"]["sm_mhz"] is not None and isinstance(d["clocks"]["reasons"], list)
+    b = d["build_roofline"]
+    assert b["bound"] == "hbm" and b["unit"] == "GB/s" and 0 < b["frac"] < 1.5
+    assert abs(b["frac"] - b["achieved"] / b["peak"]) < 1e-9
