@@ -1,15 +1,17 @@
 // Recall-driven dual-window search (Compact Attention Fig. 3: the offline
-// search shrinks the dual windows under a recall target tau and a cost weight
-// lambda; Fig. 4: it starts from full coverage in every temporal-distance
-// group). One CTA per (b*heads + h) runs the whole greedy in shared memory,
-// with no round trip to the host:
+// search shrinks the dual windows under the recall (tau) and cost (lambda)
+// constraints; Fig. 4: it starts from full coverage in every
+// temporal-distance group). One CTA per (b*heads + h) runs the whole greedy in
+// shared memory, with no round trip to the host:
 //   masses  w = floor(min(max(m, 0), 1) * 2^24) (exact integer sums);
 //   start   (ry1, rx1, ry2, rx2) = (NH-1, NW-1, NH-1, NW-1) in every group;
 //   moves   per group g: ry1-1, rx1-1, ry2-1, rx2-1, (ry1-1, ry2-1),
 //           (rx1-1, rx2-1); an extent never goes below -1;
-//   step    among moves that uncover >= 1 pair and keep
-//           covered >= ceil(double(tau) * W), the largest
-//           J = removed / Nt^2 - lambda * lost / W, ties to the lowest index
+//   value   J = removed / Nt^2 - lambda * lost / W (double, no contraction);
+//   admit   covered - lost >= ceil(double(tau) * W) and J >= 0; a move that
+//           uncovers nothing (one window shrunk inside the other) has J = 0,
+//           which is how the two windows, equal at the start, come apart;
+//   step    the admissible move with the largest J, ties to the lowest index
 //           g*6 + m; stop when none is left.
 #pragma once
 #include "sta_common.cuh"
@@ -163,10 +165,13 @@ search_windows_kernel(const float *__restrict__ mass, Geo g, int G, GroupLo glo,
           if (!search_move_valid(mi, cur)) continue;
           const unsigned int removed = mv_removed[gi][mi];
           const unsigned long long l = mv_lost[gi][mi];
-          if (removed == 0u || covered - l < thr || l > covered) continue;
+          if (l > covered || covered - l < thr) continue;  // recall constraint
           const double a = (double)removed / (double)((long long)nt * nt);
           const double b = total ? (double)l / (double)total : 0.0;
-          const double J = a - (double)lambda * b;
+          // a - lambda * b with two roundings (a fused multiply-add could
+          // change the sign of a J near zero)
+          const double J = __dsub_rn(a, __dmul_rn((double)lambda, b));
+          if (J < 0.0) continue;  // cost constraint
           if (best < 0 || J > bestJ) {
             best = gi * SEARCH_MOVES + mi;
             bestJ = J;

@@ -19,7 +19,7 @@ Sources (pages on block-sparse attention for video diffusion transformers):
   * Rectified SpaAttn (abstract): rectified attention, skipped tiles
     recovered from pooled keys and values (reading stated in the module).
 
-Parity pins: every function here is checked in tests/test_oracle_*.py
+Parity pins: every function here is checked in tests/test_oracle.py
 against closed forms, textbook routines (torch SDPA in fp64, scipy
 softmax, stable argsort) or brute force; none of the pages prints a worked
 numeric example for this path, so no pin comes from a printed value.

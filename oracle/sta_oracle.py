@@ -437,9 +437,10 @@ def block_mass(q_tiled, k_tiled, lse, row_ptr, col_idx, T, H, W, sm_scale, rows)
 
 # --------------------------------------------------------------------------
 # Recall-driven window search (Compact Attention Fig. 3: offline search that
-# iteratively shrinks the dual windows under a recall target tau and a cost
-# weight lambda; Fig. 4: it starts from full coverage in every
-# temporal-distance group; Fig. 5(c): recall target vs achieved sparsity).
+# iteratively shrinks the dual windows under the recall (tau) and cost
+# (lambda) constraints; Fig. 4: starting from full coverage in every
+# temporal-distance group, the dual windows are shrunk while the recall and
+# shrink-penalty constraints hold; Fig. 5(c): recall target vs sparsity).
 # Reading (the pages give no step rule):
 #   masses : exact block importances of one head [Nt, Nt] (e.g. from an
 #            LSE-cached dense step), as integers w = floor(min(max(m,0),1)*2^24);
@@ -447,16 +448,24 @@ def block_mass(q_tiled, k_tiled, lse, row_ptr, col_idx, T, H, W, sm_scale, rows)
 #   start  : (ry1, rx1, ry2, rx2) = (NH-1, NW-1, NH-1, NW-1) in every group;
 #   moves  : for each group g, in order: ry1-1, rx1-1, ry2-1, rx2-1,
 #            (ry1-1, ry2-1), (rx1-1, rx2-1); an extent never goes below -1;
-#   step   : among moves that uncover at least one pair and keep
-#            covered >= ceil(double(tau) * W), take the largest
-#            J = removed / Nt^2 - lambda * lost / W (double, in that order),
-#            ties to the lowest move index g*6 + m; stop when none is left.
+#   value  : J = removed / Nt^2 - lambda * lost / W (double, in that order),
+#            removed / lost = pairs / mass the move uncovers;
+#   admit  : covered - lost >= ceil(double(tau) * W)   (recall constraint)
+#            and J >= 0                                (cost constraint);
+#            a move that uncovers nothing (one window shrunk inside the
+#            other) is admissible with J = 0: it is how the two windows,
+#            equal at the start, come apart;
+#   step   : the admissible move with the largest J, ties to the lowest move
+#            index g*6 + m; stop when none is left (every move lowers an
+#            extent, so the search ends).
 # --------------------------------------------------------------------------
 SEARCH_MOVES = ((0,), (1,), (2,), (3,), (0, 2), (1, 3))
 
 
 def search_windows(mass, T, H, W, group_lo, tau, lam):
-    """Greedy window search for one head; returns (windows [G,4] int32, stats)."""
+    """Greedy window search for one head; returns (windows [G,4] int32, stats)
+    with stats = dict(recall, density, steps, covered, total, moves), moves
+    being the applied move indices g*6 + m in order."""
     m = np.clip(np.asarray(mass, dtype=np.float64), 0.0, 1.0)
     w = np.floor(m * MASS_ONE).astype(np.int64)
     total = int(w.sum())
@@ -468,7 +477,7 @@ def search_windows(mass, T, H, W, group_lo, tau, lam):
     lam = float(np.float32(lam))
     cur = window_mask(win[None], group_lo, T, H, W)[0]
     covered = int(w[cur].sum())
-    steps = 0
+    moves = []
     while True:
         best = None
         for g in range(G):
@@ -481,19 +490,19 @@ def search_windows(mass, T, H, W, group_lo, tau, lam):
                 new = window_mask(cand[None], group_lo, T, H, W)[0]
                 gone = cur & ~new
                 removed = int(gone.sum())
-                if removed == 0:
-                    continue
                 lost = int(w[gone].sum())
                 if covered - lost < thr:
                     continue
                 J = removed / float(nt * nt) - lam * (lost / float(total) if total else 0.0)
+                if J < 0.0:
+                    continue
                 if best is None or J > best[0]:
                     best = (J, g * 6 + mi, cand, new, lost)
         if best is None:
             break
-        _, _, win, cur, lost = best
+        _, idx, win, cur, lost = best
         covered -= lost
-        steps += 1
-    stats = dict(recall=covered / total if total else 1.0, density=float(cur.mean()), steps=steps,
-                 covered=covered, total=total)
+        moves.append(idx)
+    stats = dict(recall=covered / total if total else 1.0, density=float(cur.mean()), steps=len(moves),
+                 covered=covered, total=total, moves=moves)
     return win.astype(np.int32), stats

@@ -15,6 +15,9 @@ import scipy.special
 import torch
 
 import oracle as O
+from oracle import sta_oracle
+
+import _search_cases as SC
 
 RNG = np.random.default_rng(12345)
 
@@ -474,16 +477,71 @@ def _coverage(win, group_lo, T, H, W, mass):
     return m, int(w[m].sum()), int(w.sum())
 
 
+def _search_case_result(search, case):
+    T, H, W = case["grid"]
+    win, st = search(SC.mass(case), T, H, W, tuple(case["group_lo"]), case["tau"], case["lambda"])
+    nt = O.tile_grid(T, H, W)[2]
+    return dict(moves=list(st["moves"]), windows=win.tolist(), covered_units=st["covered"] / SC.UNIT,
+                total_units=st["total"] / SC.UNIT, pairs=round(st["density"] * nt * nt))
+
+
+def test_window_search_golden(golden_dir):
+    """Hand-derived move sequences (Compact Attention Figs. 3-4 as read): lambda
+    choosing the cheap move, the same masses at lambda = 0, tau stopping the
+    descent one move early, an exact tie of J across groups, and a cross grown
+    out of two full windows by moves that uncover nothing."""
+    for case in SC.load(golden_dir):
+        got = _search_case_result(O.search_windows, case)
+        assert got == {k: case[k] for k in SC.FIELDS}, (case["name"], got)
+
+
+# Each planted mistake is a plausible slip in the step rule; each must change
+# the outcome of at least one golden case.
+SEARCH_MUTANTS = {
+    "first admissible move instead of the best": ("if best is None or J > best[0]:", "if best is None:"),
+    "lambda term with the wrong sign": ("- lam * (lost", "+ lam * (lost"),
+    "ties to the highest index": ("J > best[0]", "J >= best[0]"),
+    "recall bound strict": ("if covered - lost < thr:", "if covered - lost <= thr:"),
+    "no cost constraint": ("if J < 0.0:", "if False:"),
+    "a move must uncover a pair": ("if covered - lost < thr:", "if removed == 0 or covered - lost < thr:"),
+    "lambda term dropped": ("- lam * (lost / float(total) if total else 0.0)", ""),
+    "removed pairs not normalised": ("removed / float(nt * nt)", "float(removed)"),
+}
+
+
+def _mutant(old, new):
+    import inspect
+
+    src = inspect.getsource(O.search_windows)
+    assert src.count(old) == 1, old
+    ns = dict(vars(sta_oracle))
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)
+    return ns["search_windows"]
+
+
+@pytest.mark.parametrize("name", sorted(SEARCH_MUTANTS))
+def test_window_search_planted_mistakes_fail_the_golden_cases(golden_dir, name):
+    search = _mutant(*SEARCH_MUTANTS[name])
+    wrong = 0
+    for case in SC.load(golden_dir):
+        wrong += _search_case_result(search, case) != {k: case[k] for k in SC.FIELDS}
+    assert wrong >= 1, name
+
+
 def test_window_search_keeps_everything_at_full_recall_with_dense_mass():
-    """tau = 1 and every pair carries mass: no pair can go, the windows stay full."""
+    """tau = 1 and every pair carries mass: no pair can go, so the mask stays
+    full; only the moves that uncover nothing run (the first window of every
+    group is switched off one extent at a time)."""
     rng = np.random.default_rng(1)
     T, H, W = 3, 24, 32
     nh, nw, nt, _ = O.tile_grid(T, H, W)
     mass = rng.random((nt, nt)) + 0.1
     mass /= mass.sum(1, keepdims=True)
     win, st = O.search_windows(mass, T, H, W, (0, 1), 1.0, 1.0)
-    assert st["steps"] == 0 and st["recall"] == 1.0 and st["density"] == 1.0
-    assert (win == np.array([nh - 1, nw - 1, nh - 1, nw - 1])).all()
+    assert st["recall"] == 1.0 and st["density"] == 1.0
+    assert (win == np.array([-1, -1, nh - 1, nw - 1])).all()
+    # group 0's ry1 steps first (index 0), then its rx1, then group 1's
+    assert st["moves"] == [0] * nh + [1] * nw + [6] * nh + [7] * nw
 
 
 def test_window_search_diagonal_mass_shrinks_to_the_own_tile():
@@ -504,14 +562,14 @@ def test_window_search_zero_target_removes_everything():
     nt = O.tile_grid(T, H, W)[2]
     mass = rng.random((nt, nt))
     win, st = O.search_windows(mass, T, H, W, (0, 1), 0.0, 0.0)
-    assert st["density"] == 0.0
-    assert (win == -1).any(axis=1).all() or (win[:, [0, 2]] == -1).all()
+    assert st["density"] == 0.0 and st["recall"] == 0.0
+    assert (win == -1).all()
 
 
 def test_window_search_result_is_feasible_and_locally_final():
     """On local-looking masses: the final recall (recomputed from the windows)
-    meets tau, and no single move of the move set uncovers a pair while still
-    meeting tau (checked by direct enumeration)."""
+    meets tau, and no single move of the move set meets both constraints
+    (recall >= tau and J >= 0), checked by direct enumeration."""
     T, H, W = 4, 24, 40
     nh, nw, nt, _ = O.tile_grid(T, H, W)
     idx = np.arange(nt)
@@ -520,7 +578,7 @@ def test_window_search_result_is_feasible_and_locally_final():
     mass = np.exp(-d2)
     mass /= mass.sum(1, keepdims=True)
     group_lo = (0, 1, 3)
-    for tau, lam in ((0.9, 1.0), (0.97, 0.5), (0.8, 2.0)):
+    for tau, lam in ((0.9, 1.0), (0.97, 0.5), (0.8, 2.0), (0.9, 0.0)):
         win, st = O.search_windows(mass, T, H, W, group_lo, tau, lam)
         m, cov, tot = _coverage(win, group_lo, T, H, W, mass)
         thr = math.ceil(float(np.float32(tau)) * tot)
@@ -534,7 +592,9 @@ def test_window_search_result_is_feasible_and_locally_final():
                 for e in ext:
                     cand[g, e] -= 1
                 m2, cov2, _ = _coverage(cand, group_lo, T, H, W, mass)
-                assert (m & ~m2).sum() == 0 or cov2 < thr
+                removed = int((m & ~m2).sum())
+                J = removed / float(nt * nt) - float(np.float32(lam)) * (cov - cov2) / float(tot)
+                assert cov2 < thr or J < 0.0, (tau, lam, g, ext)
 
 
 # ------------------------------------------- rectified attention (f4 reading)
