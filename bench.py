@@ -634,6 +634,8 @@ def l2_probe(sta, dev, iters=2000):
     """Rate of the attention kernel's load stream on its own (16 KB key-tile
     TMA loads at pseudo-random tiles), from an L2-resident 40 MB region and
     from a 4 GB region, at 1 and 2 CTAs per SM and 2 to 6 loads in flight."""
+    from block_sparse_attention_28_b200 import probe
+
     props = torch.cuda.get_device_properties(dev)
     rows = []
     for label, nbytes in (("L2-resident 40 MB", 40 << 20), ("4 GB (DRAM)", 4 << 30)):
@@ -642,8 +644,8 @@ def l2_probe(sta, dev, iters=2000):
             for slots in (2, 4, 6):
                 if slots * 16384 * cps > 200 * 1024:
                     continue
-                sta.sta_selftest_tma_stream(buf, cps, slots, 50)
-                ms = _median_ms(lambda: sta.sta_selftest_tma_stream(buf, cps, slots, iters), 5)
+                probe.sta_probe_tma_stream(buf, cps, slots, 50)
+                ms = _median_ms(lambda: probe.sta_probe_tma_stream(buf, cps, slots, iters), 5)
                 moved = props.multi_processor_count * cps * iters * 16384
                 line = {"source": label, "ctas_per_sm": cps, "loads_in_flight_per_cta": slots, "ms": ms,
                         "tb_per_s": moved / (ms * 1e-3) / 1e12}
@@ -651,7 +653,7 @@ def l2_probe(sta, dev, iters=2000):
                 print(json.dumps(line), flush=True)
         del buf
         torch.cuda.empty_cache()
-    assert sta.sta_get_device_error() == sta.STA_OK
+    assert probe.sta_probe_get_device_error() == sta.STA_OK
     return rows
 
 
@@ -675,17 +677,19 @@ def mma_probe(sta, iters=4096):
     256, with A from shared memory or from tensor memory: SM cycles per MMA
     (mean over the SMs, one CTA each) and multiply-adds per clock against the
     SM's dense peak of 4096."""
+    from block_sparse_attention_28_b200 import probe
+
     rows = []
     for a_tmem in (False, True):
         for n in (64, 128, 256):
-            sta.sta_selftest_mma_rate(n, a_tmem, 64)  # warm-up
-            cyc = sta.sta_selftest_mma_rate(n, a_tmem, iters).double()
+            probe.sta_probe_mma_rate(n, a_tmem, 64)  # warm-up
+            cyc = probe.sta_probe_mma_rate(n, a_tmem, iters).double()
             per = float(cyc.mean()) / iters
             line = {"n": n, "a_operand": "tmem" if a_tmem else "smem", "cycles_per_mma": per,
                     "mac_per_clock": 128 * n * 16 / per, "of_peak": 128 * n * 16 / per / 4096}
             rows.append(line)
             print(json.dumps(line), flush=True)
-    assert sta.sta_get_device_error() == sta.STA_OK
+    assert probe.sta_probe_get_device_error() == sta.STA_OK
     return rows
 
 

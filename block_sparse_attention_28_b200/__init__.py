@@ -89,10 +89,6 @@ _lib.sta_attn_fwd_block_mass.restype = ctypes.c_int
 _lib.sta_search_windows.argtypes = [_vp, _i32, _i32, Grid, _i32, ctypes.POINTER(ctypes.c_int32), _f32, _f32,
                                     _vp, _vp, _vp]
 _lib.sta_search_windows.restype = ctypes.c_int
-_lib.sta_selftest_tma_stream.argtypes = [_vp, _sz, _i32, _i32, _i32, _vp]
-_lib.sta_selftest_tma_stream.restype = ctypes.c_int
-_lib.sta_selftest_mma_rate.argtypes = [_i32, _i32, _i32, _vp, _vp]
-_lib.sta_selftest_mma_rate.restype = ctypes.c_int
 _lib.sta_selftest_wait_timeout.argtypes = [_i64, _vp]
 _lib.sta_selftest_wait_timeout.restype = ctypes.c_int
 _lib.sta_get_device_error.argtypes = [_vp]
@@ -245,23 +241,6 @@ def sta_search_windows(block_mass, B, heads, g, group_lo, tau, lam, windows, sta
     _check(_lib.sta_search_windows(_ptr(block_mass), B, heads, g, len(group_lo), lo, float(tau), float(lam),
                                    _ptr(windows), _ptr(stats), _stream(stream)),
            "sta_search_windows")
-
-
-def sta_selftest_tma_stream(buf, ctas_per_sm, slots, iters, stream=None):
-    _check(_lib.sta_selftest_tma_stream(_ptr(buf), buf.numel() * buf.element_size(), int(ctas_per_sm),
-                                        int(slots), int(iters), _stream(stream)),
-           "sta_selftest_tma_stream")
-
-
-def sta_selftest_mma_rate(n, a_in_tmem, iters, stream=None):
-    """SM cycles of `iters` back-to-back M=128, K=16 bf16 MMAs of width n on
-    every SM (one CTA each); returns a CPU int64 tensor, one entry per SM."""
-    dev = torch.device("cuda", torch.cuda.current_device())
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    cycles = torch.full((sms,), -2, dtype=torch.int64, device=dev)
-    _check(_lib.sta_selftest_mma_rate(int(n), 1 if a_in_tmem else 0, int(iters), _ptr(cycles), _stream(stream)),
-           "sta_selftest_mma_rate")
-    return cycles.cpu()
 
 
 def sta_selftest_wait_timeout(limit_cycles=2000000, stream=None):

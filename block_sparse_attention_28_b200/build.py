@@ -1,4 +1,5 @@
-"""Build libsta.so in-tree with nvcc for sm_100a.
+"""Build libsta.so (the product library) and libsta_probe.so (its measurement
+probes) in-tree with nvcc for sm_100a.
 
     python block_sparse_attention_28_b200/build.py [--force]
 
@@ -13,6 +14,9 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "csrc", "sta_lib.cu")
 OUT = os.path.join(HERE, "libsta.so")
+PROBE_SRC = os.path.join(HERE, "csrc", "sta_probe.cu")
+PROBE_OUT = os.path.join(HERE, "libsta_probe.so")
+TARGETS = ((SRC, OUT), (PROBE_SRC, PROBE_OUT))
 NVCC_FLAGS = [
     "-O3", "-std=c++17",
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -31,25 +35,29 @@ def _nvcc():
 
 def sources():
     d = os.path.join(HERE, "csrc")
+    inc = os.path.join(os.path.dirname(HERE), "include")
     return [os.path.join(d, f) for f in sorted(os.listdir(d)) if f.endswith((".cu", ".cuh"))] + [
-        os.path.join(os.path.dirname(HERE), "include", "sta.h")]
+        os.path.join(inc, f) for f in sorted(os.listdir(inc)) if f.endswith(".h")]
 
 
-def up_to_date():
-    if not os.path.exists(OUT):
+def up_to_date(out=OUT):
+    if not os.path.exists(out):
         return False
-    t = os.path.getmtime(OUT)
+    t = os.path.getmtime(out)
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
 def build(force=False, verbose=False):
-    if not force and up_to_date():
-        return OUT
-    cmd = [_nvcc(), *NVCC_FLAGS, "-o", OUT + ".tmp", SRC]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
-    os.replace(OUT + ".tmp", OUT)
+    """Compile every target that is missing or older than a source; returns
+    the path of libsta.so."""
+    for src, out in TARGETS:
+        if not force and up_to_date(out):
+            continue
+        cmd = [_nvcc(), *NVCC_FLAGS, "-o", out + ".tmp", src]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        subprocess.run(cmd, check=True)
+        os.replace(out + ".tmp", out)
     return OUT
 
 

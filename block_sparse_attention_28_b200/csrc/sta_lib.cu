@@ -7,6 +7,7 @@
 
 #include "sta_attn.cuh"
 #include "sta_common.cuh"
+#include "sta_host.cuh"
 #include "sta_mask.cuh"
 #include "sta_pool.cuh"
 #include "sta_reorder.cuh"
@@ -84,37 +85,6 @@ size_t select_smem(int d, const Geo &g, bool use_scores, int qb = SEL_QB, int mo
 
 constexpr size_t MAX_DYN_SMEM = 227 * 1024;
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// [rows, d] bf16 row-major; box = 64 rows x 64 elements (128 B), 128 B swizzle.
-bool make_tile_map(CUtensorMap *map, const void *base, unsigned long long rows, int d) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-  cuuint32_t box[2] = {64, 64};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Raster [B, L, heads, d] bf16 as the 5D tensor (d, heads, W, H, B*T): a box
 // of 64 d-values x 1 head x 8 columns x 8 rows x 1 frame is one token tile
 // (zero-filled beyond the grid edge), 128 B swizzle.
@@ -147,13 +117,6 @@ bool make_raster_pool_map(CUtensorMap *map, const void *base, const Geo &g, int 
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return 148;
-  return n > 0 ? n : 148;
 }
 
 // Pooled rows [bh, Nt, d] fp32 as a 3D tensor (d, Nt, bh); a box is 32 d-values
@@ -193,114 +156,6 @@ sta_status launch_scores_tc(const float *qhi, const float *qlo, const float *khi
   parts = (qblocks + per_part - 1) / per_part;  // no empty range
   dim3 grid((unsigned)kblocks, (unsigned)parts, (unsigned)bh);
   kern<<<grid, score::NUM_THREADS, smem, s>>>(m_khi, m_klo, m_qhi, m_qlo, S, g.Nt, scale, per_part * score::N);
-  STA_CUDA_TRY(cudaGetLastError());
-  return STA_OK;
-}
-
-bool device_is_sm100() {
-  int dev = 0, major = 0, minor = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return false;
-  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return false;
-  return major == 10 && minor == 0;
-}
-
-// The attention kernel's load stream without its compute: one thread per CTA
-// keeps `slots` 16 KB key-tile loads (two 64x64 bf16 boxes, 128 B swizzle,
-// as the kernel issues them) in flight from `tiles` tiles of buf, at
-// pseudo-random tile indices, for `iters` loads. Timed by the caller; it
-// gives the L2-to-SM rate TMA reaches on this GPU at a given depth.
-constexpr int STREAM_MAX_SLOTS = 6;
-__global__ void __launch_bounds__(32) tma_stream_kernel(const __grid_constant__ CUtensorMap tm, int tiles,
-                                                        int slots, int iters) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + slots * 16384);
-  if (threadIdx.x != 0) return;
-  for (int sl = 0; sl < slots; ++sl) tc::mbar_init(bar + sl, 1);
-  tc::fence_barrier_init();
-  uint32_t seed = blockIdx.x * 2654435761u + 12345u;
-  auto issue = [&](int sl) {
-    seed = seed * 1664525u + 1013904223u;
-    const int tile = (int)(seed % (uint32_t)tiles);
-    tc::mbar_expect_tx(bar + sl, 16384);
-    tc::tma_load_2d(tc::smem_u32(smem + sl * 16384), &tm, bar + sl, 0, tile * 64);
-    tc::tma_load_2d(tc::smem_u32(smem + sl * 16384 + 8192), &tm, bar + sl, 64, tile * 64);
-  };
-  int issued = 0;
-  for (; issued < slots && issued < iters; ++issued) issue(issued);
-  for (int i = 0; i < iters; ++i) {
-    const int sl = i % slots;
-    // spin without a suspend hint, so that the wait adds no wake-up delay to
-    // the rate being measured; bounded, then recorded like the pipeline waits
-    bool ok = false;
-    for (long long spin = 0; spin < 100000000LL && !ok; ++spin) ok = tc::mbar_try_wait(bar + sl, (i / slots) & 1);
-    if (!ok) {
-      record_error(DEV_ERR_TIMEOUT);
-      for (int j = i + 1; j < issued; ++j) tc::mbar_wait(bar + j % slots, (j / slots) & 1, nullptr, 200000000LL);
-      return;
-    }
-    if (issued < iters) issue(issued++ % slots);
-  }
-}
-
-// Back-to-back tcgen05.mma (kind::f16, bf16 x bf16 -> fp32, M = 128, K = 16)
-// of one N, A from shared memory (A_TMEM = false) or from TMEM, B from shared
-// memory, all into one accumulator; the operands are zeros (their values do
-// not change the rate). One thread issues `iters` MMAs and waits for them;
-// cycles[blockIdx.x] gets the SM cycles from the first issue to completion.
-// One CTA per SM: the dynamic shared memory asked for keeps two off one SM.
-constexpr int MMA_RATE_SMEM = 120 * 1024;
-template <int N, bool A_TMEM>
-__global__ void __launch_bounds__(128, 1) mma_rate_kernel(long long *cycles, int iters) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
-  __shared__ uint64_t bar;
-  __shared__ uint32_t taddr;
-  const int tid = threadIdx.x;
-  // A: 128 rows x 128 B; B: N rows x 128 B (K-major, 128-byte swizzle)
-  for (int i = tid; i < (16384 + N * 128) / 16; i += 128) reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0, 0, 0, 0);
-  if (tid == 0) {
-    tc::mbar_init(&bar, 1);
-    tc::fence_barrier_init();
-  }
-  if (tid < 32) {
-    tc::tmem_alloc(&taddr, 512);
-    tc::tmem_relinquish();
-  }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // zeros visible to the tensor core
-  tc::fence_before();
-  __syncthreads();
-  tc::fence_after();
-  const uint32_t tm = taddr;
-  if (tid == 0) {
-    const uint32_t sa = tc::smem_u32(smem), sb = sa + 16384;
-    constexpr uint32_t idesc = tc::idesc_bf16(128, N, false);
-    const long long t0 = clock64();
-    for (int i = 0; i < iters; ++i) {
-      const uint32_t koff = (uint32_t)((i & 3) * 32);  // the four K = 16 steps of a 128-byte row
-      if (A_TMEM)
-        tc::mma_ts(tm, tm + 256u + (uint32_t)((i & 3) * 8), tc::desc_k_sw128(sb + koff), idesc, i > 0 ? 1u : 0u);
-      else
-        tc::mma_ss(tm, tc::desc_k_sw128(sa + koff), tc::desc_k_sw128(sb + koff), idesc, i > 0 ? 1u : 0u);
-    }
-    tc::mma_commit(&bar);
-    const bool ok = tc::mbar_wait(&bar, 0, nullptr, 2000000000LL);
-    cycles[blockIdx.x] = ok ? clock64() - t0 : -1;
-  }
-  tc::fence_before();
-  __syncthreads();
-  if (tid < 32) {
-    tc::fence_after();
-    tc::tmem_dealloc(tm, 512);
-  }
-}
-
-template <int N, bool A_TMEM>
-sta_status launch_mma_rate(long long *cycles, int iters, int sms, cudaStream_t s) {
-  auto kern = mma_rate_kernel<N, A_TMEM>;
-  STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MMA_RATE_SMEM));
-  kern<<<(unsigned)sms, 128, MMA_RATE_SMEM, s>>>(cycles, iters);
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }
@@ -690,49 +545,6 @@ sta_status sta_search_windows(const float *block_mass, int32_t B, int32_t heads,
   return STA_OK;
 }
 
-sta_status sta_selftest_tma_stream(const void *buf, size_t bytes, int32_t ctas_per_sm, int32_t slots,
-                                   int32_t iters, sta_stream_t stream) {
-  if (buf == nullptr || (reinterpret_cast<uintptr_t>(buf) & 15u) != 0 || bytes < 16384) return STA_ERR_INVALID_ARG;
-  if (ctas_per_sm < 1 || ctas_per_sm > 8 || slots < 1 || slots > STREAM_MAX_SLOTS || iters < 1 ||
-      (long long)slots * 16384 * ctas_per_sm > 200 * 1024)
-    return STA_ERR_INVALID_ARG;
-  if (!device_is_sm100()) return STA_ERR_UNSUPPORTED;
-  const long long tiles = (long long)(bytes / 16384);
-  if (tiles * 64 >= (1LL << 31)) return STA_ERR_UNSUPPORTED;
-  CUtensorMap tm;
-  if (!make_tile_map(&tm, buf, (unsigned long long)tiles * 64, 128)) return STA_ERR_CUDA;
-  int dev = 0, sms = 0;
-  STA_CUDA_TRY(cudaGetDevice(&dev));
-  STA_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  const size_t smem = (size_t)slots * 16384 + 64 + 1024;
-  STA_CUDA_TRY(cudaFuncSetAttribute(tma_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)((size_t)STREAM_MAX_SLOTS * 16384 + 64 + 1024)));
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // ctas_per_sm CTAs per SM through the grid size; they fit on an SM at once
-  // (checked above)
-  tma_stream_kernel<<<(unsigned)(sms * ctas_per_sm), 32, smem, s>>>(tm, (int)tiles, slots, iters);
-  STA_CUDA_TRY(cudaGetLastError());
-  return STA_OK;
-}
-
-sta_status sta_selftest_mma_rate(int32_t n, int32_t a_in_tmem, int32_t iters, int64_t *cycles,
-                                 sta_stream_t stream) {
-  if ((n != 64 && n != 128 && n != 256) || iters < 1 || iters > (1 << 20) || cycles == nullptr)
-    return STA_ERR_INVALID_ARG;
-  if (!device_is_sm100()) return STA_ERR_UNSUPPORTED;
-  const int sms = sm_count();
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  long long *out = reinterpret_cast<long long *>(cycles);
-  if (a_in_tmem) {
-    if (n == 64) return launch_mma_rate<64, true>(out, iters, sms, s);
-    if (n == 128) return launch_mma_rate<128, true>(out, iters, sms, s);
-    return launch_mma_rate<256, true>(out, iters, sms, s);
-  }
-  if (n == 64) return launch_mma_rate<64, false>(out, iters, sms, s);
-  if (n == 128) return launch_mma_rate<128, false>(out, iters, sms, s);
-  return launch_mma_rate<256, false>(out, iters, sms, s);
-}
-
 sta_status sta_selftest_wait_timeout(int64_t limit_cycles, sta_stream_t stream) {
   if (limit_cycles < 1000 || limit_cycles > 2000000000LL) return STA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -771,25 +583,60 @@ const char *sta_status_string(sta_status s) {
 // ---------------------------------------------------------------------------
 // Allocation-free mask build: the workspace is this static device array.
 // Host code must not hand the array's name to a kernel (on the host it is only
-// a stand-in); its device address is looked up once per device with
-// cudaGetSymbolAddress and cached.
+// a stand-in); its device address is looked up with cudaGetSymbolAddress on
+// the first call on a device and cached together with the id of the device's
+// current context. A later call that finds another context current (e.g. the
+// primary context was reset and re-created, which reloads the module at a new
+// address) looks the address up again.
 namespace {
 
 constexpr int NOALLOC_MAX_DEVICES = 64;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[STA_NOALLOC_SCRATCH_BYTES];
 std::mutex g_noalloc_mutex;
 void *g_noalloc_addr[NOALLOC_MAX_DEVICES] = {};
+unsigned long long g_noalloc_ctx[NOALLOC_MAX_DEVICES] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+// Unique id of the calling thread's current context, 0 if there is none or
+// the driver cannot tell.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    looked_up = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0ull;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0ull;
+  return id;
+}
 
 sta_status noalloc_scratch_address(void **out) {
   int dev = -1;
   STA_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return STA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_noalloc_addr[dev] == nullptr || ctx == 0ull || ctx != g_noalloc_ctx[dev]) {
     void *addr = nullptr;
     STA_CUDA_TRY(cudaGetSymbolAddress(&addr, g_noalloc_scratch));
     if (addr == nullptr) return STA_ERR_CUDA;
     g_noalloc_addr[dev] = addr;
+    // the lookup makes the device's primary context current if none was
+    g_noalloc_ctx[dev] = current_context_id();
   }
   *out = g_noalloc_addr[dev];
   return STA_OK;

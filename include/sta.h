@@ -201,7 +201,11 @@ sta_status sta_attn_fwd_raster(const void *q, const void *k, const void *v, void
  *     (e.g. 40 heads of a 21x30x52 grid fit; 40 heads of 21x45x80 do not).
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress (the device must be current); make that first call
- *     before any stream capture. Later calls reuse the cached address.
+ *     before any stream capture. Later calls reuse the cached address while
+ *     the same context is current; after a device reset (a new primary
+ *     context, which reloads the library's device code at a new address) the
+ *     next call looks the address up again, and should likewise come before
+ *     any stream capture.
  *   - No allocation of any kind (no cudaMalloc / cudaFree, no allocating
  *     library routine). Nothing in the array has to start at zero: every
  *     byte the kernels read is written earlier in the same call.
@@ -256,10 +260,11 @@ sta_status sta_attn_fwd_rectified(const void *q, const void *k, const void *v, v
                                   float sm_scale, sta_stream_t stream);
 
 /* sta_search_windows -- recall-driven offline search of the dual windows
- * (Compact Attention Fig. 3: the windows are shrunk iteratively under a recall
- * target tau and a cost weight lambda, and the configurations are stored for
- * reuse; Fig. 4: the search starts from full coverage in every
- * temporal-distance group; Fig. 5(c): recall target vs achieved sparsity).
+ * (Compact Attention Fig. 3: the windows are shrunk iteratively under the
+ * recall (tau) and cost (lambda) constraints, and the configurations are
+ * stored for reuse; Fig. 4: starting from full coverage in every
+ * temporal-distance group, the dual windows are shrunk while the recall and
+ * shrink-penalty constraints hold; Fig. 5(c): recall target vs sparsity).
  * One search per (b, h) on its block importances, e.g. the masses of
  * sta_attn_fwd_block_mass over a dense list with the exact LSE:
  *   masses w = floor(min(max(m, 0), 1) * 2^24); W = sum of w; the recall of a
@@ -267,10 +272,13 @@ sta_status sta_attn_fwd_rectified(const void *q, const void *k, const void *v, v
  *   start: (ry1, rx1, ry2, rx2) = (NH-1, NW-1, NH-1, NW-1) in every group;
  *   moves, per group g in order: ry1-1, rx1-1, ry2-1, rx2-1, (ry1-1, ry2-1),
  *   (rx1-1, rx2-1); an extent never goes below -1;
- *   each step applies, among the moves that uncover at least one pair and
- *   keep covered >= ceil(double(tau) * W), the one with the largest
- *   J = removed / Nt^2 - lambda * lost / W (ties to the lowest g*6 + m), and
- *   the search stops when no move is left.
+ *   J = removed / Nt^2 - lambda * lost / W for the pairs / mass a move
+ *   uncovers; a move is admissible iff covered - lost >= ceil(double(tau) * W)
+ *   (recall) and J >= 0 (cost); a move that uncovers nothing (one window
+ *   shrunk inside the other) has J = 0, which lets the two windows, equal at
+ *   the start, come apart (e.g. into a cross of a row band and a column
+ *   band); each step applies the admissible move with the largest J (ties to
+ *   the lowest g*6 + m) and the search stops when none is left.
  *   block_mass : device fp32 [B, heads, Nt, Nt]
  *   group_lo   : HOST int32 [num_groups], ascending, group_lo[0] == 0
  *   tau in [0, 1]; lambda >= 0
@@ -290,31 +298,6 @@ sta_status sta_search_windows(const float *block_mass, int32_t B, int32_t heads,
  * caller check that a stalled pipeline is reported through
  * sta_get_device_error() and leaves the context usable. */
 sta_status sta_selftest_wait_timeout(int64_t limit_cycles, sta_stream_t stream);
-
-/* sta_selftest_tma_stream -- the attention kernel's load stream on its own:
- * ctas_per_sm CTAs per SM, each keeping `slots` (1..6) 16 KB key-tile loads
- * in flight (two 64x64 bf16 TMA boxes with 128 B swizzle, as the kernel
- * loads K and V), from pseudo-random tiles of buf (device, bytes >= 16 KB,
- * 16-byte aligned), `iters` loads per CTA; slots x 16 KB x ctas_per_sm must
- * fit in 200 KB. The caller times it; bytes moved = SMs x ctas_per_sm x
- * iters x 16384. It measures the L2-to-SM rate the hardware gives such loads
- * when nothing else runs (a denominator for the attention's load stream). */
-sta_status sta_selftest_tma_stream(const void *buf, size_t bytes, int32_t ctas_per_sm, int32_t slots,
-                                   int32_t iters, sta_stream_t stream);
-
-/* sta_selftest_mma_rate -- the tensor-core rate of one MMA shape on its own:
- * one CTA per SM of the current device issues `iters` (1..2^20) back-to-back
- * tcgen05.mma of kind::f16 (bf16 x bf16 -> fp32) with M = 128, K = 16 and
- * N = n (64, 128 or 256), A from shared memory (a_in_tmem = 0) or from
- * tensor memory (a_in_tmem != 0), B from shared memory, into one
- * accumulator. cycles: device int64 array with one entry per SM of the
- * current device, written with each CTA's SM cycles from the first issue to
- * completion (-1 if its bounded wait gave up, also recorded as
- * STA_ERR_TIMEOUT). cycles / iters is the cost of one MMA; 128 * n * 16 /
- * that is the multiply-adds per clock (4096 is the dense bf16 peak of an SM).
- * Arguments out of range give STA_ERR_INVALID_ARG before anything runs. */
-sta_status sta_selftest_mma_rate(int32_t n, int32_t a_in_tmem, int32_t iters, int64_t *cycles,
-                                 sta_stream_t stream);
 
 /* Reads and clears the device error word of the current device after
  * synchronising `stream`. STA_OK if no device-side fault was recorded. */

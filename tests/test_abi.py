@@ -9,6 +9,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "sta.h")
+PROBE_HEADER = os.path.join(ROOT, "include", "sta_probe.h")
 
 
 @pytest.fixture(scope="module")
@@ -21,8 +22,8 @@ def sta():
     return mod
 
 
-def declared_functions():
-    text = open(HEADER).read()
+def declared_functions(header=HEADER):
+    text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(sta_[a-z0-9_]+)\s*\(", text)))
 
@@ -38,6 +39,19 @@ def test_library_exports_every_declared_symbol(sta):
     lib = ctypes.CDLL(sta.LIB_PATH)
     for name in declared_functions():
         assert hasattr(lib, name), name
+
+
+def test_probe_library_exports_its_symbols_and_the_product_header_has_none(sta):
+    from block_sparse_attention_28_b200 import probe
+
+    names = declared_functions(PROBE_HEADER)
+    assert names == ["sta_probe_get_device_error", "sta_probe_mma_rate", "sta_probe_tma_stream"]
+    lib = ctypes.CDLL(probe.LIB_PATH)
+    for name in names:
+        assert hasattr(lib, name), name
+    # the measurement probes are not part of the product boundary
+    assert not [n for n in declared_functions() if "probe" in n or n.startswith("sta_selftest_") and
+                n != "sta_selftest_wait_timeout"]
 
 
 def test_tile_counts(sta):
@@ -93,10 +107,12 @@ def test_selftest_limit_is_checked_on_the_host(sta):
 
 
 def test_mma_rate_arguments_are_checked_on_the_host(sta):
+    from block_sparse_attention_28_b200 import probe
+
     buf = ctypes.c_int64(0)
     for n, iters in ((96, 10), (64, 0), (128, (1 << 20) + 1)):
-        assert sta._lib.sta_selftest_mma_rate(n, 0, iters, ctypes.byref(buf), None) == sta.STA_ERR_INVALID_ARG
-    assert sta._lib.sta_selftest_mma_rate(64, 0, 10, None, None) == sta.STA_ERR_INVALID_ARG
+        assert probe._lib.sta_probe_mma_rate(n, 0, iters, ctypes.byref(buf), None) == sta.STA_ERR_INVALID_ARG
+    assert probe._lib.sta_probe_mma_rate(64, 0, 10, None, None) == sta.STA_ERR_INVALID_ARG
 
 
 def test_binding_mirrors_the_noalloc_array_size(sta):

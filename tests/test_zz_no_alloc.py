@@ -87,12 +87,14 @@ def test_noalloc_matches_workspace_path_on_two_calls(sta):
 
 def test_noalloc_rejects_sizes_beyond_the_array(sta):
     # 40 heads of the 21x45x80 layer need ~60 MB of workspace: refused up
-    # front, before any launch (the pointers are never touched).
+    # front, before any launch. Every device pointer is NULL, so were the size
+    # check to regress the call would stop at the argument checks
+    # (STA_ERR_INVALID_ARG) instead of launching.
     g = sta.grid(21, 45, 80)
     assert sta.sta_build_mask_workspace_min(1, 40, 128, g) > (32 << 20)
     params = sta.mask_params(0.95, 8, True)
-    status = sta._lib.sta_build_mask_noalloc(256, 256, 1, 40, 128, g, sta.ctypes.byref(params), 256, 256,
-                                             256, None, None, None)
+    status = sta._lib.sta_build_mask_noalloc(None, None, 1, 40, 128, g, sta.ctypes.byref(params), None, None,
+                                             None, None, None, None)
     assert status == sta.STA_ERR_WORKSPACE
     # 40 heads of the 21x30x52 layer fit
     assert sta.sta_build_mask_workspace_min(1, 40, 128, sta.grid(21, 30, 52)) <= (32 << 20)
