@@ -89,6 +89,10 @@ _lib.sta_attn_fwd_block_mass.restype = ctypes.c_int
 _lib.sta_search_windows.argtypes = [_vp, _i32, _i32, Grid, _i32, ctypes.POINTER(ctypes.c_int32), _f32, _f32,
                                     _vp, _vp, _vp]
 _lib.sta_search_windows.restype = ctypes.c_int
+_lib.sta_set_wait_limit.argtypes = [_i64]
+_lib.sta_set_wait_limit.restype = ctypes.c_int
+_lib.sta_get_wait_limit.argtypes = []
+_lib.sta_get_wait_limit.restype = _i64
 _lib.sta_selftest_wait_timeout.argtypes = [_i64, _vp]
 _lib.sta_selftest_wait_timeout.restype = ctypes.c_int
 _lib.sta_get_device_error.argtypes = [_vp]
@@ -241,6 +245,14 @@ def sta_search_windows(block_mass, B, heads, g, group_lo, tau, lam, windows, sta
     _check(_lib.sta_search_windows(_ptr(block_mass), B, heads, g, len(group_lo), lo, float(tau), float(lam),
                                    _ptr(windows), _ptr(stats), _stream(stream)),
            "sta_search_windows")
+
+
+def sta_set_wait_limit(limit_cycles):
+    _check(_lib.sta_set_wait_limit(int(limit_cycles)), "sta_set_wait_limit")
+
+
+def sta_get_wait_limit():
+    return int(_lib.sta_get_wait_limit())
 
 
 def sta_selftest_wait_timeout(limit_cycles=2000000, stream=None):

@@ -25,6 +25,10 @@
 // TMEM columns: S0 [0,64) S1 [64,128) O [128, 128+d). Two CTAs share an SM
 // (TMEM 2 x 256 columns, shared memory 2 x 103 KB), so one CTA's softmax runs
 // while the other's MMAs do.
+// Every pipeline wait gives up after wait_limit SM cycles (set by the host):
+// it records DEV_ERR_TIMEOUT and raises the CTA's abort flag, which ends the
+// other roles' waits too; the CTA then waits (with a long, fixed limit) for
+// its own MMAs and TMA copies in flight, releases TMEM and returns.
 #pragma once
 #include "sta_common.cuh"
 #include "sta_tc.cuh"
@@ -45,8 +49,7 @@ constexpr uint32_t FLAG_A = 1u << 30;
 constexpr uint32_t FLAG_B = 1u << 31;
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t O_COL = 128;
-constexpr long long WAIT_LIMIT = 2000000000LL;   // SM cycles (~1 s)
-constexpr long long DRAIN_LIMIT = 200000000LL;   // after an abort
+constexpr long long DRAIN_LIMIT = 200000000LL;   // own copies / MMAs, after the pipeline
 constexpr float RESCALE_LOG2 = 8.0f;             // lazy O rescale threshold
 constexpr int MIN_BLOCKS_PER_SM = 2;             // two CTAs share an SM: one's softmax
                                                  // overlaps the other's MMAs
@@ -116,7 +119,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int *__restrict__ col_idx, Geo g, float scale_log2,
                 const float *__restrict__ lse_in, float *__restrict__ block_mass, int heads,
                 const __grid_constant__ CUtensorMap tm_kbar, const __grid_constant__ CUtensorMap tm_vbar,
-                int ntp) {
+                int ntp, long long wait_limit) {
   static_assert(!(MASS && RECT) && !(RASTER && RECT), "the rectified form is tiled and mass-free");
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -284,6 +287,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   }
   auto uidx = [&](int j) { const int t = j + rot; return t < n ? t : t - n; };
 
+  int issued_k = 0, issued_v = 0;  // K / V tiles the producer has loaded
   if (warp == WARP_PRODUCER) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0 && n > 0) {
@@ -313,7 +317,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       auto load_tile = [&](const CUtensorMap *map, const CUtensorMap *pooled_map, uint64_t *full,
                            uint64_t *empty, int off, int ns, int j) -> bool {
         const int s = j % ns, u = j / ns;
-        if (u > 0 && !tc::mbar_wait(empty + s, (u - 1) & 1, abort_flag, WAIT_LIMIT)) return false;
+        if (u > 0 && !tc::mbar_wait(empty + s, (u - 1) & 1, abort_flag, wait_limit)) return false;
         const uint32_t e = U[uidx(j)];
         const int kt = (int)(e & KT_MASK);
         tc::mbar_expect_tx(full + s, C::TILE_BYTES);
@@ -328,7 +332,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         return true;
       };
-      int issued_k = 0, issued_v = 0;
       bool ok = true;
       for (int j = 0; ok && j < C::KLEAD && j < n; ++j) {
         ok = load_tile(&tm_k, &tm_kbar, k_full, k_empty, C::OFF_K, C::NSK, j);
@@ -343,24 +346,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ok = load_tile(&tm_v, &tm_vbar, v_full, v_empty, C::OFF_V, C::NSV, j);
         if (ok) issued_v = j + 1;
       }
-      // Copies still in flight must land before the CTA can exit.
-      if (*abort_flag) {
-        tc::mbar_wait(q_full, 0, nullptr, DRAIN_LIMIT);
-        for (int j = (issued_k > C::NSK ? issued_k - C::NSK : 0); j < issued_k; ++j)
-          tc::mbar_wait(k_full + j % C::NSK, (j / C::NSK) & 1, nullptr, DRAIN_LIMIT);
-        for (int j = (issued_v > C::NSV ? issued_v - C::NSV : 0); j < issued_v; ++j)
-          tc::mbar_wait(v_full + j % C::NSV, (j / C::NSV) & 1, nullptr, DRAIN_LIMIT);
-      }
     }
     __syncwarp();
   } else if (warp == WARP_MMA) {
     // ------------------------------------------------------ MMA issuer
     if (lane == 0 && n > 0) {
-      bool ok = tc::mbar_wait(q_full, 0, abort_flag, WAIT_LIMIT);
+      bool ok = tc::mbar_wait(q_full, 0, abort_flag, wait_limit);
       tc::fence_after();
       auto issue_s = [&](int j) -> bool {
         const int s = j % C::NSK;
-        if (!tc::mbar_wait(k_full + s, (j / C::NSK) & 1, abort_flag, WAIT_LIMIT)) return false;
+        if (!tc::mbar_wait(k_full + s, (j / C::NSK) & 1, abort_flag, wait_limit)) return false;
         tc::fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)((j & 1) * 64);
 #pragma unroll
@@ -377,8 +372,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       };
       auto issue_pv = [&](int j) -> bool {
         const int s = j % C::NSV;
-        if (!tc::mbar_wait(p_full + (j & 1), (j >> 1) & 1, abort_flag, WAIT_LIMIT)) return false;
-        if (!tc::mbar_wait(v_full + s, (j / C::NSV) & 1, abort_flag, WAIT_LIMIT)) return false;
+        if (!tc::mbar_wait(p_full + (j & 1), (j >> 1) & 1, abort_flag, wait_limit)) return false;
+        if (!tc::mbar_wait(v_full + s, (j / C::NSV) & 1, abort_flag, wait_limit)) return false;
         tc::fence_after();
         const uint32_t p_tmem = tmem + (uint32_t)((j & 1) * 64);
 #pragma unroll
@@ -398,9 +393,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (ok) ok = issue_pv(j - 1);
       }
       if (ok) ok = issue_pv(n - 1);
-      // All issued MMAs must retire before TMEM is released.
+      // All issued MMAs must retire before TMEM is released: a wait on the
+      // CTA's own work, so the long limit whatever the pipeline limit.
       tc::mma_commit(mma_done);
-      tc::mbar_wait(mma_done, 0, nullptr, ok ? WAIT_LIMIT : DRAIN_LIMIT);
+      tc::mbar_wait(mma_done, 0, nullptr, DRAIN_LIMIT);
     }
     __syncwarp();
   } else {
@@ -423,7 +419,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     for (int j = 0; j < n; ++j) {
       const int buf = j & 1;
-      const bool got = tc::mbar_wait(s_full + buf, (j >> 1) & 1, abort_flag, WAIT_LIMIT);
+      const bool got = tc::mbar_wait(s_full + buf, (j >> 1) & 1, abort_flag, wait_limit);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
@@ -525,7 +521,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           // was issued after PV_{j-2}, so its completion proves PV_{j-2}
           // retired: o_done has completed j-1 or j phases and the parity of
           // phase j-1 is unambiguous.
-          const bool got_o = tc::mbar_wait(o_done, (j - 1) & 1, abort_flag, WAIT_LIMIT);
+          const bool got_o = tc::mbar_wait(o_done, (j - 1) & 1, abort_flag, wait_limit);
           if (!__all_sync(0xffffffffu, got_o)) {
             ok = false;
             break;
@@ -548,11 +544,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(p_full + buf);
     }
+    // a warp that left the loop early may still have its P store in flight
+    tc::tmem_wait_st();
     // ---- epilogue
     // Wait on the single-use barrier committed after the last P.V: o_done's
     // parity cannot tell PV_{n-1} from PV_{n-2} here, because the last S MMA
     // was issued before PV_{n-2} and so proves only PV_{n-3} retired.
-    if (ok && n > 0) ok = tc::mbar_wait(mma_done, 0, abort_flag, WAIT_LIMIT);
+    if (ok && n > 0) ok = tc::mbar_wait(mma_done, 0, abort_flag, wait_limit);
     ok = __all_sync(0xffffffffu, ok);
     tc::fence_after();
     const bool row_exists = !halfB || hasB;
@@ -597,6 +595,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (lse != nullptr)
         lse[orow] = (l > 0.0f) ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
     }
+  }
+  // Every role has left its loop, so a timeout in any of them has raised the
+  // abort flag by now. The copies the producer issued must land before the
+  // CTA's shared memory is released: after an abort it waits for the last
+  // use of every ring slot (an older use was consumed before its slot was
+  // refilled) and for Q.
+  __syncthreads();
+  if (warp == WARP_PRODUCER && lane == 0 && n > 0 && *abort_flag) {
+    tc::mbar_wait(q_full, 0, nullptr, DRAIN_LIMIT);
+    for (int j = (issued_k > C::NSK ? issued_k - C::NSK : 0); j < issued_k; ++j)
+      tc::mbar_wait(k_full + j % C::NSK, (j / C::NSK) & 1, nullptr, DRAIN_LIMIT);
+    for (int j = (issued_v > C::NSV ? issued_v - C::NSV : 0); j < issued_v; ++j)
+      tc::mbar_wait(v_full + j % C::NSV, (j / C::NSV) & 1, nullptr, DRAIN_LIMIT);
   }
   tc::fence_before();
   __syncthreads();

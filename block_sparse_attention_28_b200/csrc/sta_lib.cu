@@ -3,6 +3,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "sta_attn.cuh"
@@ -17,6 +18,16 @@
 using namespace sta;
 
 namespace {
+
+// SM-cycle limit of every bounded pipeline wait in the kernels launched from
+// now on (0: the default of ~1 s); see sta_set_wait_limit.
+constexpr long long DEFAULT_WAIT_LIMIT = 2000000000LL;
+std::atomic<long long> g_wait_limit{0};
+
+long long wait_limit() {
+  const long long v = g_wait_limit.load(std::memory_order_relaxed);
+  return v > 0 ? v : DEFAULT_WAIT_LIMIT;
+}
 
 bool common_sizes_ok(int32_t B, int32_t heads, int32_t d, sta_grid g, Geo *geo, sta_status *st) {
   if (B <= 0 || heads <= 0 || !make_geo(g, geo)) {
@@ -155,7 +166,8 @@ sta_status launch_scores_tc(const float *qhi, const float *qlo, const float *khi
   const int per_part = (qblocks + parts - 1) / parts;
   parts = (qblocks + per_part - 1) / per_part;  // no empty range
   dim3 grid((unsigned)kblocks, (unsigned)parts, (unsigned)bh);
-  kern<<<grid, score::NUM_THREADS, smem, s>>>(m_khi, m_klo, m_qhi, m_qlo, S, g.Nt, scale, per_part * score::N);
+  kern<<<grid, score::NUM_THREADS, smem, s>>>(m_khi, m_klo, m_qhi, m_qlo, S, g.Nt, scale, per_part * score::N,
+                                              wait_limit());
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }
@@ -211,7 +223,8 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
       STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PC::SMEM));
       const long long units = 2LL * B * g.T * g.NH * g.NW * ((heads + PC::HB - 1) / PC::HB);
       const long long ctas = units < sm_count() ? units : sm_count();
-      kern<<<(unsigned)ctas, pool::NUM_THREADS, PC::SMEM, s>>>(m_q, m_k, qbar, kbar, qlo, klo, g, heads, units);
+      kern<<<(unsigned)ctas, pool::NUM_THREADS, PC::SMEM, s>>>(m_q, m_k, qbar, kbar, qlo, klo, g, heads, units,
+                                                               wait_limit());
     } else {
       const long long warps = 2 * R;
       const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
@@ -324,7 +337,7 @@ sta_status launch_attn(const void *q, const void *k, const void *v, void *o, flo
   dim3 grid((unsigned)((g.Nt + 1) / 2), (unsigned)(B * heads));
   attn::attn_fwd_kernel<D, MASS, RASTER, RECT><<<grid, attn::NUM_THREADS, smem, s>>>(
       tq, tk, tv, static_cast<__nv_bfloat16 *>(o), lse, row_ptr, col_idx, g, scale_log2, lse_in,
-      block_mass, heads, tkb, tvb, ntp);
+      block_mass, heads, tkb, tvb, ntp, wait_limit());
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }
@@ -544,6 +557,14 @@ sta_status sta_search_windows(const float *block_mass, int32_t B, int32_t heads,
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }
+
+sta_status sta_set_wait_limit(int64_t limit_cycles) {
+  if (limit_cycles != 0 && (limit_cycles < 1000 || limit_cycles > DEFAULT_WAIT_LIMIT)) return STA_ERR_INVALID_ARG;
+  g_wait_limit.store((long long)limit_cycles, std::memory_order_relaxed);
+  return STA_OK;
+}
+
+int64_t sta_get_wait_limit(void) { return (int64_t)wait_limit(); }
 
 sta_status sta_selftest_wait_timeout(int64_t limit_cycles, sta_stream_t stream) {
   if (limit_cycles < 1000 || limit_cycles > 2000000000LL) return STA_ERR_INVALID_ARG;

@@ -17,8 +17,9 @@
 //               tf32(x - tf32(x)) in qlo / klo
 // The ring keeps up to 192 KB of loads in flight per SM without a thread per
 // outstanding load.
-// Every wait is bounded; on a timeout the kernel records DEV_ERR_TIMEOUT,
-// waits (bounded) for its own copies in flight and returns.
+// Every pipeline wait gives up after wait_limit SM cycles (set by the host);
+// on a timeout the kernel records DEV_ERR_TIMEOUT, waits (with a long, fixed
+// limit) for its own copies in flight and returns.
 #pragma once
 #include "sta_mask.cuh"
 #include "sta_tc.cuh"
@@ -30,8 +31,7 @@ constexpr int CONSUMERS = 512;                 // 16 warps: two columns x half t
 constexpr int NUM_THREADS = CONSUMERS + 32;    // + the producer warp
 constexpr int WARP_TMA = CONSUMERS / 32;
 constexpr int STAGES = 3;
-constexpr long long WAIT_LIMIT = 2000000000LL;  // SM cycles (~1 s)
-constexpr long long DRAIN_LIMIT = 200000000LL;  // after an abort
+constexpr long long DRAIN_LIMIT = 200000000LL;  // own copies, after the pipeline
 
 template <int D>
 struct Cfg {
@@ -45,64 +45,15 @@ struct Cfg {
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-// Unit u = ((((b*T + t) * NH + ty) * NW + tx) * 2 + tensor) * G + group,
-// G = ceil(heads / HB); consecutive units are neighbouring boxes of memory.
+// The consumers of pool_tma_kernel: threads 0 .. CONSUMERS-1.
 template <int D>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-pool_tma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                float *__restrict__ qbar, float *__restrict__ kbar, float *__restrict__ qlo,
-                float *__restrict__ klo, Geo g, int heads, long long units) {
+__device__ __forceinline__ void consume(uint8_t *smem, uint64_t *full, uint64_t *empty,
+                                        volatile uint32_t *abort_flag, float *__restrict__ qbar,
+                                        float *__restrict__ kbar, float *__restrict__ qlo,
+                                        float *__restrict__ klo, const Geo &g, int heads, long long units,
+                                        long long wait_limit, int G) {
   using C = Cfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t sbase = tc::smem_u32(smem);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-  uint64_t *empty = full + STAGES;
-  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(empty + STAGES);
-  if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      tc::mbar_init(full + s, 1);
-      tc::mbar_init(empty + s, CONSUMERS / 32);  // one arrival per consumer warp
-    }
-    *abort_flag = 0u;
-    tc::fence_barrier_init();
-  }
-  __syncthreads();
-  const int G = (heads + C::HB - 1) / C::HB;
-
-  if (warp == WARP_TMA) {
-    // ---------------------------------------------------------- producer
-    if (lane == 0) {
-      long long issued = 0, i = 0;
-      for (long long u = blockIdx.x; u < units; u += gridDim.x, ++i) {
-        const int s = (int)(i % STAGES);
-        const long long r = i / STAGES;
-        if (r > 0 && !tc::mbar_wait(empty + s, (uint32_t)((r - 1) & 1), abort_flag, WAIT_LIMIT)) break;
-        long long v = u;
-        const int grp = (int)(v % G);
-        v /= G;
-        const int tensor = (int)(v & 1);
-        v >>= 1;
-        const int tx = (int)(v % g.NW);
-        v /= g.NW;
-        const int ty = (int)(v % g.NH);
-        const int bt = (int)(v / g.NH);
-        tc::mbar_expect_tx(full + s, C::BOX_BYTES);
-        tc::tma_load_5d(sbase + s * C::BOX_BYTES, tensor ? &tm_k : &tm_q, full + s, 0, grp * C::HB, tx * 8,
-                        ty * 8, bt);
-        issued = i + 1;
-      }
-      // copies still in flight must land before the CTA can exit
-      if (*abort_flag) {
-        for (long long j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
-          tc::mbar_wait(full + j % STAGES, (uint32_t)((j / STAGES) & 1), nullptr, DRAIN_LIMIT);
-      }
-    }
-    __syncwarp();
-    return;
-  }
-  // ------------------------------------------------------------ consumers
+  const int tid = threadIdx.x, lane = tid & 31;
   const int pair = tid % (CONSUMERS / 2), half = tid / (CONSUMERS / 2);
   const int col = 2 * pair;  // columns col, col + 1 of the box: head col / D, dims col % D
   const int h_in = col / D, dd = col - h_in * D;
@@ -110,7 +61,7 @@ pool_tma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   long long i = 0;
   for (long long u = blockIdx.x; u < units; u += gridDim.x, ++i) {
     const int s = (int)(i % STAGES);
-    const bool got = tc::mbar_wait(full + s, (uint32_t)((i / STAGES) & 1), abort_flag, WAIT_LIMIT);
+    const bool got = tc::mbar_wait(full + s, (uint32_t)((i / STAGES) & 1), abort_flag, wait_limit);
     double a0 = 0.0, a1 = 0.0;
     if (got) {
       // box row r = 8 y + x (token of the tile), columns [head][d]; this
@@ -163,6 +114,71 @@ pool_tma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       *reinterpret_cast<float2 *>((tensor ? kbar : qbar) + row * D + dd) = make_float2(m0, m1);
     }
+  }
+}
+
+
+// Unit u = ((((b*T + t) * NH + ty) * NW + tx) * 2 + tensor) * G + group,
+// G = ceil(heads / HB); consecutive units are neighbouring boxes of memory.
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+pool_tma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                float *__restrict__ qbar, float *__restrict__ kbar, float *__restrict__ qlo,
+                float *__restrict__ klo, Geo g, int heads, long long units, long long wait_limit) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = tc::smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+  uint64_t *empty = full + STAGES;
+  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(empty + STAGES);
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(full + s, 1);
+      tc::mbar_init(empty + s, CONSUMERS / 32);  // one arrival per consumer warp
+    }
+    *abort_flag = 0u;
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  const int G = (heads + C::HB - 1) / C::HB;
+
+  long long issued = 0;  // boxes the producer has loaded
+  if (warp == WARP_TMA) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      long long i = 0;
+      for (long long u = blockIdx.x; u < units; u += gridDim.x, ++i) {
+        const int s = (int)(i % STAGES);
+        const long long r = i / STAGES;
+        if (r > 0 && !tc::mbar_wait(empty + s, (uint32_t)((r - 1) & 1), abort_flag, wait_limit)) break;
+        long long v = u;
+        const int grp = (int)(v % G);
+        v /= G;
+        const int tensor = (int)(v & 1);
+        v >>= 1;
+        const int tx = (int)(v % g.NW);
+        v /= g.NW;
+        const int ty = (int)(v % g.NH);
+        const int bt = (int)(v / g.NH);
+        tc::mbar_expect_tx(full + s, C::BOX_BYTES);
+        tc::tma_load_5d(sbase + s * C::BOX_BYTES, tensor ? &tm_k : &tm_q, full + s, 0, grp * C::HB, tx * 8,
+                        ty * 8, bt);
+        issued = i + 1;
+      }
+    }
+    __syncwarp();
+  } else {
+    consume<D>(smem, full, empty, abort_flag, qbar, kbar, qlo, klo, g, heads, units, wait_limit, G);
+  }
+  // Every thread has left its loop, so a timeout in any of them has raised
+  // the abort flag by now; the producer's boxes still in flight (the last use
+  // of every ring stage) must land before shared memory is released.
+  __syncthreads();
+  if (warp == WARP_TMA && lane == 0 && *abort_flag) {
+    for (long long j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+      tc::mbar_wait(full + j % STAGES, (uint32_t)((j / STAGES) & 1), nullptr, DRAIN_LIMIT);
   }
 }
 

@@ -26,9 +26,10 @@
 // memory, and with N = 128 it runs at the full tensor-core rate (an N = 64
 // MMA takes ~46 cycles for the work of 32). Operands in shared memory are
 // K-major with the 128-byte swizzle: a chunk of 32 fp32 along d per 128-byte
-// row, 8-row groups 1024 B apart. Every wait is bounded; on a timeout the
-// kernel records DEV_ERR_TIMEOUT, waits (bounded) for its own copies in
-// flight, releases TMEM and returns.
+// row, 8-row groups 1024 B apart. Every pipeline wait gives up after
+// wait_limit SM cycles (set by the host); on a timeout the kernel records
+// DEV_ERR_TIMEOUT, waits (with a long, fixed limit) for its own MMAs and
+// copies in flight, releases TMEM and returns.
 #pragma once
 #include "sta_tc.cuh"
 
@@ -40,8 +41,7 @@ constexpr int N = 128;           // query tiles per MMA block (TMEM columns)
 constexpr int NH = 64;           // query tiles per epilogue half
 constexpr int NUM_THREADS = 192;
 constexpr int WARP_TMA = 4, WARP_MMA = 5;
-constexpr long long WAIT_LIMIT = 2000000000LL;  // SM cycles (~1 s)
-constexpr long long DRAIN_LIMIT = 200000000LL;  // after an abort
+constexpr long long DRAIN_LIMIT = 200000000LL;  // own copies / MMAs, after the pipeline
 
 template <int D>
 struct Cfg {
@@ -114,7 +114,7 @@ template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constant__ CUtensorMap tm_klo,
                 const __grid_constant__ CUtensorMap tm_qhi, const __grid_constant__ CUtensorMap tm_qlo,
-                float *__restrict__ S, int nt, float scale, int q_per_part) {
+                float *__restrict__ S, int nt, float scale, int q_per_part, long long wait_limit) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -163,6 +163,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
   tc::fence_after();
   const uint32_t tmem = misc[0];
   const int nchunks = nblk * C::CH;  // ring items: (block j, d-chunk c) = item j * CH + c
+  int issued = 0;                    // ring items the producer has loaded
 
   if (warp == WARP_TMA) {
     // ---------------------------------------------------------- producer
@@ -173,12 +174,12 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
         tma_load_3d(sbase + c * C::A_CHUNK, &tm_khi, a_tma, 32 * c, k0, bh);
         tma_load_3d(sbase + C::A_PART + c * C::A_CHUNK, &tm_klo, a_tma, 32 * c, k0, bh);
       }
-      int issued = 0;
-      // the ring reuses the staging area once the key block is in TMEM
-      bool ok = tc::mbar_wait(a_moved, 0, abort_flag, WAIT_LIMIT);
+      // the ring reuses the staging area once the key block is in TMEM (the
+      // epilogue warps arrive after a timeout too, with the abort flag raised)
+      bool ok = tc::mbar_wait(a_moved, 0, abort_flag, wait_limit) && !*abort_flag;
       for (int it = 0; ok && it < nchunks; ++it) {
         const int s = it % C::STAGES, u = it / C::STAGES;
-        if (u > 0 && !tc::mbar_wait(empty + s, (u - 1) & 1, abort_flag, WAIT_LIMIT)) break;
+        if (u > 0 && !tc::mbar_wait(empty + s, (u - 1) & 1, abort_flag, wait_limit)) break;
         const int j = it / C::CH, c = it - j * C::CH;
         const uint32_t dst = sbase + s * C::STAGE_BYTES;
         const int q0 = q_begin + j * N;
@@ -187,26 +188,20 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
         tma_load_3d(dst + C::B_CHUNK, &tm_qlo, full + s, 32 * c, q0, bh);
         issued = it + 1;
       }
-      // copies still in flight must land before the CTA can exit
-      if (*abort_flag) {
-        tc::mbar_wait(a_tma, 0, nullptr, DRAIN_LIMIT);
-        for (int it = (issued > C::STAGES ? issued - C::STAGES : 0); it < issued; ++it)
-          tc::mbar_wait(full + it % C::STAGES, (it / C::STAGES) & 1, nullptr, DRAIN_LIMIT);
-      }
     }
     __syncwarp();
   } else if (warp == WARP_MMA) {
     // ---------------------------------------------------------- MMA issue
     if (lane == 0 && nblk > 0) {
-      bool ok = tc::mbar_wait(a_full, 0, abort_flag, WAIT_LIMIT);
+      bool ok = tc::mbar_wait(a_full, 0, abort_flag, wait_limit);
       tc::fence_after();
       for (int j = 0; ok && j < nblk; ++j) {
         const int buf = j & 1;
-        if (j >= 2 && !tc::mbar_wait(t_empty + buf, ((j >> 1) - 1) & 1, abort_flag, WAIT_LIMIT)) break;
+        if (j >= 2 && !tc::mbar_wait(t_empty + buf, ((j >> 1) - 1) & 1, abort_flag, wait_limit)) break;
         const uint32_t d_tmem = tmem + (uint32_t)(buf * N);
         for (int c = 0; ok && c < C::CH; ++c) {
           const int it = j * C::CH + c, s = it % C::STAGES;
-          if (!tc::mbar_wait(full + s, (it / C::STAGES) & 1, abort_flag, WAIT_LIMIT)) {
+          if (!tc::mbar_wait(full + s, (it / C::STAGES) & 1, abort_flag, wait_limit)) {
             ok = false;
             break;
           }
@@ -228,9 +223,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
         if (!ok) break;
         tc::mma_commit(t_full + buf);
       }
-      // every issued MMA retires before TMEM is released
+      // every issued MMA retires before TMEM is released (a wait on the
+      // CTA's own work: the long limit whatever the pipeline limit)
       tc::mma_commit(mma_done);
-      tc::mbar_wait(mma_done, 0, nullptr, *abort_flag ? DRAIN_LIMIT : WAIT_LIMIT);
+      tc::mbar_wait(mma_done, 0, nullptr, DRAIN_LIMIT);
     }
     __syncwarp();
   } else {
@@ -239,7 +235,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
     bool ok = nblk > 0;
     if (ok) {
       // row tid of each swizzled chunk: 16-byte granule g sits at g ^ (tid % 8)
-      ok = tc::mbar_wait(a_tma, 0, abort_flag, WAIT_LIMIT);
+      ok = tc::mbar_wait(a_tma, 0, abort_flag, wait_limit);
       if (ok) {
 #pragma unroll 1
         for (int part = 0; part < 2; ++part) {
@@ -274,7 +270,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
     ok = all_epilogue(ok);
     for (int j = 0; ok && j < nblk; ++j) {
       const int buf = j & 1;
-      if (!all_epilogue(tc::mbar_wait(t_full + buf, (j >> 1) & 1, abort_flag, WAIT_LIMIT))) break;
+      if (!all_epilogue(tc::mbar_wait(t_full + buf, (j >> 1) & 1, abort_flag, wait_limit))) break;
       tc::fence_after();
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
@@ -307,6 +303,16 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
         asm volatile("bar.sync 1, 128;" ::: "memory");
       }
     }
+  }
+  // Every role has left its loop, so a timeout in any of them has raised the
+  // abort flag by now; the producer's copies still in flight (the key block,
+  // the last use of every ring stage) must land before shared memory is
+  // released.
+  __syncthreads();
+  if (warp == WARP_TMA && lane == 0 && nblk > 0 && *abort_flag) {
+    tc::mbar_wait(a_tma, 0, nullptr, DRAIN_LIMIT);
+    for (int it = (issued > C::STAGES ? issued - C::STAGES : 0); it < issued; ++it)
+      tc::mbar_wait(full + it % C::STAGES, (it / C::STAGES) & 1, nullptr, DRAIN_LIMIT);
   }
   tc::fence_before();
   __syncthreads();

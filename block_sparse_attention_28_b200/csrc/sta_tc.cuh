@@ -44,7 +44,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // try_wait with a suspend-time hint: a waiting thread sleeps until the phase
 // completes (or the hint in ns runs out) instead of spinning, so waiting
 // warps take no issue slots from the softmax warps of their SM sub-partition.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
 #if STA_WAIT_SLEEP_NS > 0
   uint32_t ok;
   asm volatile(
@@ -52,7 +52,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "n"(STA_WAIT_SLEEP_NS)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0u;
 #else
@@ -61,13 +61,17 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
 }
 
 // Bounded wait: gives up after `limit` SM cycles (or when another role has
-// raised `abort`), records DEV_ERR_TIMEOUT and returns false.
+// raised `abort`), records DEV_ERR_TIMEOUT and returns false. The limit is
+// checked each time the suspended thread wakes, so the suspend hint is kept
+// at or below a quarter of the limit (in ns, which is fewer than cycles at
+// the B200's clocks) and a short limit is noticed in time.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile uint32_t *abort,
                                           long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
+  const uint32_t hint = limit >= 4LL * STA_WAIT_SLEEP_NS ? (uint32_t)STA_WAIT_SLEEP_NS : (uint32_t)(limit / 4);
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
     if (abort != nullptr && *abort) return false;
     if (clock64() - t0 > limit) {
       if (abort != nullptr) *abort = 1u;

@@ -290,6 +290,23 @@ sta_status sta_search_windows(const float *block_mass, int32_t B, int32_t heads,
                               int32_t num_groups, const int32_t *group_lo, float tau, float lambda,
                               int32_t *windows, float *stats, sta_stream_t stream);
 
+/* sta_set_wait_limit -- how long a stalled pipeline may wait before it is
+ * reported. Every pipeline wait of the kernels launched after this call by
+ * this process (the attention forms, the tensor-core scores and the raster
+ * pooling of the mask build) gives up after limit_cycles SM cycles: the kernel
+ * records STA_ERR_TIMEOUT in the device error word, waits (with a fixed limit
+ * of 2e8 cycles) for its own MMAs and TMA copies in flight, releases its
+ * tensor memory and returns, so the context stays usable; the outputs of that
+ * call are unspecified. limit_cycles in [1e3, 2e9], or 0 for the default
+ * (2e9 cycles, about a second at the B200's clocks). A limit below the
+ * pipeline's ordinary latencies (a few thousand cycles) makes every call time
+ * out: it exists to check the timeout path, or to report stalls sooner. The
+ * pages have no counterpart. Returns STA_ERR_INVALID_ARG out of range. */
+sta_status sta_set_wait_limit(int64_t limit_cycles);
+
+/* The wait limit the next launches will use (SM cycles). */
+int64_t sta_get_wait_limit(void);
+
 /* sta_selftest_wait_timeout -- exercises the bounded wait that every pipeline
  * stage of sta_attn_fwd uses, without a fault: one thread initialises a
  * shared-memory mbarrier that nothing will ever complete, waits on it for at

@@ -1055,6 +1055,85 @@ def test_bounded_wait_reports_timeout_and_context_survives(sta, gp):
     test_attn_tiny_config(sta, gp)  # a full attention call still runs and matches
 
 
+def _timeout_case(sta, gp):
+    """A small layer (4 heads, d = 128, 4 x 40 x 48 grid, every key tile
+    listed) in raster and tiled form."""
+    B, Hh, d, T, H, W = 1, 4, 128, 4, 40, 48
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    q, k, v = _structured(T, H, W, Hh, d, seed=31)
+    R = B * Hh * nt
+    rp = (torch.arange(R + 1, device="cuda", dtype=torch.int64) * nt).to(torch.int32)
+    ci = torch.arange(nt, device="cuda", dtype=torch.int32).repeat(R)
+    return B, Hh, d, g, q, k, v, rp, ci
+
+
+def test_attention_waits_run_out_drain_and_the_context_survives(sta, gp):
+    """With the pipeline wait limit cut to 1,000 SM cycles (shorter than a
+    tile load or a softmax step), the attention kernel's own waits run out:
+    the call reports STA_ERR_TIMEOUT and no fault, the CTAs drain their copies
+    and MMAs and free TMEM, and a call with the default limit afterwards, on
+    the same context, gives output bit-identical to one made before."""
+    B, Hh, d, g, q, k, v, rp, ci = _timeout_case(sta, gp)
+    o_ref, lse_ref = torch.empty_like(q), torch.empty(B, Hh, sta.sta_tiled_len(g), device="cuda")
+    sta.sta_attn_fwd_raster(q, k, v, o_ref, lse_ref, rp, ci, B, Hh, d, g)
+    assert sta.sta_get_device_error() == sta.STA_OK
+    assert sta.sta_get_wait_limit() == 2_000_000_000
+    try:
+        sta.sta_set_wait_limit(1000)
+        assert sta.sta_get_wait_limit() == 1000
+        o = torch.zeros_like(q)
+        sta.sta_attn_fwd_raster(q, k, v, o, None, rp, ci, B, Hh, d, g)
+        assert sta.sta_get_device_error() == sta.STA_ERR_TIMEOUT
+    finally:
+        sta.sta_set_wait_limit(0)
+    assert sta.sta_get_wait_limit() == 2_000_000_000
+    assert sta.sta_get_device_error() == sta.STA_OK
+    o2, lse2 = torch.full_like(q, float("nan")), torch.full_like(lse_ref, float("nan"))
+    sta.sta_attn_fwd_raster(q, k, v, o2, lse2, rp, ci, B, Hh, d, g)
+    assert sta.sta_get_device_error() == sta.STA_OK
+    assert torch.equal(o2.view(torch.int16), o_ref.view(torch.int16))
+    assert torch.equal(lse2.view(torch.int32), lse_ref.view(torch.int32))
+
+
+def test_mask_build_waits_run_out_drain_and_the_context_survives(sta, gp):
+    """The same for the mask build's pipelined kernels (the raster pooling's
+    TMA ring and the tensor-core scores): at a 1,000-cycle limit the build
+    reports STA_ERR_TIMEOUT without a fault, and with the default limit it then
+    gives the CSR, byte mask and P of a build made before, bit for bit."""
+    B, Hh, d, g, q, k, _, _, _ = _timeout_case(sta, gp)
+    params = sta.mask_params(0.9, 4, True)
+
+    def build():
+        bufs = sta.MaskBuffers(B, Hh, d, g, "cuda", with_mask=True, with_probs=True)
+        sta.build_mask(q, k, B, Hh, d, g, params, bufs, raster=True)
+        return bufs
+
+    ref = build()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    try:
+        sta.sta_set_wait_limit(1000)
+        build()
+        assert sta.sta_get_device_error() == sta.STA_ERR_TIMEOUT
+    finally:
+        sta.sta_set_wait_limit(0)
+    assert sta.sta_get_device_error() == sta.STA_OK
+    again = build()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    n = int(ref.nnz.item())
+    assert n == int(again.nnz.item())
+    assert torch.equal(again.row_ptr, ref.row_ptr) and torch.equal(again.col_idx[:n], ref.col_idx[:n])
+    assert torch.equal(again.block_mask, ref.block_mask)
+    assert torch.equal(again.block_probs.view(torch.int32), ref.block_probs.view(torch.int32))
+
+
+def test_wait_limit_is_checked_on_the_host(sta):
+    for bad in (1, 999, 2_000_000_001, -5):
+        with pytest.raises(sta.StaError):
+            sta.sta_set_wait_limit(bad)
+    assert sta.sta_get_wait_limit() == 2_000_000_000
+
+
 @pytest.mark.parametrize("a_tmem", [False, True])
 def test_mma_rate_probe(sta, a_tmem):
     """The MMA-rate probe runs on every SM and reports a cost per MMA that
