@@ -619,6 +619,76 @@ def sweep(sta, dev, peak, reps=20):
     return rows
 
 
+def per_config(sta, dev, peaks, reps=10):
+    """Compact record of every other timed layer of the workload table, for
+    the default 1-GPU line: the 480p window layer, the 129-frame layer at its
+    four window densities and the reuse layer at its five fixed densities
+    (mask built once from step-0 inputs; attention over the ten perturbed
+    steps). Per row: attention and build medians (CUDA events, each launch
+    timed alone, inputs larger than L2), kept-pair TFLOP/s as a fraction of
+    the measured burst and sustained bf16 peaks, the pairing efficiency of
+    the 128-row CTAs, and the clocks sampled while that row ran."""
+    burst = float(peaks.get("bf16_tflops", 1590.0))
+    sust = float(peaks.get("bf16_tflops_sustained", burst))
+    rows = []
+
+    def record(name, layer, attn_fn, attn_reps, extra):
+        clocks = ClockSampler(dev)
+        clocks.start()
+        h0 = time.monotonic()
+        build_ms = _median_ms(layer.build, reps)
+        ms = _median_ms(attn_fn, attn_reps)
+        clk = clocks.stop(h0, time.monotonic())
+        pairs = layer.kept_pairs()
+        tf = pairs * flops_per_pair(layer.d) / (ms * 1e-3) / 1e12
+        eff, _ = layer.pair_union_stats()
+        row = {"workload": name, "density": pairs / (layer.B * layer.Hh * layer.nt ** 2), "kept_pairs": pairs,
+               "attn_ms": ms, "attn_tflops": tf, "frac_burst": tf / burst, "frac_sustained": tf / sust,
+               "pairing_efficiency": eff, "build_ms": build_ms,
+               "clocks": {"sm_mhz": clk.get("sm_mhz"), "power_w_median": clk.get("power_w_median"),
+                          "reasons": clk.get("reasons")}}
+        row.update(extra)
+        rows.append(row)
+
+    for wl, dens in (("dit480p", (0,)), ("dit720p_129f", (0, 1, 2, 3))):
+        for di in dens:
+            layer = Layer(sta, CONFIGS[wl], dev, workload=wl, density_index=di)
+            layer.build()
+            record(CONFIGS[wl].name, layer, layer.attn, reps,
+                   {"density_target": CONFIGS[wl].window_density[di]})
+            del layer
+            torch.cuda.empty_cache()
+
+    cfg = CONFIGS["reuse480p"]
+    layer = Layer(sta, cfg, dev, workload="reuse480p")
+    gen = torch.Generator(device=dev).manual_seed(1234)
+    masters = [layer.q.float(), layer.k.float()]
+    steps_inputs = []
+    for _ in range(cfg.reuse_steps):
+        qm, qb = perturb_step(masters[0], gen)
+        km, kb = perturb_step(masters[1], gen)
+        masters = [qm, km]
+        steps_inputs.append((qb, kb))
+    del masters
+    for rho in cfg.fixed_densities:
+        k_min = int(round(rho * layer.nt))
+        layer.params = sta.mask_params(0.0, k_min, True, 0.0, cfg.group_lo, None)
+        layer.build()
+        it = iter(range(10 ** 9))
+
+        def attn_reuse():
+            qb, kb = steps_inputs[next(it) % len(steps_inputs)]
+            layer.attn(qb, kb)
+
+        # one launch per perturbed step, in turn, over the mask of step 0
+        record(cfg.name, layer, attn_reuse, 2 * len(steps_inputs),
+               {"density_target": rho, "k_min": k_min, "reuse_steps": len(steps_inputs)})
+    del layer, steps_inputs
+    torch.cuda.empty_cache()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    return rows
+
+
 def blas_threads():
     """Threads of the BLAS library numpy uses (the oracle's matmuls)."""
     try:
@@ -787,6 +857,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-mask run of the same kernel")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-config record of the other workload layers (1 GPU only)")
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(CONFIGS),
                     help="workload (profiling of smaller layers); the headline is the 720p layer")
     ap.add_argument("--density-index", type=int, default=0)
@@ -913,8 +985,12 @@ def main():
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    peak_burst = float(peaks.get("bf16_tflops", peak))
     eff, union_tiles = layer.pair_union_stats() if rank == 0 else (None, None)
     line = None
+    per_cfg = None
+    if rank == 0 and world == 1 and not args.no_per_config and args.workload == HEADLINE and args.heads == 0:
+        per_cfg = per_config(sta, dev, peaks)
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline and args.workload == HEADLINE:
@@ -944,11 +1020,13 @@ def main():
             "pairing_efficiency": eff,
             "dense_mask_run": dense,
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
-                         "frac": attn_tflops / peak, "traffic": load_traffic(),
+                         "frac": attn_tflops / peak, "frac_burst": attn_tflops / peak_burst,
+                         "peak_burst": peak_burst, "traffic": load_traffic(),
                          "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
                          "kernel": "attn_fwd_kernel<128, MASS=false, RASTER=true>",
                          "algorithmic": f"{pairs} kept pairs x 4*64*64*{cfg.d} flop"},
             "cpu_baseline": cpu,
+            "per_config": per_cfg,
             "e2e": e2e,
             "gpu_launches": K * n_launch,
             "gpu_launches_source": launch_src,

@@ -66,6 +66,8 @@ _lib.sta_build_mask_workspace.argtypes = [_i32, _i32, _i32, Grid]
 _lib.sta_build_mask_workspace.restype = _sz
 _lib.sta_build_mask_workspace_min.argtypes = [_i32, _i32, _i32, Grid]
 _lib.sta_build_mask_workspace_min.restype = _sz
+_lib.sta_build_mask_pooled_offsets.argtypes = [_i32, _i32, _i32, Grid, _sz, ctypes.POINTER(_sz)]
+_lib.sta_build_mask_pooled_offsets.restype = ctypes.c_int
 _lib.sta_build_mask.argtypes = [_vp, _vp, _i32, _i32, _i32, Grid, ctypes.POINTER(MaskParams), _vp, _vp,
                                 _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.sta_build_mask.restype = ctypes.c_int
@@ -170,6 +172,14 @@ def mask_params(top_p=0.0, k_min=0, use_scores=False, sm_scale=0.0, group_lo=(0,
     # the struct holds raw device pointers: keep the tensors alive with it
     p._keep = (windows, block_scores)
     return p
+
+
+def sta_build_mask_pooled_offsets(B, heads, d, g, ws_bytes):
+    """(qbar, kbar, qlo, klo) byte offsets of the pooled means in a mask-build
+    workspace of ws_bytes; qlo / klo are 0 when the means are not split."""
+    out = (_sz * 4)()
+    _check(_lib.sta_build_mask_pooled_offsets(B, heads, d, g, int(ws_bytes), out), "sta_build_mask_pooled_offsets")
+    return tuple(int(x) for x in out)
 
 
 def sta_build_mask(q_tiled, k_tiled, B, heads, d, g, params, row_ptr, col_idx, nnz_dev,

@@ -14,6 +14,7 @@
 #include "sta_reorder.cuh"
 #include "sta_score.cuh"
 #include "sta_search.cuh"
+#include "sta_select.cuh"
 
 using namespace sta;
 
@@ -87,7 +88,7 @@ MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
 // Dynamic shared memory of score_select_kernel<D, qb, mode>.
 size_t select_smem(int d, const Geo &g, bool use_scores, int qb = SEL_QB, int mode = SEL_FUSED) {
   const size_t q = (mode == SEL_FUSED && use_scores) ? (size_t)qb * d : 0;
-  const size_t scores = use_scores ? (size_t)(qb * g.Nt + (SEL_THREADS / 32) * 256) : 0;
+  const size_t scores = use_scores ? (size_t)(qb * g.Nt + (SEL_THREADS / 32) * 256 * 2) : 0;  // u64 histograms
   // window tables (group of each |dt|, the head's extents) and one row of
   // window bits per warp
   const size_t tables = (size_t)((g.T + 3) & ~3) + 4 * STA_MAX_GROUPS + (SEL_THREADS / 32) * ((g.Nt + 31) / 32);
@@ -185,6 +186,50 @@ __global__ void selftest_wait_kernel(long long limit) {
   }
 }
 
+// The select pass with the row in registers (sel::select_rows_kernel<NPL>,
+// NPL = ceil(Nt / 32) rounded up to a multiple of 8). With the per-head floor
+// (kfloor != nullptr) it runs twice around head_floor_kernel: first for the
+// base counts only (sel_count), then with k_min raised to the floor.
+template <int NPL>
+sta_status launch_select_regs_npl(const float *P, int logits, float *probs, int B, int heads, const Geo &g,
+                                  const sta_mask_params *p, bool use_scores, const int *windows, int G,
+                                  const GroupLo &glo, unsigned int *bits, int *counts, int wpr, int *kfloor,
+                                  int *sel, cudaStream_t s) {
+  auto kern = sel::select_rows_kernel<NPL>;
+  const size_t smem = sel::smem_bytes(NPL, wpr, g.T);
+  if (smem > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
+  STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  dim3 grid((unsigned)((g.Nt + sel::WARPS - 1) / sel::WARPS), (unsigned)(B * heads));
+  if (kfloor != nullptr) {
+    kern<<<grid, sel::THREADS, smem, s>>>(P, logits, nullptr, heads, g, p->top_p, p->k_min, 1, nullptr, 0, glo,
+                                          bits, counts, wpr, nullptr, sel);
+    STA_CUDA_TRY(cudaGetLastError());
+    head_floor_kernel<<<(unsigned)(B * heads), FLOOR_THREADS, 0, s>>>(sel, kfloor, g);
+    STA_CUDA_TRY(cudaGetLastError());
+  }
+  kern<<<grid, sel::THREADS, smem, s>>>(P, logits, probs, heads, g, p->top_p, p->k_min, use_scores ? 1 : 0, windows,
+                                        G, glo, bits, counts, wpr, kfloor, nullptr);
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
+}
+
+sta_status launch_select_regs(const float *P, int logits, float *probs, int B, int heads, const Geo &g,
+                              const sta_mask_params *p, bool use_scores, const int *windows, int G,
+                              const GroupLo &glo, unsigned int *bits, int *counts, int wpr, int *kfloor, int *sel,
+                              cudaStream_t s) {
+  switch ((g.Nt + 255) / 256) {
+    case 1: return launch_select_regs_npl<8>(P, logits, probs, B, heads, g, p, use_scores, windows, G, glo, bits, counts, wpr, kfloor, sel, s);
+    case 2: return launch_select_regs_npl<16>(P, logits, probs, B, heads, g, p, use_scores, windows, G, glo, bits, counts, wpr, kfloor, sel, s);
+    case 3: return launch_select_regs_npl<24>(P, logits, probs, B, heads, g, p, use_scores, windows, G, glo, bits, counts, wpr, kfloor, sel, s);
+    case 4: return launch_select_regs_npl<32>(P, logits, probs, B, heads, g, p, use_scores, windows, G, glo, bits, counts, wpr, kfloor, sel, s);
+    case 5: return launch_select_regs_npl<40>(P, logits, probs, B, heads, g, p, use_scores, windows, G, glo, bits, counts, wpr, kfloor, sel, s);
+    case 6: return launch_select_regs_npl<48>(P, logits, probs, B, heads, g, p, use_scores, windows, G, glo, bits, counts, wpr, kfloor, sel, s);
+    case 7: return launch_select_regs_npl<56>(P, logits, probs, B, heads, g, p, use_scores, windows, G, glo, bits, counts, wpr, kfloor, sel, s);
+    case 8: return launch_select_regs_npl<64>(P, logits, probs, B, heads, g, p, use_scores, windows, G, glo, bits, counts, wpr, kfloor, sel, s);
+  }
+  return STA_ERR_UNSUPPORTED;
+}
+
 // ws_bytes decides the layout. With the full workspace the scores run on
 // the tensor cores into a row buffer (the caller's block_probs when given)
 // and a separate, smaller select pass does the softmax and the selection;
@@ -273,22 +318,33 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
       P_sel = rows;
       logits = 1;
     }
-    const size_t smem = select_smem(D, g, use_scores, SEL_QB_SELECT, SEL_SELECT);
-    auto kern = score_select_kernel<D, SEL_QB_SELECT, SEL_SELECT>;
-    if (smem > 48 * 1024)
-      STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    dim3 grid((unsigned)((g.Nt + SEL_QB_SELECT - 1) / SEL_QB_SELECT), (unsigned)(B * heads));
-    if (floor) {
-      kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, nullptr, 0, glo,
-                                           bits, counts, nullptr, wpr, nullptr, sel, P_sel, logits);
-      STA_CUDA_TRY(cudaGetLastError());
-      head_floor_kernel<<<(unsigned)(B * heads), FLOOR_THREADS, 0, s>>>(sel, kfloor, g);
+    // Rows of up to 2048 key tiles held in registers (scores to softmax, or
+    // window-only rows); caller-given block scores, whose rows need not sum
+    // to one, and longer rows take the general select pass (64-bit sums).
+    const bool in_regs = g.Nt <= 32 * sel::MAX_NPL && (!use_scores || logits);
+    if (in_regs) {
+      const sta_status st = launch_select_regs(P_sel, logits, block_probs, B, heads, g, p, use_scores, windows, G,
+                                               glo, bits, counts, wpr, floor ? kfloor : nullptr, floor ? sel : nullptr,
+                                               s);
+      if (st != STA_OK) return st;
+    } else {
+      const size_t smem = select_smem(D, g, use_scores, SEL_QB_SELECT, SEL_SELECT);
+      auto kern = score_select_kernel<D, SEL_QB_SELECT, SEL_SELECT>;
+      if (smem > 48 * 1024)
+        STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+      dim3 grid((unsigned)((g.Nt + SEL_QB_SELECT - 1) / SEL_QB_SELECT), (unsigned)(B * heads));
+      if (floor) {
+        kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, 1, nullptr, 0, glo,
+                                             bits, counts, nullptr, wpr, nullptr, sel, P_sel, logits);
+        STA_CUDA_TRY(cudaGetLastError());
+        head_floor_kernel<<<(unsigned)(B * heads), FLOOR_THREADS, 0, s>>>(sel, kfloor, g);
+        STA_CUDA_TRY(cudaGetLastError());
+      }
+      kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, use_scores ? 1 : 0,
+                                           windows, G, glo, bits, counts, block_probs, wpr,
+                                           floor ? kfloor : nullptr, nullptr, P_sel, logits);
       STA_CUDA_TRY(cudaGetLastError());
     }
-    kern<<<grid, SEL_THREADS, smem, s>>>(qbar, kbar, heads, g, scale, p->top_p, p->k_min, use_scores ? 1 : 0,
-                                         windows, G, glo, bits, counts, block_probs, wpr,
-                                         floor ? kfloor : nullptr, nullptr, P_sel, logits);
-    STA_CUDA_TRY(cudaGetLastError());
   }
   scan_kernel<<<1, SCAN_THREADS, 0, s>>>(counts, row_ptr, reinterpret_cast<long long *>(nnz_dev), R);
   STA_CUDA_TRY(cudaGetLastError());
@@ -381,6 +437,21 @@ size_t sta_build_mask_workspace_min(int32_t B, int32_t heads, int32_t d, sta_gri
   sta_status st = STA_OK;
   if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return 0;
   return mask_ws_layout(B, heads, d, geo).total_min;
+}
+
+sta_status sta_build_mask_pooled_offsets(int32_t B, int32_t heads, int32_t d, sta_grid g, size_t ws_bytes,
+                                         size_t offsets[4]) {
+  Geo geo;
+  sta_status st = STA_OK;
+  if (offsets == nullptr) return STA_ERR_INVALID_ARG;
+  if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return st;
+  const MaskWs L = mask_ws_layout(B, heads, d, geo);
+  const bool split = ws_bytes >= L.total;
+  offsets[0] = L.qbar;
+  offsets[1] = L.kbar;
+  offsets[2] = split ? L.qlo : 0;
+  offsets[3] = split ? L.klo : 0;
+  return STA_OK;
 }
 
 static sta_status build_mask_any(const void *q_tiled, const void *k_tiled, int32_t B, int32_t heads,

@@ -184,30 +184,48 @@ struct GroupLo {
   int v[STA_MAX_GROUPS];
 };
 
+constexpr float LOG2E_F = 1.4426950408889634f;
+
+// 2^x on the MUFU unit (ex2.approx.ftz.f32: relative error below 2^-22).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// A caller-given block score clamped to [0, 1], with -0 taken to +0 (the
+// selection orders P by its bit pattern).
+__device__ __forceinline__ float clamp_unit(float x) { return __fadd_rn(fminf(fmaxf(x, 0.0f), 1.0f), 0.0f); }
+
 __device__ __forceinline__ unsigned int warp_sum_u32(unsigned int x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
 }
 
-// Row softmax in fp32 over Sr[0, nt): maximum, expf, a fixed-order sum
-// (lane-strided partial sums, then a butterfly), IEEE divide. P replaces the
-// scores in Sr and is copied to out when given.
+// Row softmax in fp32 over Sr[0, nt): the maximum m, e = 2^(s log2e - m log2e)
+// (one FFMA, ex2.approx), the sum Z in a fixed order (lane-strided partial
+// sums in index order, then a butterfly over the lanes), P = e * (1 / Z) with
+// the reciprocal rounded once. P replaces the scores in Sr and is copied to
+// out when given. The register-resident select pass computes the same P bit
+// for bit (same operations in the same order).
 __device__ __forceinline__ void row_softmax(float *Sr, int nt, int lane, float *out) {
   float mx = -INFINITY;
   for (int j = lane; j < nt; j += 32) mx = fmaxf(mx, Sr[j]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float ml = mx * LOG2E_F;
   float sum = 0.0f;
   for (int j = lane; j < nt; j += 32) {
-    const float e = expf(Sr[j] - mx);
+    const float e = ex2_approx(fmaf(Sr[j], LOG2E_F, -ml));
     Sr[j] = e;
     sum += e;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float rz = __frcp_rn(sum);
   for (int j = lane; j < nt; j += 32) {
-    const float p = Sr[j] / sum;
+    const float p = Sr[j] * rz;
     Sr[j] = p;
     if (out) out[j] = p;
   }
@@ -218,15 +236,19 @@ __device__ __forceinline__ unsigned int mass_of(float p) {
 }
 
 // Total mass (or count when `count_only`) of the row entries whose P bit
-// pattern is >= `key`. P >= 0, so float bits order like the values.
-__device__ __forceinline__ unsigned int mass_at_least(const float *row, int nt, unsigned int key,
-                                                      bool count_only, int lane) {
-  unsigned int s = 0;
+// pattern is >= `key`. P >= 0, so float bits order like the values. 64-bit:
+// a row of caller-given block scores (each clamped to [0, 1], not normalised)
+// can hold up to Nt * 2^24 of mass.
+__device__ __forceinline__ unsigned long long mass_at_least(const float *row, int nt, unsigned int key,
+                                                            bool count_only, int lane) {
+  unsigned long long s = 0;
   for (int j = lane; j < nt; j += 32) {
     const float p = row[j];
     if (__float_as_uint(p) >= key) s += count_only ? 1u : mass_of(p);
   }
-  return warp_sum_u32(s);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
 }
 
 // Radix select over the P bit patterns (P >= 0, so the bits order like the
@@ -235,40 +257,42 @@ __device__ __forceinline__ unsigned int mass_at_least(const float *row, int nt, 
 // a time from the most significant (bits 30-23, 22-15, 14-7, 6-0), with a
 // per-warp histogram of 256 bins in shared memory. Also returns f restricted
 // to entries strictly above v. target must be >= 1 and f(0) >= target.
-// All sums are integers, so the result does not depend on summation order.
-__device__ void radix_level(const float *row, int nt, unsigned int target, bool count_only, int lane,
-                            unsigned int *hist, unsigned int &v_out, unsigned int &above_out) {
-  unsigned int prefix = 0u, pmask = 0u, above = 0u;
+// All sums are 64-bit integers, so the result does not depend on summation
+// order.
+__device__ void radix_level(const float *row, int nt, unsigned long long target, bool count_only, int lane,
+                            unsigned long long *hist, unsigned int &v_out, unsigned long long &above_out) {
+  unsigned int prefix = 0u, pmask = 0u;
+  unsigned long long above = 0ull;
 #pragma unroll
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = pass == 0 ? 23 : (pass == 1 ? 15 : (pass == 2 ? 7 : 0));
     const unsigned int dmask = pass == 3 ? 0x7Fu : 0xFFu;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) hist[i * 32 + lane] = 0u;
+    for (int i = 0; i < 8; ++i) hist[i * 32 + lane] = 0ull;
     __syncwarp();
     for (int j = lane; j < nt; j += 32) {
       const unsigned int b = __float_as_uint(row[j]);
       // entries of zero mass add nothing to a mass histogram: no atomic
       const unsigned int add = count_only ? 1u : mass_of(__uint_as_float(b));
-      if ((b & pmask) == prefix && add != 0u) atomicAdd(hist + ((b >> shift) & dmask), add);
+      if ((b & pmask) == prefix && add != 0u) atomicAdd(hist + ((b >> shift) & dmask), (unsigned long long)add);
     }
     __syncwarp();
     // lane owns digits [8*lane, 8*lane + 8)
-    unsigned int hb[8], own = 0u;
+    unsigned long long hb[8], own = 0ull;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       hb[k] = hist[8 * lane + k];
       own += hb[k];
     }
-    unsigned int suffix = own;  // digits owned by this lane and all higher lanes
+    unsigned long long suffix = own;  // digits owned by this lane and all higher lanes
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const unsigned int y = __shfl_down_sync(0xffffffffu, suffix, o);
+      const unsigned long long y = __shfl_down_sync(0xffffffffu, suffix, o);
       if (lane + o < 32) suffix += y;
     }
-    unsigned int run = above + (suffix - own);
+    unsigned long long run = above + (suffix - own);
     int found = -1;
-    unsigned int above_found = 0u;
+    unsigned long long above_found = 0ull;
 #pragma unroll
     for (int k = 7; k >= 0; --k) {
       if (found < 0 && run + hb[k] >= target) {
@@ -318,11 +342,11 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
   // is a multiple of 8)
   float *qs = sm;
   float *S = qs + ((HAS_SCORES && use_scores) ? QB * D : 0);
-  unsigned int *hist = reinterpret_cast<unsigned int *>(S + (use_scores ? QB * nt : 0));
+  unsigned long long *hist = reinterpret_cast<unsigned long long *>(S + (use_scores ? QB * nt : 0));
   int *gtab = reinterpret_cast<int *>(hist + (use_scores ? (SEL_THREADS / 32) * 256 : 0));
   int *wtab = gtab + ((g.T + 3) & ~3);  // 4 ints per group
   unsigned int *wwin = reinterpret_cast<unsigned int *>(wtab + 4 * STA_MAX_GROUPS) + warp * wpr;
-  unsigned int *whist = hist + warp * 256;
+  unsigned long long *whist = hist + warp * 256;
 
   // Window tables, once per CTA: the temporal group of every |dt| and this
   // head's extents.
@@ -411,7 +435,7 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
       } else if (!HAS_SCORES || P_in != nullptr) {
         // caller-supplied block scores (e.g. exact block masses), clamped to [0, 1]
         for (int j = lane; j < nt; j += 32) {
-          const float p = fminf(fmaxf(P_in[row * nt + j], 0.0f), 1.0f);
+          const float p = clamp_unit(P_in[row * nt + j]);
           Sr[j] = p;
           if (pout) pout[j] = p;
         }
@@ -430,25 +454,26 @@ score_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
         m_p_ties = 0xFFFFFFFFu;
         m_p = nt;
       } else if (top_p > 0.0f) {
-        const unsigned int W = mass_at_least(Sr, nt, 0u, false, lane);
-        const double thr_d = ceil((double)top_p * (double)W);
-        const unsigned int thr = (unsigned int)thr_d;
-        if (thr > 0u) {
-          unsigned int v, above;
+        const unsigned long long W = mass_at_least(Sr, nt, 0u, false, lane);
+        const unsigned long long thr = (unsigned long long)ceil((double)top_p * (double)W);
+        if (thr > 0ull) {
+          unsigned int v;
+          unsigned long long above;
           radix_level(Sr, nt, thr, false, lane, whist, v, above);
-          const unsigned int wv = mass_of(__uint_as_float(v));
-          const unsigned int need = (thr - above + wv - 1u) / wv;  // tied entries at level v
-          const unsigned int cnt_above = mass_at_least(Sr, nt, v + 1u, true, lane);
+          const unsigned long long wv = mass_of(__uint_as_float(v));
+          const unsigned int need = (unsigned int)((thr - above + wv - 1ull) / wv);  // tied entries at level v
+          const unsigned int cnt_above = (unsigned int)mass_at_least(Sr, nt, v + 1u, true, lane);
           m_p_level = v;
           m_p_ties = need;
           m_p = (long long)cnt_above + need;
         }
       }
       if ((long long)kk > m_p) {
-        unsigned int u, cnt_above;
-        radix_level(Sr, nt, (unsigned int)kk, true, lane, whist, u, cnt_above);
+        unsigned int u;
+        unsigned long long cnt_above;
+        radix_level(Sr, nt, (unsigned long long)kk, true, lane, whist, u, cnt_above);
         v_f = u;
-        c_f = (unsigned int)kk - cnt_above;
+        c_f = (unsigned int)kk - (unsigned int)cnt_above;
       } else if (m_p > 0) {
         v_f = m_p_level;
         c_f = m_p_ties;

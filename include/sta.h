@@ -119,6 +119,20 @@ sta_status sta_reorder(const void *src, void *dst, int32_t B, int32_t heads, int
 size_t sta_build_mask_workspace(int32_t B, int32_t heads, int32_t d, sta_grid g);
 size_t sta_build_mask_workspace_min(int32_t B, int32_t heads, int32_t d, sta_grid g);
 
+/* Where sta_build_mask (and _raster) leaves the pooled means in its
+ * workspace, as byte offsets: offsets[0] = qbar, offsets[1] = kbar, each fp32
+ * [B*heads*Nt, d] with row (b*heads + h)*Nt + tile. They are written when
+ * use_scores is set and block_scores is NULL. With a workspace of at least
+ * sta_build_mask_workspace() bytes (the tensor-core layout) each mean x is
+ * stored split: tf32(x) at offsets[0] / [1] and tf32(x - tf32(x)) (round to
+ * nearest, ties away) at offsets[2] / [3]; with a smaller workspace x itself
+ * is stored and offsets[2] = offsets[3] = 0 (nothing written there). x is the
+ * mean over the real tokens of the tile, an exact sum rounded once to fp32
+ * (Rectified SpaAttn abstract: pooled query-key). Returns STA_ERR_INVALID_ARG
+ * or STA_ERR_UNSUPPORTED for sizes sta_build_mask rejects. */
+sta_status sta_build_mask_pooled_offsets(int32_t B, int32_t heads, int32_t d, sta_grid g, size_t ws_bytes,
+                                         size_t offsets[4]);
+
 /* sta_build_mask -- per-head tile mask as CSR lists (Compact Attention Fig. 3:
  * masks computed online are loaded into the block-sparse kernel; Fig. 4: the
  * result is a binary mask over (query tile, key tile)).

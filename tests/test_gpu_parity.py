@@ -142,6 +142,7 @@ def _check_mask(sta, gp, qt, kt, B, Hh, d, T, H, W, top_p, k_min, use_scores, wi
             _, p_ref = O.block_scores(qb, kb, scale)
             bound = gp.prob_bound(qb, kb, scale, p_ref)
             assert np.all(np.abs(probs - p_ref) <= bound)
+            assert np.max(np.abs(probs - p_ref) / bound) <= gp.PROB_ERR_CEILING
             # the oracle's own end-to-end mask differs only at near-threshold
             # tiles: a P within the error bound of a boundary tile's P (a
             # near-tie), or a prefix mass within the derived mass error of
@@ -640,6 +641,163 @@ def test_block_mass_720p_dense_sampled_rows(sta, gp):
     assert np.allclose(sums, 1.0, atol=1e-4)
 
 
+# ------------------------------------------ the two select passes, same P
+@pytest.mark.parametrize("top_p,k_min,floor", [(0.95, 8, False), (0.6, 1, False), (0.0, 37, False),
+                                               (0.9, 4, True), (1.0, 0, False)])
+def test_register_select_equals_general_select_on_the_same_p(sta, gp, top_p, k_min, floor):
+    """The select pass that holds the row in registers (rows from the scores)
+    and the general one (caller block scores, 64-bit sums) reach the same CSR
+    on the same P: the build's exported P fed back as block_scores (values in
+    [0, 1], so the clamp changes nothing), with windows, on a 720p-shaped grid
+    of 4 heads."""
+    T, H, W, Hh, d = 21, 45, 80, 4, 128
+    g = sta.grid(T, H, W)
+    q, k, _ = _structured(T, H, W, Hh, d, seed=77)
+    rng = np.random.default_rng(5)
+    win = torch.from_numpy(rng.integers(-1, 3, size=(Hh, 3, 4)).astype(np.int32)).cuda()
+    bufs = sta.MaskBuffers(1, Hh, d, g, "cuda", with_mask=True, with_probs=True)
+    sta.build_mask(q, k, 1, Hh, d, g, sta.mask_params(top_p, k_min, True, 0.0, (0, 1, 4), win, floor), bufs,
+                   raster=True)
+    P = bufs.block_probs.clone()
+    again = sta.MaskBuffers(1, Hh, d, g, "cuda", with_mask=True, with_probs=True)
+    sta.build_mask(None, None, 1, Hh, d, g,
+                   sta.mask_params(top_p, k_min, True, 0.0, (0, 1, 4), win, floor, block_scores=P), again)
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    assert torch.equal(again.block_probs.view(torch.int32), P.view(torch.int32))
+    n = int(bufs.nnz.item())
+    assert n == int(again.nnz.item())
+    assert torch.equal(bufs.row_ptr, again.row_ptr) and torch.equal(bufs.col_idx[:n], again.col_idx[:n])
+    assert torch.equal(bufs.block_mask, again.block_mask)
+
+
+def test_caller_block_scores_with_row_mass_beyond_32_bits(sta, gp):
+    """Caller block scores need not sum to one: rows of 1980 values in
+    [0.5, 1] carry ~2^34 of integer mass, beyond 32 bits. The selection (top-p
+    and the count floor) equals the oracle's, which sums in exact integers."""
+    T, H, W, Hh = 33, 45, 80, 2
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    gen = torch.Generator(device="cuda").manual_seed(9)
+    sc = (0.5 + 0.5 * torch.rand((1, Hh, nt, nt), generator=gen, device="cuda")).float()
+    sc[0, 0, 3, :] = 1.0  # a row of ties
+    sc[0, 1, 5, ::7] = 0.0
+    for top_p, k_min in ((0.7, 3), (0.3, 900), (0.999, 0)):
+        bufs = sta.MaskBuffers(1, Hh, 128, g, "cuda", with_mask=True)
+        sta.build_mask(None, None, 1, Hh, 128, g, sta.mask_params(top_p, k_min, True, block_scores=sc), bufs)
+        torch.cuda.synchronize()
+        assert sta.sta_get_device_error() == sta.STA_OK
+        want = O.select(sc.cpu().numpy().astype(np.float64), top_p, k_min)
+        assert np.array_equal(bufs.block_mask.cpu().numpy().astype(bool), want)
+        rp, ci = O.mask_to_csr(want)
+        got_rp, got_ci, nnz = gp.csr_np(bufs)
+        assert np.array_equal(got_rp, rp) and np.array_equal(got_ci, ci)
+
+
+def test_rows_longer_than_2048_tiles_take_the_general_select(sta, gp):
+    """Nt = 2304 (a 36 x 64 x 64 grid): past the register pass's 2048-tile
+    rows the general select pass runs; its CSR equals the oracle's selection
+    on the GPU's P, and P is within the bound."""
+    T, H, W, Hh, d = 36, 64, 64, 1, 64
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    assert nt > 2048
+    q, k, _ = _structured(T, H, W, Hh, d, seed=3)
+    qt, kt = gp.reorder(q, 1, Hh, d, g), gp.reorder(k, 1, Hh, d, g)
+    bufs = gp.build(qt, kt, 1, Hh, d, g, sta.mask_params(0.9, 5, True))
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    probs = bufs.block_probs.cpu().numpy()
+    rows = np.random.default_rng(0).choice(nt, 64, replace=False)
+    want = O.select(probs[0, 0, rows].astype(np.float64), 0.9, 5)
+    assert np.array_equal(bufs.block_mask.cpu().numpy()[0, 0, rows].astype(bool), want)
+    scale = 1.0 / math.sqrt(d)
+    qb, kb = O.pool(gp.to_np64(qt), T, H, W), O.pool(gp.to_np64(kt), T, H, W)
+    _, p_ref = O.block_scores(qb[:, :, rows], kb, scale)
+    bound = gp.prob_bound(qb[:, :, rows], kb, scale, p_ref)
+    assert np.all(np.abs(probs[:, :, rows] - p_ref) <= bound)
+    assert np.max(np.abs(probs[:, :, rows] - p_ref) / bound) <= gp.PROB_ERR_CEILING
+
+
+# ------------------------------------------------ pooled means (a2), directly
+def _rna_tf32(x32):
+    """fp32 -> the nearest tf32 (10 explicit mantissa bits), ties away from
+    zero: half a tf32 unit added to the magnitude bits, then the 13 low bits
+    cleared (the sign bit is untouched)."""
+    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32)
+    return ((u + np.uint32(0x1000)) & np.uint32(0xFFFFE000)).view(np.float32)
+
+
+def _pooled_from_ws(sta, ws, B, Hh, d, g, ws_bytes):
+    nt = sta.sta_num_tiles(g)
+    R = B * Hh * nt
+    off = sta.sta_build_mask_pooled_offsets(B, Hh, d, g, ws_bytes)
+
+    def at(o):
+        return ws[o:o + R * d * 4].view(torch.float32).view(B, Hh, nt, d).cpu().numpy()
+
+    return at(off[0]), at(off[1]), (at(off[2]) if off[2] else None), (at(off[3]) if off[3] else None)
+
+
+@pytest.mark.parametrize("T,H,W,Hh,d,B,raster,full_ws", [
+    (3, 19, 37, 3, 128, 2, True, True), (3, 19, 37, 3, 128, 2, False, True),
+    (3, 19, 37, 3, 128, 2, False, False), (5, 24, 37, 6, 64, 1, True, True),
+    (2, 9, 10, 10, 128, 1, True, False), (1, 8, 8, 1, 64, 1, False, True)])
+def test_pooled_means_bit_exact(sta, gp, T, H, W, Hh, d, B, raster, full_ws):
+    """q-bar and k-bar as the mask build leaves them in its workspace, against
+    the oracle's fp64 tile means: both sides sum the bf16 values exactly and
+    divide by the real-token count in fp64, so the GPU's one rounding to fp32
+    gives fp32(oracle mean) bit for bit; in the tensor-core layout the two
+    stored parts are tf32(x) and tf32(x - tf32(x)), round to nearest, ties
+    away (ragged grids, partial head boxes, raster and tiled pooling)."""
+    g = sta.grid(T, H, W)
+    q, k, _ = _structured(T, H, W, Hh, d, seed=41 + H, B=B)
+    src = (q, k) if raster else (gp.reorder(q, B, Hh, d, g), gp.reorder(k, B, Hh, d, g))
+    ws_bytes = (sta.sta_build_mask_workspace if full_ws else sta.sta_build_mask_workspace_min)(B, Hh, d, g)
+    bufs = sta.MaskBuffers(B, Hh, d, g, "cuda")
+    ws = torch.full((ws_bytes,), 0xFF, dtype=torch.uint8, device="cuda")
+    params = sta.mask_params(0.9, 2, True)
+    fn = sta.sta_build_mask_raster if raster else sta.sta_build_mask
+    fn(src[0], src[1], B, Hh, d, g, params, bufs.row_ptr, bufs.col_idx, bufs.nnz, None, None, ws, ws_bytes)
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    qb, kb, qlo, klo = _pooled_from_ws(sta, ws, B, Hh, d, g, ws_bytes)
+    for got, lo, x in ((qb, qlo, q), (kb, klo, k)):
+        want = O.pool(O.reorder_fwd(gp.to_np64(x), T, H, W), T, H, W).astype(np.float32)
+        if full_ws:
+            hi = _rna_tf32(want)
+            assert np.array_equal(got.view(np.uint32), hi.view(np.uint32))
+            assert np.array_equal(lo.view(np.uint32), _rna_tf32(want - hi).view(np.uint32))
+        else:
+            assert lo is None
+            assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+def test_pooled_means_bit_exact_720p_sampled_heads(sta, gp):
+    """The 720p layer in the benchmark's launch configuration (raster pooling
+    through the TMA ring, full workspace): three sampled heads, every tile."""
+    cfg = CONFIGS["dit720p"]
+    B, Hh, d, T, H, W = cfg.B, cfg.heads, cfg.d, cfg.T, cfg.H, cfg.W
+    g = sta.grid(T, H, W)
+    q, k, _ = make_qkv(cfg, device="cuda")
+    ws_bytes = sta.sta_build_mask_workspace(B, Hh, d, g)
+    bufs = sta.MaskBuffers(B, Hh, d, g, "cuda")
+    ws = torch.full((ws_bytes,), 0xFF, dtype=torch.uint8, device="cuda")
+    params = sta.mask_params(cfg.top_p, cfg.k_min, True)
+    sta.sta_build_mask_raster(q, k, B, Hh, d, g, params, bufs.row_ptr, bufs.col_idx, bufs.nnz, None, None, ws,
+                              ws_bytes)
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    qb, kb, qlo, klo = _pooled_from_ws(sta, ws, B, Hh, d, g, ws_bytes)
+    heads = [0, 17, 39]
+    for got, lo, x in ((qb, qlo, q), (kb, klo, k)):
+        sub = gp.to_np64(x[:, :, heads, :])
+        want = O.pool(O.reorder_fwd(sub, T, H, W), T, H, W).astype(np.float32)
+        hi = _rna_tf32(want)
+        assert np.array_equal(got[:, heads].view(np.uint32), hi.view(np.uint32))
+        assert np.array_equal(lo[:, heads].view(np.uint32), _rna_tf32(want - hi).view(np.uint32))
+
+
 # ------------------------------------------ recall-driven window search (f2)
 def _local_masses(T, H, W, shapes):
     """One [Nt, Nt] row-normalised mass per (st, sy, sx) spread of a Gaussian
@@ -799,6 +957,7 @@ def test_build_mask_fused_and_tensor_core_layouts(sta, gp, floor, d):
         probs = bufs.block_probs.cpu().numpy()
         bound = gp.prob_bound(qb, kb, scale, p_ref, fused=fused)
         assert np.all(np.abs(probs.astype(np.float64) - p_ref) <= bound)
+        assert np.max(np.abs(probs.astype(np.float64) - p_ref) / bound) <= gp.PROB_ERR_CEILING
         sel = _floor_mask(probs, top_p, k_min, sizes) if floor else O.select(probs, top_p, k_min)
         mask = sel | wmask
         assert np.array_equal(bufs.block_mask.cpu().numpy().astype(bool), mask)

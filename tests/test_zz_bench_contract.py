@@ -48,3 +48,13 @@ def test_bench_json_line():
     b = d["build_roofline"]
     assert b["bound"] == "hbm" and b["unit"] == "GB/s" and 0 < b["frac"] < 1.5
     assert abs(b["frac"] - b["achieved"] / b["peak"]) < 1e-9
+    assert abs(r["frac_burst"] - r["achieved"] / r["peak_burst"]) < 1e-9
+    # every other layer of the workload table: 480p, 129 frames at four
+    # densities, the reuse layer at five
+    rows = d["per_config"]
+    assert [x["workload"].split("_")[0] for x in rows] == ["dit480p"] + ["dit720p129f"] * 4 + ["reuse"] * 5, \
+        [x["workload"] for x in rows]
+    for x in rows:
+        assert x["attn_ms"] > 0 and x["build_ms"] > 0 and x["kept_pairs"] > 0
+        assert 0 < x["frac_burst"] <= x["frac_sustained"] < 1.5 and 0 < x["pairing_efficiency"] <= 1.0
+        assert isinstance(x["clocks"]["reasons"], list)
