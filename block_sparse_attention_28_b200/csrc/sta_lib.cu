@@ -187,7 +187,8 @@ __global__ void selftest_wait_kernel(long long limit) {
 }
 
 // The select pass with the row in registers (sel::select_rows_kernel<NPL>,
-// NPL = ceil(Nt / 32) rounded up to a multiple of 8). With the per-head floor
+// NPL = ceil(Nt / 32) rounded up to a multiple of 8), on rows of scores to be
+// softmaxed (P) or window-only rows (P unused). With the per-head floor
 // (kfloor != nullptr) it runs twice around head_floor_kernel: first for the
 // base counts only (sel_count), then with k_min raised to the floor.
 template <int NPL>
@@ -201,14 +202,14 @@ sta_status launch_select_regs_npl(const float *P, int logits, float *probs, int 
   STA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   dim3 grid((unsigned)((g.Nt + sel::WARPS - 1) / sel::WARPS), (unsigned)(B * heads));
   if (kfloor != nullptr) {
-    kern<<<grid, sel::THREADS, smem, s>>>(P, logits, nullptr, heads, g, p->top_p, p->k_min, 1, nullptr, 0, glo,
-                                          bits, counts, wpr, nullptr, sel);
+    kern<<<grid, sel::THREADS, smem, s>>>(P, nullptr, heads, g, p->top_p, p->k_min, 1, nullptr, 0, glo, bits, counts,
+                                          wpr, nullptr, sel);
     STA_CUDA_TRY(cudaGetLastError());
     head_floor_kernel<<<(unsigned)(B * heads), FLOOR_THREADS, 0, s>>>(sel, kfloor, g);
     STA_CUDA_TRY(cudaGetLastError());
   }
-  kern<<<grid, sel::THREADS, smem, s>>>(P, logits, probs, heads, g, p->top_p, p->k_min, use_scores ? 1 : 0, windows,
-                                        G, glo, bits, counts, wpr, kfloor, nullptr);
+  kern<<<grid, sel::THREADS, smem, s>>>(P, probs, heads, g, p->top_p, p->k_min, use_scores ? 1 : 0, windows, G, glo,
+                                        bits, counts, wpr, kfloor, nullptr);
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }

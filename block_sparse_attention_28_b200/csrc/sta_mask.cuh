@@ -193,6 +193,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Three-input maximum (one instruction).
+__device__ __forceinline__ float fmax3_f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // A caller-given block score clamped to [0, 1], with -0 taken to +0 (the
 // selection orders P by its bit pattern).
 __device__ __forceinline__ float clamp_unit(float x) { return __fadd_rn(fminf(fmaxf(x, 0.0f), 1.0f), 0.0f); }

@@ -53,99 +53,88 @@ inline size_t smem_bytes(int npl, int wpr, int T) {
   return (tables + (size_t)WARPS * (u + 256 + ((wpr + 3) & ~3))) * 4;
 }
 
-// Weight of a P pattern in level 1: mass w = floor(P 2^24) in bits 0-24 and
-// a count of 1 in bits 25-31 (a lane adds at most NPL <= 64 entries to a bin,
-// and its masses sum to at most 2^24 (1 + Nt 2^-24) < 2^25).
+// Level 1 of the threshold search: a private histogram per lane (its own
+// column of [32 bins][32 lanes], so no two lanes ever add to the same word)
+// of the entries' weight over 32 bins of the exponent of P. By mass: bin =
+// exponent - 103 for the entries with mass (P >= 2^-24, exponent 103 .. 127),
+// each adding its mass w = floor(P 2^24) and a count of 1 packed as
+// w + 2^25 (a lane's masses in a bin sum below 2^25). Entries of zero mass,
+// the row's padding among them (P = 0), are left out. By count (top-k):
+// bin = max(exponent - 96, 0), each valid entry adding a count of 1 (2^25).
 constexpr uint32_t CNT_ONE = 1u << 25;
 constexpr uint32_t MASS_MASK = CNT_ONE - 1u;
 
-// Level 1: private per-lane histograms over bin = exponent(P) - base,
-// clamped to [0, 31] (mass: entries with no mass are left out, and base is
-// the exponent of 2^-24, so the bins are exact exponents). Returns the bin
-// b* where the weight at or above it first reaches `target` (scanning from
-// the top bin) and the mass and count strictly above b*. target >= 1 and the
-// row's total weight is >= target.
 template <int NPL>
-__device__ __forceinline__ void level1(const uint32_t (&pb)[NPL], int nt, int lane, bool mass, uint32_t target,
-                                       uint32_t *h, int &bstar, uint32_t &mass_above, uint32_t &cnt_above) {
-  const int base = mass ? MASS_BASE : COUNT_BASE;
+__device__ __forceinline__ void hist_mass(const uint32_t (&pb)[NPL], int lane, uint32_t *h) {
 #pragma unroll
   for (int b = 0; b < 32; ++b) h[b * 32 + lane] = 0u;
   __syncwarp();
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
-    if (32 * i + lane < nt) {
-      const uint32_t b = pb[i];
-      const uint32_t w = mass_of(__uint_as_float(b));
-      int bin = (int)(b >> 23) - base;
-      bin = bin < 0 ? 0 : (bin > 31 ? 31 : bin);
-      if (!mass || w != 0u) atomicAdd(h + bin * 32 + lane, w + CNT_ONE);  // private column: no conflicts
+    const uint32_t ex = pb[i] >> 23;
+    if (ex >= (uint32_t)MASS_BASE)
+      atomicAdd(h + (ex - MASS_BASE) * 32 + lane, mass_of(__uint_as_float(pb[i])) + CNT_ONE);
+  }
+  __syncwarp();
+}
+
+template <int NPL>
+__device__ __forceinline__ void hist_count(const uint32_t (&pb)[NPL], int nv, int lane, uint32_t *h) {
+#pragma unroll
+  for (int b = 0; b < 32; ++b) h[b * 32 + lane] = 0u;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    if (i < nv) {
+      const int bin = max((int)(pb[i] >> 23) - COUNT_BASE, 0);
+      atomicAdd(h + bin * 32 + lane, CNT_ONE);
     }
   }
   __syncwarp();
-  // lane l totals bin l over the 32 columns, reading diagonally (conflict-free)
-  uint32_t m = 0u, c = 0u;
-#pragma unroll 8
-  for (int t = 0; t < 32; ++t) {
-    const uint32_t x = h[lane * 32 + ((lane + t) & 31)];
-    m += x & MASS_MASK;
-    c += x >> 25;
-  }
-  // weight at or above each bin (suffix sums from the top bin)
-  const uint32_t own = mass ? m : c;
-  uint32_t suf = own, sufc = c, sufm = m;
+}
+
+// Lane l's total of bin l over the 32 columns (read diagonally: conflict-free),
+// summed as packed words in 64 bits (mass below bit 25, count above).
+__device__ __forceinline__ unsigned long long bin_total(const uint32_t *h, int lane) {
+  unsigned long long acc = 0ull;
+  const uint32_t *rowp = h + lane * 32;
+#pragma unroll
+  for (int t = 0; t < 32; ++t) acc += rowp[(lane + t) & 31];
+  return acc;
+}
+
+// The bin b* where the weight at or above it, scanning down from the top bin,
+// first reaches `target` (1 <= target <= total), with the weight and count
+// strictly above b*.
+__device__ __forceinline__ void find_bin(uint32_t own_w, uint32_t own_c, uint32_t target, int lane, int &bstar,
+                                         uint32_t &w_above, uint32_t &c_above) {
+  uint32_t suf = own_w, sufc = own_c;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t y = __shfl_down_sync(0xffffffffu, suf, o);
     const uint32_t yc = __shfl_down_sync(0xffffffffu, sufc, o);
-    const uint32_t ym = __shfl_down_sync(0xffffffffu, sufm, o);
     if (lane + o < 32) {
       suf += y;
       sufc += yc;
-      sufm += ym;
     }
   }
   const uint32_t hit = __ballot_sync(0xffffffffu, suf >= target);
   bstar = 31 - __clz((int)hit);
-  mass_above = __shfl_sync(0xffffffffu, sufm - m, bstar);
-  cnt_above = __shfl_sync(0xffffffffu, sufc - c, bstar);
-  __syncwarp();  // the histograms are reused as candidate columns
+  w_above = __shfl_sync(0xffffffffu, suf - own_w, bstar);
+  c_above = __shfl_sync(0xffffffffu, sufc - own_c, bstar);
 }
 
-// Appends the entries of bin b* to the lane's candidate column
-// (cand[k * 32 + lane], k < returned count).
-template <int NPL>
-__device__ __forceinline__ int collect(const uint32_t (&pb)[NPL], int nt, int lane, bool mass, int bstar,
-                                       uint32_t *cand) {
-  const int base = mass ? MASS_BASE : COUNT_BASE;
-  int k = 0;
-#pragma unroll
-  for (int i = 0; i < NPL; ++i) {
-    const uint32_t b = pb[i];
-    int bin = (int)(b >> 23) - base;
-    bin = bin < 0 ? 0 : (bin > 31 ? 31 : bin);
-    const bool in = (32 * i + lane < nt) && bin == bstar && (!mass || mass_of(__uint_as_float(b)) != 0u);
-    if (in) cand[(k++) * 32 + lane] = b;
-  }
-  __syncwarp();
-  return k;
-}
-
-// Level 2: radix select over the candidates, digit passes from `first`
-// (0: bits 30-23, 1: 22-15, 2: 14-7, 3: 6-0): the largest pattern v whose
-// weight at or above reaches `target`, and the weight of the candidates
-// strictly above v. Per-warp 256-bin histogram; integer sums.
-__device__ __forceinline__ void level2(const uint32_t *cand, int k, int first, uint32_t target, bool count_only,
-                                       int lane, uint32_t *hist, uint32_t &v_out, uint32_t &above_out) {
+// Level 2: radix select over the candidates (lane l's in cand[k * 32 + l],
+// k < its count), digit passes from `first` (0: bits 30-23, 1: 22-15,
+// 2: 14-7, 3: 6-0), `prefix0` holding the bits above the first pass: the
+// largest pattern v whose weight at or above reaches `target`, and the weight
+// of the candidates strictly above v. Per-warp 256-bin histogram; integer sums.
+__device__ __forceinline__ void level2(const uint32_t *cand, int k, int first, uint32_t prefix0, uint32_t target,
+                                       bool count_only, int lane, uint32_t *hist, uint32_t &v_out,
+                                       uint32_t &above_out) {
   const int kmax = __reduce_max_sync(0xffffffffu, k);
-  uint32_t prefix = 0u, pmask = 0u, above = 0u;
-  if (first > 0) {
-    // the candidates share the bits above the first pass: take them from any
-    const int src = __ffs(__ballot_sync(0xffffffffu, k > 0)) - 1;
-    const uint32_t any = __shfl_sync(0xffffffffu, k > 0 ? cand[lane] : 0u, src);
-    pmask = first == 1 ? 0xFF800000u : (first == 2 ? 0xFFFF8000u : 0xFFFFFF80u);
-    prefix = any & pmask;
-  }
+  uint32_t prefix = prefix0, above = 0u;
+  uint32_t pmask = first == 0 ? 0u : (first == 1 ? 0xFF800000u : (first == 2 ? 0xFFFF8000u : 0xFFFFFF80u));
   for (int pass = first; pass < 4; ++pass) {
     const int shift = pass == 0 ? 23 : (pass == 1 ? 15 : (pass == 2 ? 7 : 0));
     const uint32_t dmask = pass == 3 ? 0x7Fu : 0xFFu;
@@ -156,7 +145,7 @@ __device__ __forceinline__ void level2(const uint32_t *cand, int k, int first, u
       if (j < k) {
         const uint32_t b = cand[j * 32 + lane];
         const uint32_t add = count_only ? 1u : mass_of(__uint_as_float(b));
-        if ((b & pmask) == prefix && add != 0u) atomicAdd(hist + ((b >> shift) & dmask), add);
+        if ((b & pmask) == prefix) atomicAdd(hist + ((b >> shift) & dmask), add);
       }
     }
     __syncwarp();
@@ -196,9 +185,9 @@ __device__ __forceinline__ void level2(const uint32_t *cand, int k, int first, u
   above_out = above;
 }
 
-// Number of candidates strictly above v and equal to v (warp totals).
-__device__ __forceinline__ void cand_counts(const uint32_t *cand, int k, uint32_t v, int lane, uint32_t &gt,
-                                            uint32_t &eq) {
+// Candidates strictly above v and equal to v (warp totals).
+__device__ __forceinline__ void cand_counts(const uint32_t *cand, int k, uint32_t v, uint32_t &gt, uint32_t &eq,
+                                            int lane) {
   uint32_t g = 0u, e = 0u;
   for (int j = 0; j < k; ++j) {
     const uint32_t b = cand[j * 32 + lane];
@@ -209,40 +198,17 @@ __device__ __forceinline__ void cand_counts(const uint32_t *cand, int k, uint32_
   eq = __reduce_add_sync(0xffffffffu, e);
 }
 
-// Selection by weight: the pattern v of the entry where the weight (mass or
-// count) in P-descending order first reaches target, the number of entries
-// strictly above v and equal to v, and the weight strictly above v.
+// One warp per row r = (b*heads + h)*Nt + q0 + warp; the row's scores come
+// from P_in (softmaxed here) unless the mask is window-only. kmin_head
+// (per-head floor, second pass) raises k_min; sel_count (first pass of the
+// floor) records the selected count and skips the bitset. Entries past Nt
+// get P = 0: they carry no mass, so the top-p path needs no validity test;
+// the count path (top-k) and a threshold at P = 0 test it explicitly.
 template <int NPL>
-__device__ __forceinline__ void threshold(const uint32_t (&pb)[NPL], int nt, int lane, bool mass, uint32_t target,
-                                          uint32_t *wsm, uint32_t &v, uint32_t &n_gt, uint32_t &n_eq,
-                                          uint32_t &w_above) {
-  int bstar;
-  uint32_t m_above, c_above;
-  level1<NPL>(pb, nt, lane, mass, target, wsm, bstar, m_above, c_above);
-  uint32_t *cand = wsm;
-  const int k = collect<NPL>(pb, nt, lane, mass, bstar, cand);
-  const uint32_t a1 = mass ? m_above : c_above;
-  // bins above 0 are exact exponents; bin 0 of the count mode mixes exponents
-  const int first = (!mass && bstar == 0) ? 0 : 1;
-  uint32_t above_c;
-  level2(cand, k, first, target - a1, !mass, lane, wsm + Ws<NPL>::HIST, v, above_c);
-  uint32_t gt_c, eq_c;
-  cand_counts(cand, k, v, lane, gt_c, eq_c);
-  n_gt = c_above + gt_c;
-  n_eq = eq_c;
-  w_above = a1 + above_c;
-  __syncwarp();
-}
-
-// One warp per row r = (b*heads + h)*Nt + q0 + warp; the row's scores
-// (p_logits: softmax first) or block scores (clamped to [0, 1]) come from
-// P_in. kmin_head (per-head floor, second pass) raises k_min; sel_count
-// (first pass of the floor) records the selected count and skips the bitset.
-template <int NPL>
-__global__ void __launch_bounds__(THREADS, 2)
-select_rows_kernel(const float *__restrict__ P_in, int p_logits, float *__restrict__ probs_out, int heads,
-                   Geo g, float top_p, int k_min, int use_scores, const int *__restrict__ windows, int G,
-                   GroupLo glo, unsigned int *__restrict__ bits, int *__restrict__ counts, int wpr,
+__global__ void __launch_bounds__(THREADS, NPL <= 40 ? 3 : 2)
+select_rows_kernel(const float *__restrict__ P_in, float *__restrict__ probs_out, int heads, Geo g, float top_p,
+                   int k_min, int use_scores, const int *__restrict__ windows, int G, GroupLo glo,
+                   unsigned int *__restrict__ bits, int *__restrict__ counts, int wpr,
                    const int *__restrict__ kmin_head, int *__restrict__ sel_count) {
   extern __shared__ __align__(16) uint32_t smw[];
   const int nt = g.Nt;
@@ -255,6 +221,7 @@ select_rows_kernel(const float *__restrict__ P_in, int p_logits, float *__restri
   uint32_t *wsm = reinterpret_cast<uint32_t *>(wtab + 4 * STA_MAX_GROUPS) +
                   warp * (Ws<NPL>::WIN + ((wpr + 3) & ~3));
   uint32_t *wwin = wsm + Ws<NPL>::WIN;
+  uint32_t *hist2 = wsm + Ws<NPL>::HIST;
 
   if (windows != nullptr) {
     for (int dt = tid; dt < g.T; dt += THREADS) {
@@ -270,6 +237,7 @@ select_rows_kernel(const float *__restrict__ P_in, int p_logits, float *__restri
   const int qt = blockIdx.x * WARPS + warp;
   if (qt >= nt) return;
   const long long row = (long long)bh * nt + qt;
+  const int nv = (nt - lane + 31) >> 5;  // valid entries of this lane: i < nv
 
   uint32_t v_f = NONE, c_f = 0u;  // keep P > v_f, plus the first c_f ties at v_f
   uint32_t eq_f = 0u;              // entries equal to v_f
@@ -278,37 +246,30 @@ select_rows_kernel(const float *__restrict__ P_in, int p_logits, float *__restri
     const float *src = P_in + row * nt;
     float s[NPL];
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) s[i] = (32 * i + lane < nt) ? __ldcs(src + 32 * i + lane) : -INFINITY;
-    if (p_logits) {
-      float mx = -INFINITY;
+    for (int i = 0; i < NPL; ++i) s[i] = (i < nv) ? __ldcs(src + 32 * i + lane) : -INFINITY;
+    float mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < NPL; ++i) mx = fmaxf(mx, s[i]);
+    for (int i = 0; i + 1 < NPL; i += 2) mx = fmax3_f(mx, s[i], s[i + 1]);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float ml = mx * LOG2E_F;
-      float z = 0.0f;
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float ml = mx * LOG2E_F;
+    float z = 0.0f;
 #pragma unroll
-      for (int i = 0; i < NPL; ++i) {
-        s[i] = ex2_approx(fmaf(s[i], LOG2E_F, -ml));
-        z += s[i];
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-      const float rz = __frcp_rn(z);
-#pragma unroll
-      for (int i = 0; i < NPL; ++i) s[i] *= rz;
-    } else {
-#pragma unroll
-      for (int i = 0; i < NPL; ++i) s[i] = clamp_unit(s[i]);
+    for (int i = 0; i < NPL; ++i) {
+      s[i] = ex2_approx(fmaf(s[i], LOG2E_F, -ml));
+      z += s[i];
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    const float rz = __frcp_rn(z);
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) pb[i] = __float_as_uint(s[i] * rz);
     if (probs_out != nullptr) {
       float *dst = probs_out + row * nt;
 #pragma unroll
       for (int i = 0; i < NPL; ++i)
-        if (32 * i + lane < nt) dst[32 * i + lane] = s[i];
+        if (i < nv) dst[32 * i + lane] = __uint_as_float(pb[i]);
     }
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) pb[i] = __float_as_uint(s[i]);
 
     // per-head top-k floor (second pass): k_min raised to the head's floor
     const uint32_t kk = (uint32_t)min(kmin_head != nullptr ? max(k_min, kmin_head[bh]) : k_min, nt);
@@ -319,20 +280,33 @@ select_rows_kernel(const float *__restrict__ P_in, int p_logits, float *__restri
       m_ties = NONE;
       m_p = nt;
     } else if (top_p > 0.0f) {
-      uint32_t wsum = 0u;
-#pragma unroll
-      for (int i = 0; i < NPL; ++i)
-        if (32 * i + lane < nt) wsum += mass_of(__uint_as_float(pb[i]));
-      const uint32_t W = __reduce_add_sync(0xffffffffu, wsum);
+      hist_mass<NPL>(pb, lane, wsm);
+      const unsigned long long tot = bin_total(wsm, lane);
+      const uint32_t own_w = (uint32_t)(tot & MASS_MASK), own_c = (uint32_t)(tot >> 25);
+      const uint32_t W = __reduce_add_sync(0xffffffffu, own_w);
       const uint32_t thr = (uint32_t)ceil((double)top_p * (double)W);
+      __syncwarp();  // the histogram columns become candidate columns
       if (thr > 0u) {
-        uint32_t v, n_gt, n_eq, above;
-        threshold<NPL>(pb, nt, lane, true, thr, wsm, v, n_gt, n_eq, above);
+        int bstar;
+        uint32_t w_above, c_above;
+        find_bin(own_w, own_c, thr, lane, bstar, w_above, c_above);
+        // the entries of bin b*: exponent MASS_BASE + b*
+        const uint32_t ex = (uint32_t)(MASS_BASE + bstar);
+        int k = 0;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+          if ((pb[i] >> 23) == ex) wsm[(k++) * 32 + lane] = pb[i];
+        __syncwarp();
+        uint32_t v, above_c, gt_c, eq_c;
+        level2(wsm, k, 1, ex << 23, thr - w_above, false, lane, hist2, v, above_c);
+        cand_counts(wsm, k, v, gt_c, eq_c, lane);
+        const uint32_t above = w_above + above_c;
         const uint32_t wv = mass_of(__uint_as_float(v));
         m_level = v;
         m_ties = (thr - above + wv - 1u) / wv;  // tied entries at level v
-        m_eq = n_eq;
-        m_p = (long long)n_gt + m_ties;
+        m_eq = eq_c;
+        m_p = (long long)(c_above + gt_c) + m_ties;
+        __syncwarp();
       }
     }
     if ((long long)kk > m_p) {
@@ -340,11 +314,27 @@ select_rows_kernel(const float *__restrict__ P_in, int p_logits, float *__restri
         v_f = 0u;  // every entry
         c_f = NONE;
       } else {
-        uint32_t u, n_gt, n_eq, above;
-        threshold<NPL>(pb, nt, lane, false, kk, wsm, u, n_gt, n_eq, above);
+        hist_count<NPL>(pb, nv, lane, wsm);
+        const uint32_t own_c = (uint32_t)(bin_total(wsm, lane) >> 25);
+        __syncwarp();
+        int bstar;
+        uint32_t c_above, c_above2;
+        find_bin(own_c, own_c, kk, lane, bstar, c_above, c_above2);
+        int k = 0;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i)
+          if (i < nv && max((int)(pb[i] >> 23) - COUNT_BASE, 0) == bstar) wsm[(k++) * 32 + lane] = pb[i];
+        __syncwarp();
+        // bins above 0 are exact exponents; bin 0 mixes the exponents below 97
+        const int first = bstar == 0 ? 0 : 1;
+        const uint32_t pre = bstar == 0 ? 0u : (uint32_t)(COUNT_BASE + bstar) << 23;
+        uint32_t u, above_c, gt_c, eq_c;
+        level2(wsm, k, first, pre, kk - c_above, true, lane, hist2, u, above_c);
+        cand_counts(wsm, k, u, gt_c, eq_c, lane);
         v_f = u;
-        c_f = kk - n_gt;
-        eq_f = n_eq;
+        c_f = kk - (c_above + gt_c);
+        eq_f = eq_c;
+        __syncwarp();
       }
     } else if (m_p > 0) {
       v_f = m_level;
@@ -357,46 +347,52 @@ select_rows_kernel(const float *__restrict__ P_in, int p_logits, float *__restri
     }
   }
 
-  // window tiles of the row, written as runs of bits: for each key frame, each
-  // of the two rectangles and each tile row it covers, the tile columns within
-  // the extent (clipped to the grid) are consecutive key tiles
+  // window tiles of the row, written as runs of bits: for each key frame and
+  // each of the two rectangles, every tile row the rectangle covers holds a
+  // run of consecutive key tiles (the columns within the extent, clipped to
+  // the grid)
   const int tq = qt / tpf, remq = qt - tq * tpf;
   const int yq = remq / g.NW, xq = remq - yq * g.NW;
   if (windows != nullptr) {
     for (int w = lane; w < wpr; w += 32) wwin[w] = 0u;
     __syncwarp();
-    const int items = g.T * 2 * g.NH;
-    for (int it = lane; it < items; it += 32) {
-      const int y = it % g.NH, rect = (it / g.NH) & 1, tk = it / (2 * g.NH);
+    for (int it = lane; it < 2 * g.T; it += 32) {
+      const int rect = it & 1, tk = it >> 1;
       const int grp = gtab[abs(tq - tk)];
       if (grp < 0) continue;
       const int4 w4 = reinterpret_cast<const int4 *>(wtab)[grp];
       const int ry = rect ? w4.z : w4.x, rx = rect ? w4.w : w4.y;
-      if (ry < 0 || rx < 0 || abs(y - yq) > ry) continue;
-      const int base = (tk * g.NH + y) * g.NW;
-      const int k0 = base + max(0, xq - rx), k1 = base + min(g.NW - 1, xq + rx);
-      for (int w = k0 >> 5; w <= (k1 >> 5); ++w) {
-        const int lo = max(k0 - 32 * w, 0), hi = min(k1 - 32 * w, 31);
-        atomicOr(wwin + w, (0xFFFFFFFFu >> (31 - hi + lo)) << lo);  // bits lo..hi
+      if (ry < 0 || rx < 0) continue;
+      const int y0 = max(0, yq - ry), y1 = min(g.NH - 1, yq + ry);
+      const int x0 = max(0, xq - rx), x1 = min(g.NW - 1, xq + rx);
+      for (int y = y0; y <= y1; ++y) {
+        const int base = (tk * g.NH + y) * g.NW;
+        const int k0 = base + x0, k1 = base + x1;
+        for (int w = k0 >> 5; w <= (k1 >> 5); ++w) {
+          const int lo = max(k0 - 32 * w, 0), hi = min(k1 - 32 * w, 31);
+          atomicOr(wwin + w, (0xFFFFFFFFu >> (31 - hi + lo)) << lo);  // bits lo..hi
+        }
       }
     }
     __syncwarp();
   }
 
   // membership bits: one ballot per 32 entries; ties at v_f ranked by index
-  // only when some tied entries are left out
-  const bool all_ties = c_f == NONE || c_f >= eq_f;
-  unsigned int *brow = bits + row * wpr;
-  uint32_t ties_seen = 0u, mine[(NPL + 31) / 32];
+  // only when some tied entries are left out; entries past Nt (P = 0) can
+  // only meet a threshold at P = 0, where validity is tested
+  constexpr int NW32 = (NPL + 31) / 32;
+  uint32_t mine[NW32];
 #pragma unroll
-  for (int q = 0; q < (NPL + 31) / 32; ++q) mine[q] = 0u;
-  int total = 0;
+  for (int q = 0; q < NW32; ++q) mine[q] = 0u;
+  if (use_scores && v_f != NONE) {
+    const bool all_ties = c_f == NONE || c_f >= eq_f;
+    const bool test_valid = v_f == 0u;
+    uint32_t ties_seen = 0u;
 #pragma unroll
-  for (int i = 0; i < NPL; ++i) {
-    if (32 * i >= nt) break;  // uniform: words past the row
-    const bool valid = 32 * i + lane < nt;
-    bool sel = false;
-    if (use_scores && v_f != NONE) {
+    for (int i = 0; i < NPL; ++i) {
+      if (32 * i >= nt) break;  // uniform: words past the row
+      const bool valid = !test_valid || i < nv;
+      bool sel;
       if (all_ties) {
         sel = valid && pb[i] >= v_f;
       } else {
@@ -406,14 +402,22 @@ select_rows_kernel(const float *__restrict__ P_in, int p_logits, float *__restri
         sel = valid && (pb[i] > v_f || (tie && ties_seen + before < c_f));
         ties_seen += __popc(tmask);
       }
+      const uint32_t word = __ballot_sync(0xffffffffu, sel);
+      if (lane == (i & 31)) mine[i >> 5] = word;
     }
-    const uint32_t word = __ballot_sync(0xffffffffu, sel) | (windows != nullptr ? wwin[i] : 0u);
-    if (lane == (i & 31)) mine[i >> 5] = word;
-    total += __popc(word);
   }
+  unsigned int *brow = bits + row * wpr;
+  int total = 0;
 #pragma unroll
-  for (int q = 0; q < (NPL + 31) / 32; ++q)
-    if (32 * q + lane < wpr) brow[32 * q + lane] = mine[q];
+  for (int q = 0; q < NW32; ++q) {
+    const int w = 32 * q + lane;
+    if (w < wpr) {
+      const uint32_t word = mine[q] | (windows != nullptr ? wwin[w] : 0u);
+      brow[w] = word;
+      total += __popc(word);
+    }
+  }
+  total = __reduce_add_sync(0xffffffffu, total);
   if (lane == 0) counts[row] = total;
 }
 
