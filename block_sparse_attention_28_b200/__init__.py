@@ -6,6 +6,11 @@ names: sta_reorder, sta_build_mask, sta_attn_fwd, ... Tensors are passed as
 torch tensors (device pointers are taken from them) and calls go on torch's
 current CUDA stream unless a stream is given. If the library is missing the
 import fails: there is no fallback path.
+
+With STA_CHECKED=1 in the environment the checked build libsta_debug.so
+(same kernels, compiled with -DSTA_DEBUG=1: run-time indices and addresses
+are bounds-checked on the device and reported as STA_ERR_BOUNDS) is loaded
+instead of libsta.so.
 """
 import ctypes
 import os
@@ -13,7 +18,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsta.so")
+CHECKED = os.environ.get("STA_CHECKED", "0") == "1"
+LIB_PATH = os.path.join(_HERE, "libsta_debug.so" if CHECKED else "libsta.so")
 
 STA_OK = 0
 STA_ERR_INVALID_ARG = 1
@@ -22,6 +28,7 @@ STA_ERR_WORKSPACE = 3
 STA_ERR_CUDA = 4
 STA_ERR_TIMEOUT = 5
 STA_ERR_BAD_MASK = 6
+STA_ERR_BOUNDS = 7
 MAX_GROUPS = 8
 
 
@@ -99,6 +106,8 @@ _lib.sta_selftest_wait_timeout.argtypes = [_i64, _vp]
 _lib.sta_selftest_wait_timeout.restype = ctypes.c_int
 _lib.sta_get_device_error.argtypes = [_vp]
 _lib.sta_get_device_error.restype = ctypes.c_int
+_lib.sta_debug_build.argtypes = []
+_lib.sta_debug_build.restype = _i32
 _lib.sta_status_string.argtypes = [ctypes.c_int]
 _lib.sta_status_string.restype = ctypes.c_char_p
 
@@ -126,6 +135,10 @@ def _check(status, what):
 
 def grid(T, H, W):
     return Grid(int(T), int(H), int(W))
+
+
+def sta_debug_build():
+    return int(_lib.sta_debug_build())
 
 
 def sta_status_string(status):

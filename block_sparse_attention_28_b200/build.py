@@ -1,5 +1,6 @@
-"""Build libsta.so (the product library) and libsta_probe.so (its measurement
-probes) in-tree with nvcc for sm_100a.
+"""Build libsta.so (the product library), libsta_debug.so (the same sources
+with the device-side bounds checks compiled in: -DSTA_DEBUG=1) and
+libsta_probe.so (measurement probes) in-tree with nvcc for sm_100a.
 
     python block_sparse_attention_28_b200/build.py [--force]
 
@@ -16,7 +17,9 @@ SRC = os.path.join(HERE, "csrc", "sta_lib.cu")
 OUT = os.path.join(HERE, "libsta.so")
 PROBE_SRC = os.path.join(HERE, "csrc", "sta_probe.cu")
 PROBE_OUT = os.path.join(HERE, "libsta_probe.so")
-TARGETS = ((SRC, OUT), (PROBE_SRC, PROBE_OUT))
+DEBUG_OUT = os.path.join(HERE, "libsta_debug.so")
+# (source, output, extra flags)
+TARGETS = ((SRC, OUT, ()), (SRC, DEBUG_OUT, ("-DSTA_DEBUG=1",)), (PROBE_SRC, PROBE_OUT, ()))
 NVCC_FLAGS = [
     "-O3", "-std=c++17",
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -50,14 +53,22 @@ def up_to_date(out=OUT):
 def build(force=False, verbose=False):
     """Compile every target that is missing or older than a source; returns
     the path of libsta.so."""
-    for src, out in TARGETS:
+    jobs = []
+    for src, out, extra in TARGETS:
         if not force and up_to_date(out):
             continue
-        cmd = [_nvcc(), *NVCC_FLAGS, "-o", out + ".tmp", src]
+        cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-o", out + ".tmp", src]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
-        subprocess.run(cmd, check=True)
-        os.replace(out + ".tmp", out)
+        jobs.append((subprocess.Popen(cmd), cmd, out))  # the targets compile side by side
+    failed = None
+    for proc, cmd, out in jobs:
+        if proc.wait() != 0:
+            failed = failed or subprocess.CalledProcessError(proc.returncode, cmd)
+        else:
+            os.replace(out + ".tmp", out)
+    if failed is not None:
+        raise failed
     return OUT
 
 

@@ -295,6 +295,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // for K and V, + Q_REGION for Q)
       auto load_tile_atoms = [&](const CUtensorMap *map, uint64_t *bar, uint32_t dst, uint32_t atom_step,
                                  int tile) {
+        if (!dbg_ok(tile >= 0 && tile < nt)) return;
         if (RASTER) {
           const int tpf = g.NH * g.NW;
           const int t = tile / tpf, rem = tile - t * tpf;
@@ -324,6 +325,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (RECT && (e & VIRT) != 0u) {
           // 64 pooled rows [64 kt, 64 kt + 64) of this head
           const int row = (int)((long long)bh * ntp + 64LL * kt);
+          if (!dbg_ok(kt >= 0 && 64LL * kt + 64 <= ntp)) return true;
 #pragma unroll
           for (int kb = 0; kb < C::KB; ++kb)
             tc::tma_load_2d(sbase + off + s * C::TILE_BYTES + kb * 8192, pooled_map, full + s, kb * 64, row);
@@ -513,7 +515,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
           // two warps (32 rows each) per query tile: two adds onto zero, so the
           // result does not depend on their order
-          if (lane == 0) atomicAdd(block_mass + ((long long)bh * nt + qt_half) * nt + kt, c * inv_nq);
+          if (lane == 0 && dbg_ok(qt_half < nt && kt < nt))
+            atomicAdd(block_mass + ((long long)bh * nt + qt_half) * nt + kt, c * inv_nq);
         }
         const bool need_o = rescale && (m != -INFINITY);
         if (__any_sync(0xffffffffu, need_o)) {
@@ -572,6 +575,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         store_row = y < g.H && x < g.W;
         dst_row = (((long long)(b * g.T + t) * g.H + y) * g.W + x) * heads + h;
       }
+      const bool rows_ok = dbg_ok(orow < (long long)gridDim.y * g.Lpad &&
+                                  (!RASTER || !store_row || dst_row < (long long)gridDim.y * g.T * g.H * g.W));
+      if (!rows_ok) store_row = false;
       uint4 *dst = reinterpret_cast<uint4 *>(out + dst_row * D);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -592,7 +598,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             dst[cc * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
-      if (lse != nullptr)
+      if (lse != nullptr && rows_ok)
         lse[orow] = (l > 0.0f) ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
     }
   }

@@ -14,11 +14,37 @@ namespace sta {
 enum : unsigned int {
   DEV_ERR_TIMEOUT = 1u,
   DEV_ERR_BAD_MASK = 2u,
+  DEV_ERR_BOUNDS = 4u,  // checked build only: an index or address failed its check
 };
 
 __device__ unsigned int g_dev_error;
 
 __device__ __forceinline__ void record_error(unsigned int bit) { atomicOr(&g_dev_error, bit); }
+
+// The checked build (compiled with -DSTA_DEBUG=1: libsta_debug.so) tests the
+// indices and addresses that come from run-time data before each TMA load,
+// TMEM access and global store that uses them: a failed check records
+// DEV_ERR_BOUNDS and the access is skipped (a skipped load then ends in a
+// bounded pipeline wait, never in a fault). In the product build dbg_ok() is
+// the constant true and the checks compile away.
+#ifndef STA_DEBUG
+#define STA_DEBUG 0
+#endif
+// Bytes of dynamic shared memory this CTA was launched with.
+__device__ __forceinline__ uint32_t dyn_smem_bytes() {
+  uint32_t r;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ bool dbg_ok(bool cond) {
+#if STA_DEBUG
+  if (!cond) record_error(DEV_ERR_BOUNDS);
+  return cond;
+#else
+  (void)cond;
+  return true;
+#endif
+}
 
 // Tile geometry of a T x H x W grid with 1x8x8 tiles.
 struct Geo {

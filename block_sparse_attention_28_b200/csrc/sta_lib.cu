@@ -653,10 +653,13 @@ sta_status sta_get_device_error(sta_stream_t stream) {
   STA_CUDA_TRY(cudaMemcpyFromSymbol(&word, g_dev_error, sizeof(word)));
   const unsigned int zero = 0;
   STA_CUDA_TRY(cudaMemcpyToSymbol(g_dev_error, &zero, sizeof(zero)));
+  if (word & DEV_ERR_BOUNDS) return STA_ERR_BOUNDS;
   if (word & DEV_ERR_TIMEOUT) return STA_ERR_TIMEOUT;
   if (word & DEV_ERR_BAD_MASK) return STA_ERR_BAD_MASK;
   return STA_OK;
 }
+
+int32_t sta_debug_build(void) { return STA_DEBUG ? 1 : 0; }
 
 const char *sta_status_string(sta_status s) {
   switch (s) {
@@ -667,6 +670,7 @@ const char *sta_status_string(sta_status s) {
     case STA_ERR_CUDA: return "CUDA call failed";
     case STA_ERR_TIMEOUT: return "device pipeline wait timed out";
     case STA_ERR_BAD_MASK: return "CSR column index out of range";
+    case STA_ERR_BOUNDS: return "index or address outside its buffer (checked build)";
   }
   return "unknown status";
 }

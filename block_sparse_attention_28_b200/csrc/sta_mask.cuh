@@ -646,6 +646,8 @@ fill_kernel(const unsigned int *__restrict__ bits, const int *__restrict__ row_p
   if (row >= R) return;
   const unsigned int *brow = bits + row * wpr;
   int base = row_ptr[row];
+  // checked build: every index stays inside the row's own range of col_idx
+  const int row_end = STA_DEBUG ? row_ptr[row + 1] : 0x7fffffff;
   for (int w0 = 0; w0 < wpr; w0 += 32) {
     const int w = w0 + lane;
     unsigned int word = (w < wpr) ? brow[w] : 0u;
@@ -664,7 +666,8 @@ fill_kernel(const unsigned int *__restrict__ bits, const int *__restrict__ row_p
     }
     while (word) {
       const int b = __ffs(word) - 1;
-      col_idx[pos++] = w * 32 + b;
+      if (dbg_ok(pos < row_end && (long long)pos < R * nt && w * 32 + b < nt)) col_idx[pos] = w * 32 + b;
+      ++pos;
       word &= word - 1u;
     }
     base += __shfl_sync(0xffffffffu, incl, 31);

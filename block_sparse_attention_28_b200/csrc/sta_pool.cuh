@@ -100,7 +100,8 @@ __device__ __forceinline__ void consume(uint8_t *smem, uint64_t *full, uint64_t 
     const int ty = (int)(v % g.NH);
     const int bt = (int)(v / g.NH);
     const int h = grp * C::HB + h_in;
-    if (h < heads) {
+    // checked build: the row lies in [0, B * heads * Nt) = [0, units / (2G) * heads)
+    if (h < heads && dbg_ok((long long)bt * g.NH * g.NW < units / (2 * G))) {
       const int b = bt / g.T, t = bt - b * g.T;
       const double cnt = (double)(valid_extent(g.H, ty) * valid_extent(g.W, tx));
       const long long row = ((long long)b * heads + h) * g.Nt + ((long long)t * g.NH + ty) * g.NW + tx;
@@ -163,6 +164,7 @@ pool_tma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int ty = (int)(v % g.NH);
         const int bt = (int)(v / g.NH);
         tc::mbar_expect_tx(full + s, C::BOX_BYTES);
+        if (!dbg_ok(grp < G && (long long)bt * g.NH * g.NW < units / (2 * G))) continue;
         tc::tma_load_5d(sbase + s * C::BOX_BYTES, tensor ? &tm_k : &tm_q, full + s, 0, grp * C::HB, tx * 8,
                         ty * 8, bt);
         issued = i + 1;

@@ -76,6 +76,8 @@ constexpr uint32_t IDESC = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >>
 
 // A from tensor memory (lane = row, one tf32 per column), B from shared memory.
 __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t accumulate) {
+  // A: K = 8 tf32 columns
+  if (!tc::tmem_operand_ok(d_tmem, (uint32_t)N) || !tc::tmem_operand_ok(a_tmem, 8u)) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
@@ -98,6 +100,7 @@ __device__ __forceinline__ bool all_epilogue(bool v) {
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint64_t *bar, int x, int y,
                                             int z) {
+  if (!tc::tma_args_ok(dst, x)) return;
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
@@ -291,6 +294,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tm_khi, const __grid_constan
         for (int c = warp; c < NH && q0 + c < q_end; c += 4) {
           const float4 val = reinterpret_cast<const float4 *>(T + c * M)[lane];
           float *dst = S + ((long long)bh * nt + q0 + c) * nt + kk;
+          if (!dbg_ok(q0 + c < nt && kk >= 0)) continue;
           if (vec && kk + 3 < nt) {
             *reinterpret_cast<float4 *>(dst) = val;
           } else {

@@ -237,6 +237,13 @@ select_rows_kernel(const float *__restrict__ P_in, float *__restrict__ probs_out
   const int qt = blockIdx.x * WARPS + warp;
   if (qt >= nt) return;
   const long long row = (long long)bh * nt + qt;
+  // checked build: this warp's shared-memory region lies inside the launch's
+  const uint32_t warp_end = (uint32_t)(reinterpret_cast<const uint8_t *>(wwin + ((wpr + 3) & ~3)) -
+                                       reinterpret_cast<const uint8_t *>(smw));
+  if (!dbg_ok(warp_end <= dyn_smem_bytes() && wpr * 32 >= nt)) {
+    if (lane == 0) counts[row] = 0;
+    return;
+  }
   const int nv = (nt - lane + 31) >> 5;  // valid entries of this lane: i < nv
 
   uint32_t v_f = NONE, c_f = 0u;  // keep P > v_f, plus the first c_f ties at v_f

@@ -82,10 +82,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------- TMA
+// Checked build: the box's innermost coordinate must start on 16 bytes
+// (every tensor map of this library holds 2- or 4-byte elements and its
+// inner coordinates are multiples of 8 elements) and the destination must be
+// 128-byte aligned; otherwise the load is not issued.
+__device__ __forceinline__ bool tma_args_ok(uint32_t dst, int x) {
+  return dbg_ok((x & 7) == 0 && (dst & 127u) == 0u);
+}
+
 // 2D tiled load of one box into shared memory, completing on `bar`.
 // No cluster multicast: the destination is this CTA's own shared memory.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint64_t *bar, int x,
                                             int y) {
+  if (!tma_args_ok(dst, x)) return;
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
@@ -96,6 +105,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
 // 5D tiled load (raster token grid: d, head, x, y, frame), completing on `bar`.
 __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *map, uint64_t *bar, int c0,
                                             int c1, int c2, int c3, int c4) {
+  if (!tma_args_ok(dst, c0)) return;
   asm volatile(
       "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
@@ -105,6 +115,24 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *map
 }
 
 // ---------------------------------------------------------------- TMEM
+// Checked build: a 32x32b access of ncols columns at taddr must stay inside
+// the 512 columns and use the lane quarter of the issuing warp (warp w of a
+// CTA reaches lanes 32 (w % 4) .. 32 (w % 4) + 31). Blocks are 1D.
+__device__ __forceinline__ bool tmem_access_ok(uint32_t taddr, uint32_t ncols) {
+#if STA_DEBUG
+  const uint32_t lane = taddr >> 16, col = taddr & 0xFFFFu;
+  return dbg_ok(lane == 32u * ((threadIdx.x >> 5) & 3u) && col + ncols <= 512u);
+#else
+  (void)taddr;
+  (void)ncols;
+  return true;
+#endif
+}
+// Checked build: an MMA accumulator (M = 128: every lane) of N columns, or a
+// TMEM A operand of K = 16 bf16 (8 columns), inside the 512 columns.
+__device__ __forceinline__ bool tmem_operand_ok(uint32_t taddr, uint32_t ncols) {
+  return dbg_ok((taddr >> 16) == 0u && (taddr & 0xFFFFu) + ncols <= 512u);
+}
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    smem_u32(dst_smem)),
@@ -152,6 +180,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
 
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                        uint32_t accumulate) {
+  if (!tmem_operand_ok(d_tmem, ((idesc >> 17) & 0x3Fu) << 3)) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
@@ -161,6 +190,7 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, 
 // A operand read from tensor memory (P, bf16 packed two per column).
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
                                        uint32_t accumulate) {
+  if (!tmem_operand_ok(d_tmem, ((idesc >> 17) & 0x3Fu) << 3) || !tmem_operand_ok(a_tmem, 8u)) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
@@ -178,6 +208,11 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
 // 32 lanes x 32 bit, 32 consecutive columns; the wait is inside the same asm
 // so the outputs are never used before the load has landed.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  if (!tmem_access_ok(taddr, 32u)) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) r[c] = 0u;
+    return;
+  }
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -192,6 +227,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  if (!tmem_access_ok(taddr, 32u)) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -242,6 +278,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 // 64 consecutive TMEM columns in one load (and one wait).
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  if (!tmem_access_ok(taddr, 64u)) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) r[c] = 0u;
+    return;
+  }
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,"

@@ -47,7 +47,10 @@ typedef enum {
   STA_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than required */
   STA_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
   STA_ERR_TIMEOUT = 5,     /* device: a bounded pipeline wait ran out */
-  STA_ERR_BAD_MASK = 6     /* device: a CSR column index out of range */
+  STA_ERR_BAD_MASK = 6,    /* device: a CSR column index out of range */
+  STA_ERR_BOUNDS = 7       /* device, checked build only: an index or address
+                              failed its bounds / alignment check; the access
+                              was skipped (see sta_debug_build) */
 } sta_status;
 
 typedef struct {
@@ -330,8 +333,23 @@ int64_t sta_get_wait_limit(void);
  * sta_get_device_error() and leaves the context usable. */
 sta_status sta_selftest_wait_timeout(int64_t limit_cycles, sta_stream_t stream);
 
+/* sta_debug_build -- 1 in the checked build of the library
+ * (libsta_debug.so, compiled with -DSTA_DEBUG=1), 0 in the product build
+ * (libsta.so). The checked build runs the same kernels with the same
+ * arithmetic, and in addition tests, before use, every index and address
+ * derived from run-time data: TMA box coordinates against the tensor's
+ * extents and the 16-byte rule for the innermost coordinate, shared-memory
+ * destinations against the CTA's layout, TMEM addresses against the
+ * allocation and the warp's lane quarter, and global store indices against
+ * their buffers. A failed check records STA_ERR_BOUNDS in the device error
+ * word and skips the access (a skipped load then ends in a bounded pipeline
+ * wait, reported as well). The pages have no counterpart. */
+int32_t sta_debug_build(void);
+
 /* Reads and clears the device error word of the current device after
- * synchronising `stream`. STA_OK if no device-side fault was recorded. */
+ * synchronising `stream`. STA_OK if no device-side fault was recorded;
+ * STA_ERR_BOUNDS takes precedence over STA_ERR_TIMEOUT (a skipped access is
+ * the cause of the wait that ran out), then STA_ERR_BAD_MASK. */
 sta_status sta_get_device_error(sta_stream_t stream);
 
 /* Static description of a status code. */

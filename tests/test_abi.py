@@ -41,6 +41,19 @@ def test_library_exports_every_declared_symbol(sta):
         assert hasattr(lib, name), name
 
 
+def test_checked_build_exports_the_same_boundary_and_says_so(sta):
+    """libsta_debug.so (device-side bounds checks compiled in) carries every
+    symbol of the header; sta_debug_build tells the two builds apart."""
+    checked = ctypes.CDLL(os.path.join(os.path.dirname(sta.LIB_PATH), "libsta_debug.so"))
+    for name in declared_functions():
+        assert hasattr(checked, name), name
+    product = ctypes.CDLL(os.path.join(os.path.dirname(sta.LIB_PATH), "libsta.so"))
+    checked.sta_debug_build.restype = ctypes.c_int32
+    product.sta_debug_build.restype = ctypes.c_int32
+    assert checked.sta_debug_build() == 1 and product.sta_debug_build() == 0
+    assert sta.sta_debug_build() == (1 if sta.CHECKED else 0)
+
+
 def test_probe_library_exports_its_symbols_and_the_product_header_has_none(sta):
     from block_sparse_attention_28_b200 import probe
 
@@ -96,9 +109,10 @@ def test_argument_checks_return_before_any_launch(sta):
 
 
 def test_status_strings(sta):
-    for s in range(7):
-        assert sta.sta_status_string(s)
+    for s in range(8):
+        assert sta.sta_status_string(s) != "unknown status"
     assert "out of range" in sta.sta_status_string(sta.STA_ERR_BAD_MASK)
+    assert "checked build" in sta.sta_status_string(sta.STA_ERR_BOUNDS)
 
 
 def test_selftest_limit_is_checked_on_the_host(sta):
