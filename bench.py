@@ -268,6 +268,7 @@ class Layer:
             self.win = None
         self.params = sta.mask_params(c.top_p, c.k_min, c.use_scores, 0.0, c.group_lo, self.win)
         self.bufs = sta.MaskBuffers(self.B, self.Hh, self.d, self.g, dev)
+        self.qpairs = None  # the mask build's overlap pairing, when asked for
         # pool, tensor-core scores, select, scan, fill; attention (the tile
         # gather is the TMA box, so no reorder launch)
         self.launches_per_step = 5 + 1
@@ -306,10 +307,22 @@ class Layer:
                             self.g, self.params, self.bufs, raster=True)
 
     def attn(self, q=None, k=None, v=None, o=None):
-        """Attention on raster Q, K, V into raster O (sta_attn_fwd_raster)."""
-        self.sta.sta_attn_fwd_raster(self.q if q is None else q, self.k if k is None else k,
-                                     self.v if v is None else v, self.o if o is None else o, None,
-                                     self.bufs.row_ptr, self.bufs.col_idx, self.B, self.Hh, self.d, self.g)
+        """Attention on raster Q, K, V into raster O (sta_attn_fwd_raster, or
+        sta_attn_fwd_raster_paired with the build's overlap pairing)."""
+        args = (self.q if q is None else q, self.k if k is None else k, self.v if v is None else v,
+                self.o if o is None else o, None, self.bufs.row_ptr, self.bufs.col_idx)
+        if self.qpairs is not None:
+            self.sta.sta_attn_fwd_raster_paired(*args, self.qpairs, self.B, self.Hh, self.d, self.g)
+        else:
+            self.sta.sta_attn_fwd_raster(*args, self.B, self.Hh, self.d, self.g)
+
+    def use_overlap_pairing(self, params_kw):
+        """Mask recipe with the build's query-tile pairing by list overlap
+        (sta_mask_params.query_pairs); attn() then runs the paired call."""
+        if self.qpairs is None:
+            self.qpairs = torch.empty((self.B * self.Hh, 2 * ((self.nt + 1) // 2)), dtype=torch.int32,
+                                      device=self.dev)
+        self.params = self.sta.mask_params(query_pairs=self.qpairs, **params_kw)
 
     def build_tiled(self):
         self.sta.build_mask(self.qt, self.kt, self.B, self.Hh, self.d, self.g, self.params, self.bufs)
@@ -407,10 +420,16 @@ class Layer:
     def kept_pairs(self):
         return int(self.bufs.nnz.item())
 
-    def query_pairs(self):
-        """The two query tiles of each 128-row CTA, as the attention kernel pairs
-        them: the same spatial tile in frames 2u and 2u+1, and right-hand
-        neighbours within the last frame when the frame count is odd."""
+    def query_pairs(self, bh=0, default=False):
+        """The two query tiles of each 128-row CTA of head bh: the build's
+        overlap pairing when in use (and not `default`), else the attention
+        kernel's own: the same spatial tile in frames 2u and 2u+1, and
+        right-hand neighbours within the last frame when the frame count is
+        odd."""
+        if self.qpairs is not None and not default:
+            flat = self.qpairs[bh].cpu().numpy()
+            return [(int(flat[2 * i]), int(flat[2 * i + 1]) if flat[2 * i + 1] >= 0 else None)
+                    for i in range(flat.size // 2)]
         c = self.cfg
         nh, nw = -(-c.H // 8), -(-c.W // 8)
         tpf = nh * nw
@@ -420,14 +439,14 @@ class Layer:
             pairs += [(base + i, base + i + 1 if i + 1 < tpf else None) for i in range(0, tpf, 2)]
         return pairs
 
-    def pair_union_stats(self):
+    def pair_union_stats(self, default=False):
         """Pairing efficiency (|A|+|B|) / (2 |A u B|) of the 128-row CTAs."""
         rp = self.bufs.row_ptr.cpu().numpy()
         ci = self.bufs.col_idx[: int(rp[-1])].cpu().numpy()
         nt = self.nt
         tot_ab, tot_u = 0, 0
         for bh in range(self.B * self.Hh):
-            for qa, qb in self.query_pairs():
+            for qa, qb in self.query_pairs(bh, default):
                 ra = bh * nt + qa
                 a = ci[rp[ra]:rp[ra + 1]]
                 b = ci[rp[bh * nt + qb]:rp[bh * nt + qb + 1]] if qb is not None else np.zeros(0, np.int32)
@@ -604,14 +623,17 @@ def sweep(sta, dev, peak, reps=20):
     del masters
     for rho in cfg.fixed_densities:
         k_min = int(round(rho * layer.nt))
-        layer.params = sta.mask_params(0.0, k_min, True, 0.0, cfg.group_lo, None)
+        # top-k lists of neighbouring frames overlap less at low density: the
+        # build also pairs the query tiles by list overlap, once per reused mask
+        layer.use_overlap_pairing(dict(top_p=0.0, k_min=k_min, use_scores=True, group_lo=cfg.group_lo))
         layer.build()
         extra = build_extra(layer)
         per_step = []
         for qb, kb in steps_inputs:
             per_step.append(_median_ms(lambda: layer.attn(qb, kb), max(3, reps // 4)))
         extra.update({"density_target": rho, "k_min": k_min, "reuse_steps": len(per_step),
-                      "attn_ms_per_reuse_step": per_step})
+                      "attn_ms_per_reuse_step": per_step, "pairing": "overlap (sta_mask_params.query_pairs)",
+                      "pairing_efficiency_frames": layer.pair_union_stats(default=True)[0]})
         attn_line(cfg.name, layer, extra)
     del layer, steps_inputs
     torch.cuda.empty_cache()
@@ -672,7 +694,9 @@ def per_config(sta, dev, peaks, reps=10):
     del masters
     for rho in cfg.fixed_densities:
         k_min = int(round(rho * layer.nt))
-        layer.params = sta.mask_params(0.0, k_min, True, 0.0, cfg.group_lo, None)
+        # top-k lists of neighbouring frames overlap less at low density: the
+        # build also pairs the query tiles by list overlap, once per reused mask
+        layer.use_overlap_pairing(dict(top_p=0.0, k_min=k_min, use_scores=True, group_lo=cfg.group_lo))
         layer.build()
         it = iter(range(10 ** 9))
 
@@ -682,7 +706,9 @@ def per_config(sta, dev, peaks, reps=10):
 
         # one launch per perturbed step, in turn, over the mask of step 0
         record(cfg.name, layer, attn_reuse, 2 * len(steps_inputs),
-               {"density_target": rho, "k_min": k_min, "reuse_steps": len(steps_inputs)})
+               {"density_target": rho, "k_min": k_min, "reuse_steps": len(steps_inputs),
+                "pairing": "overlap (sta_mask_params.query_pairs)",
+                "pairing_efficiency_frames": layer.pair_union_stats(default=True)[0]})
     del layer, steps_inputs
     torch.cuda.empty_cache()
     assert sta.sta_get_device_error() == sta.STA_OK

@@ -53,6 +53,7 @@ class MaskParams(ctypes.Structure):
         ("windows", ctypes.c_void_p),
         ("head_topk_floor", ctypes.c_int32),
         ("block_scores", ctypes.c_void_p),
+        ("query_pairs", ctypes.c_void_p),
     ]
 
 
@@ -87,6 +88,10 @@ _lib.sta_build_mask_raster.argtypes = _lib.sta_build_mask.argtypes
 _lib.sta_build_mask_raster.restype = ctypes.c_int
 _lib.sta_attn_fwd_raster.argtypes = _lib.sta_attn_fwd.argtypes
 _lib.sta_attn_fwd_raster.restype = ctypes.c_int
+_lib.sta_attn_fwd_paired.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, Grid, _f32, _vp]
+_lib.sta_attn_fwd_paired.restype = ctypes.c_int
+_lib.sta_attn_fwd_raster_paired.argtypes = _lib.sta_attn_fwd_paired.argtypes
+_lib.sta_attn_fwd_raster_paired.restype = ctypes.c_int
 _lib.sta_rectified_workspace.argtypes = [_i32, _i32, _i32, Grid]
 _lib.sta_rectified_workspace.restype = _sz
 _lib.sta_attn_fwd_rectified.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i32, _i32, _i32, Grid,
@@ -167,11 +172,14 @@ def sta_build_mask_workspace_min(B, heads, d, g):
 
 
 def mask_params(top_p=0.0, k_min=0, use_scores=False, sm_scale=0.0, group_lo=(0,), windows=None,
-                head_floor=False, block_scores=None):
+                head_floor=False, block_scores=None, query_pairs=None):
     """MaskParams; `windows` is a device int32 tensor [heads, G, 4] or None;
     `head_floor` turns on the per-head top-k floor of the selection;
-    `block_scores` (device fp32 [B, heads, Nt, Nt]) replaces the pooled scores."""
+    `block_scores` (device fp32 [B, heads, Nt, Nt]) replaces the pooled scores;
+    `query_pairs` (device int32 [B*heads, 2*ceil(Nt/2)]) receives the
+    overlap pairing of the query tiles for sta_attn_fwd_paired."""
     p = MaskParams()
+    p.query_pairs = _ptr(query_pairs)
     p.head_topk_floor = 1 if head_floor else 0
     p.block_scores = _ptr(block_scores)
     p.top_p = float(top_p)
@@ -183,7 +191,7 @@ def mask_params(top_p=0.0, k_min=0, use_scores=False, sm_scale=0.0, group_lo=(0,
         p.group_lo[i] = int(v)
     p.windows = _ptr(windows)
     # the struct holds raw device pointers: keep the tensors alive with it
-    p._keep = (windows, block_scores)
+    p._keep = (windows, block_scores, query_pairs)
     return p
 
 
@@ -224,6 +232,23 @@ def sta_attn_fwd(q, k, v, o, lse, row_ptr, col_idx, B, heads, d, g, sm_scale=0.0
     _check(_lib.sta_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(row_ptr), _ptr(col_idx),
                              B, heads, d, g, float(sm_scale), _stream(stream)),
            "sta_attn_fwd")
+
+
+def sta_attn_fwd_paired(q, k, v, o, lse, row_ptr, col_idx, query_pairs, B, heads, d, g, sm_scale=0.0,
+                        stream=None):
+    """sta_attn_fwd with the caller's pairing of query tiles."""
+    _check(_lib.sta_attn_fwd_paired(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(row_ptr), _ptr(col_idx),
+                                    _ptr(query_pairs), B, heads, d, g, float(sm_scale), _stream(stream)),
+           "sta_attn_fwd_paired")
+
+
+def sta_attn_fwd_raster_paired(q, k, v, o, lse, row_ptr, col_idx, query_pairs, B, heads, d, g, sm_scale=0.0,
+                               stream=None):
+    """sta_attn_fwd_raster with the caller's pairing of query tiles."""
+    _check(_lib.sta_attn_fwd_raster_paired(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(row_ptr),
+                                           _ptr(col_idx), _ptr(query_pairs), B, heads, d, g, float(sm_scale),
+                                           _stream(stream)),
+           "sta_attn_fwd_raster_paired")
 
 
 def sta_build_mask_raster(q, k, B, heads, d, g, params, row_ptr, col_idx, nnz_dev, block_mask=None,

@@ -119,7 +119,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int *__restrict__ col_idx, Geo g, float scale_log2,
                 const float *__restrict__ lse_in, float *__restrict__ block_mass, int heads,
                 const __grid_constant__ CUtensorMap tm_kbar, const __grid_constant__ CUtensorMap tm_vbar,
-                int ntp, long long wait_limit) {
+                int ntp, long long wait_limit, const int *__restrict__ query_pairs) {
   static_assert(!(MASS && RECT) && !(RASTER && RECT), "the rectified form is tiled and mass-free");
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -129,22 +129,34 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nt = g.Nt;
   const int bh = blockIdx.y;
-  // Query-tile pairing: the same spatial tile in frames 2u and 2u+1 (their
-  // lists overlap most: windows and pooled scores change little between
-  // neighbouring frames); with an odd frame count the last frame's tiles are
-  // paired with their right-hand neighbour.
-  const int tpf_q = g.NH * g.NW;
-  const int pairs_t = (g.T / 2) * tpf_q;
+  // Query-tile pairing: the caller's (query_pairs: pair blockIdx.x of this
+  // head), or by default the same spatial tile in frames 2u and 2u+1 (their
+  // lists overlap most when windows dominate: windows and pooled scores change
+  // little between neighbouring frames); with an odd frame count the last
+  // frame's tiles are paired with their right-hand neighbour.
   int qtA, qtB;
-  if ((int)blockIdx.x < pairs_t) {
-    const int u = (int)blockIdx.x / tpf_q, rem = (int)blockIdx.x - u * tpf_q;
-    qtA = 2 * u * tpf_q + rem;
-    qtB = qtA + tpf_q;
+  if (query_pairs != nullptr) {
+    const long long at = ((long long)bh * ((nt + 1) / 2) + blockIdx.x) * 2;
+    qtA = query_pairs[at];
+    qtB = query_pairs[at + 1];
+    if ((unsigned)qtA >= (unsigned)nt || (qtB != -1 && (unsigned)qtB >= (unsigned)nt)) {
+      // the whole CTA leaves before any shared state exists
+      if (threadIdx.x == 0) record_error(DEV_ERR_BAD_MASK);
+      return;
+    }
   } else {
-    qtA = (g.T - 1) * tpf_q + 2 * ((int)blockIdx.x - pairs_t);
-    qtB = qtA + 1;
+    const int tpf_q = g.NH * g.NW;
+    const int pairs_t = (g.T / 2) * tpf_q;
+    if ((int)blockIdx.x < pairs_t) {
+      const int u = (int)blockIdx.x / tpf_q, rem = (int)blockIdx.x - u * tpf_q;
+      qtA = 2 * u * tpf_q + rem;
+      qtB = qtA + tpf_q;
+    } else {
+      qtA = (g.T - 1) * tpf_q + 2 * ((int)blockIdx.x - pairs_t);
+      qtB = qtA + 1;
+    }
   }
-  const bool hasB = qtB < nt;
+  const bool hasB = qtB >= 0 && qtB < nt;
   const int wpr = (nt + 31) / 32;
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);

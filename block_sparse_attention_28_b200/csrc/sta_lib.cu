@@ -10,6 +10,7 @@
 #include "sta_common.cuh"
 #include "sta_host.cuh"
 #include "sta_mask.cuh"
+#include "sta_pair.cuh"
 #include "sta_pool.cuh"
 #include "sta_reorder.cuh"
 #include "sta_score.cuh"
@@ -54,7 +55,7 @@ bool common_sizes_ok(int32_t B, int32_t heads, int32_t d, sta_grid g, Geo *geo, 
 // the split passes (tensor-core scores, then a select pass with four CTAs
 // per SM).
 struct MaskWs {
-  size_t qbar, kbar, bits, counts, sel, kfloor, total_min, qlo, klo, prows, total;
+  size_t qbar, kbar, bits, counts, sel, kfloor, pairw, total_min, qlo, klo, prows, total;
 };
 
 MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
@@ -74,6 +75,8 @@ MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
   off = align_up(off + R * sizeof(int32_t), 256);
   w.kfloor = off;
   off = align_up(off + (size_t)B * heads * sizeof(int32_t), 256);
+  w.pairw = off;  // candidate-pair overlaps of the query-tile pairing
+  off = align_up(off + R * pairq::NOFF * sizeof(int32_t), 256);
   w.total_min = off;
   w.qlo = off;
   off = align_up(off + R * d * sizeof(float), 256);
@@ -352,6 +355,20 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
   const unsigned fblocks = (unsigned)((R * 32 + 255) / 256);
   fill_kernel<<<fblocks, 256, 0, s>>>(bits, row_ptr, col_idx, block_mask, R, g.Nt, wpr);
   STA_CUDA_TRY(cudaGetLastError());
+  if (p->query_pairs != nullptr) {
+    // query-tile pairing by list overlap, from the final row bitsets
+    int *pw = reinterpret_cast<int *>(ws + L.pairw);
+    const long long warps = R * pairq::NOFF;
+    pairq::pair_weights_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(bits, pw, R, g, wpr);
+    STA_CUDA_TRY(cudaGetLastError());
+    const size_t psmem = 2 * (size_t)g.Nt * sizeof(int);
+    if (psmem > 48 * 1024)
+      STA_CUDA_TRY(cudaFuncSetAttribute(pairq::pair_match_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)psmem));
+    pairq::pair_match_kernel<<<(unsigned)(B * heads), pairq::MATCH_THREADS, psmem, s>>>(bits, pw, counts,
+                                                                                       p->query_pairs, g, wpr);
+    STA_CUDA_TRY(cudaGetLastError());
+  }
   if (block_probs != nullptr && !use_scores)
     STA_CUDA_TRY(cudaMemsetAsync(block_probs, 0, (size_t)R * g.Nt * sizeof(float), s));
   return STA_OK;
@@ -364,7 +381,8 @@ template <int D, bool MASS, bool RASTER = false, bool RECT = false>
 sta_status launch_attn(const void *q, const void *k, const void *v, void *o, float *lse,
                        const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
                        const Geo &g, float sm_scale, cudaStream_t s, const float *lse_in = nullptr,
-                       float *block_mass = nullptr, const void *kbar = nullptr, const void *vbar = nullptr) {
+                       float *block_mass = nullptr, const void *kbar = nullptr, const void *vbar = nullptr,
+                       const int32_t *query_pairs = nullptr) {
   const unsigned long long rows = (unsigned long long)B * heads * g.Lpad;
   const int ntp = RECT ? pooled_rows(g) : 0;
   CUtensorMap tq, tk, tv, tkb, tvb;
@@ -394,7 +412,7 @@ sta_status launch_attn(const void *q, const void *k, const void *v, void *o, flo
   dim3 grid((unsigned)((g.Nt + 1) / 2), (unsigned)(B * heads));
   attn::attn_fwd_kernel<D, MASS, RASTER, RECT><<<grid, attn::NUM_THREADS, smem, s>>>(
       tq, tk, tv, static_cast<__nv_bfloat16 *>(o), lse, row_ptr, col_idx, g, scale_log2, lse_in,
-      block_mass, heads, tkb, tvb, ntp, wait_limit());
+      block_mass, heads, tkb, tvb, ntp, wait_limit(), query_pairs);
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }
@@ -478,6 +496,11 @@ static sta_status build_mask_any(const void *q_tiled, const void *k_tiled, int32
       ws_bytes < mask_ws_layout(B, heads, d, geo).total_min)
     return STA_ERR_WORKSPACE;
   if (select_smem(d, geo, p->use_scores != 0) > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
+  if (p->query_pairs != nullptr) {
+    if ((reinterpret_cast<uintptr_t>(p->query_pairs) & 3u) != 0) return STA_ERR_INVALID_ARG;
+    // the pairing keeps two int32 per tile of a head in shared memory
+    if (2 * (size_t)geo.Nt * sizeof(int) > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
+  }
   // window tables pack (t, tile row, tile column) into 12 + 10 + 10 bits
   if (p->windows != nullptr && (geo.T >= 4096 || geo.NH >= 1024 || geo.NW >= 1024)) return STA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -506,7 +529,8 @@ sta_status sta_build_mask_raster(const void *q, const void *k, int32_t B, int32_
 
 static sta_status attn_fwd_any(const void *q, const void *k, const void *v, void *o, float *lse,
                                const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
-                               int32_t d, sta_grid g, float sm_scale, sta_stream_t stream, bool raster) {
+                               int32_t d, sta_grid g, float sm_scale, sta_stream_t stream, bool raster,
+                               const int32_t *query_pairs = nullptr) {
   Geo geo;
   sta_status st = STA_OK;
   if (!common_sizes_ok(B, heads, d, g, &geo, &st)) return st;
@@ -519,11 +543,15 @@ static sta_status attn_fwd_any(const void *q, const void *k, const void *v, void
   if (raster) {
     // TMA coordinates of the 5D map are 32-bit: B*T frames, W columns, H rows
     if ((long long)B * geo.T >= (1LL << 31)) return STA_ERR_UNSUPPORTED;
-    return (d == 128) ? launch_attn<128, false, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s)
-                      : launch_attn<64, false, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s);
+    return (d == 128) ? launch_attn<128, false, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s,
+                                                      nullptr, nullptr, nullptr, nullptr, query_pairs)
+                      : launch_attn<64, false, true>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s,
+                                                     nullptr, nullptr, nullptr, nullptr, query_pairs);
   }
-  return (d == 128) ? launch_attn<128, false>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s)
-                    : launch_attn<64, false>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s);
+  return (d == 128) ? launch_attn<128, false>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s, nullptr,
+                                              nullptr, nullptr, nullptr, query_pairs)
+                    : launch_attn<64, false>(q, k, v, o, lse, row_ptr, col_idx, B, heads, geo, sm_scale, s, nullptr,
+                                             nullptr, nullptr, nullptr, query_pairs);
 }
 
 sta_status sta_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
@@ -536,6 +564,22 @@ sta_status sta_attn_fwd_raster(const void *q, const void *k, const void *v, void
                                const int32_t *row_ptr, const int32_t *col_idx, int32_t B, int32_t heads,
                                int32_t d, sta_grid g, float sm_scale, sta_stream_t stream) {
   return attn_fwd_any(q, k, v, o, lse, row_ptr, col_idx, B, heads, d, g, sm_scale, stream, true);
+}
+
+sta_status sta_attn_fwd_paired(const void *q, const void *k, const void *v, void *o, float *lse,
+                               const int32_t *row_ptr, const int32_t *col_idx, const int32_t *query_pairs,
+                               int32_t B, int32_t heads, int32_t d, sta_grid g, float sm_scale,
+                               sta_stream_t stream) {
+  if (query_pairs == nullptr || (reinterpret_cast<uintptr_t>(query_pairs) & 3u) != 0) return STA_ERR_INVALID_ARG;
+  return attn_fwd_any(q, k, v, o, lse, row_ptr, col_idx, B, heads, d, g, sm_scale, stream, false, query_pairs);
+}
+
+sta_status sta_attn_fwd_raster_paired(const void *q, const void *k, const void *v, void *o, float *lse,
+                                      const int32_t *row_ptr, const int32_t *col_idx,
+                                      const int32_t *query_pairs, int32_t B, int32_t heads, int32_t d,
+                                      sta_grid g, float sm_scale, sta_stream_t stream) {
+  if (query_pairs == nullptr || (reinterpret_cast<uintptr_t>(query_pairs) & 3u) != 0) return STA_ERR_INVALID_ARG;
+  return attn_fwd_any(q, k, v, o, lse, row_ptr, col_idx, B, heads, d, g, sm_scale, stream, true, query_pairs);
 }
 
 sta_status sta_attn_fwd_block_mass(const void *q, const void *k, const void *v, void *o, float *lse,

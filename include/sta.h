@@ -94,6 +94,11 @@ typedef struct {
                               e.g. the masses of sta_attn_fwd_block_mass;
                               values are clamped to [0, 1] and q_tiled, k_tiled
                               are not read */
+  int32_t *query_pairs;   /* optional output, device int32 [B*heads][2*NP],
+                              NP = ceil(Nt/2), or NULL: the query tiles of
+                              each head paired into the 128-row tiles of
+                              sta_attn_fwd_paired, chosen by list overlap
+                              (see sta_attn_fwd_paired) */
 } sta_mask_params;
 
 /* Number of tiles per head (Nt) and padded rows per head (Lpad) of a grid;
@@ -198,6 +203,47 @@ sta_status sta_attn_fwd_raster(const void *q, const void *k, const void *v, void
                                const int32_t *row_ptr, const int32_t *col_idx, int32_t B,
                                int32_t heads, int32_t d, sta_grid g, float sm_scale,
                                sta_stream_t stream);
+
+/* sta_attn_fwd_paired, sta_attn_fwd_raster_paired -- sta_attn_fwd and
+ * sta_attn_fwd_raster with the query tiles paired as the caller says. The
+ * kernels run 128 query rows (two 64-token query tiles) per tensor-core tile
+ * over the union of the two tiles' key lists; a tile gets P = 0 for the key
+ * tiles its own list lacks, so the union steps it does not need are wasted
+ * work. The default pairing (frames 2u and 2u+1 of one spatial tile; the last
+ * odd frame's tiles with their right-hand neighbour) suits window masks;
+ * lists from a top-k selection at low density overlap less between frames.
+ * The pages have no counterpart: the results are those of the unpaired calls
+ * up to the fp32 summation order of each row.
+ *   query_pairs : device int32 [B*heads][2*NP], NP = ceil(Nt/2): pair i of
+ *                 head (b, h) is (query_pairs[2i], query_pairs[2i+1]), the
+ *                 second -1 for a tile without a partner; every tile of the
+ *                 head must appear exactly once. sta_build_mask writes such
+ *                 an array when sta_mask_params.query_pairs is set:
+ *                 - candidates: tile a = (t, y, x) with b = a + (dt, dy, dx)
+ *                   for (dt, dy, dx) in {1} x {-1, 0, 1}^2, (0, 1, -1..1),
+ *                   (0, 0, 1) and (2, 0, 0), inside the grid; weight
+ *                   |L_a n L_b| of the two final key-tile lists;
+ *                 - greedy matching: candidate pairs by weight descending,
+ *                   ties to the lower smaller tile, then the lower larger
+ *                   tile, each taken if both tiles are free; the tiles left
+ *                   over are paired in ascending order (a last one alone if
+ *                   their count is odd);
+ *                 - per head, if the total union size sum(|L_a u L_b|) of
+ *                   this pairing is not below that of the default pairing,
+ *                   the default pairing is written instead;
+ *                 pairs are written in ascending order of their first tile
+ *                 (the default pairing in its own order).
+ * A tile index out of range in query_pairs is reported as STA_ERR_BAD_MASK
+ * (the pair is skipped). Every other argument, output and error is that of
+ * sta_attn_fwd / sta_attn_fwd_raster. */
+sta_status sta_attn_fwd_paired(const void *q, const void *k, const void *v, void *o, float *lse,
+                               const int32_t *row_ptr, const int32_t *col_idx, const int32_t *query_pairs,
+                               int32_t B, int32_t heads, int32_t d, sta_grid g, float sm_scale,
+                               sta_stream_t stream);
+sta_status sta_attn_fwd_raster_paired(const void *q, const void *k, const void *v, void *o, float *lse,
+                                      const int32_t *row_ptr, const int32_t *col_idx,
+                                      const int32_t *query_pairs, int32_t B, int32_t heads, int32_t d,
+                                      sta_grid g, float sm_scale, sta_stream_t stream);
 
 /* Size in bytes of the static device scratch behind sta_build_mask_noalloc. */
 #define STA_NOALLOC_SCRATCH_BYTES (32u << 20)

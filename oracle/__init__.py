@@ -18,6 +18,9 @@ Sources (pages on block-sparse attention for video diffusion transformers):
   * Compact Attention Figs. 3-5: recall-driven offline window search.
   * Rectified SpaAttn (abstract): rectified attention, skipped tiles
     recovered from pooled keys and values (reading stated in the module).
+  * The query-tile pairing the library emits with a mask (no counterpart in
+    the pages; a scheduling choice of its attention kernels, restated so
+    that the GPU's output can be checked).
 
 Parity pins: every function here is checked in tests/test_oracle.py
 against closed forms, textbook routines (torch SDPA in fp64, scipy
@@ -48,4 +51,8 @@ from .sta_oracle import (  # noqa: F401
     pooled_kv,
     rectified_attention_rows,
     SEARCH_MOVES,
+    PAIR_OFFSETS,
+    default_pairs,
+    pairs_union,
+    pair_query_tiles,
 )

@@ -506,3 +506,84 @@ def search_windows(mass, T, H, W, group_lo, tau, lam):
     stats = dict(recall=covered / total if total else 1.0, density=float(cur.mean()), steps=len(moves),
                  covered=covered, total=total, moves=moves)
     return win.astype(np.int32), stats
+
+
+# --------------------------------------------------------------------------
+# Query-tile pairing by list overlap. The pages have no counterpart: this is
+# how the library groups two 64-token query tiles into one 128-row block of
+# its attention kernels (Compact Attention Fig. 3: precomputed masks loaded
+# into block-sparse kernels), and the attention result does not depend on it
+# beyond fp32 summation order. Restated here because sta_build_mask emits
+# it as an output (sta_mask_params.query_pairs).
+# Rule: candidate pairs (a, a + o) for the offsets o of PAIR_OFFSETS inside
+# the tile grid, weight |L_a n L_b| of the final key-tile lists; taken
+# greedily in the order (weight descending, smaller tile ascending, larger
+# tile ascending) when both tiles are free; tiles left over paired in
+# ascending order, a last one alone; kept only if its total union
+# sum |L_a u L_b| is below that of the default pairing (frames 2u, 2u+1 of
+# one spatial tile; in a last odd frame, neighbours 2i, 2i+1), else the
+# default pairing is returned. Pairs come in ascending order of their first
+# tile (the default pairing in its own order).
+# --------------------------------------------------------------------------
+PAIR_OFFSETS = ([(1, dy, dx) for dy in (-1, 0, 1) for dx in (-1, 0, 1)]
+                + [(0, 1, -1), (0, 1, 0), (0, 1, 1), (0, 0, 1), (2, 0, 0)])
+
+
+def default_pairs(T, H, W):
+    """The attention kernels' own pairing: list of (a, b or -1)."""
+    nh, nw, nt, _ = tile_grid(T, H, W)
+    tpf = nh * nw
+    pairs = []
+    for u in range(T // 2):
+        for rem in range(tpf):
+            a = 2 * u * tpf + rem
+            pairs.append((a, a + tpf))
+    if T % 2:
+        base = (T - 1) * tpf
+        for i in range(0, tpf, 2):
+            a = base + i
+            pairs.append((a, a + 1 if a + 1 < nt else -1))
+    return pairs
+
+
+def pairs_union(mask, pairs):
+    """Total union size sum |L_a u L_b| over the pairs (|L_a| for a lone tile)."""
+    total = 0
+    for a, b in pairs:
+        total += int((mask[a] | mask[b]).sum()) if b >= 0 else int(mask[a].sum())
+    return total
+
+
+def pair_query_tiles(mask, T, H, W):
+    """mask: bool [Nt, Nt] of one head (row = query tile). Returns the pairs
+    as a flat int array [2 * ceil(Nt/2)]."""
+    mask = np.asarray(mask, dtype=bool)
+    nh, nw, nt, _ = tile_grid(T, H, W)
+    edges = []
+    for a in range(nt):
+        t, rem = divmod(a, nh * nw)
+        y, x = divmod(rem, nw)
+        for dt, dy, dx in PAIR_OFFSETS:
+            t2, y2, x2 = t + dt, y + dy, x + dx
+            if t2 < T and 0 <= y2 < nh and 0 <= x2 < nw:
+                b = (t2 * nh + y2) * nw + x2
+                w = int((mask[a] & mask[b]).sum())
+                edges.append((-w, min(a, b), max(a, b)))
+    edges.sort()
+    mate = [-1] * nt
+    for _, a, b in edges:
+        if mate[a] < 0 and mate[b] < 0:
+            mate[a], mate[b] = b, a
+    left = [v for v in range(nt) if mate[v] < 0]
+    pairs = []
+    for i in range(0, len(left) - 1, 2):
+        mate[left[i]], mate[left[i + 1]] = left[i + 1], left[i]
+    for v in range(nt):
+        if mate[v] < 0:
+            pairs.append((v, -1))
+        elif mate[v] > v:
+            pairs.append((v, mate[v]))
+    dflt = default_pairs(T, H, W)
+    if pairs_union(mask, pairs) >= pairs_union(mask, dflt):
+        pairs = dflt
+    return np.array([i for p in pairs for i in p], dtype=np.int64)

@@ -108,6 +108,17 @@ def test_argument_checks_return_before_any_launch(sta):
     assert lib.sta_reorder(16, 32, 1, 2, 64, too_big, 0, None) != sta.STA_OK
 
 
+def test_paired_attention_needs_its_pairs(sta):
+    """sta_attn_fwd_paired / _raster_paired refuse a NULL or misaligned pair
+    array before anything runs."""
+    lib = ctypes.CDLL(sta.LIB_PATH)
+    g = sta.grid(2, 16, 16)
+    for fn in (lib.sta_attn_fwd_paired, lib.sta_attn_fwd_raster_paired):
+        fn.argtypes = sta._lib.sta_attn_fwd_paired.argtypes
+        assert fn(16, 16, 16, 16, None, 16, 16, None, 1, 1, 64, g, 0.0, None) == sta.STA_ERR_INVALID_ARG
+        assert fn(16, 16, 16, 16, None, 16, 16, 18, 1, 1, 64, g, 0.0, None) == sta.STA_ERR_INVALID_ARG
+
+
 def test_status_strings(sta):
     for s in range(8):
         assert sta.sta_status_string(s) != "unknown status"

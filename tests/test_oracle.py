@@ -673,3 +673,108 @@ def test_rectified_weights_sum_to_one_and_pool_over_real_tokens():
     # tile 1 is cut by the right edge (W = 12): 8 x 4 real tokens
     real = kt[0, 0, 64:128][O.valid_rows(T, H, W)[64:128]]
     assert real.shape[0] == n[1] == 32 and np.allclose(kb[0, 0, 1], real.mean(0))
+
+
+# ---------------------------------------------------------------- query-tile pairing
+def _pair_cases(golden_dir):
+    import json
+
+    return json.load(open(os.path.join(golden_dir, "pair_cases.json")))["cases"]
+
+
+def _lists_mask(lists):
+    nt = len(lists)
+    m = np.zeros((nt, nt), dtype=bool)
+    for i, l in enumerate(lists):
+        m[i, list(l)] = True
+    return m
+
+
+def test_pairing_golden(golden_dir):
+    """Hand-derived pairings: equal lists found across non-frame neighbours,
+    the frame pairing kept on a tie, left-overs paired in ascending order, the
+    tie order of equal weights, and an odd tile count."""
+    for case in _pair_cases(golden_dir):
+        got = O.pair_query_tiles(_lists_mask(case["lists"]), case["T"], case["H"], case["W"])
+        assert got.tolist() == case["pairs"], (case["name"], got.tolist())
+
+
+PAIR_MUTANTS = {
+    "ties to the higher smaller tile": ("edges.append((-w, min(a, b), max(a, b)))",
+                                        "edges.append((-w, -min(a, b), max(a, b)))"),
+    "lightest pairs first": ("edges.append((-w, min(a, b), max(a, b)))", "edges.append((w, min(a, b), max(a, b)))"),
+    "greedy kept on a tie with the frame pairing": ("if pairs_union(mask, pairs) >= pairs_union(mask, dflt):",
+                                                    "if pairs_union(mask, pairs) > pairs_union(mask, dflt):"),
+    "left-overs paired from the top": ("left = [v for v in range(nt) if mate[v] < 0]",
+                                       "left = [v for v in range(nt) if mate[v] < 0][::-1]"),
+    "no frame-pairing fallback": ("pairs = dflt", "pass"),
+}
+
+
+def _pair_mutant(old, new):
+    import inspect
+
+    src = inspect.getsource(O.pair_query_tiles)
+    assert src.count(old) == 1, old
+    ns = dict(vars(sta_oracle))
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)
+    return ns["pair_query_tiles"]
+
+
+@pytest.mark.parametrize("name", sorted(PAIR_MUTANTS))
+def test_pairing_planted_mistakes_fail_the_golden_cases(golden_dir, name):
+    fn = _pair_mutant(*PAIR_MUTANTS[name])
+    wrong = 0
+    for case in _pair_cases(golden_dir):
+        wrong += fn(_lists_mask(case["lists"]), case["T"], case["H"], case["W"]).tolist() != case["pairs"]
+    assert wrong >= 1, name
+
+
+def test_pairing_is_a_partition_never_worse_than_the_default():
+    """Random top-k masks on ragged grids: every tile appears exactly once,
+    ceil(Nt/2) pairs, and the total union is at most the default pairing's.
+    The greedy part is maximal: no two tiles left over (before the
+    left-over pairing) are candidate partners."""
+    rng = np.random.default_rng(7)
+    for T, H, W, k in ((3, 19, 37, 3), (4, 16, 24, 2), (1, 40, 40, 5), (5, 8, 8, 2)):
+        nh, nw, nt, _ = O.tile_grid(T, H, W)
+        scores = rng.random((nt, nt))
+        mask = np.zeros((nt, nt), dtype=bool)
+        np.put_along_axis(mask, np.argsort(-scores, axis=1)[:, :k], True, axis=1)
+        flat = O.pair_query_tiles(mask, T, H, W)
+        assert flat.size == 2 * ((nt + 1) // 2)
+        tiles = flat[flat >= 0]
+        assert sorted(tiles.tolist()) == list(range(nt))
+        pairs = [(int(flat[2 * i]), int(flat[2 * i + 1])) for i in range(flat.size // 2)]
+        assert O.pairs_union(mask, pairs) <= O.pairs_union(mask, O.default_pairs(T, H, W))
+        # brute-force: the sequential greedy over every candidate pair, by
+        # exhaustive scan for the heaviest free pair each time
+        cand = {}
+        for a in range(nt):
+            t, rem = divmod(a, nh * nw)
+            y, x = divmod(rem, nw)
+            for dt, dy, dx in O.PAIR_OFFSETS:
+                if t + dt < T and 0 <= y + dy < nh and 0 <= x + dx < nw:
+                    b = ((t + dt) * nh + y + dy) * nw + x + dx
+                    cand[(min(a, b), max(a, b))] = int((mask[a] & mask[b]).sum())
+        free = set(range(nt))
+        matched = []
+        while True:
+            live = [(w, e) for e, w in cand.items() if e[0] in free and e[1] in free]
+            if not live:
+                break
+            w, e = max(live, key=lambda we: (we[0], -we[1][0], -we[1][1]))
+            matched.append(e)
+            free -= set(e)
+        if pairs != O.default_pairs(T, H, W):
+            for e in matched:
+                assert e in pairs, (T, H, W, e)
+
+
+def test_default_pairs_cover_every_tile():
+    for T, H, W in ((1, 8, 8), (2, 8, 24), (3, 19, 37), (5, 17, 9)):
+        nt = O.tile_grid(T, H, W)[2]
+        dp = O.default_pairs(T, H, W)
+        assert len(dp) == (nt + 1) // 2
+        tiles = sorted(t for p in dp for t in p if t >= 0)
+        assert tiles == list(range(nt))
