@@ -55,7 +55,7 @@ bool common_sizes_ok(int32_t B, int32_t heads, int32_t d, sta_grid g, Geo *geo, 
 // the split passes (tensor-core scores, then a select pass with four CTAs
 // per SM).
 struct MaskWs {
-  size_t qbar, kbar, bits, counts, sel, kfloor, pairw, total_min, qlo, klo, prows, total;
+  size_t qbar, kbar, bits, counts, sel, kfloor, pairc, total_min, qlo, klo, prows, total;
 };
 
 MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
@@ -75,8 +75,8 @@ MaskWs mask_ws_layout(int32_t B, int32_t heads, int32_t d, const Geo &g) {
   off = align_up(off + R * sizeof(int32_t), 256);
   w.kfloor = off;
   off = align_up(off + (size_t)B * heads * sizeof(int32_t), 256);
-  w.pairw = off;  // candidate-pair overlaps of the query-tile pairing
-  off = align_up(off + R * pairq::NOFF * sizeof(int32_t), 256);
+  w.pairc = off;  // each tile's pairing candidates, in the pairing's order
+  off = align_up(off + R * 2 * pairq::NOFF * sizeof(int32_t), 256);
   w.total_min = off;
   w.qlo = off;
   off = align_up(off + R * d * sizeof(float), 256);
@@ -357,15 +357,14 @@ sta_status launch_build(const void *q_tiled, const void *k_tiled, int32_t B, int
   STA_CUDA_TRY(cudaGetLastError());
   if (p->query_pairs != nullptr) {
     // query-tile pairing by list overlap, from the final row bitsets
-    int *pw = reinterpret_cast<int *>(ws + L.pairw);
-    const long long warps = R * pairq::NOFF;
-    pairq::pair_weights_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(bits, pw, R, g, wpr);
+    int *pc = reinterpret_cast<int *>(ws + L.pairc);
+    pairq::pair_candidates_kernel<<<(unsigned)((R * 32 + 255) / 256), 256, 0, s>>>(bits, pc, R, g, wpr);
     STA_CUDA_TRY(cudaGetLastError());
-    const size_t psmem = 2 * (size_t)g.Nt * sizeof(int);
+    const size_t psmem = 2 * (size_t)g.Nt * sizeof(int) + (size_t)g.Nt;
     if (psmem > 48 * 1024)
       STA_CUDA_TRY(cudaFuncSetAttribute(pairq::pair_match_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)psmem));
-    pairq::pair_match_kernel<<<(unsigned)(B * heads), pairq::MATCH_THREADS, psmem, s>>>(bits, pw, counts,
+    pairq::pair_match_kernel<<<(unsigned)(B * heads), pairq::MATCH_THREADS, psmem, s>>>(bits, counts, pc,
                                                                                        p->query_pairs, g, wpr);
     STA_CUDA_TRY(cudaGetLastError());
   }
@@ -498,8 +497,8 @@ static sta_status build_mask_any(const void *q_tiled, const void *k_tiled, int32
   if (select_smem(d, geo, p->use_scores != 0) > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
   if (p->query_pairs != nullptr) {
     if ((reinterpret_cast<uintptr_t>(p->query_pairs) & 3u) != 0) return STA_ERR_INVALID_ARG;
-    // the pairing keeps two int32 per tile of a head in shared memory
-    if (2 * (size_t)geo.Nt * sizeof(int) > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
+    // the pairing keeps two int32 and a byte per tile of a head in shared memory
+    if (2 * (size_t)geo.Nt * sizeof(int) + (size_t)geo.Nt > MAX_DYN_SMEM) return STA_ERR_UNSUPPORTED;
   }
   // window tables pack (t, tile row, tile column) into 12 + 10 + 10 bits
   if (p->windows != nullptr && (geo.T >= 4096 || geo.NH >= 1024 || geo.NW >= 1024)) return STA_ERR_UNSUPPORTED;

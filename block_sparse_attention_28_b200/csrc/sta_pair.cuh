@@ -11,8 +11,9 @@
 // gives the sequential greedy result; the tiles left over are paired in
 // ascending order; and the pairing is kept only if its total union is below
 // that of the attention's default frame pairing.
-//   pair_weights_kernel  one warp per (tile, offset): |L_a n L_b| from the row
-//                        bitsets of the mask build (AND + popcount over words)
+//   pair_candidates_kernel  one warp per tile: the overlaps of its candidates
+//                        from the row bitsets of the mask build (AND + popcount
+//                        over words), sorted in the total order
 //   pair_match_kernel    one CTA per head: the matching, the left-over tiles,
 //                        the comparison with the frame pairing, the output
 #pragma once
@@ -46,49 +47,13 @@ __device__ __forceinline__ void offset(int k, int &dt, int &dy, int &dx) {
   }
 }
 
-// Tile a + offset k, or -1 outside the grid.
-__device__ __forceinline__ int neighbour(const Geo &g, int a, int k) {
+// Tile (t, y, x) + sign * offset k, or -1 outside the grid.
+__device__ __forceinline__ int step(const Geo &g, int t, int y, int x, int k, int sign) {
   int dt, dy, dx;
   offset(k, dt, dy, dx);
-  const int tpf = g.NH * g.NW;
-  const int t = a / tpf, rem = a - t * tpf;
-  const int y = rem / g.NW, x = rem - y * g.NW;
-  const int t2 = t + dt, y2 = y + dy, x2 = x + dx;
-  if (t2 >= g.T || y2 < 0 || y2 >= g.NH || x2 < 0 || x2 >= g.NW) return -1;
+  const int t2 = t + sign * dt, y2 = y + sign * dy, x2 = x + sign * dx;
+  if (t2 < 0 || t2 >= g.T || y2 < 0 || y2 >= g.NH || x2 < 0 || x2 >= g.NW) return -1;
   return (t2 * g.NH + y2) * g.NW + x2;
-}
-
-// Tile a - offset k (the tile whose candidate k is a), or -1.
-__device__ __forceinline__ int back_neighbour(const Geo &g, int a, int k) {
-  int dt, dy, dx;
-  offset(k, dt, dy, dx);
-  const int tpf = g.NH * g.NW;
-  const int t = a / tpf, rem = a - t * tpf;
-  const int y = rem / g.NW, x = rem - y * g.NW;
-  const int t2 = t - dt, y2 = y - dy, x2 = x - dx;
-  if (t2 < 0 || y2 < 0 || y2 >= g.NH || x2 < 0 || x2 >= g.NW) return -1;
-  return (t2 * g.NH + y2) * g.NW + x2;
-}
-
-// w[(bh*Nt + a)*NOFF + k] = |L_a n L_b| for b = a + offset k, -1 if b is off
-// the grid.
-__global__ void __launch_bounds__(256)
-pair_weights_kernel(const unsigned int *__restrict__ bits, int *__restrict__ w, long long R, Geo g, int wpr) {
-  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (gw >= R * NOFF) return;
-  const long long row = gw / NOFF;
-  const int k = (int)(gw - row * NOFF);
-  const int a = (int)(row % g.Nt);
-  const int b = neighbour(g, a, k);
-  int c = 0;
-  if (b >= 0) {
-    const unsigned int *ra = bits + row * wpr;
-    const unsigned int *rb = bits + (row - a + b) * wpr;
-    for (int i = lane; i < wpr; i += 32) c += __popc(ra[i] & rb[i]);
-    c = __reduce_add_sync(0xffffffffu, c);
-  }
-  if (lane == 0 && dbg_ok(gw < R * NOFF)) w[gw] = b >= 0 ? c : -1;
 }
 
 // Strict total order of candidate pairs: larger weight first, then the lower
@@ -100,12 +65,46 @@ __device__ __forceinline__ bool before(int w1, int a1, int b1, int w2, int a2, i
   return hi1 < hi2;
 }
 
-// |L_a n L_b| of two rows of one head, by one warp.
-__device__ __forceinline__ int overlap(const unsigned int *__restrict__ bits, long long r0, int a, int b, int wpr,
-                                      int lane) {
-  int c = 0;
-  for (int i = lane; i < wpr; i += 32) c += __popc(bits[(r0 + a) * wpr + i] & bits[(r0 + b) * wpr + i]);
-  return __reduce_add_sync(0xffffffffu, c);
+// One warp per tile v of a head: the overlaps |L_v n L_u| of its (up to
+// 2 * NOFF) candidates u = v +- offset k (AND + popcount of the two row
+// bitsets; the words of row v are loaded once), then the candidates in the
+// total order into cand[(bh*Nt + v)*2*NOFF + rank], -1 after the last. Lane j
+// holds candidate j; its rank is the number of candidates that come first.
+__global__ void __launch_bounds__(256)
+pair_candidates_kernel(const unsigned int *__restrict__ bits, int *__restrict__ cand, long long R, Geo g,
+                       int wpr) {
+  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= R) return;
+  const int v = (int)(row % g.Nt);
+  const int tpf = g.NH * g.NW;
+  const int t = v / tpf, rem = v - t * tpf;
+  const int y = rem / g.NW, x = rem - y * g.NW;
+  const unsigned int *rv = bits + row * wpr;
+  const unsigned int v0 = lane < wpr ? rv[lane] : 0u;  // rows of up to 32 words in one load
+  int my_u = -1, my_w = 0, n = 0;
+#pragma unroll 1
+  for (int j = 0; j < 2 * NOFF; ++j) {
+    const int u = step(g, t, y, x, j >> 1, (j & 1) ? -1 : 1);
+    if (u < 0) continue;  // uniform over the warp
+    const unsigned int *ru = bits + (row - v + u) * wpr;
+    int c = __popc(v0 & (lane < wpr ? ru[lane] : 0u));
+    for (int i = lane + 32; i < wpr; i += 32) c += __popc(rv[i] & ru[i]);
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (lane == n) {
+      my_u = u;
+      my_w = c;
+    }
+    ++n;
+  }
+  int rank = 0;
+  for (int i = 0; i < n; ++i) {
+    const int ui = __shfl_sync(0xffffffffu, my_u, i), wi = __shfl_sync(0xffffffffu, my_w, i);
+    if (lane < n && i != lane && before(wi, v, ui, my_w, v, my_u)) ++rank;
+  }
+  int *out = cand + row * 2 * NOFF;
+  if (lane < n && dbg_ok(rank < 2 * NOFF)) out[rank] = my_u;
+  if (lane >= n && lane < 2 * NOFF) out[lane] = -1;
 }
 
 // The default pairing of the attention kernels: pair i -> (qtA, qtB), qtB
@@ -124,45 +123,68 @@ __device__ __forceinline__ void frame_pair(const Geo &g, int i, int &qa, int &qb
   if (qb >= g.Nt) qb = -1;
 }
 
-// One CTA per (b, h). Shared memory: mate[Nt], best[Nt] (int32).
+// Exclusive prefix sum over the MATCH_THREADS threads of the block (all of
+// them call it); returns this thread's offset and the total in `total`.
+__device__ __forceinline__ int block_exclusive_scan(int x, int *tmp, int &total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) tmp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < MATCH_THREADS / 32 ? tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < MATCH_THREADS / 32) tmp[lane] = t;  // inclusive per warp
+  }
+  __syncthreads();
+  total = tmp[MATCH_THREADS / 32 - 1];
+  const int before = (warp > 0 ? tmp[warp - 1] : 0) + incl - x;
+  __syncthreads();  // tmp is reused by the next call
+  return before;
+}
+
+// One CTA per (b, h), on the candidate lists of pair_candidates_kernel: a
+// round only advances each free tile's pointer past candidates that got
+// matched, so a round costs a few loads per free tile however many rounds
+// ties make. Shared memory: mate[Nt], best[Nt] (int32), ptr[Nt] (uint8).
 __global__ void __launch_bounds__(MATCH_THREADS)
-pair_match_kernel(const unsigned int *__restrict__ bits, const int *__restrict__ w, const int *__restrict__ counts,
-                  int *__restrict__ pairs, Geo g, int wpr) {
+pair_match_kernel(const unsigned int *__restrict__ bits, const int *__restrict__ counts,
+                  const int *__restrict__ cand, int *__restrict__ pairs, Geo g, int wpr) {
   extern __shared__ int psm[];
   const int nt = g.Nt;
   int *mate = psm;       // partner, -1 while free
   int *best = psm + nt;  // this round's choice
+  uint8_t *ptr = reinterpret_cast<uint8_t *>(psm + 2 * nt);
   __shared__ long long cost[2];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ int scan_tmp[MATCH_THREADS / 32];
+  const int tid = threadIdx.x, lane = tid & 31;
   const long long r0 = (long long)blockIdx.x * nt;
-  const int *wh = w + r0 * NOFF;
-  for (int v = tid; v < nt; v += MATCH_THREADS) mate[v] = -1;
+  const int *ch = cand + r0 * 2 * NOFF;
+  for (int v = tid; v < nt; v += MATCH_THREADS) {
+    mate[v] = -1;
+    ptr[v] = 0;
+  }
   if (tid == 0) cost[0] = cost[1] = 0;
   __syncthreads();
   // locally-dominant matching: at most nt / 2 rounds (each round matches the
   // heaviest free candidate pair, if any)
   for (int round = 0; round <= nt / 2; ++round) {
     for (int v = tid; v < nt; v += MATCH_THREADS) {
-      int bu = -1, bw = 0;
+      int bu = -1;
       if (mate[v] < 0) {
-        for (int k = 0; k < NOFF; ++k) {
-          const int u = neighbour(g, v, k);
-          if (u >= 0 && mate[u] < 0) {
-            const int wt = wh[(long long)v * NOFF + k];
-            if (bu < 0 || before(wt, v, u, bw, v, bu)) {
-              bu = u;
-              bw = wt;
-            }
-          }
-          const int u2 = back_neighbour(g, v, k);
-          if (u2 >= 0 && mate[u2] < 0) {
-            const int wt = wh[(long long)u2 * NOFF + k];
-            if (bu < 0 || before(wt, v, u2, bw, v, bu)) {
-              bu = u2;
-              bw = wt;
-            }
-          }
-        }
+        const int *cv = ch + (long long)v * 2 * NOFF;
+        int p = ptr[v];
+        while (p < 2 * NOFF && cv[p] >= 0 && mate[cv[p]] >= 0) ++p;
+        ptr[v] = (uint8_t)p;
+        bu = (p < 2 * NOFF) ? cv[p] : -1;
       }
       best[v] = bu;
     }
@@ -177,39 +199,52 @@ pair_match_kernel(const unsigned int *__restrict__ bits, const int *__restrict__
     }
     if (!__syncthreads_or(changed)) break;
   }
-  // tiles left over: paired in ascending order (serial; Nt is small)
-  if (tid == 0) {
-    int prev = -1;
-    for (int v = 0; v < nt; ++v) {
-      if (mate[v] >= 0) continue;
-      if (prev < 0) {
-        prev = v;
-      } else {
-        mate[prev] = v;
-        mate[v] = prev;
-        prev = -1;
-      }
+  // tiles left over: paired in ascending order of their rank among the free
+  // tiles (2i with 2i + 1; a last one alone); best[] now lists them by rank
+  const int CH = (nt + MATCH_THREADS - 1) / MATCH_THREADS;  // tiles per thread, contiguous
+  const int v0 = tid * CH, v1 = min(nt, v0 + CH);
+  int nfree = 0;
+  for (int v = v0; v < v1; ++v) nfree += mate[v] < 0;
+  int total_free;
+  int rank = block_exclusive_scan(nfree, scan_tmp, total_free);
+  __syncthreads();  // every thread has read mate[] for the scan
+  for (int v = v0; v < v1; ++v)
+    if (mate[v] < 0) best[rank++] = v;
+  __syncthreads();
+  for (int r = 2 * tid; r < total_free; r += 2 * MATCH_THREADS) {
+    const int a = best[r];
+    if (r + 1 < total_free) {
+      const int b = best[r + 1];
+      mate[a] = b;
+      mate[b] = a;
+    } else {
+      mate[a] = nt;  // alone (odd count): marked past the end
     }
-    if (prev >= 0) mate[prev] = nt;  // alone (odd count): marked past the end
   }
   __syncthreads();
   // total union of this pairing (pairs led by their lower tile) and of the
-  // default pairing, one warp per pair
+  // default pairing; a thread per pair, the overlap over the row words
   const int np = (nt + 1) / 2;
-  const int nwarps = MATCH_THREADS / 32;
   long long c_greedy = 0, c_frame = 0;
-  for (int v = warp; v < nt; v += nwarps) {
+  auto ovl = [&](int x, int y) {
+    int c = 0;
+    for (int i = 0; i < wpr; ++i) c += __popc(bits[(r0 + x) * wpr + i] & bits[(r0 + y) * wpr + i]);
+    return c;
+  };
+  for (int v = tid; v < nt; v += MATCH_THREADS) {
     const int u = mate[v];
     if (u < v) continue;  // led by the partner
     const int ca = counts[r0 + v];
-    c_greedy += (u >= nt) ? ca : ca + counts[r0 + u] - overlap(bits, r0, v, u, wpr, lane);
+    c_greedy += (u >= nt) ? ca : ca + counts[r0 + u] - ovl(v, u);
   }
-  for (int i = warp; i < np; i += nwarps) {
+  for (int i = tid; i < np; i += MATCH_THREADS) {
     int qa, qb;
     frame_pair(g, i, qa, qb);
     const int ca = counts[r0 + qa];
-    c_frame += (qb < 0) ? ca : ca + counts[r0 + qb] - overlap(bits, r0, qa, qb, wpr, lane);
+    c_frame += (qb < 0) ? ca : ca + counts[r0 + qb] - ovl(qa, qb);
   }
+  c_greedy = __reduce_add_sync(0xffffffffu, (unsigned)c_greedy);  // < 2^32 per warp: Nt^2 < 2^31
+  c_frame = __reduce_add_sync(0xffffffffu, (unsigned)c_frame);
   if (lane == 0) {
     atomicAdd(reinterpret_cast<unsigned long long *>(&cost[0]), (unsigned long long)c_greedy);
     atomicAdd(reinterpret_cast<unsigned long long *>(&cost[1]), (unsigned long long)c_frame);
@@ -217,19 +252,20 @@ pair_match_kernel(const unsigned int *__restrict__ bits, const int *__restrict__
   __syncthreads();
   int *out = pairs + (long long)blockIdx.x * 2 * np;
   if (cost[0] < cost[1]) {
-    // pairs in ascending order of their lower tile: the rank of a leader is
-    // the number of leaders before it (serial count; Nt is small)
-    if (tid == 0) {
-      int i = 0;
-      for (int v = 0; v < nt; ++v) {
-        const int u = mate[v];
-        if (u < v) continue;
-        if (dbg_ok(i < np)) {
-          out[2 * i] = v;
-          out[2 * i + 1] = (u >= nt) ? -1 : u;
-        }
-        ++i;
+    // pairs in ascending order of their lower tile: a leader's slot is the
+    // number of leaders before it
+    int nlead = 0;
+    for (int v = v0; v < v1; ++v) nlead += mate[v] >= v;
+    int total_lead;
+    int slot = block_exclusive_scan(nlead, scan_tmp, total_lead);
+    for (int v = v0; v < v1; ++v) {
+      const int u = mate[v];
+      if (u < v) continue;
+      if (dbg_ok(slot < np)) {
+        out[2 * slot] = v;
+        out[2 * slot + 1] = (u >= nt) ? -1 : u;
       }
+      ++slot;
     }
   } else {
     for (int i = tid; i < np; i += MATCH_THREADS) {
