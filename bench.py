@@ -765,7 +765,7 @@ def build_roofline(layer, build_ms, peaks):
     achieved = nbytes / (build_ms * 1e-3) / 1e9
     peak = float(peaks.get("hbm_gbs", 6650.0))
     return {"bound": "hbm", "algorithmic_bytes": nbytes, "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "kernels": "pool_tma, score_tc, score_select, scan, fill"}
+            "frac": achieved / peak, "kernels": "pool_tma, score_tc, select_rows, scan, fill"}
 
 
 def mma_probe(sta, iters=4096):

@@ -96,6 +96,22 @@ def case(tag, T, H, W, Hh, d, top_p, k_min, seed, G=2, head_floor=False):
     status(tag + "_rectified")
     keep(tag + "_o_rect", o_x.view(torch.int16))
 
+    # the overlap pairing of the query tiles and the paired calls
+    qp = torch.full((B * Hh, 2 * ((nt + 1) // 2)), -7, dtype=torch.int32, device="cuda")
+    pb = sta.MaskBuffers(B, Hh, d, g, "cuda")
+    sta.build_mask(qt, kt, B, Hh, d, g, sta.mask_params(0.0, max(1, nt // 8), True, 0.0, cfg.group_lo,
+                                                        query_pairs=qp), pb)
+    status(tag + "_build_pairs")
+    keep(tag + "_query_pairs", qp)
+    o_p = torch.zeros_like(qt)
+    sta.sta_attn_fwd_paired(qt, kt, vt, o_p, None, pb.row_ptr, pb.col_idx, qp, B, Hh, d, g)
+    status(tag + "_attn_paired")
+    keep(tag + "_o_paired", o_p.view(torch.int16))
+    o_pr = torch.zeros_like(q)
+    sta.sta_attn_fwd_raster_paired(q, k, v, o_pr, None, pb.row_ptr, pb.col_idx, qp, B, Hh, d, g)
+    status(tag + "_attn_raster_paired")
+    keep(tag + "_o_raster_paired", o_pr.view(torch.int16))
+
     w_out = torch.zeros((B * Hh, len(cfg.group_lo), 4), dtype=torch.int32, device="cuda")
     stats = torch.zeros((B * Hh, 2), dtype=torch.float32, device="cuda")
     sta.sta_search_windows(mass, B, Hh, g, cfg.group_lo, 0.9, 0.5, w_out, stats)
