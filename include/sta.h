@@ -95,10 +95,11 @@ typedef struct {
                               values are clamped to [0, 1] and q_tiled, k_tiled
                               are not read */
   int32_t *query_pairs;   /* optional output, device int32 [B*heads][2*NP],
-                              NP = ceil(Nt/2), or NULL: the query tiles of
-                              each head paired into the 128-row tiles of
-                              sta_attn_fwd_paired, chosen by list overlap
-                              (see sta_attn_fwd_paired) */
+                              NP = ceil(Nt/2), 4-byte aligned, or NULL: the
+                              query tiles of each head paired into the 128-row
+                              tiles of sta_attn_fwd_paired, chosen by list
+                              overlap (see sta_attn_fwd_paired); needs
+                              9*Nt <= 227 KB (STA_ERR_UNSUPPORTED otherwise) */
 } sta_mask_params;
 
 /* Number of tiles per head (Nt) and padded rows per head (Lpad) of a grid;
