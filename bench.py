@@ -43,6 +43,26 @@ HEADLINE = "dit720p"  # the 75,600-token 720p layer
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+NVTX = False  # --nvtx: name the calls of each step on the profiler timeline
+
+
+class nvtx_range:
+    """An NVTX range around one library call when --nvtx is given (for nsys /
+    ncu timelines); nothing otherwise."""
+
+    def __init__(self, name):
+        self.name = name
+
+    def __enter__(self):
+        if NVTX:
+            torch.cuda.nvtx.range_push(self.name)
+
+    def __exit__(self, *exc):
+        if NVTX:
+            torch.cuda.nvtx.range_pop()
+        return False
+
+
 def flops_per_pair(d):
     return 4.0 * 64 * 64 * d
 
@@ -386,10 +406,12 @@ class Layer:
         if ev is not None:
             ev[0].record()
             ev[1].record()
-        self.build()
+        with nvtx_range("sta_build_mask_raster"):
+            self.build()
         if ev is not None:
             ev[2].record()
-        self.attn()
+        with nvtx_range("sta_attn_fwd_raster"):
+            self.attn()
         if ev is not None:
             ev[3].record()
             ev[4].record()
@@ -883,6 +905,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-mask run of the same kernel")
+    ap.add_argument("--nvtx", action="store_true", help="NVTX ranges around the calls of each step")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per-config record of the other workload layers (1 GPU only)")
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(CONFIGS),
@@ -899,6 +922,8 @@ def main():
     ap.add_argument("--search-curve", action="store_true",
                     help="print the recall-target vs density curve of the window search and exit")
     args = ap.parse_args()
+    global NVTX
+    NVTX = args.nvtx
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
