@@ -111,6 +111,8 @@ _lib.sta_selftest_wait_timeout.argtypes = [_i64, _vp]
 _lib.sta_selftest_wait_timeout.restype = ctypes.c_int
 _lib.sta_get_device_error.argtypes = [_vp]
 _lib.sta_get_device_error.restype = ctypes.c_int
+_lib.sta_validate_csr.argtypes = [_vp, _vp, _i64, _i32, _i32, Grid, _vp]
+_lib.sta_validate_csr.restype = ctypes.c_int
 _lib.sta_debug_build.argtypes = []
 _lib.sta_debug_build.restype = _i32
 _lib.sta_status_string.argtypes = [ctypes.c_int]
@@ -140,6 +142,14 @@ def _check(status, what):
 
 def grid(T, H, W):
     return Grid(int(T), int(H), int(W))
+
+
+def sta_validate_csr(row_ptr, col_idx, B, heads, g, col_capacity=None, stream=None):
+    """Checks a caller's CSR on the device (result in sta_get_device_error);
+    col_capacity defaults to col_idx.numel()."""
+    cap = col_idx.numel() if col_capacity is None else int(col_capacity)
+    _check(_lib.sta_validate_csr(_ptr(row_ptr), _ptr(col_idx), cap, B, heads, g, _stream(stream)),
+           "sta_validate_csr")
 
 
 def sta_debug_build():

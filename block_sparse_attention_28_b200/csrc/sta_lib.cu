@@ -689,6 +689,20 @@ sta_status sta_selftest_wait_timeout(int64_t limit_cycles, sta_stream_t stream) 
   return STA_OK;
 }
 
+sta_status sta_validate_csr(const int32_t *row_ptr, const int32_t *col_idx, int64_t col_capacity, int32_t B,
+                            int32_t heads, sta_grid g, sta_stream_t stream) {
+  Geo geo;
+  if (!make_geo(g, &geo) || B <= 0 || heads <= 0) return STA_ERR_INVALID_ARG;
+  if (row_ptr == nullptr || col_idx == nullptr || col_capacity < 0) return STA_ERR_INVALID_ARG;
+  if (!device_is_sm100()) return STA_ERR_UNSUPPORTED;
+  const long long R = (long long)B * heads * geo.Nt;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  validate_csr_kernel<<<(unsigned)((R * 32 + 255) / 256), 256, 0, s>>>(row_ptr, col_idx, (long long)col_capacity,
+                                                                       R, geo.Nt);
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
+}
+
 sta_status sta_get_device_error(sta_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   STA_CUDA_TRY(cudaStreamSynchronize(s));

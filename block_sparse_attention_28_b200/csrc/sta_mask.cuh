@@ -635,6 +635,29 @@ scan_kernel(const int *__restrict__ counts, int *__restrict__ row_ptr, long long
   if (tid == 0) *nnz = carry;
 }
 
+// ---------------------------------------------------------------- validate
+// One warp per row of a caller's CSR: the offsets are read first and checked
+// (row_ptr[0] == 0, non-decreasing, at most Nt entries per row, inside the
+// column array's capacity), and only then the row's columns, which must be
+// strictly ascending and in [0, Nt). Any violation sets DEV_ERR_BAD_MASK.
+__global__ void __launch_bounds__(256)
+validate_csr_kernel(const int *__restrict__ row_ptr, const int *__restrict__ col_idx, long long capacity,
+                    long long R, int nt) {
+  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= R) return;
+  const long long a0 = row_ptr[row], a1 = row_ptr[row + 1];
+  bool bad = (row == 0 && a0 != 0) || a0 < 0 || a1 < a0 || a1 - a0 > nt || a1 > capacity;
+  if (!bad) {
+    for (long long i = a0 + lane; i < a1; i += 32) {
+      const int c = col_idx[i];
+      const int prev = (i > a0) ? col_idx[i - 1] : -1;
+      if (c < 0 || c >= nt || c <= prev) bad = true;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(DEV_ERR_BAD_MASK);
+}
+
 // ---------------------------------------------------------------- fill
 // One warp per row: word prefix popcounts -> ascending column indices.
 __global__ void __launch_bounds__(256)

@@ -393,6 +393,20 @@ sta_status sta_selftest_wait_timeout(int64_t limit_cycles, sta_stream_t stream);
  * wait, reported as well). The pages have no counterpart. */
 int32_t sta_debug_build(void);
 
+/* sta_validate_csr -- checks a caller's CSR lists before they are handed to
+ * the attention calls (the pages have no counterpart: masks the library
+ * builds are valid by construction). One warp per row
+ * r < B*heads*Nt reads row_ptr[r], row_ptr[r+1] first and checks
+ * row_ptr[0] == 0, row_ptr[r] <= row_ptr[r+1] <= col_capacity and at most Nt
+ * entries per row; only then it reads the row's columns, which must be
+ * strictly ascending and in [0, Nt). Any violation records STA_ERR_BAD_MASK
+ * in the device error word (read it with sta_get_device_error); nothing is
+ * written. row_ptr must hold B*heads*Nt + 1 entries; col_capacity is the
+ * number of int32 the col_idx array holds, so that no read leaves it.
+ * Asynchronous on `stream`; argument errors are returned at once. */
+sta_status sta_validate_csr(const int32_t *row_ptr, const int32_t *col_idx, int64_t col_capacity, int32_t B,
+                            int32_t heads, sta_grid g, sta_stream_t stream);
+
 /* Reads and clears the device error word of the current device after
  * synchronising `stream`. STA_OK if no device-side fault was recorded;
  * STA_ERR_BOUNDS takes precedence over STA_ERR_TIMEOUT (a skipped access is

@@ -119,6 +119,17 @@ def test_paired_attention_needs_its_pairs(sta):
         assert fn(16, 16, 16, 16, None, 16, 16, 18, 1, 1, 64, g, 0.0, None) == sta.STA_ERR_INVALID_ARG
 
 
+def test_csr_validation_checks_its_arguments_on_the_host(sta):
+    lib = ctypes.CDLL(sta.LIB_PATH)
+    lib.sta_validate_csr.argtypes = sta._lib.sta_validate_csr.argtypes
+    g = sta.grid(2, 16, 16)
+    assert lib.sta_validate_csr(None, 16, 8, 1, 1, g, None) == sta.STA_ERR_INVALID_ARG
+    assert lib.sta_validate_csr(16, None, 8, 1, 1, g, None) == sta.STA_ERR_INVALID_ARG
+    assert lib.sta_validate_csr(16, 16, -1, 1, 1, g, None) == sta.STA_ERR_INVALID_ARG
+    assert lib.sta_validate_csr(16, 16, 8, 0, 1, g, None) == sta.STA_ERR_INVALID_ARG
+    assert lib.sta_validate_csr(16, 16, 8, 1, 1, sta.grid(0, 16, 16), None) == sta.STA_ERR_INVALID_ARG
+
+
 def test_status_strings(sta):
     for s in range(8):
         assert sta.sta_status_string(s) != "unknown status"

@@ -162,3 +162,51 @@ def test_pair_index_out_of_range_is_reported(sta, gp):
     a, b = int(pairs[0, 0]), int(pairs[0, 1])
     for t in (a, b):
         assert torch.equal(o[0, 0, 64 * t:64 * t + 64], o2[0, 0, 64 * t:64 * t + 64])
+
+
+def test_csr_validation(sta, gp):
+    """sta_validate_csr: a mask the library built passes; each kind of
+    corruption of a caller's CSR is reported as STA_ERR_BAD_MASK, and the
+    offsets are checked against the column capacity before any column is
+    read."""
+    T, H, W, Hh, B, d = 3, 19, 37, 2, 1, 128
+    g = sta.grid(T, H, W)
+    nt = sta.sta_num_tiles(g)
+    gen = torch.Generator(device="cuda").manual_seed(4)
+    sc = torch.rand((B, Hh, nt, nt), generator=gen, device="cuda")
+    bufs = sta.MaskBuffers(B, Hh, d, g, "cuda")
+    sta.build_mask(None, None, B, Hh, d, g, sta.mask_params(0.0, 5, True, block_scores=sc), bufs)
+    torch.cuda.synchronize()
+    assert sta.sta_get_device_error() == sta.STA_OK
+    nnz = int(bufs.nnz.item())
+    sta.sta_validate_csr(bufs.row_ptr, bufs.col_idx, B, Hh, g)
+    assert sta.sta_get_device_error() == sta.STA_OK
+    sta.sta_validate_csr(bufs.row_ptr, bufs.col_idx, B, Hh, g, col_capacity=nnz)
+    assert sta.sta_get_device_error() == sta.STA_OK
+
+    def corrupt(fn, cap=None):
+        rp, ci = bufs.row_ptr.clone(), bufs.col_idx.clone()
+        fn(rp, ci)
+        sta.sta_validate_csr(rp, ci, B, Hh, g, col_capacity=cap)
+        return sta.sta_get_device_error()
+
+    def swap_cols(rp, ci):
+        a = int(rp[7])
+        ci[a], ci[a + 1] = ci[a + 1].clone(), ci[a].clone()
+
+    def dup_col(rp, ci):
+        a = int(rp[9])
+        ci[a + 1] = ci[a]
+
+    cases = {
+        "first offset not zero": lambda rp, ci: rp.__setitem__(0, 1),
+        "offsets decrease": lambda rp, ci: rp.__setitem__(5, int(rp[4]) - 1),
+        "column past Nt": lambda rp, ci: ci.__setitem__(int(rp[3]), nt),
+        "negative column": lambda rp, ci: ci.__setitem__(int(rp[3]), -1),
+        "columns out of order": swap_cols,
+        "repeated column": dup_col,
+    }
+    for name, fn in cases.items():
+        assert corrupt(fn) == sta.STA_ERR_BAD_MASK, name
+    # offsets beyond the column capacity: refused before the columns are read
+    assert corrupt(lambda rp, ci: None, cap=nnz - 1) == sta.STA_ERR_BAD_MASK
