@@ -33,7 +33,7 @@ def load_mask(path, device="cuda"):
     on `device`: row_ptr, col_idx (capacity B*heads*Nt*Nt, as sta_build_mask
     writes it, the first nnz entries filled), nnz (device int64 [1]), and
     windows / query_pairs when saved."""
-    blob = torch.load(path, map_location="cpu", weights_only=False)
+    blob = torch.load(path, map_location="cpu", weights_only=True)  # tensors and plain values only
     if blob.get("format") != FORMAT:
         raise ValueError(f"{path}: not a saved sta mask")
     T, H, W = blob["grid"]
