@@ -243,7 +243,9 @@ pair_match_kernel(const unsigned int *__restrict__ bits, const int *__restrict__
     const int ca = counts[r0 + qa];
     c_frame += (qb < 0) ? ca : ca + counts[r0 + qb] - ovl(qa, qb);
   }
-  c_greedy = __reduce_add_sync(0xffffffffu, (unsigned)c_greedy);  // < 2^32 per warp: Nt^2 < 2^31
+  // a warp's sum is at most 32 (Nt/512 + 1) 2 Nt < 2^32 for every Nt whose
+  // 9 Nt bytes of shared memory the launch allows
+  c_greedy = __reduce_add_sync(0xffffffffu, (unsigned)c_greedy);
   c_frame = __reduce_add_sync(0xffffffffu, (unsigned)c_frame);
   if (lane == 0) {
     atomicAdd(reinterpret_cast<unsigned long long *>(&cost[0]), (unsigned long long)c_greedy);
