@@ -58,3 +58,8 @@ def test_bench_json_line():
         assert x["attn_ms"] > 0 and x["build_ms"] > 0 and x["kept_pairs"] > 0
         assert 0 < x["frac_burst"] <= x["frac_sustained"] < 1.5 and 0 < x["pairing_efficiency"] <= 1.0
         assert isinstance(x["clocks"]["reasons"], list)
+    # the reuse rows run the overlap pairing, which never does worse than the
+    # frame pairing it is compared with
+    for x in rows[-5:]:
+        assert x["pairing"].startswith("overlap")
+        assert x["pairing_efficiency"] >= x["pairing_efficiency_frames"] - 1e-12
