@@ -47,7 +47,8 @@ typedef enum {
   STA_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than required */
   STA_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed */
   STA_ERR_TIMEOUT = 5,     /* device: a bounded pipeline wait ran out */
-  STA_ERR_BAD_MASK = 6,    /* device: a CSR column index out of range */
+  STA_ERR_BAD_MASK = 6,    /* device: a CSR column index or query pair out of
+                              range, or a CSR that sta_validate_csr rejects */
   STA_ERR_BOUNDS = 7       /* device, checked build only: an index or address
                               failed its bounds / alignment check; the access
                               was skipped (see sta_debug_build) */
